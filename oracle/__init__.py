@@ -1,0 +1,211 @@
+"""fp64 CPU oracle for the fused DiT per-token operators (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU baseline and
+reference arm may import this package.  The product library (``dit_block_b200``)
+never imports it and shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP over rows); this module
+only marshals numpy arrays into it.  Inputs are numpy arrays of ``float32``,
+``float64`` or ``uint16`` (the raw bits of bf16 values); every output is ``float64``.
+Each function names the operator it computes; the definitions and the page passages
+they follow are in the header of ``oracle.c``.
+
+Parity status: every function is pinned by ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32, BF16, F64 = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c with gcc (-O2, OpenMP, no fast-math) into liboracle.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P, I64, I32, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+        I = ctypes.c_int
+        lib.oracle_num_threads.restype = I
+        lib.oracle_adaln_modulate.argtypes = [P, I64, P, I64, I, P, P, I64, I, P, I32, I64, I64, I64, D]
+        lib.oracle_adaln_modulate.restype = None
+        lib.oracle_gated_residual.argtypes = [P, I64, P, I64, P, I64, I, P, I64, I, P, I32, I64, I64, I64]
+        lib.oracle_gated_residual.restype = None
+        lib.oracle_swiglu.argtypes = [P, I64, P, P, I64, I, I64, I64]
+        lib.oracle_swiglu.restype = None
+        lib.oracle_qk_rmsnorm_rope3d.argtypes = [P, P, I64, I64, P, P, I64, I64, I, P, P, I, P,
+                                                 I32, I32, I32, I64, I32, I32, I32, D, I64, I32, I32, D]
+        lib.oracle_qk_rmsnorm_rope3d.restype = I
+        lib.oracle_dit_prologue.argtypes = [P, P, P, P, I, P, P, P, I64, I64, I, P, I32, I64, I64, I64, D]
+        lib.oracle_dit_prologue.restype = None
+        lib.oracle_dit_epilogue.argtypes = [P, P, I64, I, P, P, I, P, I32, I32, I32, I64,
+                                            I32, I32, I32, D, I64, I32, I32, D]
+        lib.oracle_dit_epilogue.restype = I
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle runs on."""
+    return int(_load().oracle_num_threads())
+
+
+def _code(a: np.ndarray | None) -> int:
+    if a is None:
+        return F32
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    if a.dtype == np.float64:
+        return F64
+    raise TypeError(f"oracle inputs are float32, float64 or uint16 (bf16 bits), got {a.dtype}")
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags.c_contiguous, "oracle inputs must be C-contiguous"
+    return a.ctypes.data
+
+
+def _ld(a: np.ndarray) -> int:
+    return a.shape[-1] if a.ndim > 1 else a.shape[0]
+
+
+def _mod_args(mod: np.ndarray | None, stream_id, n_streams, tokens_per_sample):
+    ld_mod = _ld(mod) if mod is not None else 0
+    sid = None
+    if stream_id is not None:
+        sid = np.ascontiguousarray(stream_id, dtype=np.uint8)
+    return ld_mod, sid, int(n_streams), int(tokens_per_sample)
+
+
+def adaln_modulate(x, shift=None, scale=None, *, eps=1e-6, stream_id=None, n_streams=1,
+                   tokens_per_sample=0, n_tokens=None, d=None):
+    """h = LN(x) * (1 + scale[r]) + shift[r] per token row of x ([N, ld_x], first d columns)."""
+    n = x.shape[0] if n_tokens is None else n_tokens
+    d = x.shape[1] if d is None else d
+    mod = shift if shift is not None else scale
+    ld_mod, sid, S, tps = _mod_args(mod, stream_id, n_streams, tokens_per_sample)
+    out = np.empty((n, d), np.float64)
+    _load().oracle_adaln_modulate(out.ctypes.data, d, _ptr(x), _ld(x), _code(x), _ptr(shift),
+                                  _ptr(scale), ld_mod, _code(mod), _ptr(sid), S, tps, n, d,
+                                  float(eps))
+    return out
+
+
+def gated_residual(x, y, gate=None, *, stream_id=None, n_streams=1, tokens_per_sample=0,
+                   n_tokens=None, d=None):
+    """o = x + gate[r] * y per token row."""
+    assert x.dtype == y.dtype
+    n = x.shape[0] if n_tokens is None else n_tokens
+    d = x.shape[1] if d is None else d
+    ld_mod, sid, S, tps = _mod_args(gate, stream_id, n_streams, tokens_per_sample)
+    out = np.empty((n, d), np.float64)
+    _load().oracle_gated_residual(out.ctypes.data, d, _ptr(x), _ld(x), _ptr(y), _ld(y), _code(x),
+                                  _ptr(gate), ld_mod, _code(gate), _ptr(sid), S, tps, n, d)
+    return out
+
+
+def swiglu(u, inner=None, *, n_tokens=None):
+    """o[:, j] = silu(u[:, j]) * u[:, inner + j] for the packed up-projection u [N, 2*inner]."""
+    n = u.shape[0] if n_tokens is None else n_tokens
+    inner = u.shape[1] // 2 if inner is None else inner
+    out = np.empty((n, inner), np.float64)
+    esz = u.dtype.itemsize
+    _load().oracle_swiglu(out.ctypes.data, inner, _ptr(u), u.ctypes.data + inner * esz,
+                          _ld(u), _code(u), n, inner)
+    return out
+
+
+def swiglu_ab(a, b):
+    """o = silu(a) * b for two separate [N, inner] tensors of one dtype."""
+    assert a.shape == b.shape and a.dtype == b.dtype
+    n, inner = a.shape
+    out = np.empty((n, inner), np.float64)
+    _load().oracle_swiglu(out.ctypes.data, inner, _ptr(a), _ptr(b), inner, _code(a), n, inner)
+    return out
+
+
+def _pos_ptr(pos):
+    if pos is None:
+        return None, None
+    p = np.ascontiguousarray(pos, dtype=np.int32)
+    assert p.ndim == 2 and p.shape[1] == 3
+    return p, p.ctypes.data
+
+
+def qk_rmsnorm_rope3d(q, k, wq=None, wk=None, *, n_heads, head_dim, pos=None, grid=(0, 0, 0),
+                      tokens_per_sample=0, dims=(32, 48, 48), theta=10000.0, eps=1e-6):
+    """QK RMSNorm then 3D RoPE on each head vector of q [N, ld_q] and k [N, ld_k].
+
+    Either q or k may be None.  Returns (q_out, k_out) as [N, n_heads*head_dim] float64."""
+    src = q if q is not None else k
+    n = src.shape[0]
+    hd = n_heads * head_dim
+    qo = np.empty((n, hd), np.float64) if q is not None else None
+    ko = np.empty((n, hd), np.float64) if k is not None else None
+    w = wq if wq is not None else wk
+    pos_arr, pos_p = _pos_ptr(pos)
+    rc = _load().oracle_qk_rmsnorm_rope3d(
+        _ptr(qo), _ptr(ko), hd, hd, _ptr(q), _ptr(k), _ld(q) if q is not None else 0,
+        _ld(k) if k is not None else 0, _code(src), _ptr(wq), _ptr(wk), _code(w), pos_p,
+        int(grid[0]), int(grid[1]), int(grid[2]), int(tokens_per_sample), int(dims[0]),
+        int(dims[1]), int(dims[2]), float(theta), n, int(n_heads), int(head_dim), float(eps))
+    if rc != 0:
+        raise ValueError("RoPE split does not fit head_dim (dims must be even and sum to it)")
+    return qo, ko
+
+
+def dit_prologue(x, y=None, gate=None, shift=None, scale=None, *, eps=1e-6, stream_id=None,
+                 n_streams=1, tokens_per_sample=0):
+    """Fused prologue: x' = x + gate*y (when y is given), h = AdaLN(x').  Returns (x', h);
+    x' is None when y is None."""
+    n, d = x.shape
+    mod = next((m for m in (gate, shift, scale) if m is not None), None)
+    ld_mod, sid, S, tps = _mod_args(mod, stream_id, n_streams, tokens_per_sample)
+    xo = np.empty((n, d), np.float64) if y is not None else None
+    h = np.empty((n, d), np.float64)
+    _load().oracle_dit_prologue(_ptr(xo), h.ctypes.data, _ptr(x), _ptr(y), _code(x), _ptr(gate),
+                                _ptr(shift), _ptr(scale), d, ld_mod, _code(mod), _ptr(sid), S, tps,
+                                n, d, float(eps))
+    return xo, h
+
+
+def dit_epilogue(qkv, wq=None, wk=None, *, n_heads, head_dim, pos=None, grid=(0, 0, 0),
+                 tokens_per_sample=0, dims=(32, 48, 48), theta=10000.0, eps=1e-6):
+    """Fused QKV epilogue on packed rows [q | k | v]: returns [N, 2*n_heads*head_dim] with the
+    normed+rotated q then k."""
+    n = qkv.shape[0]
+    hd = n_heads * head_dim
+    out = np.empty((n, 2 * hd), np.float64)
+    w = wq if wq is not None else wk
+    pos_arr, pos_p = _pos_ptr(pos)
+    rc = _load().oracle_dit_epilogue(
+        out.ctypes.data, _ptr(qkv), _ld(qkv), _code(qkv), _ptr(wq), _ptr(wk), _code(w), pos_p,
+        int(grid[0]), int(grid[1]), int(grid[2]), int(tokens_per_sample), int(dims[0]),
+        int(dims[1]), int(dims[2]), float(theta), n, int(n_heads), int(head_dim), float(eps))
+    if rc != 0:
+        raise ValueError("RoPE split does not fit head_dim (dims must be even and sum to it)")
+    return out
