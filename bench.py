@@ -1,0 +1,444 @@
+"""Throughput of the fused DiT-block per-token hot path on B200.
+
+One step = one pass of the whole path over the workload, five libsol launches on one
+stream (AdaLN -> QKV epilogue -> prologue -> SwiGLU -> gated residual; see
+dit_block_b200/block.py).  Default workload: the full-resolution 10 s grid, 61x48x84 =
+245,952 tokens, d=5120, 40x128 heads, SwiGLU width 13,824, bf16, 0.1% +-50 outliers.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+N > 1 is launched by torchrun, one rank per GPU; every rank processes its own copy of
+the workload (weak scaling, no collective on the data path) and the time is the max
+over ranks.  Rank 0 prints one JSON line.
+
+value       algorithmic HBM bytes of all ranks' steps / device time (GB/s); every tensor
+            element an op must read or write counts once (216,064 B per token per step).
+e2e         the same metric through the public API with host buffers: per step, pinned
+            host -> device copies of every input, the five launches, device -> host
+            copies of every output, all inside the timed region.
+roofline    the SwiGLU launch (the largest byte mover): achieved GB/s from CUDA events
+            around each launch in the timed steps, against the measured HBM copy peak.
+cpu_baseline / --impl reference
+            the fp64 oracle (C, OpenMP on all host cores) on a bounded token sample.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from dit_block_b200 import workloads  # noqa: E402
+
+METRIC = "fused DiT-op HBM GB/s & tokens/s at 125k/246k tokens; % of B200 HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_swiglu_fullres_10s.md")
+OPS = ("adaln_modulate", "dit_epilogue", "dit_prologue", "swiglu", "gated_residual")
+DOMINANT = "swiglu"
+
+
+def bytes_per_token(w) -> dict:
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    return {"adaln_modulate": 2 * w.d * e, "dit_epilogue": 4 * w.hd * e, "dit_prologue": 4 * w.d * e,
+            "swiglu": 3 * w.inner * e, "gated_residual": 3 * w.d * e}
+
+
+def dtype_name(w) -> str:
+    return "bf16" if w.dtype == torch.bfloat16 else "f32"
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device: torch.device, period_s: float = 0.01):
+        self.period = period_s
+        self.samples: list[int] = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that the clocks are unknown
+            self.err = str(e)
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        self._stop.set()
+        self._t.join()
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------ helpers
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("k_stream.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "dit_block_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(n_tokens: int):
+    """DRAM bytes of one SwiGLU launch from the committed ncu summary, scaled to n_tokens;
+    None if absent or taken on different kernel source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            text = f.read()
+    except OSError:
+        return None
+    kv = {}
+    for line in text.splitlines():
+        line = line.strip().strip("`")
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            kv[k.strip()] = v.strip()
+    try:
+        if kv.get("kernel_source_sha256_16") != source_digest():
+            return None
+        per_token = float(kv["dram_bytes_per_token"])
+        return per_token * n_tokens
+    except (KeyError, ValueError):
+        return None
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(vals: list[float], world: int, device) -> list[float]:
+    if world == 1:
+        return vals
+    import torch.distributed as dist
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+# -------------------------------------------------------------------------- CPU oracle
+
+def _bits(t):
+    c = t.detach().contiguous().cpu()
+    if c.dtype == torch.bfloat16:
+        return c.view(torch.int16).numpy().view(np.uint16).copy()
+    return c.numpy().copy()
+
+
+class OracleChain:
+    """The oracle's pass over a token sample (same five operators, same shapes)."""
+
+    def __init__(self, w, n_tokens: int):
+        import oracle
+        oracle.build()
+        self.o = oracle
+        self.w = w
+        inp = workloads.block_inputs(w, "cpu", n_tokens=n_tokens)
+        self.n = n_tokens
+        self.a = {k: _bits(v) for k, v in inp.items() if isinstance(v, torch.Tensor)}
+        self.pos = None if inp["pos"] is None else inp["pos"].numpy()
+
+    def step(self):
+        o, w, a = self.o, self.w, self.a
+        sel = dict(stream_id=a.get("stream_id"), n_streams=w.n_streams,
+                   tokens_per_sample=w.tokens_per_sample)
+        o.adaln_modulate(a["x"], a["shift_msa"], a["scale_msa"], eps=w.eps, **sel)
+        o.dit_epilogue(a["qkv"], a["wq"], a["wk"], n_heads=w.n_heads, head_dim=w.head_dim,
+                       pos=self.pos, grid=w.grid, tokens_per_sample=w.tokens_per_sample,
+                       dims=w.rope_dims, theta=w.theta, eps=w.eps)
+        o.dit_prologue(a["x"], a["y_attn"], a["gate_msa"], a["shift_mlp"], a["scale_mlp"], eps=w.eps,
+                       **sel)
+        o.swiglu(a["u"], w.inner)
+        o.gated_residual(a["x"], a["y_mlp"], a["gate_mlp"], **sel)
+
+    def bytes_per_step(self) -> int:
+        return sum(bytes_per_token(self.w).values()) * self.n
+
+
+def cpu_baseline(w, target_s: float = 10.0, sample_tokens: int = 1024) -> dict:
+    chain = OracleChain(w, sample_tokens)
+    chain.step()  # warm-up (page faults, thread pool)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        chain.step()
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= target_s or reps >= 1000:
+            break
+    gbs = chain.bytes_per_step() * reps / el / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": chain.o.num_threads(), "kind": "oracle",
+            "sample": f"{reps} passes of the 5-op chain over {sample_tokens} tokens of {w.name} "
+                      f"({el:.1f} s, fp64, OpenMP)",
+            "tokens_per_s": round(sample_tokens * reps / el, 1)}
+
+
+# ------------------------------------------------------------------------- arms
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    chain = OracleChain(w, args.ref_tokens)
+    for _ in range(args.warmup):
+        chain.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        chain.step()
+    el = time.perf_counter() - t0
+    gbs = chain.bytes_per_step() * args.steps / el / 1e9
+    cores = chain.o.num_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "tokens": w.n_tokens, "sample_tokens": args.ref_tokens,
+                   "d": w.d, "heads": f"{w.n_heads}x{w.head_dim}", "swiglu_inner": w.inner,
+                   "parallelism": "replicas", "l2": "host run"},
+        "tokens_per_s": round(args.ref_tokens * args.steps / el, 1),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{args.ref_tokens} tokens of {w.name} per step"},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w):
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    from dit_block_b200 import block, build, sol
+    build.build()
+    sol.lib()
+
+    bufs = block.BlockBuffers.allocate(w, dev, n_tokens=args.tokens)
+    n = bufs.n_tokens
+    bpt = bytes_per_token(w)
+    step_bytes = sum(bpt.values()) * n
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local])
+
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        bufs.step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(OPS) + 1)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.start()
+    start.record(stream)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        for j, op in enumerate(OPS):
+            bufs.launch(op)
+            ev[s][j + 1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(end)
+    per_op_ms = {op: sum(ev[s][j].elapsed_time(ev[s][j + 1]) for s in range(args.steps)) / args.steps
+                 for j, op in enumerate(OPS)}
+    total_ms, = max_over_ranks([total_ms], world, dev)
+    ms_step = total_ms / args.steps
+    value = step_bytes * world * args.steps / (total_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, bufs, dev, world, step_bytes)
+
+    peak, peak_kind = measured_peak()
+    dom_ms = per_op_ms[DOMINANT]
+    dom_bytes = bpt[DOMINANT] * n
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(n)
+    per_op = {op: {"ms": round(per_op_ms[op], 4),
+                   "GB_s": round(bpt[op] * n / (per_op_ms[op] * 1e-3) / 1e9, 1),
+                   "frac_of_measured_peak": round(bpt[op] * n / (per_op_ms[op] * 1e-3) / 1e9 / peak, 4),
+                   "bytes_per_token": bpt[op]} for op in OPS}
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(w),
+        "data": "synthetic",
+        "config": {"workload": w.name, "tokens": n, "grid": list(w.grid), "batch": w.batch,
+                   "d": w.d, "heads": f"{w.n_heads}x{w.head_dim}", "swiglu_inner": w.inner,
+                   "bytes_per_token": sum(bpt.values()),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "no flush: every op streams >= 2.5 GB, far above the 126 MB L2"},
+        "tokens_per_s": round(n * world * args.steps / (total_ms * 1e-3), 1),
+        "frac_of_measured_hbm_peak": round(value / world / peak, 4),
+        "frac_of_spec_hbm_peak": round(value / world / SPEC_HBM_GBS, 4),
+        "per_op": per_op,
+        "roofline": {"bound": "hbm", "kernel": "k_swiglu", "achieved": round(achieved, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": None if traffic is None else int(traffic),
+                     "algorithmic_bytes": dom_bytes},
+        "clocks": clk,
+        "gpu_launches": len(OPS) * args.steps,
+        "e2e": e2e,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    bufs.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, bufs, dev, world, step_bytes):
+    """Pinned host buffers in, five launches, host buffers out; copies inside the timing."""
+    i = bufs.inp
+    in_names = [k for k in ("x", "qkv", "y_attn", "u", "y_mlp", "shift_msa", "scale_msa", "gate_msa",
+                            "shift_mlp", "scale_mlp", "gate_mlp", "wq", "wk", "pos", "stream_id")
+                if i.get(k) is not None]
+    outs = {"h1": bufs.h1, "qkv": i["qkv"], "x1": bufs.x1, "h2": bufs.h2, "act": bufs.act, "x2": bufs.x2}
+    need = sum(i[k].numel() * i[k].element_size() for k in in_names) + \
+        sum(t.numel() * t.element_size() for t in outs.values())
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = 0
+    if need > 0.4 * avail:
+        return {"value": None, "unit": "GB/s",
+                "error": f"skipped: {need / 1e9:.1f} GB of pinned host buffers > 40% of the "
+                         f"{avail / 1e9:.1f} GB available host memory"}
+    try:
+        host_in = {k: torch.empty(i[k].shape, dtype=i[k].dtype, pin_memory=True) for k in in_names}
+        host_out = {k: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for k, t in outs.items()}
+    except RuntimeError as e:
+        return {"value": None, "unit": "GB/s", "error": f"pinned host allocation failed: {e}"[:200]}
+    for k in in_names:
+        host_in[k].copy_(i[k])
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        for k in in_names:
+            i[k].copy_(host_in[k], non_blocking=True)
+        bufs.step()
+        for k, t in outs.items():
+            host_out[k].copy_(t, non_blocking=True)
+
+    for _ in range(args.e2e_warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[dev.index])
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.e2e_steps):
+        one()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(end)
+    ms, = max_over_ranks([ms], world, dev)
+    val = step_bytes * world * args.e2e_steps / (ms * 1e-3) / 1e9
+    del host_in, host_out
+    return {"value": round(val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": args.e2e_steps, "ms_per_step": round(ms / args.e2e_steps, 2)}
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="fullres_10s", choices=sorted(workloads.WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--tokens", type=int, default=None,
+                   help="run only the first N tokens of the workload (small profiling cases)")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-warmup", type=int, default=1)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--ref-tokens", type=int, default=256, help="oracle token sample per reference step")
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        p.error("--warmup must be >= 3")
+    w = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

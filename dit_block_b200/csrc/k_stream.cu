@@ -1,0 +1,220 @@
+// k_stream.cu -- streaming per-token kernels: the gated residual and the SwiGLU
+// activation.  Both are pure HBM streams (2 reads : 1 write per element), so the design
+// is about bytes in flight and coalescing, not arithmetic:
+//   * every access is a 16-byte vector; consecutive threads touch consecutive vectors;
+//   * a CTA owns one fixed column chunk (blockDim.x * U vectors) of a row and walks rows
+//     with a grid stride; the grid is (resident CTAs per SM * SMs) rounded to a multiple
+//     of the chunks per row, so a CTA never changes columns;
+//   * each thread issues all U x inputs loads before the first use (U * 32 or 48 bytes
+//     in flight per thread); inputs use evict-first loads, outputs evict-first stores;
+//   * the gate row is re-read through the read-only path and stays L1/L2 resident.
+#include "common.cuh"
+#include "launch.h"
+
+namespace sol {
+
+// Gated residual [XHH-QA "门控残差"]: out = x + gate[r] * y, fp32 inside.
+template <typename T, int U>
+__global__ void __launch_bounds__(512)
+k_gated_residual(T* __restrict__ out, int64_t ld_out, const T* x, int64_t ld_x,
+                 const T* __restrict__ y, int64_t ld_y, const T* __restrict__ gate,
+                 int64_t ld_mod, ModSel sel, int64_t n_tokens, int32_t vpr, int32_t cpr)
+{
+    constexpr int E = Vec<T>::N;
+    const int chunk = blockIdx.x % cpr;
+    const int64_t row_step = gridDim.x / cpr;
+    const int col0 = chunk * blockDim.x * U + threadIdx.x;
+    for (int64_t row = blockIdx.x / cpr; row < n_tokens; row += row_step) {
+        const int64_t mr = mod_row(row, sel);
+        uint4 xv[U], yv[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int col = col0 + k * blockDim.x;
+            if (col < vpr) {
+                xv[k] = ld_stream(x + row * ld_x + (int64_t)col * E);
+                yv[k] = ld_stream(y + row * ld_y + (int64_t)col * E);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int col = col0 + k * blockDim.x;
+            if (col < vpr) {
+                float fx[E], fy[E], fg[E];
+                unpack<T>(xv[k], fx);
+                unpack<T>(yv[k], fy);
+                if (gate) {
+                    unpack<T>(ld_cached(gate + mr * ld_mod + (int64_t)col * E), fg);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) fg[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) fx[e] = fmaf(fg[e], fy[e], fx[e]);
+                st_stream(out + row * ld_out + (int64_t)col * E, pack<T>(fx));
+            }
+        }
+    }
+}
+
+// silu(a) * b.  bf16 outputs: ex2.approx-based exponential and approximate division
+// (one MUFU op each); the relative error is a few 1e-7, far below a bf16 ulp.  f32
+// outputs: expf and IEEE division.
+template <typename T> __device__ __forceinline__ float silu_mul(float a, float b);
+template <> __device__ __forceinline__ float silu_mul<bf16>(float a, float b)
+{
+    return __fdividef(a, 1.f + __expf(-a)) * b;
+}
+template <> __device__ __forceinline__ float silu_mul<float>(float a, float b)
+{
+    return a / (1.f + expf(-a)) * b;
+}
+
+// SwiGLU [XHH-QA, STM-GAN]: out_j = silu(a_j) * b_j.
+template <typename T, int U>
+__global__ void __launch_bounds__(512)
+k_swiglu(T* __restrict__ out, int64_t ld_out, const T* __restrict__ a, const T* __restrict__ b,
+         int64_t ld_in, int64_t n_tokens, int32_t vpr, int32_t cpr)
+{
+    constexpr int E = Vec<T>::N;
+    const int chunk = blockIdx.x % cpr;
+    const int64_t row_step = gridDim.x / cpr;
+    const int col0 = chunk * blockDim.x * U + threadIdx.x;
+    for (int64_t row = blockIdx.x / cpr; row < n_tokens; row += row_step) {
+        uint4 av[U], bv[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int col = col0 + k * blockDim.x;
+            if (col < vpr) {
+                av[k] = ld_stream(a + row * ld_in + (int64_t)col * E);
+                bv[k] = ld_stream(b + row * ld_in + (int64_t)col * E);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int col = col0 + k * blockDim.x;
+            if (col < vpr) {
+                float fa[E], fb[E];
+                unpack<T>(av[k], fa);
+                unpack<T>(bv[k], fb);
+#pragma unroll
+                for (int e = 0; e < E; ++e) fa[e] = silu_mul<T>(fa[e], fb[e]);
+                st_stream(out + row * ld_out + (int64_t)col * E, pack<T>(fa));
+            }
+        }
+    }
+}
+
+namespace {
+
+struct StreamShape {
+    int threads, U, cpr;
+};
+
+// Column chunking of a row of `vpr` vectors: the fewest idle lanes, then U in the
+// preference order below, then blockDim nearest 256.
+StreamShape choose_stream_shape(int64_t vpr)
+{
+    static const int kU[] = {4, 6, 8, 3, 2, 1};
+    StreamShape best{0, 0, 0};
+    int64_t best_waste = -1;
+    int best_rank = 0, best_tdist = 0;
+    for (int ui = 0; ui < 6; ++ui) {
+        for (int t = 32; t <= 512; t += 32) {
+            const int64_t chunk = (int64_t)t * kU[ui];
+            const int64_t cpr = (vpr + chunk - 1) / chunk;
+            const int64_t waste = cpr * chunk - vpr;
+            const int tdist = t > 256 ? t - 256 : 256 - t;
+            const bool better = best_waste < 0 || waste < best_waste ||
+                                (waste == best_waste &&
+                                 (ui < best_rank || (ui == best_rank && tdist < best_tdist)));
+            if (better) {
+                best = StreamShape{t, kU[ui], (int)cpr};
+                best_waste = waste;
+                best_rank = ui;
+                best_tdist = tdist;
+            }
+        }
+    }
+    return best;
+}
+
+int64_t stream_grid(const void* kernel, const StreamShape& sh, int64_t n_tokens)
+{
+    const int64_t resident = (int64_t)ctas_per_sm(kernel, sh.threads, 0) * sm_count();
+    int64_t rows = resident / sh.cpr;
+    if (rows < 1) rows = 1;
+    if (rows > n_tokens) rows = n_tokens;
+    return rows * sh.cpr;
+}
+
+template <typename T, int U>
+cudaError_t run_gated(void* out, int64_t ld_out, const void* x, int64_t ld_x, const void* y,
+                      int64_t ld_y, const void* gate, int64_t ld_mod, const ModSel& sel,
+                      int64_t n_tokens, int64_t vpr, const StreamShape& sh, cudaStream_t s)
+{
+    const void* kfn = (const void*)k_gated_residual<T, U>;
+    const int64_t grid = stream_grid(kfn, sh, n_tokens);
+    k_gated_residual<T, U><<<(unsigned)grid, sh.threads, 0, s>>>(
+        (T*)out, ld_out, (const T*)x, ld_x, (const T*)y, ld_y, (const T*)gate, ld_mod, sel,
+        n_tokens, (int32_t)vpr, sh.cpr);
+    return cudaGetLastError();
+}
+
+template <typename T, int U>
+cudaError_t run_swiglu(void* out, int64_t ld_out, const void* a, const void* b, int64_t ld_in,
+                       int64_t n_tokens, int64_t vpr, const StreamShape& sh, cudaStream_t s)
+{
+    const void* kfn = (const void*)k_swiglu<T, U>;
+    const int64_t grid = stream_grid(kfn, sh, n_tokens);
+    k_swiglu<T, U><<<(unsigned)grid, sh.threads, 0, s>>>((T*)out, ld_out, (const T*)a,
+                                                           (const T*)b, ld_in, n_tokens,
+                                                           (int32_t)vpr, sh.cpr);
+    return cudaGetLastError();
+}
+
+#define SOL_DISPATCH_U(U_, CALL) \
+    switch (U_) {                \
+    case 1: return CALL(1);      \
+    case 2: return CALL(2);      \
+    case 3: return CALL(3);      \
+    case 4: return CALL(4);      \
+    case 6: return CALL(6);      \
+    case 8: return CALL(8);      \
+    default: return cudaErrorInvalidConfiguration; \
+    }
+
+}  // namespace
+
+cudaError_t launch_gated_residual(sol_dtype dt, void* out, int64_t ld_out, const void* x,
+                                  int64_t ld_x, const void* y, int64_t ld_y, const void* gate,
+                                  int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
+                                  cudaStream_t s)
+{
+    const int64_t vpr = d / (dt == SOL_DTYPE_BF16 ? 8 : 4);
+    const StreamShape sh = choose_stream_shape(vpr);
+#define CALL_B(U) run_gated<bf16, U>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, sel, n_tokens, vpr, sh, s)
+#define CALL_F(U) run_gated<float, U>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, sel, n_tokens, vpr, sh, s)
+    if (dt == SOL_DTYPE_BF16) {
+        SOL_DISPATCH_U(sh.U, CALL_B)
+    }
+    SOL_DISPATCH_U(sh.U, CALL_F)
+#undef CALL_B
+#undef CALL_F
+}
+
+cudaError_t launch_swiglu(sol_dtype dt, void* out, int64_t ld_out, const void* a, const void* b,
+                          int64_t ld_in, int64_t n_tokens, int64_t inner, cudaStream_t s)
+{
+    const int64_t vpr = inner / (dt == SOL_DTYPE_BF16 ? 8 : 4);
+    const StreamShape sh = choose_stream_shape(vpr);
+#define CALL_B(U) run_swiglu<bf16, U>(out, ld_out, a, b, ld_in, n_tokens, vpr, sh, s)
+#define CALL_F(U) run_swiglu<float, U>(out, ld_out, a, b, ld_in, n_tokens, vpr, sh, s)
+    if (dt == SOL_DTYPE_BF16) {
+        SOL_DISPATCH_U(sh.U, CALL_B)
+    }
+    SOL_DISPATCH_U(sh.U, CALL_F)
+#undef CALL_B
+#undef CALL_F
+}
+
+}  // namespace sol

@@ -1,0 +1,53 @@
+// launch.h -- host-side launchers of the libsol kernels (internal to the library).
+// Arguments reach these only after sol_api.cu validated them.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sol.h"
+
+namespace sol {
+
+struct ModSel;
+
+// Device view of a sol_rope3d: per axis (t, h, w), a [max_c, dim_c/2] table of
+// (cos, sin) pairs.
+struct RopeDev {
+    const float2* tab[3];
+    int32_t max[3];
+    int32_t half[3];
+};
+
+// Resident CTAs per SM for `kernel` at `block` threads on the current device (cached).
+int ctas_per_sm(const void* kernel, int block, size_t smem);
+// SM count of the current device (cached).
+int sm_count();
+
+cudaError_t launch_gated_residual(sol_dtype dt, void* out, int64_t ld_out, const void* x,
+                                  int64_t ld_x, const void* y, int64_t ld_y, const void* gate,
+                                  int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
+                                  cudaStream_t s);
+
+cudaError_t launch_swiglu(sol_dtype dt, void* out, int64_t ld_out, const void* a, const void* b,
+                          int64_t ld_in, int64_t n_tokens, int64_t inner, cudaStream_t s);
+
+// AdaLN with an optional fused gated residual in front (y == nullptr: plain AdaLN).
+cudaError_t launch_adaln_rows(sol_dtype dt, void* x_out, int64_t ld_xo, void* h, int64_t ld_h,
+                              const void* x, int64_t ld_x, const void* y, int64_t ld_y,
+                              const void* gate, const void* shift, const void* scale,
+                              int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
+                              float eps, cudaStream_t s);
+
+cudaError_t launch_qk_rmsnorm_rope3d(sol_dtype dt, void* q_out, void* k_out, int64_t ld_qo,
+                                     int64_t ld_ko, const void* q, const void* k, int64_t ld_q,
+                                     int64_t ld_k, const void* wq, const void* wk,
+                                     const int32_t* pos, int32_t grid_T, int32_t grid_H,
+                                     int32_t grid_W, int64_t tokens_per_sample,
+                                     const RopeDev& rope, int64_t n_tokens, int32_t n_heads,
+                                     int32_t head_dim, float eps, cudaStream_t s);
+
+// Whether a row of `vpr` 16-byte vectors fits the register-resident AdaLN kernel.
+bool adaln_row_fits(int64_t vpr);
+
+}  // namespace sol

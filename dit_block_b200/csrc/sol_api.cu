@@ -1,0 +1,441 @@
+// sol_api.cu -- the C ABI of libsol (declared in include/sol.h): argument validation,
+// the RoPE table handle, launch bookkeeping, and dispatch to the kernel launchers.
+// Every check runs on the host before anything is launched, so a rejected call has no
+// side effect on the device.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "launch.h"
+#include "sol.h"
+
+struct sol_rope3d {
+    float2* dev;           // one allocation holding the three axis tables
+    int32_t dims[3];       // chunk widths (t, h, w)
+    int32_t max[3];        // positions per axis
+    double theta;
+    int device;
+    sol::RopeDev view;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sol_status fail(sol_status st, const char* fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+sol_status cuda_status(cudaError_t e, const char* what)
+{
+    if (e == cudaSuccess) return SOL_OK;
+    return fail(SOL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elems16(sol_dtype dt) { return dt == SOL_DTYPE_BF16 ? 8 : 4; }
+
+#define CHECK(cond, st, ...)                      \
+    do {                                          \
+        if (!(cond)) return fail(st, __VA_ARGS__); \
+    } while (0)
+
+sol_status check_dtype(sol_dtype dt)
+{
+    CHECK(dt == SOL_DTYPE_F32 || dt == SOL_DTYPE_BF16, SOL_ERR_UNSUPPORTED,
+          "dtype %d is not SOL_DTYPE_F32 or SOL_DTYPE_BF16", (int)dt);
+    return SOL_OK;
+}
+
+// A required [rows, ld] tensor whose rows hold `width` used elements.
+sol_status check_tensor(const char* name, const void* p, int64_t ld, int64_t width, sol_dtype dt,
+                        bool required)
+{
+    if (!p) {
+        CHECK(!required, SOL_ERR_INVALID_ARGUMENT, "%s is NULL", name);
+        return SOL_OK;
+    }
+    CHECK(aligned16(p), SOL_ERR_MISALIGNED, "%s is not 16-byte aligned", name);
+    CHECK(ld >= width, SOL_ERR_INVALID_ARGUMENT, "ld of %s (%lld) is below the row width %lld",
+          name, (long long)ld, (long long)width);
+    CHECK(ld % elems16(dt) == 0, SOL_ERR_MISALIGNED,
+          "ld of %s (%lld) is not a multiple of %d elements (16 bytes)", name, (long long)ld,
+          elems16(dt));
+    return SOL_OK;
+}
+
+sol_status check_modsel(const sol_modsel& sel)
+{
+    CHECK(sel.n_streams >= 1 && sel.n_streams <= 256, SOL_ERR_INVALID_ARGUMENT,
+          "sel.n_streams (%d) must be in [1, 256]", (int)sel.n_streams);
+    CHECK(sel.tokens_per_sample >= 0, SOL_ERR_INVALID_ARGUMENT,
+          "sel.tokens_per_sample (%lld) is negative", (long long)sel.tokens_per_sample);
+    return SOL_OK;
+}
+
+sol::ModSel to_dev(const sol_modsel& sel)
+{
+    return sol::ModSel{sel.stream_id, sel.n_streams, sel.tokens_per_sample};
+}
+
+// Byte ranges [p, p + rows*ld*esz) overlap?  Used to reject forbidden aliasing.
+bool overlap(const void* a, int64_t lda, const void* b, int64_t ldb, int64_t rows, size_t esz)
+{
+    if (!a || !b || rows == 0) return false;
+    const char* a0 = (const char*)a;
+    const char* b0 = (const char*)b;
+    const char* a1 = a0 + (size_t)rows * (size_t)lda * esz;
+    const char* b1 = b0 + (size_t)rows * (size_t)ldb * esz;
+    return a0 < b1 && b0 < a1;
+}
+
+size_t esize(sol_dtype dt) { return dt == SOL_DTYPE_BF16 ? 2 : 4; }
+
+#define TRY(expr)                          \
+    do {                                   \
+        const sol_status st_ = (expr);     \
+        if (st_ != SOL_OK) return st_;     \
+    } while (0)
+
+sol_status check_rows(int64_t n_tokens, int64_t d, sol_dtype dt, const char* dname)
+{
+    CHECK(n_tokens >= 0, SOL_ERR_INVALID_ARGUMENT, "n_tokens (%lld) is negative", (long long)n_tokens);
+    CHECK(d >= elems16(dt), SOL_ERR_INVALID_ARGUMENT, "%s (%lld) is below %d", dname, (long long)d,
+          elems16(dt));
+    CHECK(d % elems16(dt) == 0, SOL_ERR_UNSUPPORTED, "%s (%lld) is not a multiple of %d", dname,
+          (long long)d, elems16(dt));
+    CHECK(d / elems16(dt) < (int64_t)1 << 30, SOL_ERR_UNSUPPORTED, "%s (%lld) is too wide", dname,
+          (long long)d);
+    return SOL_OK;
+}
+
+}  // namespace
+
+namespace sol {
+
+namespace {
+struct OccEntry {
+    const void* fn;
+    int block;
+    size_t smem;
+    int device;
+    int ctas;
+};
+std::mutex g_occ_mu;
+std::vector<OccEntry> g_occ;
+int g_sms[64];
+}  // namespace
+
+int ctas_per_sm(const void* kernel, int block, size_t smem)
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    for (const OccEntry& e : g_occ)
+        if (e.fn == kernel && e.block == block && e.smem == smem && e.device == dev) return e.ctas;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, smem) != cudaSuccess || n < 1)
+        n = 1;
+    g_occ.push_back(OccEntry{kernel, block, smem, dev, n});
+    return n;
+}
+
+int sm_count()
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    if (g_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 1;
+        g_sms[dev] = n;
+    }
+    return g_sms[dev];
+}
+
+}  // namespace sol
+
+extern "C" {
+
+const char* sol_status_string(sol_status status)
+{
+    switch (status) {
+    case SOL_OK: return "ok";
+    case SOL_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case SOL_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+    case SOL_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SOL_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char* sol_last_error(void) { return g_last_error.c_str(); }
+
+int32_t sol_abi_version(void) { return 1; }
+
+sol_status sol_adaln_modulate(void* h, int64_t ld_h, const void* x, int64_t ld_x,
+                              const void* shift, const void* scale, int64_t ld_mod,
+                              sol_modsel sel, int64_t n_tokens, int64_t d, float eps,
+                              sol_dtype dt, sol_stream_t stream)
+{
+    TRY(check_dtype(dt));
+    TRY(check_rows(n_tokens, d, dt, "d"));
+    CHECK(sol::adaln_row_fits(d / elems16(dt)), SOL_ERR_UNSUPPORTED,
+          "d (%lld) is wider than one CTA row holds (max 4096 16-byte vectors)", (long long)d);
+    CHECK(std::isfinite(eps) && eps >= 0.f, SOL_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
+    TRY(check_tensor("h", h, ld_h, d, dt, true));
+    TRY(check_tensor("x", x, ld_x, d, dt, true));
+    TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
+    TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
+    TRY(check_modsel(sel));
+    CHECK(h == x ? ld_h == ld_x : !overlap(h, ld_h, x, ld_x, n_tokens, esize(dt)),
+          SOL_ERR_INVALID_ARGUMENT, "h overlaps x without being the same tensor");
+    if (n_tokens == 0) return SOL_OK;
+    const sol::ModSel ms = to_dev(sel);
+    return cuda_status(sol::launch_adaln_rows(dt, nullptr, 0, h, ld_h, x, ld_x, nullptr, 0, nullptr,
+                                              shift, scale, ld_mod, ms, n_tokens, d, eps,
+                                              (cudaStream_t)stream),
+                       "sol_adaln_modulate launch");
+}
+
+sol_status sol_gated_residual(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                              const void* y, int64_t ld_y, const void* gate, int64_t ld_mod,
+                              sol_modsel sel, int64_t n_tokens, int64_t d, sol_dtype dt,
+                              sol_stream_t stream)
+{
+    TRY(check_dtype(dt));
+    TRY(check_rows(n_tokens, d, dt, "d"));
+    TRY(check_tensor("out", out, ld_out, d, dt, true));
+    TRY(check_tensor("x", x, ld_x, d, dt, true));
+    TRY(check_tensor("y", y, ld_y, d, dt, true));
+    TRY(check_tensor("gate", gate, ld_mod, d, dt, false));
+    TRY(check_modsel(sel));
+    CHECK(out == x ? ld_out == ld_x : !overlap(out, ld_out, x, ld_x, n_tokens, esize(dt)),
+          SOL_ERR_INVALID_ARGUMENT, "out overlaps x without being the same tensor");
+    CHECK(!overlap(out, ld_out, y, ld_y, n_tokens, esize(dt)), SOL_ERR_INVALID_ARGUMENT,
+          "out overlaps y");
+    if (n_tokens == 0) return SOL_OK;
+    const sol::ModSel ms = to_dev(sel);
+    return cuda_status(sol::launch_gated_residual(dt, out, ld_out, x, ld_x, y, ld_y, gate, ld_mod,
+                                                  ms, n_tokens, d, (cudaStream_t)stream),
+                       "sol_gated_residual launch");
+}
+
+sol_status sol_swiglu(void* out, int64_t ld_out, const void* a, const void* b, int64_t ld_in,
+                      int64_t n_tokens, int64_t inner, sol_dtype dt, sol_stream_t stream)
+{
+    TRY(check_dtype(dt));
+    TRY(check_rows(n_tokens, inner, dt, "inner"));
+    TRY(check_tensor("out", out, ld_out, inner, dt, true));
+    TRY(check_tensor("a", a, ld_in, inner, dt, true));
+    TRY(check_tensor("b", b, ld_in, inner, dt, true));
+    // a and b may be two halves of one row: the row extent of each is ld_in wide
+    CHECK(!overlap(out, ld_out, a, ld_in, n_tokens, esize(dt)) &&
+              !overlap(out, ld_out, b, ld_in, n_tokens, esize(dt)),
+          SOL_ERR_INVALID_ARGUMENT, "out overlaps a or b");
+    if (n_tokens == 0) return SOL_OK;
+    return cuda_status(sol::launch_swiglu(dt, out, ld_out, a, b, ld_in, n_tokens, inner,
+                                          (cudaStream_t)stream),
+                       "sol_swiglu launch");
+}
+
+sol_status sol_rope3d_create(sol_rope3d** out, int32_t dim_t, int32_t dim_h, int32_t dim_w,
+                             double theta, int32_t max_t, int32_t max_h, int32_t max_w)
+{
+    CHECK(out, SOL_ERR_INVALID_ARGUMENT, "out is NULL");
+    *out = nullptr;
+    const int32_t dims[3] = {dim_t, dim_h, dim_w};
+    const int32_t maxp[3] = {max_t, max_h, max_w};
+    for (int c = 0; c < 3; ++c) {
+        CHECK(dims[c] >= 0 && dims[c] % 2 == 0 && dims[c] <= 1024, SOL_ERR_INVALID_ARGUMENT,
+              "RoPE chunk width %d of axis %d must be even and in [0, 1024]", (int)dims[c], c);
+        CHECK(maxp[c] >= 1 && maxp[c] <= (1 << 20), SOL_ERR_INVALID_ARGUMENT,
+              "max position %d of axis %d must be in [1, 2^20]", (int)maxp[c], c);
+    }
+    CHECK(dim_t + dim_h + dim_w >= 2, SOL_ERR_INVALID_ARGUMENT, "RoPE chunk widths sum to 0");
+    CHECK(std::isfinite(theta) && theta > 1.0, SOL_ERR_INVALID_ARGUMENT, "theta must be finite and > 1");
+
+    size_t off[4] = {0, 0, 0, 0};
+    for (int c = 0; c < 3; ++c) off[c + 1] = off[c] + (size_t)maxp[c] * (size_t)(dims[c] / 2);
+    // tables on the host in fp64, rounded once to fp32: phi = p * theta^(-2j/D_c)
+    std::vector<float2> host(off[3] > 0 ? off[3] : 1);
+    for (int c = 0; c < 3; ++c) {
+        const int half = dims[c] / 2;
+        for (int32_t p = 0; p < maxp[c]; ++p) {
+            for (int j = 0; j < half; ++j) {
+                const double inv_freq = std::pow(theta, -2.0 * (double)j / (double)dims[c]);
+                const double phi = (double)p * inv_freq;
+                host[off[c] + (size_t)p * half + j] = make_float2((float)std::cos(phi), (float)std::sin(phi));
+            }
+        }
+    }
+    sol_rope3d* r = new (std::nothrow) sol_rope3d();
+    CHECK(r, SOL_ERR_INVALID_ARGUMENT, "host allocation failed");
+    cudaGetDevice(&r->device);
+    cudaError_t e = cudaMalloc((void**)&r->dev, host.size() * sizeof(float2));
+    if (e != cudaSuccess) {
+        delete r;
+        return cuda_status(e, "sol_rope3d_create cudaMalloc");
+    }
+    e = cudaMemcpy(r->dev, host.data(), host.size() * sizeof(float2), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaFree(r->dev);
+        delete r;
+        return cuda_status(e, "sol_rope3d_create cudaMemcpy");
+    }
+    for (int c = 0; c < 3; ++c) {
+        r->dims[c] = dims[c];
+        r->max[c] = maxp[c];
+        r->view.tab[c] = r->dev + off[c];
+        r->view.max[c] = maxp[c];
+        r->view.half[c] = dims[c] / 2;
+    }
+    r->theta = theta;
+    *out = r;
+    return SOL_OK;
+}
+
+sol_status sol_rope3d_destroy(sol_rope3d* rope)
+{
+    if (!rope) return SOL_OK;
+    const cudaError_t e = cudaFree(rope->dev);
+    delete rope;
+    return cuda_status(e, "sol_rope3d_destroy cudaFree");
+}
+
+static sol_status check_qk_common(const sol_rope3d* rope, const int32_t* pos, int32_t grid_T,
+                                  int32_t grid_H, int32_t grid_W, int64_t tps, int64_t n_tokens,
+                                  int32_t n_heads, int32_t head_dim, float eps, sol_dtype dt,
+                                  const void* wq, const void* wk)
+{
+    TRY(check_dtype(dt));
+    CHECK(rope, SOL_ERR_INVALID_ARGUMENT, "rope is NULL");
+    CHECK(n_tokens >= 0, SOL_ERR_INVALID_ARGUMENT, "n_tokens is negative");
+    CHECK(n_heads >= 1 && n_heads <= 4096, SOL_ERR_INVALID_ARGUMENT, "n_heads (%d) must be in [1, 4096]",
+          (int)n_heads);
+    const int lph = head_dim / elems16(dt);
+    CHECK(head_dim % elems16(dt) == 0 && (lph == 8 || lph == 16 || lph == 32), SOL_ERR_UNSUPPORTED,
+          "head_dim %d is not built for this dtype (bf16: 64/128/256, f32: 32/64/128)", (int)head_dim);
+    CHECK(rope->dims[0] + rope->dims[1] + rope->dims[2] == head_dim, SOL_ERR_INVALID_ARGUMENT,
+          "RoPE chunk widths (%d, %d, %d) do not sum to head_dim %d", (int)rope->dims[0],
+          (int)rope->dims[1], (int)rope->dims[2], (int)head_dim);
+    CHECK(std::isfinite(eps) && eps >= 0.f, SOL_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
+    CHECK(!wq || aligned16(wq), SOL_ERR_MISALIGNED, "wq is not 16-byte aligned");
+    CHECK(!wk || aligned16(wk), SOL_ERR_MISALIGNED, "wk is not 16-byte aligned");
+    CHECK(tps >= 0, SOL_ERR_INVALID_ARGUMENT, "tokens_per_sample is negative");
+    if (!pos) {
+        CHECK(grid_T >= 1 && grid_H >= 1 && grid_W >= 1, SOL_ERR_INVALID_ARGUMENT,
+              "implicit positions need grid_T, grid_H, grid_W >= 1");
+        CHECK(grid_T <= rope->max[0] && grid_H <= rope->max[1] && grid_W <= rope->max[2],
+              SOL_ERR_INVALID_ARGUMENT, "grid %dx%dx%d exceeds the RoPE tables (%d, %d, %d)",
+              (int)grid_T, (int)grid_H, (int)grid_W, (int)rope->max[0], (int)rope->max[1],
+              (int)rope->max[2]);
+        const int64_t cells = (int64_t)grid_T * grid_H * grid_W;
+        const int64_t span = tps > 0 ? tps : n_tokens;
+        CHECK(span <= cells, SOL_ERR_INVALID_ARGUMENT,
+              "%lld tokens per sample do not fit the %lld-cell grid", (long long)span, (long long)cells);
+    }
+    int dev = 0;
+    cudaGetDevice(&dev);
+    CHECK(dev == rope->device, SOL_ERR_INVALID_ARGUMENT,
+          "rope tables live on device %d, current device is %d", rope->device, dev);
+    return SOL_OK;
+}
+
+sol_status sol_qk_rmsnorm_rope3d(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko,
+                                 const void* q, const void* k, int64_t ld_q, int64_t ld_k,
+                                 const void* wq, const void* wk, const int32_t* pos,
+                                 int32_t grid_T, int32_t grid_H, int32_t grid_W,
+                                 int64_t tokens_per_sample, const sol_rope3d* rope,
+                                 int64_t n_tokens, int32_t n_heads, int32_t head_dim, float eps,
+                                 sol_dtype dt, sol_stream_t stream)
+{
+    TRY(check_qk_common(rope, pos, grid_T, grid_H, grid_W, tokens_per_sample, n_tokens, n_heads,
+                        head_dim, eps, dt, wq, wk));
+    const int64_t hd = (int64_t)n_heads * head_dim;
+    TRY(check_tensor("q", q, ld_q, hd, dt, true));
+    TRY(check_tensor("k", k, ld_k, hd, dt, true));
+    TRY(check_tensor("q_out", q_out, ld_qo, hd, dt, true));
+    TRY(check_tensor("k_out", k_out, ld_ko, hd, dt, true));
+    const size_t es = esize(dt);
+    CHECK(q_out == q ? ld_qo == ld_q : !overlap(q_out, ld_qo, q, ld_q, n_tokens, es),
+          SOL_ERR_INVALID_ARGUMENT, "q_out overlaps q without being the same tensor");
+    CHECK(k_out == k ? ld_ko == ld_k : !overlap(k_out, ld_ko, k, ld_k, n_tokens, es),
+          SOL_ERR_INVALID_ARGUMENT, "k_out overlaps k without being the same tensor");
+    if (n_tokens == 0) return SOL_OK;
+    return cuda_status(sol::launch_qk_rmsnorm_rope3d(dt, q_out, k_out, ld_qo, ld_ko, q, k, ld_q, ld_k,
+                                                     wq, wk, pos, grid_T, grid_H, grid_W,
+                                                     tokens_per_sample, rope->view, n_tokens,
+                                                     n_heads, head_dim, eps, (cudaStream_t)stream),
+                       "sol_qk_rmsnorm_rope3d launch");
+}
+
+sol_status sol_dit_prologue(void* x_out, void* h, const void* x, const void* y,
+                            const void* gate, const void* shift, const void* scale, int64_t ld,
+                            int64_t ld_mod, sol_modsel sel, int64_t n_tokens, int64_t d,
+                            float eps, sol_dtype dt, sol_stream_t stream)
+{
+    TRY(check_dtype(dt));
+    TRY(check_rows(n_tokens, d, dt, "d"));
+    CHECK(sol::adaln_row_fits(d / elems16(dt)), SOL_ERR_UNSUPPORTED,
+          "d (%lld) is wider than one CTA row holds (max 4096 16-byte vectors)", (long long)d);
+    CHECK(std::isfinite(eps) && eps >= 0.f, SOL_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
+    TRY(check_tensor("h", h, ld, d, dt, true));
+    TRY(check_tensor("x", x, ld, d, dt, true));
+    TRY(check_tensor("y", y, ld, d, dt, false));
+    TRY(check_tensor("x_out", x_out, ld, d, dt, y != nullptr));
+    TRY(check_tensor("gate", gate, ld_mod, d, dt, false));
+    TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
+    TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
+    TRY(check_modsel(sel));
+    const size_t es = esize(dt);
+    CHECK(!overlap(h, ld, x, ld, n_tokens, es) && !overlap(h, ld, y, ld, n_tokens, es) &&
+              !overlap(h, ld, x_out, ld, n_tokens, es),
+          SOL_ERR_INVALID_ARGUMENT, "h overlaps x, y or x_out");
+    CHECK(!y || x_out == x || !overlap(x_out, ld, x, ld, n_tokens, es), SOL_ERR_INVALID_ARGUMENT,
+          "x_out overlaps x without being the same tensor");
+    CHECK(!y || !overlap(x_out, ld, y, ld, n_tokens, es), SOL_ERR_INVALID_ARGUMENT, "x_out overlaps y");
+    if (n_tokens == 0) return SOL_OK;
+    const sol::ModSel ms = to_dev(sel);
+    return cuda_status(sol::launch_adaln_rows(dt, y ? x_out : nullptr, ld, h, ld, x, ld, y, ld, gate,
+                                              shift, scale, ld_mod, ms, n_tokens, d, eps,
+                                              (cudaStream_t)stream),
+                       "sol_dit_prologue launch");
+}
+
+sol_status sol_dit_epilogue(void* qkv, int64_t ld_qkv, const void* wq, const void* wk,
+                            const int32_t* pos, int32_t grid_T, int32_t grid_H, int32_t grid_W,
+                            int64_t tokens_per_sample, const sol_rope3d* rope, int64_t n_tokens,
+                            int32_t n_heads, int32_t head_dim, float eps, sol_dtype dt,
+                            sol_stream_t stream)
+{
+    TRY(check_qk_common(rope, pos, grid_T, grid_H, grid_W, tokens_per_sample, n_tokens, n_heads,
+                        head_dim, eps, dt, wq, wk));
+    const int64_t hd = (int64_t)n_heads * head_dim;
+    TRY(check_tensor("qkv", qkv, ld_qkv, 2 * hd, dt, true));
+    if (n_tokens == 0) return SOL_OK;
+    void* k = (char*)qkv + (size_t)hd * esize(dt);
+    return cuda_status(sol::launch_qk_rmsnorm_rope3d(dt, qkv, k, ld_qkv, ld_qkv, qkv, k, ld_qkv,
+                                                     ld_qkv, wq, wk, pos, grid_T, grid_H, grid_W,
+                                                     tokens_per_sample, rope->view, n_tokens,
+                                                     n_heads, head_dim, eps, (cudaStream_t)stream),
+                       "sol_dit_epilogue launch");
+}
+
+}  // extern "C"

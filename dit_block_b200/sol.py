@@ -1,0 +1,245 @@
+"""ctypes binding of libsol (include/sol.h), same names without the ``sol_`` prefix.
+
+Argument marshalling only: every op runs in the CUDA kernels of ``libsol.so``.  Tensors
+are torch CUDA tensors, 2-D with unit column stride; their row stride is passed as the
+leading dimension.  Ops run on torch's current CUDA stream unless ``stream`` is given
+(a ``torch.cuda.Stream`` or a raw ``cudaStream_t`` integer).  A non-OK status raises
+:class:`SolError` with the library's one-line reason.  If ``libsol.so`` is missing the
+first call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsol.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "sol.h")
+
+OK, ERR_INVALID_ARGUMENT, ERR_MISALIGNED, ERR_UNSUPPORTED, ERR_CUDA = range(5)
+F32, BF16 = 0, 1
+
+
+class SolError(RuntimeError):
+    def __init__(self, status: int, func: str, detail: str):
+        super().__init__(f"{func}: status {status}: {detail}")
+        self.status = status
+
+
+class ModSel(ctypes.Structure):
+    _fields_ = [("stream_id", ctypes.c_void_p), ("n_streams", ctypes.c_int32),
+                ("tokens_per_sample", ctypes.c_int64)]
+
+
+_P, _I64, _I32, _F, _D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_double
+_E = ctypes.c_int  # enums
+
+# argument types per exported function, in header order
+SIGNATURES = {
+    "sol_status_string": ([_E], ctypes.c_char_p),
+    "sol_last_error": ([], ctypes.c_char_p),
+    "sol_abi_version": ([], _I32),
+    "sol_adaln_modulate": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _I64, _I64, _F, _E, _P], _E),
+    "sol_gated_residual": ([_P, _I64, _P, _I64, _P, _I64, _P, _I64, ModSel, _I64, _I64, _E, _P], _E),
+    "sol_swiglu": ([_P, _I64, _P, _P, _I64, _I64, _I64, _E, _P], _E),
+    "sol_rope3d_create": ([ctypes.POINTER(_P), _I32, _I32, _I32, _D, _I32, _I32, _I32], _E),
+    "sol_rope3d_destroy": ([_P], _E),
+    "sol_qk_rmsnorm_rope3d": ([_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _P, _P, _I32, _I32,
+                               _I32, _I64, _P, _I64, _I32, _I32, _F, _E, _P], _E),
+    "sol_dit_prologue": ([_P, _P, _P, _P, _P, _P, _P, _I64, _I64, ModSel, _I64, _I64, _F, _E, _P], _E),
+    "sol_dit_epilogue": ([_P, _I64, _P, _P, _P, _I32, _I32, _I32, _I64, _P, _I64, _I32, _I32, _F,
+                          _E, _P], _E),
+}
+
+_lib = None
+
+
+def header_functions() -> list[str]:
+    """Names of every function include/sol.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"\b(sol_[a-z0-9_]+)\s*\(", text)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libsol.so with argument types set (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libsol.so is not built at {LIB_PATH}; run "
+                              "`python -m dit_block_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(status: int, func: str):
+    if status != OK:
+        raise SolError(status, func, lib().sol_last_error().decode())
+
+
+def status_string(status: int) -> str:
+    return lib().sol_status_string(status).decode()
+
+
+def abi_version() -> int:
+    return int(lib().sol_abi_version())
+
+
+# ------------------------------------------------------------------------- marshalling
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"libsol takes float32 or bfloat16 tensors, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _ld(t: torch.Tensor | None) -> int:
+    if t is None:
+        return 0
+    if t.dim() == 1:
+        return t.shape[0]
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("tensors must be 2-D with unit column stride")
+    return t.stride(0)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _sel(stream_id: torch.Tensor | None, n_streams: int, tokens_per_sample: int) -> ModSel:
+    if stream_id is not None and stream_id.dtype != torch.uint8:
+        raise TypeError("stream_id must be uint8")
+    return ModSel(_ptr(stream_id), int(n_streams), int(tokens_per_sample))
+
+
+def _mod_ld(*mods) -> int:
+    for m in mods:
+        if m is not None:
+            return _ld(m)
+    return 0
+
+
+# ----------------------------------------------------------------------------- the ops
+
+def adaln_modulate(h, x, shift=None, scale=None, *, eps=1e-6, stream_id=None, n_streams=1,
+                   tokens_per_sample=0, d=None, stream=None):
+    """h = LN(x) * (1 + scale[r]) + shift[r]  (sol_adaln_modulate)."""
+    n = x.shape[0]
+    d = x.shape[1] if d is None else d
+    _check(lib().sol_adaln_modulate(_ptr(h), _ld(h), _ptr(x), _ld(x), _ptr(shift), _ptr(scale),
+                                    _mod_ld(shift, scale), _sel(stream_id, n_streams, tokens_per_sample),
+                                    n, d, eps, _dtype(x), _stream(stream)), "sol_adaln_modulate")
+    return h
+
+
+def gated_residual(out, x, y, gate=None, *, stream_id=None, n_streams=1, tokens_per_sample=0,
+                   d=None, stream=None):
+    """out = x + gate[r] * y  (sol_gated_residual)."""
+    n = x.shape[0]
+    d = x.shape[1] if d is None else d
+    _check(lib().sol_gated_residual(_ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(y), _ld(y), _ptr(gate),
+                                    _mod_ld(gate), _sel(stream_id, n_streams, tokens_per_sample), n, d,
+                                    _dtype(x), _stream(stream)), "sol_gated_residual")
+    return out
+
+
+def swiglu(out, u, *, inner=None, stream=None):
+    """out = silu(u[:, :inner]) * u[:, inner:2*inner] for the packed up-projection u."""
+    inner = u.shape[1] // 2 if inner is None else inner
+    b = u.data_ptr() + inner * u.element_size()
+    _check(lib().sol_swiglu(_ptr(out), _ld(out), u.data_ptr(), b, _ld(u), u.shape[0], inner,
+                            _dtype(u), _stream(stream)), "sol_swiglu")
+    return out
+
+
+def swiglu_ab(out, a, b, *, stream=None):
+    """out = silu(a) * b for two tensors with the same leading dimension."""
+    if _ld(a) != _ld(b):
+        raise ValueError("a and b must share a leading dimension")
+    _check(lib().sol_swiglu(_ptr(out), _ld(out), _ptr(a), _ptr(b), _ld(a), a.shape[0], a.shape[1],
+                            _dtype(a), _stream(stream)), "sol_swiglu")
+    return out
+
+
+class Rope3D:
+    """Library-owned 3D RoPE cos/sin tables on the current device (sol_rope3d_create)."""
+
+    def __init__(self, dims=(32, 48, 48), theta=10000.0, max_pos=(64, 64, 128)):
+        h = ctypes.c_void_p()
+        _check(lib().sol_rope3d_create(ctypes.byref(h), int(dims[0]), int(dims[1]), int(dims[2]),
+                                       float(theta), int(max_pos[0]), int(max_pos[1]),
+                                       int(max_pos[2])), "sol_rope3d_create")
+        self.handle = h.value
+        self.dims = tuple(dims)
+        self.theta = theta
+        self.max_pos = tuple(max_pos)
+
+    def close(self):
+        if self.handle:
+            _check(lib().sol_rope3d_destroy(self.handle), "sol_rope3d_destroy")
+            self.handle = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def qk_rmsnorm_rope3d(q_out, k_out, q, k, rope: Rope3D, *, n_heads, head_dim, wq=None, wk=None,
+                      pos=None, grid=(0, 0, 0), tokens_per_sample=0, eps=1e-6, stream=None):
+    """QK RMSNorm then 3D RoPE on every head vector of q and k (sol_qk_rmsnorm_rope3d)."""
+    if pos is not None and (pos.dtype != torch.int32 or not pos.is_contiguous()):
+        raise TypeError("pos must be a contiguous int32 [N, 3] tensor")
+    _check(lib().sol_qk_rmsnorm_rope3d(
+        _ptr(q_out), _ptr(k_out), _ld(q_out), _ld(k_out), _ptr(q), _ptr(k), _ld(q), _ld(k),
+        _ptr(wq), _ptr(wk), _ptr(pos), int(grid[0]), int(grid[1]), int(grid[2]),
+        int(tokens_per_sample), rope.handle, q.shape[0], int(n_heads), int(head_dim), eps,
+        _dtype(q), _stream(stream)), "sol_qk_rmsnorm_rope3d")
+
+
+def dit_prologue(x_out, h, x, y=None, gate=None, shift=None, scale=None, *, eps=1e-6,
+                 stream_id=None, n_streams=1, tokens_per_sample=0, stream=None):
+    """x' = x + gate*y (if y), h = AdaLN(x') in one pass (sol_dit_prologue)."""
+    ld = _ld(x)
+    _check(lib().sol_dit_prologue(_ptr(x_out), _ptr(h), _ptr(x), _ptr(y), _ptr(gate), _ptr(shift),
+                                  _ptr(scale), ld, _mod_ld(gate, shift, scale),
+                                  _sel(stream_id, n_streams, tokens_per_sample), x.shape[0],
+                                  x.shape[1], eps, _dtype(x), _stream(stream)), "sol_dit_prologue")
+
+
+def dit_epilogue(qkv, rope: Rope3D, *, n_heads, head_dim, wq=None, wk=None, pos=None,
+                 grid=(0, 0, 0), tokens_per_sample=0, eps=1e-6, stream=None):
+    """QK RMSNorm + 3D RoPE on the q and k parts of packed [q | k | v] rows, in place."""
+    if pos is not None and (pos.dtype != torch.int32 or not pos.is_contiguous()):
+        raise TypeError("pos must be a contiguous int32 [N, 3] tensor")
+    _check(lib().sol_dit_epilogue(_ptr(qkv), _ld(qkv), _ptr(wq), _ptr(wk), _ptr(pos), int(grid[0]),
+                                  int(grid[1]), int(grid[2]), int(tokens_per_sample), rope.handle,
+                                  qkv.shape[0], int(n_heads), int(head_dim), eps, _dtype(qkv),
+                                  _stream(stream)), "sol_dit_epilogue")

@@ -1,0 +1,188 @@
+/*
+ * sol.h -- C ABI of libsol, the B200 (sm_100a) library of fused DiT-block per-token
+ * operators: AdaLN modulation, the gated residual, the SwiGLU activation, QK RMSNorm
+ * fused with 3D RoPE, and two fused chains of them (a block prologue and a QKV
+ * epilogue).
+ *
+ * Sources.  The operators are the ones the SGLang Diffusion write-ups single out as
+ * fused kernels for MiniMax-H3:
+ *   [XHH-QA]  "8xH200 上的 MiniMax-H3: 无损加速 1.95 倍, SSIM 0.76-0.91 下最高 6.24 倍"
+ *             (xhh.club), Q&A, the answer on which operations the fused kernels
+ *             optimise: AdaLN modulation, gated residual, SwiGLU activation, and QK
+ *             RMSNorm fused with 3D RoPE.
+ *   [STM-GAN] "SGLang acelera video do MiniMax-H3 em ate 6,2x em GPUs H200"
+ *             (stamatios.com), section "De onde vem os ganhos".
+ *   [STM-RES] same page, section "Resultado principal": fused kernels cut memory
+ *             traffic, intermediate tensors and launches without changing the math;
+ *             video and audio tokens run through one packed DiT stack.
+ * The pages name the operators but print no formula; each function below states the
+ * formula it computes.
+ *
+ * Common conventions
+ *   Layout.    Token-major: row n of a tensor starts at element n*ld.  Leading
+ *              dimensions (ld*) count ELEMENTS and must be multiples of 8 (bf16) or
+ *              4 (f32), so that every row starts on a 16-byte boundary.
+ *   Pointers.  Device pointers (memory the GPU can address), 16-byte aligned.  The
+ *              caller owns every buffer; no op allocates, frees or synchronises.
+ *   Dtypes.    All tensors of one call share `dt`.  Arithmetic is fp32 inside every
+ *              kernel; each output element is rounded once (round to nearest even)
+ *              when stored.  The RoPE tables are always fp32.
+ *   Streams.   Every op is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *              legacy default stream).  A returned SOL_OK means the launch was
+ *              accepted, not that it finished.
+ *   Errors.    Arguments are validated on the host before anything is launched; on
+ *              failure the call returns a SOL_ERR_* code with no side effect, and
+ *              sol_last_error() gives a one-line reason (per host thread).
+ *              SOL_ERR_CUDA reports a launch failure.
+ *   n_tokens == 0 is valid and launches nothing.
+ *   Aliasing.  Only the aliases each function lists are allowed (every row is read
+ *              completely before it is written).  Any other overlap is undefined.
+ */
+#ifndef SOL_H
+#define SOL_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* sol_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    SOL_OK = 0,
+    SOL_ERR_INVALID_ARGUMENT = 1, /* NULL where a tensor is required, bad size or ld  */
+    SOL_ERR_MISALIGNED = 2,       /* pointer not 16-byte aligned                        */
+    SOL_ERR_UNSUPPORTED = 3,      /* valid but not built: dtype, head_dim, ...           */
+    SOL_ERR_CUDA = 4              /* the CUDA runtime refused the launch or allocation */
+} sol_status;
+
+typedef enum { SOL_DTYPE_F32 = 0, SOL_DTYPE_BF16 = 1 } sol_dtype;
+
+/* Which modulation row (shift / scale / gate) a token uses.  One packed sequence holds
+ * `B` samples of `tokens_per_sample` tokens each; inside a sample each token belongs
+ * to one of `n_streams` streams (video, audio, ...) [STM-RES].  Token n uses row
+ *     r = (n / tokens_per_sample) * n_streams + stream_id[n]
+ * of every modulation tensor, so those tensors hold B*n_streams rows of `ld_mod`.
+ *   stream_id          device uint8 [n_tokens], or NULL (every token in stream 0);
+ *                      ids >= n_streams are clamped to n_streams - 1.
+ *   n_streams          >= 1.
+ *   tokens_per_sample  > 0, or 0 meaning the whole call is one sample. */
+typedef struct {
+    const uint8_t* stream_id;
+    int32_t n_streams;
+    int64_t tokens_per_sample;
+} sol_modsel;
+
+/* Fixed description of a status code (never NULL). */
+const char* sol_status_string(sol_status status);
+
+/* One-line reason for the last non-SOL_OK status returned on this host thread ("" if
+ * none).  The pointer stays valid until the next sol_* call on this thread. */
+const char* sol_last_error(void);
+
+/* Version of this ABI (incremented on any incompatible change). */
+int32_t sol_abi_version(void);
+
+/* AdaLN modulation [XHH-QA, STM-GAN]:
+ *     mu = mean_i x_i,  var = mean_i (x_i - mu)^2  (biased, two passes),
+ *     h_i = (x_i - mu) / sqrt(var + eps) * (1 + scale[r]_i) + shift[r]_i
+ * for every token row of x (width d); r from `sel`.  LayerNorm has no affine weights:
+ * the modulation is its affine part.
+ *   h, ld_h        output [n_tokens, ld_h]; may equal x (then ld_h must equal ld_x).
+ *   x, ld_x        input  [n_tokens, ld_x].
+ *   shift, scale   [rows, ld_mod] or NULL (read as all zero).
+ *   d              row width: multiple of 8 (bf16) / 4 (f32), 8 <= d <= 16384.
+ *   eps            >= 0, finite. */
+sol_status sol_adaln_modulate(void* h, int64_t ld_h, const void* x, int64_t ld_x,
+                              const void* shift, const void* scale, int64_t ld_mod,
+                              sol_modsel sel, int64_t n_tokens, int64_t d, float eps,
+                              sol_dtype dt, sol_stream_t stream);
+
+/* Gated residual [XHH-QA]:  out_i = x_i + gate[r]_i * y_i  (gate is a plain multiplier).
+ *   out, ld_out    output [n_tokens, ld_out]; may equal x (then ld_out == ld_x).
+ *   x, y           inputs [n_tokens, ld_x] and [n_tokens, ld_y].
+ *   gate           [rows, ld_mod] or NULL (zero: out = x, bit for bit, for finite y).
+ *   d              multiple of 8 (bf16) / 4 (f32), >= 8. */
+sol_status sol_gated_residual(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                              const void* y, int64_t ld_y, const void* gate, int64_t ld_mod,
+                              sol_modsel sel, int64_t n_tokens, int64_t d, sol_dtype dt,
+                              sol_stream_t stream);
+
+/* SwiGLU activation [XHH-QA, STM-GAN]:  out_j = silu(a_j) * b_j,  silu(v) = v/(1+e^-v),
+ * j < inner, for every token row.  For the packed up-projection u = [a | b] of width
+ * 2*inner pass a = u, b = u + inner (elements) and ld_in = ld of u.
+ *   out, ld_out    output [n_tokens, ld_out], must not overlap a or b.
+ *   a, b, ld_in    inputs; row n of a (b) starts at a + n*ld_in (b + n*ld_in).
+ *   inner          multiple of 8 (bf16) / 4 (f32), >= 8. */
+sol_status sol_swiglu(void* out, int64_t ld_out, const void* a, const void* b, int64_t ld_in,
+                      int64_t n_tokens, int64_t inner, sol_dtype dt, sol_stream_t stream);
+
+/* 3D RoPE tables (library-owned).  The head vector is split into three chunks of widths
+ * dim_t, dim_h, dim_w (in this order, each even, summing to head_dim).  Inside chunk c,
+ * the interleaved pair (2j, 2j+1) of a token at integer position p_c on axis c turns by
+ *     phi = p_c * theta^(-2j / dim_c).
+ * The tables hold cos(phi), sin(phi) for p_c in [0, max_c), computed on the host in fp64
+ * and rounded to fp32.  Create allocates device memory on the CURRENT device (one
+ * cudaMalloc, one synchronous copy); use the handle only on that device.  Destroy
+ * frees it (NULL is accepted) and must not run while a kernel using it is in flight. */
+typedef struct sol_rope3d sol_rope3d;
+sol_status sol_rope3d_create(sol_rope3d** out, int32_t dim_t, int32_t dim_h, int32_t dim_w,
+                             double theta, int32_t max_t, int32_t max_h, int32_t max_w);
+sol_status sol_rope3d_destroy(sol_rope3d* rope);
+
+/* QK RMSNorm fused with 3D RoPE [XHH-QA "QK RMSNorm 与 3D RoPE 的融合", STM-GAN]:
+ * for every head vector v (head_dim wide) of q and of k:
+ *     v^_i = v_i / sqrt(mean_i v_i^2 + eps) * w_i         (w = wq for q, wk for k)
+ * then every pair of v^ is turned by the RoPE angle of the token's (t, h, w) position.
+ *   q_out, k_out   outputs, ld_qo / ld_ko; may equal q / k (in place) with the same ld.
+ *   q, k           [n_tokens, ld_q] / [n_tokens, ld_k]: n_heads vectors per row, the
+ *                  row may sit inside a packed QKV row (ld = 3*n_heads*head_dim).
+ *   wq, wk         [head_dim] RMSNorm weights, or NULL (all ones).
+ *   pos            device int32 [n_tokens, 3] (t, h, w) positions, or NULL: then token
+ *                  n of each sample sits at n_local = n mod tokens_per_sample in a
+ *                  row-major grid_T x grid_H x grid_W grid:
+ *                  t = n_local / (H*W), h = (n_local / W) mod H, w = n_local mod W.
+ *                  Explicit positions outside [0, max_c) are clamped into it.
+ *   grid_*         used when pos == NULL; each must be <= the table's max on its axis.
+ *   tokens_per_sample  > 0, or 0 = one sample (used only when pos == NULL).
+ *   rope           tables from sol_rope3d_create, dims summing to head_dim.
+ *   head_dim       64, 128 or 256 for bf16; 32, 64 or 128 for f32.
+ *   n_heads        >= 1. */
+sol_status sol_qk_rmsnorm_rope3d(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko,
+                                 const void* q, const void* k, int64_t ld_q, int64_t ld_k,
+                                 const void* wq, const void* wk, const int32_t* pos,
+                                 int32_t grid_T, int32_t grid_H, int32_t grid_W,
+                                 int64_t tokens_per_sample, const sol_rope3d* rope,
+                                 int64_t n_tokens, int32_t n_heads, int32_t head_dim,
+                                 float eps, sol_dtype dt, sol_stream_t stream);
+
+/* Fused block prologue [STM-RES: one pass instead of two, same math]:
+ *     x'_i = x_i + gate[r]_i * y_i             (skipped when y == NULL: x' = x)
+ *     h_i  = AdaLN(x')_i  as in sol_adaln_modulate, on the UNROUNDED fp32 x'.
+ * One read of x (and y), one write of x' (when y != NULL) and of h.
+ *   x_out          [n_tokens, ld] receives x' (rounded); required iff y != NULL; may
+ *                  equal x.
+ *   h              [n_tokens, ld]; must not overlap x, y or x_out.
+ *   gate, shift, scale  [rows, ld_mod] or NULL (zero).
+ *   ld             shared leading dimension of x_out, h, x, y. */
+sol_status sol_dit_prologue(void* x_out, void* h, const void* x, const void* y,
+                            const void* gate, const void* shift, const void* scale, int64_t ld,
+                            int64_t ld_mod, sol_modsel sel, int64_t n_tokens, int64_t d,
+                            float eps, sol_dtype dt, sol_stream_t stream);
+
+/* Fused QKV-projection epilogue: sol_qk_rmsnorm_rope3d on the q and k parts of packed
+ * rows [q | k | v] (q at element 0, k at n_heads*head_dim), IN PLACE, in one launch;
+ * v is neither read nor written.  Arguments as in sol_qk_rmsnorm_rope3d. */
+sol_status sol_dit_epilogue(void* qkv, int64_t ld_qkv, const void* wq, const void* wk,
+                            const int32_t* pos, int32_t grid_T, int32_t grid_H, int32_t grid_W,
+                            int64_t tokens_per_sample, const sol_rope3d* rope, int64_t n_tokens,
+                            int32_t n_heads, int32_t head_dim, float eps, sol_dtype dt,
+                            sol_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOL_H */

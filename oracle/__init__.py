@@ -47,19 +47,20 @@ def _load():
         P, I64, I32, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double
         I = ctypes.c_int
         lib.oracle_num_threads.restype = I
-        lib.oracle_adaln_modulate.argtypes = [P, I64, P, I64, I, P, P, I64, I, P, I32, I64, I64, I64, D]
+        lib.oracle_adaln_modulate.argtypes = [P, I64, P, I64, I, P, P, I64, I, P, I32, I64, P, I64, I64, D]
         lib.oracle_adaln_modulate.restype = None
-        lib.oracle_gated_residual.argtypes = [P, I64, P, I64, P, I64, I, P, I64, I, P, I32, I64, I64, I64]
+        lib.oracle_gated_residual.argtypes = [P, I64, P, I64, P, I64, I, P, I64, I, P, I32, I64, P, I64, I64]
         lib.oracle_gated_residual.restype = None
         lib.oracle_swiglu.argtypes = [P, I64, P, P, I64, I, I64, I64]
         lib.oracle_swiglu.restype = None
         lib.oracle_qk_rmsnorm_rope3d.argtypes = [P, P, I64, I64, P, P, I64, I64, I, P, P, I, P,
-                                                 I32, I32, I32, I64, I32, I32, I32, D, I64, I32, I32, D]
+                                                 I32, I32, I32, I64, I32, I32, I32, D, P, I64, I32,
+                                                 I32, D]
         lib.oracle_qk_rmsnorm_rope3d.restype = I
-        lib.oracle_dit_prologue.argtypes = [P, P, P, P, I, P, P, P, I64, I64, I, P, I32, I64, I64, I64, D]
+        lib.oracle_dit_prologue.argtypes = [P, P, P, P, I, P, P, P, I64, I64, I, P, I32, I64, P, I64, I64, D]
         lib.oracle_dit_prologue.restype = None
         lib.oracle_dit_epilogue.argtypes = [P, P, I64, I, P, P, I, P, I32, I32, I32, I64,
-                                            I32, I32, I32, D, I64, I32, I32, D]
+                                            I32, I32, I32, D, P, I64, I32, I32, D]
         lib.oracle_dit_epilogue.restype = I
         _lib = lib
     return _lib
@@ -89,6 +90,15 @@ def _ptr(a: np.ndarray | None):
     return a.ctypes.data
 
 
+def _rows(rows, n):
+    """Global token index of each row passed (None: rows are tokens 0..n-1)."""
+    if rows is None:
+        return None
+    r = np.ascontiguousarray(rows, dtype=np.int64)
+    assert r.shape == (n,), "rows must hold one global token index per row"
+    return r
+
+
 def _ld(a: np.ndarray) -> int:
     return a.shape[-1] if a.ndim > 1 else a.shape[0]
 
@@ -102,29 +112,34 @@ def _mod_args(mod: np.ndarray | None, stream_id, n_streams, tokens_per_sample):
 
 
 def adaln_modulate(x, shift=None, scale=None, *, eps=1e-6, stream_id=None, n_streams=1,
-                   tokens_per_sample=0, n_tokens=None, d=None):
-    """h = LN(x) * (1 + scale[r]) + shift[r] per token row of x ([N, ld_x], first d columns)."""
+                   tokens_per_sample=0, rows=None, n_tokens=None, d=None):
+    """h = LN(x) * (1 + scale[r]) + shift[r] per token row of x ([N, ld_x], first d columns).
+
+    rows: optional global token index of each row of x (stream_id is then indexed by it)."""
     n = x.shape[0] if n_tokens is None else n_tokens
     d = x.shape[1] if d is None else d
     mod = shift if shift is not None else scale
     ld_mod, sid, S, tps = _mod_args(mod, stream_id, n_streams, tokens_per_sample)
+    rw = _rows(rows, n)
     out = np.empty((n, d), np.float64)
     _load().oracle_adaln_modulate(out.ctypes.data, d, _ptr(x), _ld(x), _code(x), _ptr(shift),
-                                  _ptr(scale), ld_mod, _code(mod), _ptr(sid), S, tps, n, d,
-                                  float(eps))
+                                  _ptr(scale), ld_mod, _code(mod), _ptr(sid), S, tps, _ptr(rw), n,
+                                  d, float(eps))
     return out
 
 
 def gated_residual(x, y, gate=None, *, stream_id=None, n_streams=1, tokens_per_sample=0,
-                   n_tokens=None, d=None):
+                   rows=None, n_tokens=None, d=None):
     """o = x + gate[r] * y per token row."""
     assert x.dtype == y.dtype
     n = x.shape[0] if n_tokens is None else n_tokens
     d = x.shape[1] if d is None else d
     ld_mod, sid, S, tps = _mod_args(gate, stream_id, n_streams, tokens_per_sample)
+    rw = _rows(rows, n)
     out = np.empty((n, d), np.float64)
     _load().oracle_gated_residual(out.ctypes.data, d, _ptr(x), _ld(x), _ptr(y), _ld(y), _code(x),
-                                  _ptr(gate), ld_mod, _code(gate), _ptr(sid), S, tps, n, d)
+                                  _ptr(gate), ld_mod, _code(gate), _ptr(sid), S, tps, _ptr(rw),
+                                  n, d)
     return out
 
 
@@ -157,7 +172,8 @@ def _pos_ptr(pos):
 
 
 def qk_rmsnorm_rope3d(q, k, wq=None, wk=None, *, n_heads, head_dim, pos=None, grid=(0, 0, 0),
-                      tokens_per_sample=0, dims=(32, 48, 48), theta=10000.0, eps=1e-6):
+                      tokens_per_sample=0, dims=(32, 48, 48), theta=10000.0, eps=1e-6,
+                      rows=None):
     """QK RMSNorm then 3D RoPE on each head vector of q [N, ld_q] and k [N, ld_k].
 
     Either q or k may be None.  Returns (q_out, k_out) as [N, n_heads*head_dim] float64."""
@@ -168,18 +184,20 @@ def qk_rmsnorm_rope3d(q, k, wq=None, wk=None, *, n_heads, head_dim, pos=None, gr
     ko = np.empty((n, hd), np.float64) if k is not None else None
     w = wq if wq is not None else wk
     pos_arr, pos_p = _pos_ptr(pos)
+    rw = _rows(rows, n)
     rc = _load().oracle_qk_rmsnorm_rope3d(
         _ptr(qo), _ptr(ko), hd, hd, _ptr(q), _ptr(k), _ld(q) if q is not None else 0,
         _ld(k) if k is not None else 0, _code(src), _ptr(wq), _ptr(wk), _code(w), pos_p,
         int(grid[0]), int(grid[1]), int(grid[2]), int(tokens_per_sample), int(dims[0]),
-        int(dims[1]), int(dims[2]), float(theta), n, int(n_heads), int(head_dim), float(eps))
+        int(dims[1]), int(dims[2]), float(theta), _ptr(rw), n, int(n_heads), int(head_dim),
+        float(eps))
     if rc != 0:
         raise ValueError("RoPE split does not fit head_dim (dims must be even and sum to it)")
     return qo, ko
 
 
 def dit_prologue(x, y=None, gate=None, shift=None, scale=None, *, eps=1e-6, stream_id=None,
-                 n_streams=1, tokens_per_sample=0):
+                 n_streams=1, tokens_per_sample=0, rows=None):
     """Fused prologue: x' = x + gate*y (when y is given), h = AdaLN(x').  Returns (x', h);
     x' is None when y is None."""
     n, d = x.shape
@@ -187,14 +205,15 @@ def dit_prologue(x, y=None, gate=None, shift=None, scale=None, *, eps=1e-6, stre
     ld_mod, sid, S, tps = _mod_args(mod, stream_id, n_streams, tokens_per_sample)
     xo = np.empty((n, d), np.float64) if y is not None else None
     h = np.empty((n, d), np.float64)
+    rw = _rows(rows, n)
     _load().oracle_dit_prologue(_ptr(xo), h.ctypes.data, _ptr(x), _ptr(y), _code(x), _ptr(gate),
                                 _ptr(shift), _ptr(scale), d, ld_mod, _code(mod), _ptr(sid), S, tps,
-                                n, d, float(eps))
+                                _ptr(rw), n, d, float(eps))
     return xo, h
 
 
 def dit_epilogue(qkv, wq=None, wk=None, *, n_heads, head_dim, pos=None, grid=(0, 0, 0),
-                 tokens_per_sample=0, dims=(32, 48, 48), theta=10000.0, eps=1e-6):
+                 tokens_per_sample=0, dims=(32, 48, 48), theta=10000.0, eps=1e-6, rows=None):
     """Fused QKV epilogue on packed rows [q | k | v]: returns [N, 2*n_heads*head_dim] with the
     normed+rotated q then k."""
     n = qkv.shape[0]
@@ -202,10 +221,12 @@ def dit_epilogue(qkv, wq=None, wk=None, *, n_heads, head_dim, pos=None, grid=(0,
     out = np.empty((n, 2 * hd), np.float64)
     w = wq if wq is not None else wk
     pos_arr, pos_p = _pos_ptr(pos)
+    rw = _rows(rows, n)
     rc = _load().oracle_dit_epilogue(
         out.ctypes.data, _ptr(qkv), _ld(qkv), _code(qkv), _ptr(wq), _ptr(wk), _code(w), pos_p,
         int(grid[0]), int(grid[1]), int(grid[2]), int(tokens_per_sample), int(dims[0]),
-        int(dims[1]), int(dims[2]), float(theta), n, int(n_heads), int(head_dim), float(eps))
+        int(dims[1]), int(dims[2]), float(theta), _ptr(rw), n, int(n_heads), int(head_dim),
+        float(eps))
     if rc != 0:
         raise ValueError("RoPE split does not fit head_dim (dims must be even and sum to it)")
     return out

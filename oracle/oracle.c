@@ -30,6 +30,12 @@
  *   Implicit positions (pos == NULL): n_local = n mod tokens_per_sample,
  *            t = n_local / (H*W), h = (n_local / W) mod H, w = n_local mod W.
  *
+ * Row subsets: every function takes `rows`, NULL or the global token index of each row
+ * passed (row n of the inputs and outputs is token rows[n] of the sequence).  The global
+ * index selects the modulation row, the stream id (stream_id and pos are indexed by it)
+ * and the implicit grid position; it lets a caller check sampled rows of a long
+ * sequence without handing over the whole sequence.
+ *
  * Every input element is read through load(), which widens f32 / bf16 / f64 to double
  * exactly.  Everything after that is fp64; nothing is rounded until the caller reads
  * the fp64 output.  Rows run in parallel with OpenMP; nothing else is reordered.
@@ -85,11 +91,11 @@ void oracle_adaln_modulate(double* h, int64_t ld_h,
                            const void* x, int64_t ld_x, int dt_x,
                            const void* shift, const void* scale, int64_t ld_mod, int dt_mod,
                            const uint8_t* stream_id, int32_t n_streams, int64_t tokens_per_sample,
-                           int64_t n_tokens, int64_t d, double eps)
+                           const int64_t* rows, int64_t n_tokens, int64_t d, double eps)
 {
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < n_tokens; ++n) {
-        const int64_t r = mod_row(n, stream_id, n_streams, tokens_per_sample);
+        const int64_t r = mod_row(rows ? rows[n] : n, stream_id, n_streams, tokens_per_sample);
         double mu = 0.0;
         for (int64_t i = 0; i < d; ++i) mu += load(x, dt_x, n * ld_x + i);
         mu /= (double)d;
@@ -114,11 +120,11 @@ void oracle_gated_residual(double* o, int64_t ld_o,
                            const void* x, int64_t ld_x, const void* y, int64_t ld_y, int dt_xy,
                            const void* gate, int64_t ld_mod, int dt_mod,
                            const uint8_t* stream_id, int32_t n_streams, int64_t tokens_per_sample,
-                           int64_t n_tokens, int64_t d)
+                           const int64_t* rows, int64_t n_tokens, int64_t d)
 {
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < n_tokens; ++n) {
-        const int64_t r = mod_row(n, stream_id, n_streams, tokens_per_sample);
+        const int64_t r = mod_row(rows ? rows[n] : n, stream_id, n_streams, tokens_per_sample);
         for (int64_t i = 0; i < d; ++i) {
             const double g = gate ? load(gate, dt_mod, r * ld_mod + i) : 0.0;
             o[n * ld_o + i] = load(x, dt_xy, n * ld_x + i) + g * load(y, dt_xy, n * ld_y + i);
@@ -201,7 +207,8 @@ int oracle_qk_rmsnorm_rope3d(double* q_out, double* k_out, int64_t ld_qo, int64_
                              const int32_t* pos, int32_t grid_T, int32_t grid_H, int32_t grid_W,
                              int64_t tokens_per_sample,
                              int32_t dim_t, int32_t dim_h, int32_t dim_w, double theta,
-                             int64_t n_tokens, int32_t n_heads, int32_t head_dim, double eps)
+                             const int64_t* rows, int64_t n_tokens, int32_t n_heads,
+                             int32_t head_dim, double eps)
 {
     const int32_t dims[3] = {dim_t, dim_h, dim_w};
     if (dim_t + dim_h + dim_w != head_dim || (dim_t | dim_h | dim_w) & 1 || head_dim > 1024)
@@ -209,7 +216,7 @@ int oracle_qk_rmsnorm_rope3d(double* q_out, double* k_out, int64_t ld_qo, int64_
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < n_tokens; ++n) {
         int64_t p[3];
-        token_position(n, pos, grid_T, grid_H, grid_W, tokens_per_sample, p);
+        token_position(rows ? rows[n] : n, pos, grid_T, grid_H, grid_W, tokens_per_sample, p);
         for (int32_t hh = 0; hh < n_heads; ++hh) {
             if (q)
                 rmsnorm_rope_head(q_out + n * ld_qo + (int64_t)hh * head_dim, q,
@@ -233,16 +240,16 @@ void oracle_dit_prologue(double* x_out, double* h,
                          const void* gate, const void* shift, const void* scale,
                          int64_t ld, int64_t ld_mod, int dt_mod,
                          const uint8_t* stream_id, int32_t n_streams, int64_t tokens_per_sample,
-                         int64_t n_tokens, int64_t d, double eps)
+                         const int64_t* rows, int64_t n_tokens, int64_t d, double eps)
 {
     if (y) {
         oracle_gated_residual(x_out, d, x, ld, y, ld, dt, gate, ld_mod, dt_mod, stream_id,
-                              n_streams, tokens_per_sample, n_tokens, d);
+                              n_streams, tokens_per_sample, rows, n_tokens, d);
         oracle_adaln_modulate(h, d, x_out, d, OR_F64, shift, scale, ld_mod, dt_mod, stream_id,
-                              n_streams, tokens_per_sample, n_tokens, d, eps);
+                              n_streams, tokens_per_sample, rows, n_tokens, d, eps);
     } else {
         oracle_adaln_modulate(h, d, x, ld, dt, shift, scale, ld_mod, dt_mod, stream_id,
-                              n_streams, tokens_per_sample, n_tokens, d, eps);
+                              n_streams, tokens_per_sample, rows, n_tokens, d, eps);
     }
 }
 
@@ -253,13 +260,14 @@ int oracle_dit_epilogue(double* qk_out, const void* qkv, int64_t ld_qkv, int dt,
                         const int32_t* pos, int32_t grid_T, int32_t grid_H, int32_t grid_W,
                         int64_t tokens_per_sample,
                         int32_t dim_t, int32_t dim_h, int32_t dim_w, double theta,
-                        int64_t n_tokens, int32_t n_heads, int32_t head_dim, double eps)
+                        const int64_t* rows, int64_t n_tokens, int32_t n_heads, int32_t head_dim,
+                        double eps)
 {
     const int64_t hd = (int64_t)n_heads * head_dim;
     const size_t esz = dt == OR_F64 ? 8 : dt == OR_F32 ? 4 : 2;
     const void* k = (const char*)qkv + (size_t)hd * esz;
     return oracle_qk_rmsnorm_rope3d(qk_out, qk_out + hd, 2 * hd, 2 * hd, qkv, k, ld_qkv, ld_qkv,
                                     dt, wq, wk, dt_w, pos, grid_T, grid_H, grid_W,
-                                    tokens_per_sample, dim_t, dim_h, dim_w, theta, n_tokens,
+                                    tokens_per_sample, dim_t, dim_h, dim_w, theta, rows, n_tokens,
                                     n_heads, head_dim, eps);
 }

@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+function include/sol.h declares, and rejects bad arguments before any CUDA call.
+
+The pointers passed here are fake addresses; every call below fails validation on the
+host, so none of them reaches the CUDA runtime or the device."""
+from __future__ import annotations
+
+import ctypes
+
+import pytest
+
+from dit_block_b200 import build, sol
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return sol.lib()
+
+
+FAKE = 1 << 20  # 16-byte aligned fake address (never dereferenced)
+SEL = sol.ModSel(None, 1, 0)
+
+
+def last(L):
+    return L.sol_last_error().decode()
+
+
+def test_exports_every_declared_symbol(L):
+    names = sol.header_functions()
+    assert len(names) == 11
+    for n in names:
+        assert hasattr(L, n), f"libsol.so does not export {n}"
+        assert n in sol.SIGNATURES, f"binding has no signature for {n}"
+
+
+def test_status_strings_and_version(L):
+    assert L.sol_abi_version() == 1
+    assert L.sol_status_string(0) == b"ok"
+    for s in range(1, 5):
+        assert L.sol_status_string(s) and L.sol_status_string(s) != b"ok"
+    assert L.sol_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("dt", [sol.F32, sol.BF16])
+def test_adaln_validation(L, dt):
+    bad_d = 7
+    assert L.sol_adaln_modulate(FAKE, 8, FAKE, 8, None, None, 0, SEL, 4, bad_d, 1e-6, dt, None) \
+        in (sol.ERR_INVALID_ARGUMENT, sol.ERR_UNSUPPORTED)
+    assert L.sol_adaln_modulate(None, 8, FAKE, 8, None, None, 0, SEL, 4, 8, 1e-6, dt, None) \
+        == sol.ERR_INVALID_ARGUMENT
+    assert "h is NULL" in last(L)
+    assert L.sol_adaln_modulate(FAKE + 4, 8, FAKE, 8, None, None, 0, SEL, 4, 8, 1e-6, dt, None) \
+        == sol.ERR_MISALIGNED
+    assert L.sol_adaln_modulate(FAKE, 6, FAKE, 8, None, None, 0, SEL, 4, 8, 1e-6, dt, None) \
+        == sol.ERR_INVALID_ARGUMENT  # ld below width
+    assert L.sol_adaln_modulate(FAKE, 8, FAKE, 8, None, None, 0, SEL, -1, 8, 1e-6, dt, None) \
+        == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_adaln_modulate(FAKE, 8, FAKE, 8, None, None, 0, SEL, 4, 8, -1.0, dt, None) \
+        == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_adaln_modulate(FAKE, 8, FAKE, 8, None, None, 0, SEL, 4, 8, float("nan"), dt, None) \
+        == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_adaln_modulate(FAKE, 1 << 20, FAKE, 1 << 20, None, None, 0, SEL, 4, 1 << 20, 1e-6,
+                                dt, None) == sol.ERR_UNSUPPORTED  # wider than one CTA row holds
+    assert "wider" in last(L)
+
+
+def test_leading_dimension_must_keep_rows_16_byte_aligned(L):
+    # bf16 rows of ld 12 elements are 24 bytes apart: rejected; f32 ld 12 is 48 bytes: fine
+    assert L.sol_gated_residual(FAKE, 12, FAKE, 16, FAKE, 16, None, 0, SEL, 2, 8, sol.BF16, None) \
+        == sol.ERR_MISALIGNED
+    assert "multiple of 8" in last(L)
+
+
+def test_overlap_rules(L):
+    # h partially overlapping x is rejected; h == x is allowed (passes validation; with
+    # n_tokens = 0 nothing is launched)
+    n, d = 4, 64
+    assert L.sol_adaln_modulate(FAKE + 128, d, FAKE, d, None, None, 0, SEL, n, d, 1e-6, sol.BF16, None) \
+        == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_adaln_modulate(FAKE, d, FAKE, d, None, None, 0, SEL, 0, d, 1e-6, sol.BF16, None) == sol.OK
+    # prologue: h may not alias x
+    assert L.sol_dit_prologue(FAKE, FAKE, FAKE, None, None, None, None, d, 0, SEL, n, d, 1e-6,
+                              sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    # swiglu output may not overlap its inputs
+    assert L.sol_swiglu(FAKE, 64, FAKE, FAKE + 64, 128, 4, 32, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+
+
+def test_modsel_validation(L):
+    bad = sol.ModSel(None, 0, 0)
+    assert L.sol_gated_residual(FAKE, 8, FAKE + 4096, 8, FAKE + 8192, 8, None, 0, bad, 2, 8, sol.BF16,
+                                None) == sol.ERR_INVALID_ARGUMENT
+    bad = sol.ModSel(None, 1, -5)
+    assert L.sol_gated_residual(FAKE, 8, FAKE + 4096, 8, FAKE + 8192, 8, None, 0, bad, 2, 8, sol.BF16,
+                                None) == sol.ERR_INVALID_ARGUMENT
+
+
+def test_dtype_and_required_tensors(L):
+    assert L.sol_swiglu(FAKE, 8, FAKE + 4096, FAKE + 8192, 8, 2, 8, 7, None) == sol.ERR_UNSUPPORTED
+    assert L.sol_swiglu(FAKE, 8, None, FAKE + 8192, 8, 2, 8, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_gated_residual(FAKE, 8, FAKE + 4096, 8, None, 8, None, 0, SEL, 2, 8, sol.BF16, None) \
+        == sol.ERR_INVALID_ARGUMENT
+    # prologue with a residual needs x_out
+    assert L.sol_dit_prologue(None, FAKE, FAKE + 4096, FAKE + 8192, None, None, None, 8, 0, SEL, 2, 8,
+                              1e-6, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+
+
+def test_rope_create_validation(L):
+    h = ctypes.c_void_p()
+    assert L.sol_rope3d_create(ctypes.byref(h), 32, 47, 48, 1e4, 8, 8, 8) == sol.ERR_INVALID_ARGUMENT
+    assert h.value is None
+    assert L.sol_rope3d_create(ctypes.byref(h), 32, 48, 48, 1.0, 8, 8, 8) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_rope3d_create(ctypes.byref(h), 32, 48, 48, 1e4, 0, 8, 8) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_rope3d_create(None, 32, 48, 48, 1e4, 8, 8, 8) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_rope3d_destroy(None) == sol.OK
+
+
+def test_qk_validation_without_tables(L):
+    assert L.sol_qk_rmsnorm_rope3d(FAKE, FAKE, 256, 256, FAKE, FAKE, 256, 256, None, None, None, 2, 4, 4,
+                                   32, None, 32, 2, 128, 1e-6, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    assert "rope is NULL" in last(L)
+    assert L.sol_dit_epilogue(FAKE, 768, None, None, None, 2, 4, 4, 32, None, 32, 2, 128, 1e-6,
+                              sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+
+
+def test_binding_raises_with_reason():
+    with pytest.raises(sol.SolError) as e:
+        sol._check(sol.lib().sol_swiglu(None, 8, None, None, 8, 1, 8, sol.BF16, None), "sol_swiglu")
+    assert e.value.status == sol.ERR_INVALID_ARGUMENT
+    assert "NULL" in str(e.value)

@@ -417,3 +417,28 @@ def test_bad_split_rejected(oracle_mod):
     with pytest.raises(ValueError):
         oracle_mod.qk_rmsnorm_rope3d(np.zeros((1, 128)), None, n_heads=1, head_dim=128,
                                      pos=np.zeros((1, 3), np.int32), dims=(32, 48, 47))
+
+
+def test_row_subsets_equal_rows_of_the_full_sequence(oracle_mod):
+    """Evaluating a subset of rows with their global token indices gives exactly those
+    rows of the full evaluation (modulation row, stream id and implicit position all
+    follow the global index)."""
+    B, T, H, W, d, Hh, Dh = 2, 2, 3, 4, 64, 2, 128
+    tps = T * H * W
+    n = B * tps
+    x = RNG.standard_normal((n, d)); y = RNG.standard_normal((n, d))
+    S = 2
+    mods = [RNG.standard_normal((B * S, d)) for _ in range(3)]
+    sid = RNG.integers(0, S, size=n).astype(np.uint8)
+    qkv = RNG.standard_normal((n, 3 * Hh * Dh))
+    rows = np.array([0, 5, tps - 1, tps, tps + 7, n - 1])
+    kw = dict(stream_id=sid, n_streams=S, tokens_per_sample=tps)
+    full = oracle_mod.dit_prologue(x, y, *mods, **kw)
+    sub = oracle_mod.dit_prologue(np.ascontiguousarray(x[rows]), np.ascontiguousarray(y[rows]),
+                                  *mods, rows=rows, **kw)
+    np.testing.assert_array_equal(sub[0], full[0][rows])
+    np.testing.assert_array_equal(sub[1], full[1][rows])
+    ek = dict(n_heads=Hh, head_dim=Dh, grid=(T, H, W), tokens_per_sample=tps)
+    e_full = oracle_mod.dit_epilogue(qkv, **ek)
+    e_sub = oracle_mod.dit_epilogue(np.ascontiguousarray(qkv[rows]), rows=rows, **ek)
+    np.testing.assert_array_equal(e_sub, e_full[rows])
