@@ -92,14 +92,17 @@ sol::ModSel to_dev(const sol_modsel& sel)
     return sol::ModSel{sel.stream_id, sel.n_streams, sel.tokens_per_sample};
 }
 
-// Byte ranges [p, p + rows*ld*esz) overlap?  Used to reject forbidden aliasing.
-bool overlap(const void* a, int64_t lda, const void* b, int64_t ldb, int64_t rows, size_t esz)
+// Do the element ranges of two [rows, width] tensors (row strides lda / ldb) overlap?
+// A tensor spans from its first element to the end of its last row:
+// ((rows - 1) * ld + width) elements.  Used to reject forbidden aliasing.
+bool overlap(const void* a, int64_t lda, const void* b, int64_t ldb, int64_t rows, int64_t width,
+             size_t esz)
 {
     if (!a || !b || rows == 0) return false;
     const char* a0 = (const char*)a;
     const char* b0 = (const char*)b;
-    const char* a1 = a0 + (size_t)rows * (size_t)lda * esz;
-    const char* b1 = b0 + (size_t)rows * (size_t)ldb * esz;
+    const char* a1 = a0 + (size_t)((rows - 1) * lda + width) * esz;
+    const char* b1 = b0 + (size_t)((rows - 1) * ldb + width) * esz;
     return a0 < b1 && b0 < a1;
 }
 
@@ -204,7 +207,7 @@ sol_status sol_adaln_modulate(void* h, int64_t ld_h, const void* x, int64_t ld_x
     TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
     TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
     TRY(check_modsel(sel));
-    CHECK(h == x ? ld_h == ld_x : !overlap(h, ld_h, x, ld_x, n_tokens, esize(dt)),
+    CHECK(h == x ? ld_h == ld_x : !overlap(h, ld_h, x, ld_x, n_tokens, d, esize(dt)),
           SOL_ERR_INVALID_ARGUMENT, "h overlaps x without being the same tensor");
     if (n_tokens == 0) return SOL_OK;
     const sol::ModSel ms = to_dev(sel);
@@ -226,9 +229,9 @@ sol_status sol_gated_residual(void* out, int64_t ld_out, const void* x, int64_t 
     TRY(check_tensor("y", y, ld_y, d, dt, true));
     TRY(check_tensor("gate", gate, ld_mod, d, dt, false));
     TRY(check_modsel(sel));
-    CHECK(out == x ? ld_out == ld_x : !overlap(out, ld_out, x, ld_x, n_tokens, esize(dt)),
+    CHECK(out == x ? ld_out == ld_x : !overlap(out, ld_out, x, ld_x, n_tokens, d, esize(dt)),
           SOL_ERR_INVALID_ARGUMENT, "out overlaps x without being the same tensor");
-    CHECK(!overlap(out, ld_out, y, ld_y, n_tokens, esize(dt)), SOL_ERR_INVALID_ARGUMENT,
+    CHECK(!overlap(out, ld_out, y, ld_y, n_tokens, d, esize(dt)), SOL_ERR_INVALID_ARGUMENT,
           "out overlaps y");
     if (n_tokens == 0) return SOL_OK;
     const sol::ModSel ms = to_dev(sel);
@@ -246,8 +249,8 @@ sol_status sol_swiglu(void* out, int64_t ld_out, const void* a, const void* b, i
     TRY(check_tensor("a", a, ld_in, inner, dt, true));
     TRY(check_tensor("b", b, ld_in, inner, dt, true));
     // a and b may be two halves of one row: the row extent of each is ld_in wide
-    CHECK(!overlap(out, ld_out, a, ld_in, n_tokens, esize(dt)) &&
-              !overlap(out, ld_out, b, ld_in, n_tokens, esize(dt)),
+    CHECK(!overlap(out, ld_out, a, ld_in, n_tokens, inner, esize(dt)) &&
+              !overlap(out, ld_out, b, ld_in, n_tokens, inner, esize(dt)),
           SOL_ERR_INVALID_ARGUMENT, "out overlaps a or b");
     if (n_tokens == 0) return SOL_OK;
     return cuda_status(sol::launch_swiglu(dt, out, ld_out, a, b, ld_in, n_tokens, inner,
@@ -374,9 +377,9 @@ sol_status sol_qk_rmsnorm_rope3d(void* q_out, void* k_out, int64_t ld_qo, int64_
     TRY(check_tensor("q_out", q_out, ld_qo, hd, dt, true));
     TRY(check_tensor("k_out", k_out, ld_ko, hd, dt, true));
     const size_t es = esize(dt);
-    CHECK(q_out == q ? ld_qo == ld_q : !overlap(q_out, ld_qo, q, ld_q, n_tokens, es),
+    CHECK(q_out == q ? ld_qo == ld_q : !overlap(q_out, ld_qo, q, ld_q, n_tokens, hd, es),
           SOL_ERR_INVALID_ARGUMENT, "q_out overlaps q without being the same tensor");
-    CHECK(k_out == k ? ld_ko == ld_k : !overlap(k_out, ld_ko, k, ld_k, n_tokens, es),
+    CHECK(k_out == k ? ld_ko == ld_k : !overlap(k_out, ld_ko, k, ld_k, n_tokens, hd, es),
           SOL_ERR_INVALID_ARGUMENT, "k_out overlaps k without being the same tensor");
     if (n_tokens == 0) return SOL_OK;
     return cuda_status(sol::launch_qk_rmsnorm_rope3d(dt, q_out, k_out, ld_qo, ld_ko, q, k, ld_q, ld_k,
@@ -405,12 +408,12 @@ sol_status sol_dit_prologue(void* x_out, void* h, const void* x, const void* y,
     TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
     TRY(check_modsel(sel));
     const size_t es = esize(dt);
-    CHECK(!overlap(h, ld, x, ld, n_tokens, es) && !overlap(h, ld, y, ld, n_tokens, es) &&
-              !overlap(h, ld, x_out, ld, n_tokens, es),
+    CHECK(!overlap(h, ld, x, ld, n_tokens, d, es) && !overlap(h, ld, y, ld, n_tokens, d, es) &&
+              !overlap(h, ld, x_out, ld, n_tokens, d, es),
           SOL_ERR_INVALID_ARGUMENT, "h overlaps x, y or x_out");
-    CHECK(!y || x_out == x || !overlap(x_out, ld, x, ld, n_tokens, es), SOL_ERR_INVALID_ARGUMENT,
+    CHECK(!y || x_out == x || !overlap(x_out, ld, x, ld, n_tokens, d, es), SOL_ERR_INVALID_ARGUMENT,
           "x_out overlaps x without being the same tensor");
-    CHECK(!y || !overlap(x_out, ld, y, ld, n_tokens, es), SOL_ERR_INVALID_ARGUMENT, "x_out overlaps y");
+    CHECK(!y || !overlap(x_out, ld, y, ld, n_tokens, d, es), SOL_ERR_INVALID_ARGUMENT, "x_out overlaps y");
     if (n_tokens == 0) return SOL_OK;
     const sol::ModSel ms = to_dev(sel);
     return cuda_status(sol::launch_adaln_rows(dt, y ? x_out : nullptr, ld, h, ld, x, ld, y, ld, gate,

@@ -366,3 +366,19 @@ def test_block_step_full_workload(orc, name):
     bufs.close()
     del bufs
     torch.cuda.empty_cache()
+
+
+def test_adjacent_buffers_are_not_overlaps(orc):
+    """An output that starts right where the input's last row ends is legal."""
+    n, inner = 9, 64
+    buf = torch.empty(n * 2 * inner + n * inner, dtype=BF, device=DEV)
+    u = buf[:n * 2 * inner].view(n, 2 * inner)
+    u.copy_(randn((n, 2 * inner), BF, 3))
+    out = buf[n * 2 * inner:].view(n, inner)
+    sol.swiglu(out, u, inner=inner)
+    x = buf[:n * 2 * inner].view(n, 2 * inner)[:, :inner]  # strided rows, ld = 2*inner
+    o2 = torch.empty((n, inner), dtype=BF, device=DEV)
+    sol.gated_residual(o2, x, out, None)
+    torch.cuda.synchronize()
+    assert_close(to_f64(out), orc.swiglu(to_oracle(u), inner), BF, "adjacent swiglu")
+    assert torch.equal(o2, x)
