@@ -202,14 +202,14 @@ sol_status sol_adaln_modulate(void* h, int64_t ld_h, const void* x, int64_t ld_x
     CHECK(sol::adaln_row_fits(d / elems16(dt)), SOL_ERR_UNSUPPORTED,
           "d (%lld) is wider than one CTA row holds (max 4096 16-byte vectors)", (long long)d);
     CHECK(std::isfinite(eps) && eps >= 0.f, SOL_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
+    TRY(check_modsel(sel));
+    if (n_tokens == 0) return SOL_OK;  // nothing to do; empty tensors may be NULL
     TRY(check_tensor("h", h, ld_h, d, dt, true));
     TRY(check_tensor("x", x, ld_x, d, dt, true));
     TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
     TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
-    TRY(check_modsel(sel));
     CHECK(h == x ? ld_h == ld_x : !overlap(h, ld_h, x, ld_x, n_tokens, d, esize(dt)),
           SOL_ERR_INVALID_ARGUMENT, "h overlaps x without being the same tensor");
-    if (n_tokens == 0) return SOL_OK;
     const sol::ModSel ms = to_dev(sel);
     return cuda_status(sol::launch_adaln_rows(dt, nullptr, 0, h, ld_h, x, ld_x, nullptr, 0, nullptr,
                                               shift, scale, ld_mod, ms, n_tokens, d, eps,
@@ -224,16 +224,16 @@ sol_status sol_gated_residual(void* out, int64_t ld_out, const void* x, int64_t 
 {
     TRY(check_dtype(dt));
     TRY(check_rows(n_tokens, d, dt, "d"));
+    TRY(check_modsel(sel));
+    if (n_tokens == 0) return SOL_OK;  // nothing to do; empty tensors may be NULL
     TRY(check_tensor("out", out, ld_out, d, dt, true));
     TRY(check_tensor("x", x, ld_x, d, dt, true));
     TRY(check_tensor("y", y, ld_y, d, dt, true));
     TRY(check_tensor("gate", gate, ld_mod, d, dt, false));
-    TRY(check_modsel(sel));
     CHECK(out == x ? ld_out == ld_x : !overlap(out, ld_out, x, ld_x, n_tokens, d, esize(dt)),
           SOL_ERR_INVALID_ARGUMENT, "out overlaps x without being the same tensor");
     CHECK(!overlap(out, ld_out, y, ld_y, n_tokens, d, esize(dt)), SOL_ERR_INVALID_ARGUMENT,
           "out overlaps y");
-    if (n_tokens == 0) return SOL_OK;
     const sol::ModSel ms = to_dev(sel);
     return cuda_status(sol::launch_gated_residual(dt, out, ld_out, x, ld_x, y, ld_y, gate, ld_mod,
                                                   ms, n_tokens, d, (cudaStream_t)stream),
@@ -245,6 +245,7 @@ sol_status sol_swiglu(void* out, int64_t ld_out, const void* a, const void* b, i
 {
     TRY(check_dtype(dt));
     TRY(check_rows(n_tokens, inner, dt, "inner"));
+    if (n_tokens == 0) return SOL_OK;  // nothing to do; empty tensors may be NULL
     TRY(check_tensor("out", out, ld_out, inner, dt, true));
     TRY(check_tensor("a", a, ld_in, inner, dt, true));
     TRY(check_tensor("b", b, ld_in, inner, dt, true));
@@ -252,7 +253,6 @@ sol_status sol_swiglu(void* out, int64_t ld_out, const void* a, const void* b, i
     CHECK(!overlap(out, ld_out, a, ld_in, n_tokens, inner, esize(dt)) &&
               !overlap(out, ld_out, b, ld_in, n_tokens, inner, esize(dt)),
           SOL_ERR_INVALID_ARGUMENT, "out overlaps a or b");
-    if (n_tokens == 0) return SOL_OK;
     return cuda_status(sol::launch_swiglu(dt, out, ld_out, a, b, ld_in, n_tokens, inner,
                                           (cudaStream_t)stream),
                        "sol_swiglu launch");
@@ -371,6 +371,7 @@ sol_status sol_qk_rmsnorm_rope3d(void* q_out, void* k_out, int64_t ld_qo, int64_
 {
     TRY(check_qk_common(rope, pos, grid_T, grid_H, grid_W, tokens_per_sample, n_tokens, n_heads,
                         head_dim, eps, dt, wq, wk));
+    if (n_tokens == 0) return SOL_OK;  // nothing to do; empty tensors may be NULL
     const int64_t hd = (int64_t)n_heads * head_dim;
     TRY(check_tensor("q", q, ld_q, hd, dt, true));
     TRY(check_tensor("k", k, ld_k, hd, dt, true));
@@ -381,7 +382,6 @@ sol_status sol_qk_rmsnorm_rope3d(void* q_out, void* k_out, int64_t ld_qo, int64_
           SOL_ERR_INVALID_ARGUMENT, "q_out overlaps q without being the same tensor");
     CHECK(k_out == k ? ld_ko == ld_k : !overlap(k_out, ld_ko, k, ld_k, n_tokens, hd, es),
           SOL_ERR_INVALID_ARGUMENT, "k_out overlaps k without being the same tensor");
-    if (n_tokens == 0) return SOL_OK;
     return cuda_status(sol::launch_qk_rmsnorm_rope3d(dt, q_out, k_out, ld_qo, ld_ko, q, k, ld_q, ld_k,
                                                      wq, wk, pos, grid_T, grid_H, grid_W,
                                                      tokens_per_sample, rope->view, n_tokens,
@@ -399,6 +399,8 @@ sol_status sol_dit_prologue(void* x_out, void* h, const void* x, const void* y,
     CHECK(sol::adaln_row_fits(d / elems16(dt)), SOL_ERR_UNSUPPORTED,
           "d (%lld) is wider than one CTA row holds (max 4096 16-byte vectors)", (long long)d);
     CHECK(std::isfinite(eps) && eps >= 0.f, SOL_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
+    TRY(check_modsel(sel));
+    if (n_tokens == 0) return SOL_OK;  // nothing to do; empty tensors may be NULL
     TRY(check_tensor("h", h, ld, d, dt, true));
     TRY(check_tensor("x", x, ld, d, dt, true));
     TRY(check_tensor("y", y, ld, d, dt, false));
@@ -406,7 +408,6 @@ sol_status sol_dit_prologue(void* x_out, void* h, const void* x, const void* y,
     TRY(check_tensor("gate", gate, ld_mod, d, dt, false));
     TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
     TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
-    TRY(check_modsel(sel));
     const size_t es = esize(dt);
     CHECK(!overlap(h, ld, x, ld, n_tokens, d, es) && !overlap(h, ld, y, ld, n_tokens, d, es) &&
               !overlap(h, ld, x_out, ld, n_tokens, d, es),
@@ -414,7 +415,6 @@ sol_status sol_dit_prologue(void* x_out, void* h, const void* x, const void* y,
     CHECK(!y || x_out == x || !overlap(x_out, ld, x, ld, n_tokens, d, es), SOL_ERR_INVALID_ARGUMENT,
           "x_out overlaps x without being the same tensor");
     CHECK(!y || !overlap(x_out, ld, y, ld, n_tokens, d, es), SOL_ERR_INVALID_ARGUMENT, "x_out overlaps y");
-    if (n_tokens == 0) return SOL_OK;
     const sol::ModSel ms = to_dev(sel);
     return cuda_status(sol::launch_adaln_rows(dt, y ? x_out : nullptr, ld, h, ld, x, ld, y, ld, gate,
                                               shift, scale, ld_mod, ms, n_tokens, d, eps,
@@ -430,9 +430,9 @@ sol_status sol_dit_epilogue(void* qkv, int64_t ld_qkv, const void* wq, const voi
 {
     TRY(check_qk_common(rope, pos, grid_T, grid_H, grid_W, tokens_per_sample, n_tokens, n_heads,
                         head_dim, eps, dt, wq, wk));
+    if (n_tokens == 0) return SOL_OK;  // nothing to do; an empty tensor may be NULL
     const int64_t hd = (int64_t)n_heads * head_dim;
     TRY(check_tensor("qkv", qkv, ld_qkv, 2 * hd, dt, true));
-    if (n_tokens == 0) return SOL_OK;
     void* k = (char*)qkv + (size_t)hd * esize(dt);
     return cuda_status(sol::launch_qk_rmsnorm_rope3d(dt, qkv, k, ld_qkv, ld_qkv, qkv, k, ld_qkv,
                                                      ld_qkv, wq, wk, pos, grid_T, grid_H, grid_W,

@@ -34,7 +34,7 @@
  *              failure the call returns a SOL_ERR_* code with no side effect, and
  *              sol_last_error() gives a one-line reason (per host thread).
  *              SOL_ERR_CUDA reports a launch failure.
- *   n_tokens == 0 is valid and launches nothing.
+ *   n_tokens == 0 is valid and launches nothing; tensor pointers may then be NULL.
  *   Aliasing.  Only the aliases each function lists are allowed (every row is read
  *              completely before it is written).  Any other overlap is undefined.
  */
