@@ -47,6 +47,9 @@ cudaError_t launch_qk_rmsnorm_rope3d(sol_dtype dt, void* q_out, void* k_out, int
                                      const RopeDev& rope, int64_t n_tokens, int32_t n_heads,
                                      int32_t head_dim, float eps, cudaStream_t s);
 
+// Store a one-line reason for sol_last_error() on this host thread.
+void record_error(const char* msg);
+
 // Whether a row of `vpr` 16-byte vectors fits the register-resident AdaLN kernel.
 bool adaln_row_fits(int64_t vpr);
 

@@ -157,6 +157,8 @@ int ctas_per_sm(const void* kernel, int block, size_t smem)
     return n;
 }
 
+void record_error(const char* msg) { g_last_error = msg; }
+
 int sm_count()
 {
     int dev = 0;

@@ -52,6 +52,9 @@ SIGNATURES = {
     "sol_dit_prologue": ([_P, _P, _P, _P, _P, _P, _P, _I64, _I64, ModSel, _I64, _I64, _F, _E, _P], _E),
     "sol_dit_epilogue": ([_P, _I64, _P, _P, _P, _I32, _I32, _I32, _I64, _P, _I64, _I32, _I32, _F,
                           _E, _P], _E),
+    "sol_qk_rmsnorm_rope3d_noalloc": ([_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _P, _P, _I32, _I32,
+                                       _I32, _I64, _I32, _I32, _I32, _D, _I32, _I32, _I32, _I64,
+                                       _I32, _I32, _F, _E, _P], _E),
 }
 
 _lib = None
@@ -243,3 +246,23 @@ def dit_epilogue(qkv, rope: Rope3D, *, n_heads, head_dim, wq=None, wk=None, pos=
                                   int(grid[1]), int(grid[2]), int(tokens_per_sample), rope.handle,
                                   qkv.shape[0], int(n_heads), int(head_dim), eps, _dtype(qkv),
                                   _stream(stream)), "sol_dit_epilogue")
+
+
+NOALLOC_MAX_ROPE_ENTRIES = 65536
+
+
+def qk_rmsnorm_rope3d_noalloc(q_out, k_out, q, k, *, n_heads, head_dim, dims=(32, 48, 48),
+                              theta=10000.0, max_pos, wq=None, wk=None, pos=None, grid=(0, 0, 0),
+                              tokens_per_sample=0, eps=1e-6, stream=None):
+    """sol_qk_rmsnorm_rope3d without a sol_rope3d handle: for callers that cannot allocate
+    device memory.  The cos/sin table for (dims, theta, max_pos) is rebuilt by every call
+    in a fixed library array (at most NOALLOC_MAX_ROPE_ENTRIES pairs); calls that overlap
+    on the GPU race on it."""
+    if pos is not None and (pos.dtype != torch.int32 or not pos.is_contiguous()):
+        raise TypeError("pos must be a contiguous int32 [N, 3] tensor")
+    _check(lib().sol_qk_rmsnorm_rope3d_noalloc(
+        _ptr(q_out), _ptr(k_out), _ld(q_out), _ld(k_out), _ptr(q), _ptr(k), _ld(q), _ld(k),
+        _ptr(wq), _ptr(wk), _ptr(pos), int(grid[0]), int(grid[1]), int(grid[2]),
+        int(tokens_per_sample), int(dims[0]), int(dims[1]), int(dims[2]), float(theta),
+        int(max_pos[0]), int(max_pos[1]), int(max_pos[2]), q.shape[0], int(n_heads),
+        int(head_dim), eps, _dtype(q), _stream(stream)), "sol_qk_rmsnorm_rope3d_noalloc")

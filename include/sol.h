@@ -181,6 +181,35 @@ sol_status sol_dit_epilogue(void* qkv, int64_t ld_qkv, const void* wq, const voi
                             int32_t n_heads, int32_t head_dim, float eps, sol_dtype dt,
                             sol_stream_t stream);
 
+/* QK RMSNorm + 3D RoPE for callers that cannot allocate device memory.  The pages have
+ * no counterpart: this entry point exists for hosts that reserve device memory up front
+ * and forbid allocation while they run work (inference engines whose pool already holds
+ * nearly all of HBM, plugin execute callbacks, latency-critical loops that cannot afford
+ * cudaMalloc's device synchronisation).  sol_qk_rmsnorm_rope3d needs a sol_rope3d handle,
+ * and creating one calls cudaMalloc; this function allocates nothing.
+ *
+ * It computes exactly what sol_qk_rmsnorm_rope3d computes, with the table described by
+ * (dim_t, dim_h, dim_w, theta, max_t, max_h, max_w) as in sol_rope3d_create.  The table
+ * is rebuilt on `stream` by every call inside a fixed device array of
+ * SOL_NOALLOC_MAX_ROPE_ENTRIES (cos, sin) pairs (512 KiB, held by every GPU that loads
+ * the library until the process exits); a table needing more entries,
+ * max_t*dim_t/2 + max_h*dim_h/2 + max_w*dim_w/2, is rejected with SOL_ERR_UNSUPPORTED.
+ * All calls share that array: calls whose kernels overlap on the GPU (other streams,
+ * unordered host threads) race on it and must be serialised by the caller.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * current device); make that first call before any stream capture.
+ * Other arguments, layouts, aliasing and errors as in sol_qk_rmsnorm_rope3d. */
+#define SOL_NOALLOC_MAX_ROPE_ENTRIES 65536
+sol_status sol_qk_rmsnorm_rope3d_noalloc(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko,
+                                         const void* q, const void* k, int64_t ld_q, int64_t ld_k,
+                                         const void* wq, const void* wk, const int32_t* pos,
+                                         int32_t grid_T, int32_t grid_H, int32_t grid_W,
+                                         int64_t tokens_per_sample, int32_t dim_t, int32_t dim_h,
+                                         int32_t dim_w, double theta, int32_t max_t,
+                                         int32_t max_h, int32_t max_w, int64_t n_tokens,
+                                         int32_t n_heads, int32_t head_dim, float eps,
+                                         sol_dtype dt, sol_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
