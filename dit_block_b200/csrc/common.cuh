@@ -58,16 +58,73 @@ template <> __device__ __forceinline__ uint4 pack<bf16>(const float* f)
                       pack2_bf16(f[6], f[7]));
 }
 
+// Widen / narrow one 16-byte vector as fp32 pairs, for the packed f32x2 arithmetic of
+// sm_100 (__fadd2_rn, __fmul2_rn, __ffma2_rn: two IEEE fp32 operations per instruction).
+template <typename T> __device__ __forceinline__ void unpack2(const uint4& r, float2* f);
+template <> __device__ __forceinline__ void unpack2<float>(const uint4& r, float2* f)
+{
+    f[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
+    f[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
+}
+template <> __device__ __forceinline__ void unpack2<bf16>(const uint4& r, float2* f)
+{
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+}
+template <typename T> __device__ __forceinline__ uint4 pack2(const float2* f);
+template <> __device__ __forceinline__ uint4 pack2<float>(const float2* f)
+{
+    return make_uint4(__float_as_uint(f[0].x), __float_as_uint(f[0].y), __float_as_uint(f[1].x),
+                      __float_as_uint(f[1].y));
+}
+template <> __device__ __forceinline__ uint4 pack2<bf16>(const float2* f)
+{
+    return make_uint4(pack2_bf16(f[0].x, f[0].y), pack2_bf16(f[1].x, f[1].y), pack2_bf16(f[2].x, f[2].y),
+                      pack2_bf16(f[3].x, f[3].y));
+}
+
 // Modulation-row selection for packed multi-sample, multi-stream sequences.
+// The sample index n / tokens_per_sample uses a precomputed multiply-and-shift
+// (division by an invariant integer, Granlund and Montgomery 1994) when every token
+// index is below 2^31: q = (umulhi(n, m) + n) >> s with s = ceil(log2 d) and
+// m = floor(2^32 * (2^s - d) / d) + 1; otherwise a plain 64-bit division.
 struct ModSel {
     const uint8_t* stream_id;   // [n_tokens] or nullptr
     int32_t n_streams;          // >= 1
     int64_t tokens_per_sample;  // > 0, or 0 = one sample
+    uint32_t div_m;             // multiplier for the 32-bit fast path
+    uint32_t div_s;             // shift for the 32-bit fast path
+    int32_t div_fast;           // 1: use the fast path
 };
+
+// Host side: fill the fast-division fields for `n_tokens` tokens.
+inline void modsel_prepare(ModSel& m, int64_t n_tokens)
+{
+    m.div_fast = 0;
+    m.div_m = 0;
+    m.div_s = 0;
+    const int64_t d = m.tokens_per_sample;
+    if (d <= 0 || d >= (int64_t)1 << 31 || n_tokens >= (int64_t)1 << 31) return;
+    uint32_t s = 0;
+    while (((uint64_t)1 << s) < (uint64_t)d) ++s;
+    const uint64_t two32 = (uint64_t)1 << 32;
+    m.div_m = (uint32_t)((two32 * (((uint64_t)1 << s) - (uint64_t)d)) / (uint64_t)d + 1);
+    m.div_s = s;
+    m.div_fast = 1;
+}
 
 __device__ __forceinline__ int64_t mod_row(int64_t n, const ModSel& m)
 {
-    const int64_t sample = m.tokens_per_sample > 0 ? n / m.tokens_per_sample : 0;
+    int64_t sample = 0;
+    if (m.tokens_per_sample > 0) {
+        if (m.div_fast) {
+            const uint32_t nn = (uint32_t)n;
+            sample = (int64_t)((__umulhi(nn, m.div_m) + nn) >> m.div_s);
+        } else {
+            sample = n / m.tokens_per_sample;
+        }
+    }
     int32_t s = 0;
     if (m.stream_id) {
         s = m.stream_id[n];
@@ -96,6 +153,74 @@ __device__ __forceinline__ float block_sum(float v, float* buf)
     float t = 0.f;
     for (int i = 0; i < nw; ++i) t += buf[i];
     return t;
+}
+
+}  // namespace sol
+
+// ---------------------------------------------------------------------------------
+// Bulk asynchronous copies (global -> shared, no multicast) completed on an mbarrier.
+namespace sol {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Make initialised mbarriers visible to the async proxy before the first bulk copy.
+__device__ __forceinline__ void mbar_fence_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+// One non-multicast bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned)
+// from global memory into this CTA's shared memory, counted on mbarrier `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before its later
+// async-proxy ones (a bulk copy refilling a buffer other threads just read).
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// One poll of phase `parity`; a thread whose phase is not complete may be suspended for
+// up to ~1 ms (the hint, in ns) instead of spinning, so waiting warps leave the issue
+// slots to the warps that have work.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(1000000u)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete, giving up after `limit` polls (each poll
+// suspends for at most about a millisecond).  Returns false on give-up.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t limit)
+{
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
 }
 
 }  // namespace sol

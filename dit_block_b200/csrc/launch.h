@@ -47,6 +47,10 @@ cudaError_t launch_qk_rmsnorm_rope3d(sol_dtype dt, void* q_out, void* k_out, int
                                      const RopeDev& rope, int64_t n_tokens, int32_t n_heads,
                                      int32_t head_dim, float eps, cudaStream_t s);
 
+// Error flags raised on the device by the AdaLN / prologue kernels (bit 0: a bounded
+// wait on a bulk copy gave up); optionally cleared.  Synchronous.
+uint32_t rows_device_error(bool clear);
+
 // Store a one-line reason for sol_last_error() on this host thread.
 void record_error(const char* msg);
 

@@ -87,9 +87,11 @@ sol_status check_modsel(const sol_modsel& sel)
     return SOL_OK;
 }
 
-sol::ModSel to_dev(const sol_modsel& sel)
+sol::ModSel to_dev(const sol_modsel& sel, int64_t n_tokens)
 {
-    return sol::ModSel{sel.stream_id, sel.n_streams, sel.tokens_per_sample};
+    sol::ModSel m{sel.stream_id, sel.n_streams, sel.tokens_per_sample, 0u, 0u, 0};
+    sol::modsel_prepare(m, n_tokens);
+    return m;
 }
 
 // Do the element ranges of two [rows, width] tensors (row strides lda / ldb) overlap?
@@ -194,6 +196,16 @@ const char* sol_last_error(void) { return g_last_error.c_str(); }
 
 int32_t sol_abi_version(void) { return 1; }
 
+sol_status sol_device_errors(uint32_t* flags, int32_t clear)
+{
+    CHECK(flags, SOL_ERR_INVALID_ARGUMENT, "flags is NULL");
+    const cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e, "sol_device_errors");
+    *flags = sol::rows_device_error(clear != 0);
+    CHECK(*flags != 0xffffffffu, SOL_ERR_CUDA, "reading the device error flags failed");
+    return SOL_OK;
+}
+
 sol_status sol_adaln_modulate(void* h, int64_t ld_h, const void* x, int64_t ld_x,
                               const void* shift, const void* scale, int64_t ld_mod,
                               sol_modsel sel, int64_t n_tokens, int64_t d, float eps,
@@ -212,7 +224,7 @@ sol_status sol_adaln_modulate(void* h, int64_t ld_h, const void* x, int64_t ld_x
     TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
     CHECK(h == x ? ld_h == ld_x : !overlap(h, ld_h, x, ld_x, n_tokens, d, esize(dt)),
           SOL_ERR_INVALID_ARGUMENT, "h overlaps x without being the same tensor");
-    const sol::ModSel ms = to_dev(sel);
+    const sol::ModSel ms = to_dev(sel, n_tokens);
     return cuda_status(sol::launch_adaln_rows(dt, nullptr, 0, h, ld_h, x, ld_x, nullptr, 0, nullptr,
                                               shift, scale, ld_mod, ms, n_tokens, d, eps,
                                               (cudaStream_t)stream),
@@ -236,7 +248,7 @@ sol_status sol_gated_residual(void* out, int64_t ld_out, const void* x, int64_t 
           SOL_ERR_INVALID_ARGUMENT, "out overlaps x without being the same tensor");
     CHECK(!overlap(out, ld_out, y, ld_y, n_tokens, d, esize(dt)), SOL_ERR_INVALID_ARGUMENT,
           "out overlaps y");
-    const sol::ModSel ms = to_dev(sel);
+    const sol::ModSel ms = to_dev(sel, n_tokens);
     return cuda_status(sol::launch_gated_residual(dt, out, ld_out, x, ld_x, y, ld_y, gate, ld_mod,
                                                   ms, n_tokens, d, (cudaStream_t)stream),
                        "sol_gated_residual launch");
@@ -417,7 +429,7 @@ sol_status sol_dit_prologue(void* x_out, void* h, const void* x, const void* y,
     CHECK(!y || x_out == x || !overlap(x_out, ld, x, ld, n_tokens, d, es), SOL_ERR_INVALID_ARGUMENT,
           "x_out overlaps x without being the same tensor");
     CHECK(!y || !overlap(x_out, ld, y, ld, n_tokens, d, es), SOL_ERR_INVALID_ARGUMENT, "x_out overlaps y");
-    const sol::ModSel ms = to_dev(sel);
+    const sol::ModSel ms = to_dev(sel, n_tokens);
     return cuda_status(sol::launch_adaln_rows(dt, y ? x_out : nullptr, ld, h, ld, x, ld, y, ld, gate,
                                               shift, scale, ld_mod, ms, n_tokens, d, eps,
                                               (cudaStream_t)stream),

@@ -42,6 +42,7 @@ SIGNATURES = {
     "sol_status_string": ([_E], ctypes.c_char_p),
     "sol_last_error": ([], ctypes.c_char_p),
     "sol_abi_version": ([], _I32),
+    "sol_device_errors": ([ctypes.POINTER(ctypes.c_uint32), _I32], _E),
     "sol_adaln_modulate": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _I64, _I64, _F, _E, _P], _E),
     "sol_gated_residual": ([_P, _I64, _P, _I64, _P, _I64, _P, _I64, ModSel, _I64, _I64, _E, _P], _E),
     "sol_swiglu": ([_P, _I64, _P, _P, _I64, _I64, _I64, _E, _P], _E),
@@ -95,6 +96,13 @@ def status_string(status: int) -> str:
 
 def abi_version() -> int:
     return int(lib().sol_abi_version())
+
+
+def device_errors(clear: bool = False) -> int:
+    """Error flags libsol kernels raised on the current device (0 in normal operation)."""
+    f = ctypes.c_uint32(0)
+    _check(lib().sol_device_errors(ctypes.byref(f), int(clear)), "sol_device_errors")
+    return int(f.value)
 
 
 # ------------------------------------------------------------------------- marshalling

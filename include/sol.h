@@ -85,6 +85,12 @@ const char* sol_last_error(void);
 /* Version of this ABI (incremented on any incompatible change). */
 int32_t sol_abi_version(void);
 
+/* Error flags raised on the current device by libsol kernels since the last clear:
+ * bit 0 = a kernel's bounded wait on its own asynchronous copy gave up (the kernel
+ * recorded it, stopped early and left its outputs incomplete).  Synchronises the current
+ * device first; clear != 0 resets the flags.  Never set in normal operation. */
+sol_status sol_device_errors(uint32_t* flags, int32_t clear);
+
 /* AdaLN modulation [XHH-QA, STM-GAN]:
  *     mu = mean_i x_i,  var = mean_i (x_i - mu)^2  (biased, two passes),
  *     h_i = (x_i - mu) / sqrt(var + eps) * (1 + scale[r]_i) + shift[r]_i
