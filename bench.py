@@ -13,9 +13,10 @@ over ranks.  Rank 0 prints one JSON line.
 
 value       algorithmic HBM bytes of all ranks' steps / device time (GB/s); every tensor
             element an op must read or write counts once (216,064 B per token per step).
-e2e         the same metric through the public API with host buffers: per step, pinned
-            host -> device copies of every input, the five launches, device -> host
-            copies of every output, all inside the timed region.
+e2e         the same metric through the public host-buffer API (HostBlockPipeline): per
+            step, pinned host -> device copies of every input, the five launches,
+            device -> host copies of every output, all inside the timed region, chunked
+            and overlapped across three streams.
 roofline    the SwiGLU launch (the largest byte mover): achieved GB/s from CUDA events
             around each launch in the timed steps, against the measured HBM copy peak.
 cpu_baseline / --impl reference
@@ -361,43 +362,33 @@ def run_ours(args, w):
 
 
 def run_e2e(args, bufs, dev, world, step_bytes):
-    """Pinned host buffers in, five launches, host buffers out; copies inside the timing."""
-    i = bufs.inp
-    in_names = [k for k in ("x", "qkv", "y_attn", "u", "y_mlp", "shift_msa", "scale_msa", "gate_msa",
-                            "shift_mlp", "scale_mlp", "gate_mlp", "wq", "wk", "pos", "stream_id")
-                if i.get(k) is not None]
-    outs = {"h1": bufs.h1, "qkv": i["qkv"], "x1": bufs.x1, "h2": bufs.h2, "act": bufs.act, "x2": bufs.x2}
-    need = sum(i[k].numel() * i[k].element_size() for k in in_names) + \
-        sum(t.numel() * t.element_size() for t in outs.values())
+    """The pass through the public host-buffer API (dit_block_b200.pipeline): pinned host
+    inputs in, five launches per chunk, pinned host outputs back; every copy is inside
+    the timed region and overlapped with compute across three streams."""
+    from dit_block_b200 import pipeline
+    w, i = bufs.w, bufs.inp
+    n = bufs.n_tokens
+    pipe = pipeline.HostBlockPipeline(w, dev, chunk_tokens=args.e2e_chunk)
+    h2d, d2h = pipe.bytes_per_pass(n)
     try:
         import psutil
         avail = psutil.virtual_memory().available
     except Exception:
         avail = 0
-    if need > 0.4 * avail:
+    if h2d + d2h > 0.4 * avail:
+        pipe.close()
         return {"value": None, "unit": "GB/s",
-                "error": f"skipped: {need / 1e9:.1f} GB of pinned host buffers > 40% of the "
+                "error": f"skipped: {(h2d + d2h) / 1e9:.1f} GB of pinned host buffers > 40% of the "
                          f"{avail / 1e9:.1f} GB available host memory"}
-    try:
-        host_in = {k: torch.empty(i[k].shape, dtype=i[k].dtype, pin_memory=True) for k in in_names}
-        host_out = {k: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for k, t in outs.items()}
-    except RuntimeError as e:
-        return {"value": None, "unit": "GB/s", "error": f"pinned host allocation failed: {e}"[:200]}
-    for k in in_names:
+    host_in, host_out, host_mod = pipeline.host_buffers(w, n)
+    for k in pipeline.IN_NAMES:
         host_in[k].copy_(i[k])
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    for k in pipeline.MOD_NAMES:
+        host_mod[k].copy_(i[k])
+    pipe.set_weights(i["wq"], i["wk"])
     stream = torch.cuda.current_stream(dev)
-
-    def one():
-        for k in in_names:
-            i[k].copy_(host_in[k], non_blocking=True)
-        bufs.step()
-        for k, t in outs.items():
-            host_out[k].copy_(t, non_blocking=True)
-
     for _ in range(args.e2e_warmup):
-        one()
+        pipe.run(host_in, host_out, host_mod)
     torch.cuda.synchronize(dev)
     if world > 1:
         import torch.distributed as dist
@@ -405,15 +396,18 @@ def run_e2e(args, bufs, dev, world, step_bytes):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for _ in range(args.e2e_steps):
-        one()
+        pipe.run(host_in, host_out, host_mod)
     end.record(stream)
     torch.cuda.synchronize(dev)
     ms = start.elapsed_time(end)
     ms, = max_over_ranks([ms], world, dev)
     val = step_bytes * world * args.e2e_steps / (ms * 1e-3) / 1e9
-    del host_in, host_out
+    pipe.close()
+    del host_in, host_out, host_mod
     return {"value": round(val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": args.e2e_steps, "ms_per_step": round(ms / args.e2e_steps, 2)}
+            "steps": args.e2e_steps, "ms_per_step": round(ms / args.e2e_steps, 2),
+            "api": "dit_block_b200.pipeline.HostBlockPipeline.run (pinned host buffers)",
+            "chunk_tokens": args.e2e_chunk}
 
 
 def main(argv=None):
@@ -427,6 +421,7 @@ def main(argv=None):
                    help="run only the first N tokens of the workload (small profiling cases)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--e2e-warmup", type=int, default=1)
+    p.add_argument("--e2e-chunk", type=int, default=8192, help="tokens per pipelined chunk")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)

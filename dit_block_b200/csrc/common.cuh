@@ -16,11 +16,22 @@ template <typename T> struct Vec;
 template <> struct Vec<float> { static constexpr int N = 4; };
 template <> struct Vec<bf16> { static constexpr int N = 8; };
 
-// Streaming load / store of data touched once (evict-first in L1 and L2) and a
-// read-only cached load for small tensors every CTA re-reads (modulation rows, weights).
+// 16-byte loads and stores of data touched once:
+//   ld_stream     ld.global.cs (evict first) -- for inputs the same kernel may overwrite
+//                 in place (each element is read once, before its owner writes it);
+//   ld_stream_ro  ld.global.nc (read-only path) -- for inputs nothing in the kernel writes;
+//   st_stream     st.global.L1::no_allocate -- outputs are never re-read by the kernel.
+// ld_cached: read-only cached load for small tensors every CTA re-reads (modulation
+// rows, weights).  The forms were chosen by timing each op on B200.
 __device__ __forceinline__ uint4 ld_stream(const void* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
+__device__ __forceinline__ uint4 ld_stream_ro(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 __device__ __forceinline__ uint4 ld_cached(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
-__device__ __forceinline__ void st_stream(void* p, const uint4& v) { __stcs(reinterpret_cast<uint4*>(p), v); }
+__device__ __forceinline__ void st_stream(void* p, const uint4& v)
+{
+    asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
 
 // Widen one 16-byte vector to fp32.  bf16 -> fp32 is exact: the bf16 bits are the high
 // half of the binary32 with the same value.

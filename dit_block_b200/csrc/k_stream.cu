@@ -5,16 +5,22 @@
 //   * a CTA owns one fixed column chunk (blockDim.x * U vectors) of a row and walks rows
 //     with a grid stride; the grid is (resident CTAs per SM * SMs) rounded to a multiple
 //     of the chunks per row, so a CTA never changes columns;
-//   * each thread issues all U x inputs loads before the first use (U * 32 or 48 bytes
-//     in flight per thread); inputs use evict-first loads, outputs evict-first stores;
+//   * each thread issues all U x inputs loads before the first use (U * 32 bytes in
+//     flight per thread); inputs nothing in the kernel writes come through the
+//     read-only path, outputs are stored without L1 allocation;
 //   * the gate row is re-read through the read-only path and stays L1/L2 resident.
 #include "common.cuh"
 #include "launch.h"
 
+#ifndef SOL_STREAM_UPREF_FIRST
+#define SOL_STREAM_UPREF_FIRST 4  // first choice of 16-byte vectors per thread and input
+#endif
+
 namespace sol {
 
-// Gated residual [XHH-QA "门控残差"]: out = x + gate[r] * y, fp32 inside.
-template <typename T, int U>
+// Gated residual [XHH-QA "门控残差"]: out = x + gate[r] * y, fp32 inside.  RO: out does
+// not alias x, so x may come through the read-only path (y never aliases out).
+template <typename T, int U, bool RO>
 __global__ void __launch_bounds__(512)
 k_gated_residual(T* __restrict__ out, int64_t ld_out, const T* x, int64_t ld_x,
                  const T* __restrict__ y, int64_t ld_y, const T* __restrict__ gate,
@@ -31,8 +37,9 @@ k_gated_residual(T* __restrict__ out, int64_t ld_out, const T* x, int64_t ld_x,
         for (int k = 0; k < U; ++k) {
             const int col = col0 + k * blockDim.x;
             if (col < vpr) {
-                xv[k] = ld_stream(x + row * ld_x + (int64_t)col * E);
-                yv[k] = ld_stream(y + row * ld_y + (int64_t)col * E);
+                xv[k] = RO ? ld_stream_ro(x + row * ld_x + (int64_t)col * E)
+                           : ld_stream(x + row * ld_x + (int64_t)col * E);
+                yv[k] = ld_stream_ro(y + row * ld_y + (int64_t)col * E);
             }
         }
 #pragma unroll
@@ -54,6 +61,22 @@ k_gated_residual(T* __restrict__ out, int64_t ld_out, const T* x, int64_t ld_x,
             }
         }
     }
+}
+
+// The two MUFU operations of the bf16 SwiGLU: 2^x and 1/x, approximate (relative
+// error ~2^-22), flushing subnormal results to zero.  1/inf = 0, so a very negative
+// pre-activation gives silu = -0 as its limit.
+__device__ __forceinline__ float exp2f_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // silu(a) * b.  bf16 outputs: ex2.approx-based exponential and approximate division
@@ -85,20 +108,38 @@ k_swiglu(T* __restrict__ out, int64_t ld_out, const T* __restrict__ a, const T* 
         for (int k = 0; k < U; ++k) {
             const int col = col0 + k * blockDim.x;
             if (col < vpr) {
-                av[k] = ld_stream(a + row * ld_in + (int64_t)col * E);
-                bv[k] = ld_stream(b + row * ld_in + (int64_t)col * E);
+                av[k] = ld_stream_ro(a + row * ld_in + (int64_t)col * E);
+                bv[k] = ld_stream_ro(b + row * ld_in + (int64_t)col * E);
             }
         }
 #pragma unroll
         for (int k = 0; k < U; ++k) {
             const int col = col0 + k * blockDim.x;
             if (col < vpr) {
-                float fa[E], fb[E];
-                unpack<T>(av[k], fa);
-                unpack<T>(bv[k], fb);
+                if constexpr (sizeof(T) == 2) {
+                    // a * b / (1 + 2^(-a*log2 e)): products and the sum in packed f32x2,
+                    // exp2 and the reciprocal on the MUFU pipe
+                    float2 fa[E / 2], fb[E / 2];
+                    unpack2<T>(av[k], fa);
+                    unpack2<T>(bv[k], fb);
+                    const float2 nl2e = make_float2(-1.4426950408889634f, -1.4426950408889634f);
 #pragma unroll
-                for (int e = 0; e < E; ++e) fa[e] = silu_mul<T>(fa[e], fb[e]);
-                st_stream(out + row * ld_out + (int64_t)col * E, pack<T>(fa));
+                    for (int i = 0; i < E / 2; ++i) {
+                        const float2 t = __fmul2_rn(fa[i], nl2e);
+                        const float2 den = __fadd2_rn(make_float2(exp2f_approx(t.x), exp2f_approx(t.y)),
+                                                      make_float2(1.f, 1.f));
+                        const float2 ab = __fmul2_rn(fa[i], fb[i]);
+                        fa[i] = __fmul2_rn(ab, make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+                    }
+                    st_stream(out + row * ld_out + (int64_t)col * E, pack2<T>(fa));
+                } else {
+                    float fa[E], fb[E];
+                    unpack<T>(av[k], fa);
+                    unpack<T>(bv[k], fb);
+#pragma unroll
+                    for (int e = 0; e < E; ++e) fa[e] = silu_mul<T>(fa[e], fb[e]);
+                    st_stream(out + row * ld_out + (int64_t)col * E, pack<T>(fa));
+                }
             }
         }
     }
@@ -114,7 +155,12 @@ struct StreamShape {
 // preference order below, then blockDim nearest 256.
 StreamShape choose_stream_shape(int64_t vpr)
 {
-    static const int kU[] = {4, 6, 8, 3, 2, 1};
+    int kU[] = {4, 6, 8, 3, 2, 1};
+    for (int i = 0; i < 6; ++i)  // move the configured first choice to the front
+        if (kU[i] == SOL_STREAM_UPREF_FIRST) {
+            for (int j = i; j > 0; --j) kU[j] = kU[j - 1];
+            kU[0] = SOL_STREAM_UPREF_FIRST;
+        }
     StreamShape best{0, 0, 0};
     int64_t best_waste = -1;
     int best_rank = 0, best_tdist = 0;
@@ -147,17 +193,29 @@ int64_t stream_grid(const void* kernel, const StreamShape& sh, int64_t n_tokens)
     return rows * sh.cpr;
 }
 
+template <typename T, int U, bool RO>
+cudaError_t run_gated_ro(void* out, int64_t ld_out, const void* x, int64_t ld_x, const void* y,
+                         int64_t ld_y, const void* gate, int64_t ld_mod, const ModSel& sel,
+                         int64_t n_tokens, int64_t vpr, const StreamShape& sh, cudaStream_t s)
+{
+    const void* kfn = (const void*)k_gated_residual<T, U, RO>;
+    const int64_t grid = stream_grid(kfn, sh, n_tokens);
+    k_gated_residual<T, U, RO><<<(unsigned)grid, sh.threads, 0, s>>>(
+        (T*)out, ld_out, (const T*)x, ld_x, (const T*)y, ld_y, (const T*)gate, ld_mod, sel,
+        n_tokens, (int32_t)vpr, sh.cpr);
+    return cudaGetLastError();
+}
+
 template <typename T, int U>
 cudaError_t run_gated(void* out, int64_t ld_out, const void* x, int64_t ld_x, const void* y,
                       int64_t ld_y, const void* gate, int64_t ld_mod, const ModSel& sel,
                       int64_t n_tokens, int64_t vpr, const StreamShape& sh, cudaStream_t s)
 {
-    const void* kfn = (const void*)k_gated_residual<T, U>;
-    const int64_t grid = stream_grid(kfn, sh, n_tokens);
-    k_gated_residual<T, U><<<(unsigned)grid, sh.threads, 0, s>>>(
-        (T*)out, ld_out, (const T*)x, ld_x, (const T*)y, ld_y, (const T*)gate, ld_mod, sel,
-        n_tokens, (int32_t)vpr, sh.cpr);
-    return cudaGetLastError();
+    if (out == x)
+        return run_gated_ro<T, U, false>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, sel, n_tokens,
+                                         vpr, sh, s);
+    return run_gated_ro<T, U, true>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, sel, n_tokens, vpr,
+                                    sh, s);
 }
 
 template <typename T, int U>
