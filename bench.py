@@ -313,6 +313,9 @@ def run_ours(args, w):
     ms_step = total_ms / args.steps
     value = step_bytes * world * args.steps / (total_ms * 1e-3) / 1e9
 
+    # ---- ops beyond the block pass, each timed alone on the same workload
+    next_ops = {} if args.no_next else time_next_ops(bufs, dev, args)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -347,6 +350,7 @@ def run_ours(args, w):
                      "traffic": None if traffic is None else int(traffic),
                      "algorithmic_bytes": dom_bytes},
         "clocks": clk,
+        "next_ops": next_ops,
         "gpu_launches": len(OPS) * args.steps,
         "e2e": e2e,
     }
@@ -359,6 +363,45 @@ def run_ours(args, w):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def _time(fn, reps: int, stream) -> float:
+    """Median milliseconds of `fn` over `reps` launches (CUDA events on `stream`)."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    for i in range(reps):
+        ev[i].record(stream)
+        fn()
+    ev[reps].record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(reps))
+
+
+def time_next_ops(bufs, dev, args) -> dict:
+    """Each op outside the block pass, timed alone at the workload's size (median of
+    20 launches), with its algorithmic bytes per token."""
+    from dit_block_b200 import sol
+    w, i = bufs.w, bufs.inp
+    n = bufs.n_tokens
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    peak, _ = measured_peak()
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    cache = torch.empty_like(bufs.x2)
+    cache.copy_(i["y_attn"])
+    sums = torch.empty((w.batch, 2), dtype=torch.float64, device=dev)
+    sel = bufs.sel()
+    fn = lambda: sol.gated_residual_cache_diff(bufs.x2, bufs.x1, i["y_mlp"], i["gate_mlp"], cache, sums,
+                                               refresh=True, **sel)
+    ms = _time(fn, 20, stream)
+    b = 5 * w.d * e  # read x, y, cache; write out, cache
+    out["gated_residual_cache_diff"] = {"ms": round(ms, 4), "bytes_per_token": b,
+                                        "GB_s": round(b * n / (ms * 1e-3) / 1e9, 1),
+                                        "frac_of_measured_peak": round(b * n / (ms * 1e-3) / 1e9 / peak, 4)}
+    del cache
+    return out
 
 
 def run_e2e(args, bufs, dev, world, step_bytes):
@@ -423,6 +466,7 @@ def main(argv=None):
     p.add_argument("--e2e-warmup", type=int, default=1)
     p.add_argument("--e2e-chunk", type=int, default=8192, help="tokens per pipelined chunk")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-next", action="store_true", help="skip timing the ops outside the block pass")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-tokens", type=int, default=256, help="oracle token sample per reference step")

@@ -125,6 +125,17 @@ inline void modsel_prepare(ModSel& m, int64_t n_tokens)
     m.div_fast = 1;
 }
 
+// Sample index of token n (0 when the call is one sample).
+__device__ __forceinline__ int64_t sample_of(int64_t n, const ModSel& m)
+{
+    if (m.tokens_per_sample <= 0) return 0;
+    if (m.div_fast) {
+        const uint32_t nn = (uint32_t)n;
+        return (int64_t)((__umulhi(nn, m.div_m) + nn) >> m.div_s);
+    }
+    return n / m.tokens_per_sample;
+}
+
 __device__ __forceinline__ int64_t mod_row(int64_t n, const ModSel& m)
 {
     int64_t sample = 0;

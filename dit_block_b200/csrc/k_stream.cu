@@ -63,6 +63,88 @@ k_gated_residual(T* __restrict__ out, int64_t ld_out, const T* x, int64_t ld_x,
     }
 }
 
+// Gated residual fused with the Cache-DiT residual-change statistics: out = x + gate*y as
+// in k_gated_residual; r = gate*y is compared with the cached residual of the previous
+// step, sums[s] += (sum |r - cache|, sum |cache|) over sample s, and with REFRESH the
+// cache is overwritten by r.  Each thread keeps fp32 partials per row and folds them into
+// fp64 accumulators; when a CTA moves to another sample (and at the end) every warp adds
+// its fp64 totals with one atomicAdd per sum, so no block barrier is needed.
+template <typename T, int U, bool REFRESH>
+__global__ void __launch_bounds__(512)
+k_gated_residual_diff(T* __restrict__ out, int64_t ld_out, const T* x, int64_t ld_x,
+                      const T* __restrict__ y, int64_t ld_y, const T* __restrict__ gate,
+                      int64_t ld_mod, T* cache, int64_t ld_c, double* __restrict__ sums,
+                      ModSel sel, int64_t n_tokens, int32_t vpr, int32_t cpr)
+{
+    constexpr int E = Vec<T>::N;
+    const int chunk = blockIdx.x % cpr;
+    const int64_t row_step = gridDim.x / cpr;
+    const int col0 = chunk * blockDim.x * U + threadIdx.x;
+    double acc_d = 0.0, acc_c = 0.0;
+    int64_t cur = -1;
+    auto flush = [&]() {
+        double td = acc_d, tc = acc_c;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            td += __shfl_xor_sync(0xffffffffu, td, off);
+            tc += __shfl_xor_sync(0xffffffffu, tc, off);
+        }
+        if ((threadIdx.x & 31) == 0 && cur >= 0) {
+            atomicAdd(sums + 2 * cur, td);
+            atomicAdd(sums + 2 * cur + 1, tc);
+        }
+        acc_d = 0.0;
+        acc_c = 0.0;
+    };
+    for (int64_t row = blockIdx.x / cpr; row < n_tokens; row += row_step) {
+        const int64_t mr = mod_row(row, sel);
+        const int64_t sample = sample_of(row, sel);
+        if (sample != cur) {  // uniform across the CTA
+            flush();
+            cur = sample;
+        }
+        uint4 xv[U], yv[U], cv[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int col = col0 + k * blockDim.x;
+            if (col < vpr) {
+                xv[k] = ld_stream(x + row * ld_x + (int64_t)col * E);
+                yv[k] = ld_stream_ro(y + row * ld_y + (int64_t)col * E);
+                cv[k] = ld_stream(cache + row * ld_c + (int64_t)col * E);
+            }
+        }
+        float pd = 0.f, pc = 0.f;
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int col = col0 + k * blockDim.x;
+            if (col < vpr) {
+                float fx[E], fy[E], fg[E], fc[E], fr[E];
+                unpack<T>(xv[k], fx);
+                unpack<T>(yv[k], fy);
+                unpack<T>(cv[k], fc);
+                if (gate) {
+                    unpack<T>(ld_cached(gate + mr * ld_mod + (int64_t)col * E), fg);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) fg[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    fr[e] = fg[e] * fy[e];
+                    fx[e] = fmaf(fg[e], fy[e], fx[e]);
+                    pd += fabsf(fr[e] - fc[e]);
+                    pc += fabsf(fc[e]);
+                }
+                st_stream(out + row * ld_out + (int64_t)col * E, pack<T>(fx));
+                if constexpr (REFRESH) st_stream(cache + row * ld_c + (int64_t)col * E, pack<T>(fr));
+            }
+        }
+        acc_d += (double)pd;
+        acc_c += (double)pc;
+    }
+    flush();
+}
+
 // The two MUFU operations of the bf16 SwiGLU: 2^x and 1/x, approximate (relative
 // error ~2^-22), flushing subnormal results to zero.  1/inf = 0, so a very negative
 // pre-activation gives silu = -0 as its limit.
@@ -252,6 +334,53 @@ cudaError_t launch_gated_residual(sol_dtype dt, void* out, int64_t ld_out, const
     const StreamShape sh = choose_stream_shape(vpr);
 #define CALL_B(U) run_gated<bf16, U>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, sel, n_tokens, vpr, sh, s)
 #define CALL_F(U) run_gated<float, U>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, sel, n_tokens, vpr, sh, s)
+    if (dt == SOL_DTYPE_BF16) {
+        SOL_DISPATCH_U(sh.U, CALL_B)
+    }
+    SOL_DISPATCH_U(sh.U, CALL_F)
+#undef CALL_B
+#undef CALL_F
+}
+
+namespace {
+template <typename T, int U, bool REFRESH>
+cudaError_t run_diff(void* out, int64_t ld_out, const void* x, int64_t ld_x, const void* y,
+                     int64_t ld_y, const void* gate, int64_t ld_mod, void* cache, int64_t ld_c,
+                     double* sums, const ModSel& sel, int64_t n_tokens, int64_t vpr,
+                     const StreamShape& sh, cudaStream_t s)
+{
+    const void* kfn = (const void*)k_gated_residual_diff<T, U, REFRESH>;
+    const int64_t grid = stream_grid(kfn, sh, n_tokens);
+    k_gated_residual_diff<T, U, REFRESH><<<(unsigned)grid, sh.threads, 0, s>>>(
+        (T*)out, ld_out, (const T*)x, ld_x, (const T*)y, ld_y, (const T*)gate, ld_mod, (T*)cache, ld_c,
+        sums, sel, n_tokens, (int32_t)vpr, sh.cpr);
+    return cudaGetLastError();
+}
+
+template <typename T, int U>
+cudaError_t run_diff_r(bool refresh, void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                       const void* y, int64_t ld_y, const void* gate, int64_t ld_mod, void* cache,
+                       int64_t ld_c, double* sums, const ModSel& sel, int64_t n_tokens, int64_t vpr,
+                       const StreamShape& sh, cudaStream_t s)
+{
+    if (refresh)
+        return run_diff<T, U, true>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, cache, ld_c, sums, sel,
+                                    n_tokens, vpr, sh, s);
+    return run_diff<T, U, false>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, cache, ld_c, sums, sel,
+                                 n_tokens, vpr, sh, s);
+}
+}  // namespace
+
+cudaError_t launch_gated_residual_diff(sol_dtype dt, void* out, int64_t ld_out, const void* x,
+                                       int64_t ld_x, const void* y, int64_t ld_y, const void* gate,
+                                       int64_t ld_mod, void* cache, int64_t ld_c, bool refresh,
+                                       double* sums, const ModSel& sel, int64_t n_tokens, int64_t d,
+                                       cudaStream_t s)
+{
+    const int64_t vpr = d / (dt == SOL_DTYPE_BF16 ? 8 : 4);
+    const StreamShape sh = choose_stream_shape(vpr);
+#define CALL_B(U) run_diff_r<bf16, U>(refresh, out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, cache, ld_c, sums, sel, n_tokens, vpr, sh, s)
+#define CALL_F(U) run_diff_r<float, U>(refresh, out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, cache, ld_c, sums, sel, n_tokens, vpr, sh, s)
     if (dt == SOL_DTYPE_BF16) {
         SOL_DISPATCH_U(sh.U, CALL_B)
     }

@@ -29,6 +29,12 @@ cudaError_t launch_gated_residual(sol_dtype dt, void* out, int64_t ld_out, const
                                   int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
                                   cudaStream_t s);
 
+cudaError_t launch_gated_residual_diff(sol_dtype dt, void* out, int64_t ld_out, const void* x,
+                                       int64_t ld_x, const void* y, int64_t ld_y, const void* gate,
+                                       int64_t ld_mod, void* cache, int64_t ld_c, bool refresh,
+                                       double* sums, const ModSel& sel, int64_t n_tokens, int64_t d,
+                                       cudaStream_t s);
+
 cudaError_t launch_swiglu(sol_dtype dt, void* out, int64_t ld_out, const void* a, const void* b,
                           int64_t ld_in, int64_t n_tokens, int64_t inner, cudaStream_t s);
 

@@ -254,6 +254,51 @@ sol_status sol_gated_residual(void* out, int64_t ld_out, const void* x, int64_t 
                        "sol_gated_residual launch");
 }
 
+sol_status sol_gated_residual_cache_diff(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                                         const void* y, int64_t ld_y, const void* gate,
+                                         int64_t ld_mod, sol_modsel sel, void* cache,
+                                         int64_t ld_cache, int32_t refresh, double* sums,
+                                         int64_t n_samples, int64_t n_tokens, int64_t d,
+                                         sol_dtype dt, sol_stream_t stream)
+{
+    TRY(check_dtype(dt));
+    TRY(check_rows(n_tokens, d, dt, "d"));
+    TRY(check_modsel(sel));
+    CHECK(sums, SOL_ERR_INVALID_ARGUMENT, "sums is NULL");
+    CHECK((reinterpret_cast<uintptr_t>(sums) & 7u) == 0, SOL_ERR_MISALIGNED, "sums is not 8-byte aligned");
+    CHECK(n_samples >= 1, SOL_ERR_INVALID_ARGUMENT, "n_samples (%lld) must be >= 1", (long long)n_samples);
+    const int64_t needed = sel.tokens_per_sample > 0
+                               ? (n_tokens + sel.tokens_per_sample - 1) / sel.tokens_per_sample
+                               : 1;
+    CHECK(needed <= n_samples, SOL_ERR_INVALID_ARGUMENT,
+          "%lld tokens at %lld per sample need %lld sample sums, n_samples is %lld",
+          (long long)n_tokens, (long long)sel.tokens_per_sample, (long long)needed, (long long)n_samples);
+    if (n_tokens > 0) {  // empty tensors may be NULL
+        TRY(check_tensor("out", out, ld_out, d, dt, true));
+        TRY(check_tensor("x", x, ld_x, d, dt, true));
+        TRY(check_tensor("y", y, ld_y, d, dt, true));
+        TRY(check_tensor("gate", gate, ld_mod, d, dt, false));
+        TRY(check_tensor("cache", cache, ld_cache, d, dt, true));
+        const size_t es = esize(dt);
+        CHECK(out == x ? ld_out == ld_x : !overlap(out, ld_out, x, ld_x, n_tokens, d, es),
+              SOL_ERR_INVALID_ARGUMENT, "out overlaps x without being the same tensor");
+        CHECK(!overlap(out, ld_out, y, ld_y, n_tokens, d, es), SOL_ERR_INVALID_ARGUMENT, "out overlaps y");
+        CHECK(!overlap(cache, ld_cache, out, ld_out, n_tokens, d, es) &&
+                  !overlap(cache, ld_cache, x, ld_x, n_tokens, d, es) &&
+                  !overlap(cache, ld_cache, y, ld_y, n_tokens, d, es),
+              SOL_ERR_INVALID_ARGUMENT, "cache overlaps out, x or y");
+    }
+    // all arguments valid: clear the sums on the stream, then accumulate into them
+    cudaError_t e = cudaMemsetAsync(sums, 0, (size_t)n_samples * 2 * sizeof(double), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_status(e, "sol_gated_residual_cache_diff clearing sums");
+    if (n_tokens == 0) return SOL_OK;
+    const sol::ModSel ms = to_dev(sel, n_tokens);
+    return cuda_status(sol::launch_gated_residual_diff(dt, out, ld_out, x, ld_x, y, ld_y, gate, ld_mod,
+                                                       cache, ld_cache, refresh != 0, sums, ms,
+                                                       n_tokens, d, (cudaStream_t)stream),
+                       "sol_gated_residual_cache_diff launch");
+}
+
 sol_status sol_swiglu(void* out, int64_t ld_out, const void* a, const void* b, int64_t ld_in,
                       int64_t n_tokens, int64_t inner, sol_dtype dt, sol_stream_t stream)
 {

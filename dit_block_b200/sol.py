@@ -45,6 +45,8 @@ SIGNATURES = {
     "sol_device_errors": ([ctypes.POINTER(ctypes.c_uint32), _I32], _E),
     "sol_adaln_modulate": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _I64, _I64, _F, _E, _P], _E),
     "sol_gated_residual": ([_P, _I64, _P, _I64, _P, _I64, _P, _I64, ModSel, _I64, _I64, _E, _P], _E),
+    "sol_gated_residual_cache_diff": ([_P, _I64, _P, _I64, _P, _I64, _P, _I64, ModSel, _P, _I64, _I32,
+                                       _P, _I64, _I64, _I64, _E, _P], _E),
     "sol_swiglu": ([_P, _I64, _P, _P, _I64, _I64, _I64, _E, _P], _E),
     "sol_rope3d_create": ([ctypes.POINTER(_P), _I32, _I32, _I32, _D, _I32, _I32, _I32], _E),
     "sol_rope3d_destroy": ([_P], _E),
@@ -171,6 +173,22 @@ def gated_residual(out, x, y, gate=None, *, stream_id=None, n_streams=1, tokens_
     _check(lib().sol_gated_residual(_ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(y), _ld(y), _ptr(gate),
                                     _mod_ld(gate), _sel(stream_id, n_streams, tokens_per_sample), n, d,
                                     _dtype(x), _stream(stream)), "sol_gated_residual")
+    return out
+
+
+def gated_residual_cache_diff(out, x, y, gate, cache, sums, *, refresh=True, stream_id=None,
+                              n_streams=1, tokens_per_sample=0, d=None, stream=None):
+    """out = x + gate[r]*y and, per sample, sums[s] = (sum |gate*y - cache|, sum |cache|);
+    with refresh the cache becomes gate*y (sol_gated_residual_cache_diff).  sums is a
+    float64 device tensor [n_samples, 2]."""
+    if sums.dtype != torch.float64 or not sums.is_contiguous():
+        raise TypeError("sums must be a contiguous float64 tensor [n_samples, 2]")
+    n = x.shape[0]
+    d = x.shape[1] if d is None else d
+    _check(lib().sol_gated_residual_cache_diff(
+        _ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(y), _ld(y), _ptr(gate), _mod_ld(gate),
+        _sel(stream_id, n_streams, tokens_per_sample), _ptr(cache), _ld(cache), int(bool(refresh)),
+        _ptr(sums), sums.numel() // 2, n, d, _dtype(x), _stream(stream)), "sol_gated_residual_cache_diff")
     return out
 
 

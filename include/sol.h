@@ -116,6 +116,30 @@ sol_status sol_gated_residual(void* out, int64_t ld_out, const void* x, int64_t 
                               sol_modsel sel, int64_t n_tokens, int64_t d, sol_dtype dt,
                               sol_stream_t stream);
 
+/* Gated residual fused with the Cache-DiT residual-change statistics [XHH-QA, the answer
+ * on how Cache-DiT reuses computation between denoising steps: boundary blocks compare
+ * the normalised residual change with the cached state; below a threshold the middle
+ * blocks reuse the cache, otherwise they recompute and refresh it; STM-RES: one joint
+ * decision for the packed video+audio stack].  In one pass over the tokens:
+ *     out_i = x_i + gate[r]_i * y_i                  (exactly as sol_gated_residual)
+ *     r_i   = gate[r]_i * y_i                        (the block's residual contribution)
+ *     sums[s][0] = sum |r_i - cache_i|,  sums[s][1] = sum |cache_i|
+ * over every element of every token of sample s (all streams together); the change is
+ * sums[s][0] / sums[s][1] and the reuse decision is the caller's.  With refresh != 0
+ * the cache is overwritten by r (rounded to dt), so the next step compares against it.
+ *   cache, ld_cache  [n_tokens, ld_cache] device tensor, read (and written if refresh);
+ *                    must not overlap out, x or y.
+ *   sums             device double [n_samples][2], cleared and filled by this call
+ *                    (accumulated with fp64 atomics, so the last bits may vary run to
+ *                    run); n_samples >= the samples the tokens span.
+ * Everything else as in sol_gated_residual. */
+sol_status sol_gated_residual_cache_diff(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                                         const void* y, int64_t ld_y, const void* gate,
+                                         int64_t ld_mod, sol_modsel sel, void* cache,
+                                         int64_t ld_cache, int32_t refresh, double* sums,
+                                         int64_t n_samples, int64_t n_tokens, int64_t d,
+                                         sol_dtype dt, sol_stream_t stream);
+
 /* SwiGLU activation [XHH-QA, STM-GAN]:  out_j = silu(a_j) * b_j,  silu(v) = v/(1+e^-v),
  * j < inner, for every token row.  For the packed up-projection u = [a | b] of width
  * 2*inner pass a = u, b = u + inner (elements) and ld_in = ld of u.

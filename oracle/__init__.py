@@ -51,6 +51,9 @@ def _load():
         lib.oracle_adaln_modulate.restype = None
         lib.oracle_gated_residual.argtypes = [P, I64, P, I64, P, I64, I, P, I64, I, P, I32, I64, P, I64, I64]
         lib.oracle_gated_residual.restype = None
+        lib.oracle_gated_residual_cache_diff.argtypes = [P, P, P, I64, P, I64, P, I64, I, P, I64, I,
+                                                         P, I64, I, P, I32, I64, P, I64, I64]
+        lib.oracle_gated_residual_cache_diff.restype = None
         lib.oracle_swiglu.argtypes = [P, I64, P, P, I64, I, I64, I64]
         lib.oracle_swiglu.restype = None
         lib.oracle_qk_rmsnorm_rope3d.argtypes = [P, P, I64, I64, P, P, I64, I64, I, P, P, I, P,
@@ -141,6 +144,26 @@ def gated_residual(x, y, gate=None, *, stream_id=None, n_streams=1, tokens_per_s
                                   _ptr(gate), ld_mod, _code(gate), _ptr(sid), S, tps, _ptr(rw),
                                   n, d)
     return out
+
+
+def gated_residual_cache_diff(x, y, gate, cache, *, n_samples=1, stream_id=None, n_streams=1,
+                              tokens_per_sample=0, rows=None):
+    """Gated residual plus Cache-DiT residual-change sums.  Returns (out, r, sums) with
+    out = x + gate*y, r = gate*y (the refreshed cache) and sums [n_samples, 2] =
+    (sum |r - cache|, sum |cache|) per sample."""
+    assert x.dtype == y.dtype
+    n, d = x.shape
+    ld_mod, sid, S, tps = _mod_args(gate, stream_id, n_streams, tokens_per_sample)
+    rw = _rows(rows, n)
+    out = np.empty((n, d), np.float64)
+    r = np.empty((n, d), np.float64)
+    sums = np.empty((n_samples, 2), np.float64)
+    _load().oracle_gated_residual_cache_diff(out.ctypes.data, r.ctypes.data, sums.ctypes.data,
+                                             int(n_samples), _ptr(x), _ld(x), _ptr(y), _ld(y),
+                                             _code(x), _ptr(gate), ld_mod, _code(gate), _ptr(cache),
+                                             _ld(cache), _code(cache), _ptr(sid), S, tps, _ptr(rw),
+                                             n, d)
+    return out, r, sums
 
 
 def swiglu(u, inner=None, *, n_tokens=None):

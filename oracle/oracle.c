@@ -132,6 +132,44 @@ void oracle_gated_residual(double* o, int64_t ld_o,
     }
 }
 
+/* Gated residual with the Cache-DiT residual-change statistics [XHH-QA, the answer on
+ * how Cache-DiT reuses computation: after warm-up steps it compares the normalised
+ * residual change of boundary blocks with the cached state and reuses the cache when
+ * the change is below a threshold].  Read here as: the block's residual contribution
+ * r = gate * y, compared with the cached r of the previous step, per sample:
+ *     sums[s][0] = sum |r - cache|,   sums[s][1] = sum |cache|
+ * over every element of the sample's tokens (video and audio together: one joint
+ * decision for the packed stack [STM-RES]); the change is sums[s][0] / sums[s][1].
+ * out = x + r as in oracle_gated_residual; r_out receives r (the refreshed cache).
+ * sums must hold 2 * n_samples doubles and is overwritten. */
+void oracle_gated_residual_cache_diff(double* o, double* r_out, double* sums, int64_t n_samples,
+                                      const void* x, int64_t ld_x, const void* y, int64_t ld_y,
+                                      int dt_xy, const void* gate, int64_t ld_mod, int dt_mod,
+                                      const void* cache, int64_t ld_c, int dt_c,
+                                      const uint8_t* stream_id, int32_t n_streams,
+                                      int64_t tokens_per_sample, const int64_t* rows,
+                                      int64_t n_tokens, int64_t d)
+{
+    for (int64_t s = 0; s < 2 * n_samples; ++s) sums[s] = 0.0;
+    for (int64_t n = 0; n < n_tokens; ++n) {
+        const int64_t g_n = rows ? rows[n] : n;
+        const int64_t r_row = mod_row(g_n, stream_id, n_streams, tokens_per_sample);
+        const int64_t sample = tokens_per_sample > 0 ? g_n / tokens_per_sample : 0;
+        double dsum = 0.0, csum = 0.0;
+        for (int64_t i = 0; i < d; ++i) {
+            const double g = gate ? load(gate, dt_mod, r_row * ld_mod + i) : 0.0;
+            const double r = g * load(y, dt_xy, n * ld_y + i);
+            const double c = load(cache, dt_c, n * ld_c + i);
+            o[n * d + i] = load(x, dt_xy, n * ld_x + i) + r;
+            r_out[n * d + i] = r;
+            dsum += fabs(r - c);
+            csum += fabs(c);
+        }
+        sums[2 * sample] += dsum;
+        sums[2 * sample + 1] += csum;
+    }
+}
+
 /* SwiGLU activation [XHH-QA, STM-GAN]: o_j = a_j / (1 + exp(-a_j)) * b_j.  a and b are
  * separate row pointers so the caller can pass the two halves of one up-projection row
  * (b = a + inner) or two tensors. */

@@ -442,3 +442,63 @@ def test_row_subsets_equal_rows_of_the_full_sequence(oracle_mod):
     e_full = oracle_mod.dit_epilogue(qkv, **ek)
     e_sub = oracle_mod.dit_epilogue(np.ascontiguousarray(qkv[rows]), rows=rows, **ek)
     np.testing.assert_array_equal(e_sub, e_full[rows])
+
+
+# ------------------------------------------------------- Cache-DiT residual change
+
+
+def test_cache_diff_golden(oracle_mod):
+    g = read_golden("cache_diff_d2.txt")
+    x = np.array(g["x"]).reshape(2, 2); y = np.array(g["y"]).reshape(2, 2)
+    gate = np.array(g["gate"]).reshape(2, 2); cache = np.array(g["cache"]).reshape(2, 2)
+    out, r, sums = oracle_mod.gated_residual_cache_diff(x, y, gate, cache, n_samples=2,
+                                                        tokens_per_sample=1)
+    np.testing.assert_array_equal(out.reshape(-1), g["out"])
+    np.testing.assert_array_equal(sums.reshape(-1), g["sums"])
+    np.testing.assert_array_equal(r, gate * y)
+
+
+def test_cache_diff_invariants(oracle_mod):
+    d, B, tps = 96, 3, 7
+    n = B * tps
+    x = RNG.standard_normal((n, d)); y = RNG.standard_normal((n, d))
+    gate = RNG.standard_normal((B, d)) * 0.1
+    # the output is the plain gated residual
+    out, r, sums = oracle_mod.gated_residual_cache_diff(x, y, gate, np.zeros((n, d)), n_samples=B,
+                                                        tokens_per_sample=tps)
+    np.testing.assert_array_equal(out, oracle_mod.gated_residual(x, y, gate, tokens_per_sample=tps))
+    # an all-zero cache: no reference mass, the change is the residual's own L1 mass
+    np.testing.assert_array_equal(sums[:, 1], 0.0)
+    for b in range(B):
+        np.testing.assert_allclose(sums[b, 0], np.abs(r[b * tps:(b + 1) * tps]).sum(), rtol=1e-13)
+    # comparing against its own refreshed cache: no change
+    _, r2, sums2 = oracle_mod.gated_residual_cache_diff(x, y, gate, r, n_samples=B, tokens_per_sample=tps)
+    np.testing.assert_array_equal(sums2[:, 0], 0.0)
+    np.testing.assert_allclose(sums2[:, 1], sums[:, 0], rtol=1e-13)
+    # scaling y and the cache together scales both sums (the ratio is scale free)
+    c = RNG.standard_normal((n, d)) * 0.1
+    _, _, s1 = oracle_mod.gated_residual_cache_diff(x, y, gate, c, n_samples=B, tokens_per_sample=tps)
+    _, _, s2 = oracle_mod.gated_residual_cache_diff(x, 4 * y, gate, 4 * c, n_samples=B, tokens_per_sample=tps)
+    np.testing.assert_allclose(s2, 4 * s1, rtol=1e-12)
+    # samples are independent: sample b's sums depend only on its rows
+    c2 = c.copy(); c2[tps:2 * tps] += 1.0
+    _, _, s3 = oracle_mod.gated_residual_cache_diff(x, y, gate, c2, n_samples=B, tokens_per_sample=tps)
+    np.testing.assert_array_equal(s3[[0, 2]], s1[[0, 2]])
+    assert not np.allclose(s3[1], s1[1])
+
+
+def test_cache_diff_packed_streams_share_one_decision(oracle_mod):
+    """Video and audio tokens of a sample use their own gates but add into one sum."""
+    d, B, S, tps = 32, 2, 2, 9
+    n = B * tps
+    x = RNG.standard_normal((n, d)); y = RNG.standard_normal((n, d)); c = RNG.standard_normal((n, d))
+    gate = RNG.standard_normal((B * S, d))
+    sid = np.array(([0] * 6 + [1] * 3) * B, np.uint8)
+    _, r, sums = oracle_mod.gated_residual_cache_diff(x, y, gate, c, n_samples=B, stream_id=sid,
+                                                      n_streams=S, tokens_per_sample=tps)
+    for b in range(B):
+        blk = slice(b * tps, (b + 1) * tps)
+        np.testing.assert_allclose(sums[b, 0], np.abs(r[blk] - c[blk]).sum(), rtol=1e-13)
+        np.testing.assert_allclose(sums[b, 1], np.abs(c[blk]).sum(), rtol=1e-13)
+    # the audio rows of sample 1 took gate row 3
+    np.testing.assert_allclose(r[tps + 6], gate[3] * y[tps + 6], rtol=0, atol=0)
