@@ -401,6 +401,19 @@ def time_next_ops(bufs, dev, args) -> dict:
                                         "GB_s": round(b * n / (ms * 1e-3) / 1e9, 1),
                                         "frac_of_measured_peak": round(b * n / (ms * 1e-3) / 1e9 / peak, 4)}
     del cache
+    blk = 64
+    nb = sol.subblock_count(n, w.tokens_per_sample, blk)
+    pq = torch.empty((nb, w.hd), dtype=w.dtype, device=dev)
+    pk = torch.empty((nb, w.hd), dtype=w.dtype, device=dev)
+    fn = lambda: sol.dit_epilogue_pool(i["qkv"], pq, pk, bufs.rope, n_heads=w.n_heads, head_dim=w.head_dim,
+                                       wq=i["wq"], wk=i["wk"], pos=i["pos"], grid=w.grid,
+                                       tokens_per_sample=w.tokens_per_sample, block_tokens=blk, eps=w.eps)
+    ms = _time(fn, 20, stream)
+    b = 4 * w.hd * e  # read and write q and k
+    pooled = 2 * nb * w.hd * e  # the pooled rows
+    out["dit_epilogue_pool"] = {"ms": round(ms, 4), "bytes_per_token": b, "pooled_bytes": pooled,
+                                "GB_s": round((b * n + pooled) / (ms * 1e-3) / 1e9, 1),
+                                "frac_of_measured_peak": round((b * n + pooled) / (ms * 1e-3) / 1e9 / peak, 4)}
     return out
 
 

@@ -53,6 +53,16 @@ cudaError_t launch_qk_rmsnorm_rope3d(sol_dtype dt, void* q_out, void* k_out, int
                                      const RopeDev& rope, int64_t n_tokens, int32_t n_heads,
                                      int32_t head_dim, float eps, cudaStream_t s);
 
+// QKV epilogue fused with SubBlock block means (k_qk_pool.cu).  In place on q and k.
+cudaError_t launch_qk_rope_pool(sol_dtype dt, void* q, void* k, int64_t ld_q, int64_t ld_k, void* pq,
+                                void* pk, int64_t ld_pq, int64_t ld_pk, const void* wq, const void* wk,
+                                const int32_t* pos, int32_t grid_H, int32_t grid_W, int64_t tps,
+                                int32_t block, int64_t bps, int64_t n_blocks, const RopeDev& rope,
+                                int64_t n_tokens, int32_t n_heads, int32_t head_dim, float eps,
+                                cudaStream_t s);
+int qk_pool_vectors_per_lane(sol_dtype dt, int32_t n_heads, int32_t head_dim);
+int qk_pool_max_vectors_per_lane();
+
 // Error flags raised on the device by the AdaLN / prologue kernels (bit 0: a bounded
 // wait on a bulk copy gave up); optionally cleared.  Synchronous.
 uint32_t rows_device_error(bool clear);

@@ -481,6 +481,49 @@ sol_status sol_dit_prologue(void* x_out, void* h, const void* x, const void* y,
                        "sol_dit_prologue launch");
 }
 
+int64_t sol_subblock_count(int64_t n_tokens, int64_t tokens_per_sample, int32_t block_tokens)
+{
+    if (n_tokens <= 0 || block_tokens <= 0 || tokens_per_sample < 0) return 0;
+    const int64_t tps = tokens_per_sample > 0 ? tokens_per_sample : n_tokens;
+    const int64_t samples = (n_tokens + tps - 1) / tps;
+    return samples * ((tps + block_tokens - 1) / block_tokens);
+}
+
+sol_status sol_dit_epilogue_pool(void* qkv, int64_t ld_qkv, const void* wq, const void* wk,
+                                 const int32_t* pos, int32_t grid_T, int32_t grid_H, int32_t grid_W,
+                                 int64_t tokens_per_sample, const sol_rope3d* rope, int64_t n_tokens,
+                                 int32_t n_heads, int32_t head_dim, float eps, void* pooled_q,
+                                 void* pooled_k, int64_t ld_pool, int32_t block_tokens, sol_dtype dt,
+                                 sol_stream_t stream)
+{
+    TRY(check_qk_common(rope, pos, grid_T, grid_H, grid_W, tokens_per_sample, n_tokens, n_heads,
+                        head_dim, eps, dt, wq, wk));
+    CHECK(block_tokens >= 1 && block_tokens <= (1 << 20), SOL_ERR_INVALID_ARGUMENT,
+          "block_tokens (%d) must be in [1, 2^20]", (int)block_tokens);
+    CHECK(sol::qk_pool_vectors_per_lane(dt, n_heads, head_dim) <= sol::qk_pool_max_vectors_per_lane(),
+          SOL_ERR_UNSUPPORTED, "%d heads of %d are more than the pooled epilogue is built for",
+          (int)n_heads, (int)head_dim);
+    if (n_tokens == 0) return SOL_OK;  // nothing to do; empty tensors may be NULL
+    const int64_t hd = (int64_t)n_heads * head_dim;
+    TRY(check_tensor("qkv", qkv, ld_qkv, 2 * hd, dt, true));
+    const int64_t n_blocks = sol_subblock_count(n_tokens, tokens_per_sample, block_tokens);
+    TRY(check_tensor("pooled_q", pooled_q, ld_pool, hd, dt, true));
+    TRY(check_tensor("pooled_k", pooled_k, ld_pool, hd, dt, true));
+    const size_t es = esize(dt);
+    CHECK(!overlap(pooled_q, ld_pool, pooled_k, ld_pool, n_blocks, hd, es) &&
+              !overlap(pooled_q, ld_pool, qkv, ld_qkv, n_blocks < n_tokens ? n_blocks : n_tokens, hd, es) &&
+              !overlap(pooled_k, ld_pool, qkv, ld_qkv, n_blocks < n_tokens ? n_blocks : n_tokens, hd, es),
+          SOL_ERR_INVALID_ARGUMENT, "pooled outputs overlap each other or qkv");
+    const int64_t tps = tokens_per_sample > 0 ? tokens_per_sample : n_tokens;
+    const int64_t bps = (tps + block_tokens - 1) / block_tokens;
+    void* k = (char*)qkv + (size_t)hd * es;
+    return cuda_status(sol::launch_qk_rope_pool(dt, qkv, k, ld_qkv, ld_qkv, pooled_q, pooled_k, ld_pool,
+                                                ld_pool, wq, wk, pos, grid_H, grid_W, tps, block_tokens,
+                                                bps, n_blocks, rope->view, n_tokens, n_heads, head_dim,
+                                                eps, (cudaStream_t)stream),
+                       "sol_dit_epilogue_pool launch");
+}
+
 sol_status sol_dit_epilogue(void* qkv, int64_t ld_qkv, const void* wq, const void* wk,
                             const int32_t* pos, int32_t grid_T, int32_t grid_H, int32_t grid_W,
                             int64_t tokens_per_sample, const sol_rope3d* rope, int64_t n_tokens,

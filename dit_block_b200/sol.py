@@ -55,6 +55,9 @@ SIGNATURES = {
     "sol_dit_prologue": ([_P, _P, _P, _P, _P, _P, _P, _I64, _I64, ModSel, _I64, _I64, _F, _E, _P], _E),
     "sol_dit_epilogue": ([_P, _I64, _P, _P, _P, _I32, _I32, _I32, _I64, _P, _I64, _I32, _I32, _F,
                           _E, _P], _E),
+    "sol_subblock_count": ([_I64, _I64, _I32], _I64),
+    "sol_dit_epilogue_pool": ([_P, _I64, _P, _P, _P, _I32, _I32, _I32, _I64, _P, _I64, _I32, _I32, _F,
+                               _P, _P, _I64, _I32, _E, _P], _E),
     "sol_qk_rmsnorm_rope3d_noalloc": ([_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _P, _P, _I32, _I32,
                                        _I32, _I64, _I32, _I32, _I32, _D, _I32, _I32, _I32, _I64,
                                        _I32, _I32, _F, _E, _P], _E),
@@ -292,3 +295,23 @@ def qk_rmsnorm_rope3d_noalloc(q_out, k_out, q, k, *, n_heads, head_dim, dims=(32
         int(tokens_per_sample), int(dims[0]), int(dims[1]), int(dims[2]), float(theta),
         int(max_pos[0]), int(max_pos[1]), int(max_pos[2]), q.shape[0], int(n_heads),
         int(head_dim), eps, _dtype(q), _stream(stream)), "sol_qk_rmsnorm_rope3d_noalloc")
+
+
+def subblock_count(n_tokens: int, tokens_per_sample: int = 0, block_tokens: int = 64) -> int:
+    """Blocks of block_tokens tokens in the sequence (blocks restart at each sample)."""
+    return int(lib().sol_subblock_count(int(n_tokens), int(tokens_per_sample), int(block_tokens)))
+
+
+def dit_epilogue_pool(qkv, pooled_q, pooled_k, rope: Rope3D, *, n_heads, head_dim, wq=None, wk=None,
+                      pos=None, grid=(0, 0, 0), tokens_per_sample=0, block_tokens=64, eps=1e-6,
+                      stream=None):
+    """sol_dit_epilogue plus per-block means of the normalised, rotated q and k."""
+    if pos is not None and (pos.dtype != torch.int32 or not pos.is_contiguous()):
+        raise TypeError("pos must be a contiguous int32 [N, 3] tensor")
+    if _ld(pooled_q) != _ld(pooled_k):
+        raise ValueError("pooled_q and pooled_k must share a leading dimension")
+    _check(lib().sol_dit_epilogue_pool(
+        _ptr(qkv), _ld(qkv), _ptr(wq), _ptr(wk), _ptr(pos), int(grid[0]), int(grid[1]), int(grid[2]),
+        int(tokens_per_sample), rope.handle, qkv.shape[0], int(n_heads), int(head_dim), eps,
+        _ptr(pooled_q), _ptr(pooled_k), _ld(pooled_q), int(block_tokens), _dtype(qkv), _stream(stream)),
+        "sol_dit_epilogue_pool")

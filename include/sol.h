@@ -229,6 +229,31 @@ sol_status sol_dit_epilogue(void* qkv, int64_t ld_qkv, const void* wq, const voi
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
  * current device); make that first call before any stream capture.
  * Other arguments, layouts, aliasing and errors as in sol_qk_rmsnorm_rope3d. */
+/* Number of SubBlock blocks of `block_tokens` tokens in a packed sequence: blocks
+ * restart at every sample boundary, so it is n_samples * ceil(tokens_per_sample /
+ * block_tokens) (tokens_per_sample 0 = one sample); 0 for invalid arguments. */
+int64_t sol_subblock_count(int64_t n_tokens, int64_t tokens_per_sample, int32_t block_tokens);
+
+/* The QKV epilogue fused with the block means SubBlock sparse attention routes on
+ * [XHH-QA, the answer on SubBlock: 64-token blocks, a router keeps a fraction of the key
+ * blocks; STM-GAN, SubBlock splits the sequence into blocks of 64 tokens].  Does exactly
+ * what sol_dit_epilogue does (q and k of packed [q | k | v] rows normalised and rotated
+ * in place) and, in the same pass, writes the mean of the resulting q (k) rows of every
+ * block into pooled_q (pooled_k): block b of sample s is row
+ * s * ceil(tokens_per_sample / block_tokens) + b; the last block of a sample averages
+ * the tokens it has.  Means are taken over the fp32 results before their rounding.
+ *   pooled_q, pooled_k  [sol_subblock_count(...), ld_pool] each; must not overlap
+ *                       each other or qkv.
+ *   block_tokens        tokens per block (64 on the pages), >= 1.
+ * Other arguments as in sol_dit_epilogue; n_heads is limited to what one CTA's warps
+ * cover (bf16 head_dim 128: up to 80 heads; f32 head_dim 128: up to 40). */
+sol_status sol_dit_epilogue_pool(void* qkv, int64_t ld_qkv, const void* wq, const void* wk,
+                                 const int32_t* pos, int32_t grid_T, int32_t grid_H, int32_t grid_W,
+                                 int64_t tokens_per_sample, const sol_rope3d* rope, int64_t n_tokens,
+                                 int32_t n_heads, int32_t head_dim, float eps, void* pooled_q,
+                                 void* pooled_k, int64_t ld_pool, int32_t block_tokens, sol_dtype dt,
+                                 sol_stream_t stream);
+
 #define SOL_NOALLOC_MAX_ROPE_ENTRIES 65536
 sol_status sol_qk_rmsnorm_rope3d_noalloc(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko,
                                          const void* q, const void* k, int64_t ld_q, int64_t ld_k,

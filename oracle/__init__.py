@@ -54,6 +54,8 @@ def _load():
         lib.oracle_gated_residual_cache_diff.argtypes = [P, P, P, I64, P, I64, P, I64, I, P, I64, I,
                                                          P, I64, I, P, I32, I64, P, I64, I64]
         lib.oracle_gated_residual_cache_diff.restype = None
+        lib.oracle_block_mean.argtypes = [P, P, I64, I64, I64, I64]
+        lib.oracle_block_mean.restype = I64
         lib.oracle_swiglu.argtypes = [P, I64, P, P, I64, I, I64, I64]
         lib.oracle_swiglu.restype = None
         lib.oracle_qk_rmsnorm_rope3d.argtypes = [P, P, I64, I64, P, P, I64, I64, I, P, P, I, P,
@@ -253,3 +255,17 @@ def dit_epilogue(qkv, wq=None, wk=None, *, n_heads, head_dim, pos=None, grid=(0,
     if rc != 0:
         raise ValueError("RoPE split does not fit head_dim (dims must be even and sum to it)")
     return out
+
+
+def block_mean(v, *, tokens_per_sample=0, block=64):
+    """Means of `block`-token blocks of the fp64 rows v [N, width]; blocks restart at every
+    sample boundary.  Returns [n_blocks, width]."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    n, width = v.shape
+    tps = tokens_per_sample if tokens_per_sample > 0 else n
+    per_sample = -(-tps // block)
+    n_blocks = -(-n // tps) * per_sample if n else 0
+    out = np.full((n_blocks, width), np.nan)
+    got = _load().oracle_block_mean(out.ctypes.data, v.ctypes.data, n, width, int(tokens_per_sample),
+                                    int(block))
+    return out[:got]

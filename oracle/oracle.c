@@ -309,3 +309,34 @@ int oracle_dit_epilogue(double* qk_out, const void* qkv, int64_t ld_qkv, int dt,
                                     tokens_per_sample, dim_t, dim_h, dim_w, theta, rows, n_tokens,
                                     n_heads, head_dim, eps);
 }
+
+/* Block means for SubBlock routing [XHH-QA on SubBlock sparse attention: the sequence
+ * is split into 64-token blocks and a router keeps a fraction of the key blocks;
+ * "SGLang acelera video do MiniMax-H3", "De onde vem os ganhos": SubBlock splits the
+ * sequence into blocks of 64 tokens].  Read here as: blocks of `block` consecutive
+ * tokens that restart at every sample boundary (the last block of a sample holds the
+ * remainder); the pooled row of a block is the mean of its tokens' rows of `v`
+ * (n_tokens x width, fp64, e.g. the normalised and rotated q or k).  Block b of sample
+ * s is row s * ceil(tokens_per_sample / block) + b of `pooled` (width wide).  Returns
+ * the number of blocks written. */
+int64_t oracle_block_mean(double* pooled, const double* v, int64_t n_tokens, int64_t width,
+                          int64_t tokens_per_sample, int64_t block)
+{
+    const int64_t tps = tokens_per_sample > 0 ? tokens_per_sample : n_tokens;
+    const int64_t per_sample = (tps + block - 1) / block;
+    int64_t written = 0;
+    for (int64_t s0 = 0; s0 < n_tokens; s0 += tps) {
+        const int64_t s1 = s0 + tps < n_tokens ? s0 + tps : n_tokens;
+        for (int64_t b0 = s0; b0 < s1; b0 += block) {
+            const int64_t b1 = b0 + block < s1 ? b0 + block : s1;
+            const int64_t row = (s0 / tps) * per_sample + (b0 - s0) / block;
+            for (int64_t i = 0; i < width; ++i) {
+                double acc = 0.0;
+                for (int64_t t = b0; t < b1; ++t) acc += v[t * width + i];
+                pooled[row * width + i] = acc / (double)(b1 - b0);
+            }
+            if (row + 1 > written) written = row + 1;
+        }
+    }
+    return written;
+}

@@ -28,7 +28,7 @@ def last(L):
 
 def test_exports_every_declared_symbol(L):
     names = sol.header_functions()
-    assert len(names) == 14
+    assert len(names) == 16
     for n in names:
         assert hasattr(L, n), f"libsol.so does not export {n}"
         assert n in sol.SIGNATURES, f"binding has no signature for {n}"
@@ -128,3 +128,11 @@ def test_binding_raises_with_reason():
         sol._check(sol.lib().sol_swiglu(None, 8, None, None, 8, 1, 8, sol.BF16, None), "sol_swiglu")
     assert e.value.status == sol.ERR_INVALID_ARGUMENT
     assert "NULL" in str(e.value)
+
+
+def test_subblock_count(L):
+    assert L.sol_subblock_count(245952, 245952, 64) == 3843
+    assert L.sol_subblock_count(2 * 130, 130, 64) == 6     # 64 + 64 + 2 per sample
+    assert L.sol_subblock_count(100, 0, 64) == 2
+    assert L.sol_subblock_count(0, 0, 64) == 0
+    assert L.sol_subblock_count(10, 0, 0) == 0

@@ -155,3 +155,79 @@ def test_cache_diff_full_workload(orc):
                                               tokens_per_sample=w.tokens_per_sample, rows=R)
     assert_close(to_f64(out[rows]), wo, BF, "full out")
     assert_close(to_f64(cache[rows]), wr, BF, "full refreshed cache")
+
+
+# --------------------------------------------------------- SubBlock pooled epilogue
+
+POOL_CASES = [  # dtype, head_dim, dims, n_heads, grid, samples, audio tokens per sample, block
+    (BF, 128, (32, 48, 48), 40, (3, 4, 6), 2, 0, 64),
+    (BF, 128, (32, 48, 48), 3, (2, 5, 7), 1, 0, 16),     # ragged last block (70 = 16*4 + 6)
+    (BF, 64, (16, 24, 24), 5, (4, 3, 3), 3, 0, 8),
+    (BF, 128, (32, 48, 48), 40, (2, 3, 4), 2, 5, 64),    # packed video+audio, explicit positions
+    (torch.float32, 128, (32, 48, 48), 2, (2, 4, 4), 1, 0, 64),
+    (torch.float32, 32, (8, 12, 12), 7, (3, 3, 3), 2, 0, 5),
+]
+
+
+@pytest.mark.parametrize("dtype,head_dim,dims,Hh,grid,B,audio,block", POOL_CASES)
+def test_epilogue_pool(orc, dtype, head_dim, dims, Hh, grid, B, audio, block):
+    w = workloads.Workload("p", 13, dtype, B, grid, audio, 64, Hh, head_dim, 64, rope_dims=dims)
+    pos, _ = workloads.token_layout(w)
+    n, tps, hd = w.n_tokens, w.tokens_per_sample, Hh * head_dim
+    qkv = randn((n, 3 * hd), dtype, 21, std=1.5)
+    wq = randn((head_dim,), dtype, 22, std=0.02, mean=1.0)
+    wk = randn((head_dim,), dtype, 23, std=0.02, mean=1.0)
+    rope = sol.Rope3D(dims, 10000.0, w.max_pos)
+    P = None if pos is None else pos.to(DEV)
+    nb = sol.subblock_count(n, tps, block)
+    pq = torch.full((nb, hd), 99.0, dtype=dtype, device=DEV)
+    pk = torch.full((nb, hd), 99.0, dtype=dtype, device=DEV)
+    common = dict(n_heads=Hh, head_dim=head_dim, wq=wq, wk=wk, pos=P, grid=grid, tokens_per_sample=tps)
+    got = qkv.clone()
+    sol.dit_epilogue_pool(got, pq, pk, rope, block_tokens=block, **common)
+    ref = qkv.clone()
+    sol.dit_epilogue(ref, rope, **common)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref), "the fused pooling changed the epilogue's results"
+    want = orc.dit_epilogue(to_oracle(qkv), to_oracle(wq), to_oracle(wk), n_heads=Hh, head_dim=head_dim,
+                            pos=None if pos is None else pos.numpy(), grid=grid, tokens_per_sample=tps,
+                            dims=dims)
+    wpq = orc.block_mean(want[:, :hd], tokens_per_sample=tps, block=block)
+    wpk = orc.block_mean(want[:, hd:], tokens_per_sample=tps, block=block)
+    assert wpq.shape[0] == nb
+    assert_close(to_f64(pq), wpq, dtype, "pooled q")
+    assert_close(to_f64(pk), wpk, dtype, "pooled k")
+    rope.close()
+
+
+def test_epilogue_pool_full_workload(orc):
+    """fullres_10s in the bench's launch configuration: in-place results equal the plain
+    epilogue's bit for bit; pooled rows of sampled blocks match the oracle's means."""
+    w = workloads.WORKLOADS["fullres_10s"]
+    n, tps, hd, blk = w.n_tokens, w.tokens_per_sample, w.hd, 64
+    qkv = workloads.activation(w, "qkv", n, 3 * w.hd, DEV)
+    wq = workloads.norm_weight(w, "wq", DEV)
+    wk = workloads.norm_weight(w, "wk", DEV)
+    rope = sol.Rope3D(w.rope_dims, w.theta, w.max_pos)
+    nb = sol.subblock_count(n, tps, blk)
+    assert nb == 3843
+    pq = torch.empty((nb, hd), dtype=BF, device=DEV)
+    pk = torch.empty((nb, hd), dtype=BF, device=DEV)
+    common = dict(n_heads=w.n_heads, head_dim=w.head_dim, wq=wq, wk=wk, grid=w.grid, tokens_per_sample=tps)
+    picks = [0, 1, 1000, nb - 1]
+    rows = np.concatenate([np.arange(b * blk, (b + 1) * blk) for b in picks])
+    R = torch.from_numpy(rows).to(DEV)
+    qkv_rows = to_oracle(qkv.index_select(0, R))
+    ref = qkv.clone()
+    sol.dit_epilogue(ref, rope, **common)
+    sol.dit_epilogue_pool(qkv, pq, pk, rope, block_tokens=blk, **common)
+    torch.cuda.synchronize()
+    assert torch.equal(qkv, ref)
+    del ref
+    want = orc.dit_epilogue(qkv_rows, to_oracle(wq), to_oracle(wk), n_heads=w.n_heads, head_dim=w.head_dim,
+                            grid=w.grid, tokens_per_sample=tps, dims=w.rope_dims, rows=rows)
+    for i, b in enumerate(picks):
+        seg = want[i * blk:(i + 1) * blk]
+        assert_close(to_f64(pq[b:b + 1]), seg[:, :hd].mean(axis=0, keepdims=True), BF, f"pooled q {b}")
+        assert_close(to_f64(pk[b:b + 1]), seg[:, hd:].mean(axis=0, keepdims=True), BF, f"pooled k {b}")
+    rope.close()

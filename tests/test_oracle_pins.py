@@ -502,3 +502,32 @@ def test_cache_diff_packed_streams_share_one_decision(oracle_mod):
         np.testing.assert_allclose(sums[b, 1], np.abs(c[blk]).sum(), rtol=1e-13)
     # the audio rows of sample 1 took gate row 3
     np.testing.assert_allclose(r[tps + 6], gate[3] * y[tps + 6], rtol=0, atol=0)
+
+
+# ------------------------------------------------------------- SubBlock block means
+
+
+def test_block_mean_layout_and_ragged_tail(oracle_mod):
+    """A 130-token sample in 64-token blocks gives blocks of 64, 64 and 2 tokens; the
+    next sample starts a new block.  Rows are filled with their token index, so each
+    block mean is the mean of a run of integers (closed form (first + last) / 2)."""
+    tps, B, blk = 130, 2, 64
+    n = B * tps
+    v = np.repeat(np.arange(n, dtype=np.float64)[:, None], 3, axis=1)
+    p = oracle_mod.block_mean(v, tokens_per_sample=tps, block=blk)
+    assert p.shape == (6, 3)
+    starts_ends = [(0, 63), (64, 127), (128, 129), (130, 193), (194, 257), (258, 259)]
+    for row, (a, b) in enumerate(starts_ends):
+        np.testing.assert_array_equal(p[row], (a + b) / 2.0)
+
+
+def test_block_mean_constant_blocks_and_linearity(oracle_mod):
+    n, w = 200, 16
+    base = RNG.standard_normal((4, w))
+    v = np.repeat(base, [64, 64, 64, 8], axis=0)
+    p = oracle_mod.block_mean(v, block=64)
+    np.testing.assert_allclose(p, base, rtol=1e-14)
+    a = RNG.standard_normal((n, w)); b = RNG.standard_normal((n, w))
+    np.testing.assert_allclose(oracle_mod.block_mean(2 * a - b, block=64),
+                               2 * oracle_mod.block_mean(a, block=64) - oracle_mod.block_mean(b, block=64),
+                               rtol=1e-13, atol=1e-14)
