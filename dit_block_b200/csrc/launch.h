@@ -60,8 +60,8 @@ cudaError_t launch_qk_rope_pool(sol_dtype dt, void* q, void* k, int64_t ld_q, in
                                 int32_t block, int64_t bps, int64_t n_blocks, const RopeDev& rope,
                                 int64_t n_tokens, int32_t n_heads, int32_t head_dim, float eps,
                                 cudaStream_t s);
-int qk_pool_vectors_per_lane(sol_dtype dt, int32_t n_heads, int32_t head_dim);
-int qk_pool_max_vectors_per_lane();
+size_t qk_pool_smem_bytes(sol_dtype dt, int32_t n_heads, int32_t head_dim);
+size_t qk_pool_smem_limit();
 
 // Error flags raised on the device by the AdaLN / prologue kernels (bit 0: a bounded
 // wait on a bulk copy gave up); optionally cleared.  Synchronous.

@@ -500,9 +500,9 @@ sol_status sol_dit_epilogue_pool(void* qkv, int64_t ld_qkv, const void* wq, cons
                         head_dim, eps, dt, wq, wk));
     CHECK(block_tokens >= 1 && block_tokens <= (1 << 20), SOL_ERR_INVALID_ARGUMENT,
           "block_tokens (%d) must be in [1, 2^20]", (int)block_tokens);
-    CHECK(sol::qk_pool_vectors_per_lane(dt, n_heads, head_dim) <= sol::qk_pool_max_vectors_per_lane(),
-          SOL_ERR_UNSUPPORTED, "%d heads of %d are more than the pooled epilogue is built for",
-          (int)n_heads, (int)head_dim);
+    CHECK(sol::qk_pool_smem_bytes(dt, n_heads, head_dim) <= sol::qk_pool_smem_limit(), SOL_ERR_UNSUPPORTED,
+          "%d heads of %d need a larger block accumulator than the pooled epilogue holds", (int)n_heads,
+          (int)head_dim);
     if (n_tokens == 0) return SOL_OK;  // nothing to do; empty tensors may be NULL
     const int64_t hd = (int64_t)n_heads * head_dim;
     TRY(check_tensor("qkv", qkv, ld_qkv, 2 * hd, dt, true));

@@ -245,8 +245,8 @@ int64_t sol_subblock_count(int64_t n_tokens, int64_t tokens_per_sample, int32_t 
  *   pooled_q, pooled_k  [sol_subblock_count(...), ld_pool] each; must not overlap
  *                       each other or qkv.
  *   block_tokens        tokens per block (64 on the pages), >= 1.
- * Other arguments as in sol_dit_epilogue; n_heads is limited to what one CTA's warps
- * cover (bf16 head_dim 128: up to 80 heads; f32 head_dim 128: up to 40). */
+ * Other arguments as in sol_dit_epilogue; the per-block fp32 accumulator,
+ * 2 * n_heads * (head_dim + 16) floats, must fit 110 KiB (head_dim 128: up to 95 heads). */
 sol_status sol_dit_epilogue_pool(void* qkv, int64_t ld_qkv, const void* wq, const void* wk,
                                  const int32_t* pos, int32_t grid_T, int32_t grid_H, int32_t grid_W,
                                  int64_t tokens_per_sample, const sol_rope3d* rope, int64_t n_tokens,
