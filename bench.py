@@ -414,6 +414,25 @@ def time_next_ops(bufs, dev, args) -> dict:
     out["dit_epilogue_pool"] = {"ms": round(ms, 4), "bytes_per_token": b, "pooled_bytes": pooled,
                                 "GB_s": round((b * n + pooled) / (ms * 1e-3) / 1e9, 1),
                                 "frac_of_measured_peak": round((b * n + pooled) / (ms * 1e-3) / 1e9 / peak, 4)}
+    del pq, pk
+    # convention variants: q, k of the packed row -> head-major [sample, head, token, dim]
+    tps = w.tokens_per_sample
+    qh = torch.empty((w.batch, w.n_heads, tps, w.head_dim), dtype=w.dtype, device=dev)
+    kh = torch.empty_like(qh)
+    q, k = i["qkv"][:, :w.hd], i["qkv"][:, w.hd:2 * w.hd]
+    wfull = torch.ones((w.hd,), dtype=w.dtype, device=dev)
+    for name, kw in (("qk_ex_head_major_output", dict(wq=i["wq"], wk=i["wk"])),
+                     ("qk_ex_across_heads_rotate_half", dict(wq=wfull, wk=wfull, norm_span=sol.NORM_ACROSS_HEADS,
+                                                             pairing=sol.ROPE_HALF))):
+        fn = lambda: sol.qk_rmsnorm_rope3d_ex(qh, kh, q, k, bufs.rope, n_heads=w.n_heads, head_dim=w.head_dim,
+                                              pos=i["pos"], grid=w.grid, tokens_per_sample=tps, eps=w.eps,
+                                              out_strides=(w.head_dim, tps * w.head_dim,
+                                                           w.n_heads * tps * w.head_dim), **kw)
+        ms = _time(fn, 20, stream)
+        out[name] = {"ms": round(ms, 4), "bytes_per_token": b,
+                     "GB_s": round(b * n / (ms * 1e-3) / 1e9, 1),
+                     "frac_of_measured_peak": round(b * n / (ms * 1e-3) / 1e9 / peak, 4)}
+    del qh, kh
     return out
 
 

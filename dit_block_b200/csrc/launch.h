@@ -19,6 +19,12 @@ struct RopeDev {
     int32_t half[3];
 };
 
+// Element strides of a q/k output: element (token n, head h, dim i) of sample s lives at
+// s * sample + (n - s * tokens_per_sample) * token + h * head + i.
+struct QkOutStrides {
+    int64_t token, head, sample;
+};
+
 // Resident CTAs per SM for `kernel` at `block` threads on the current device (cached).
 int ctas_per_sm(const void* kernel, int block, size_t smem);
 // SM count of the current device (cached).
@@ -52,6 +58,14 @@ cudaError_t launch_qk_rmsnorm_rope3d(sol_dtype dt, void* q_out, void* k_out, int
                                      int32_t grid_W, int64_t tokens_per_sample,
                                      const RopeDev& rope, int64_t n_tokens, int32_t n_heads,
                                      int32_t head_dim, float eps, cudaStream_t s);
+
+// QK RMSNorm + 3D RoPE, convention variants (k_qk_ex.cu): `across` = RMS over all heads
+// with weights [n_heads * head_dim]; `half` = rotate-half pairs; any output strides.
+cudaError_t launch_qk_ex(sol_dtype dt, bool across, bool half, void* q_out, void* k_out,
+                         const QkOutStrides& os, const void* q, const void* k, int64_t ld_q, int64_t ld_k,
+                         const void* wq, const void* wk, const int32_t* pos, int32_t grid_H, int32_t grid_W,
+                         int64_t tps, const RopeDev& rope, int64_t n_tokens, int32_t n_heads,
+                         int32_t head_dim, float eps, cudaStream_t s);
 
 // QKV epilogue fused with SubBlock block means (k_qk_pool.cu).  In place on q and k.
 cudaError_t launch_qk_rope_pool(sol_dtype dt, void* q, void* k, int64_t ld_q, int64_t ld_k, void* pq,

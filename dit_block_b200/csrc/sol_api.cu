@@ -448,6 +448,60 @@ sol_status sol_qk_rmsnorm_rope3d(void* q_out, void* k_out, int64_t ld_qo, int64_
                        "sol_qk_rmsnorm_rope3d launch");
 }
 
+sol_status sol_qk_rmsnorm_rope3d_ex(const sol_qk_desc* d, sol_stream_t stream)
+{
+    CHECK(d, SOL_ERR_INVALID_ARGUMENT, "desc is NULL");
+    TRY(check_qk_common(d->rope, d->pos, d->grid_T, d->grid_H, d->grid_W, d->tokens_per_sample, d->n_tokens,
+                        d->n_heads, d->head_dim, d->eps, d->dt, d->wq, d->wk));
+    CHECK(d->norm_span == SOL_NORM_PER_HEAD || d->norm_span == SOL_NORM_ACROSS_HEADS, SOL_ERR_INVALID_ARGUMENT,
+          "norm_span %d is not a sol_norm_span", (int)d->norm_span);
+    CHECK(d->rope_pairing == SOL_ROPE_INTERLEAVED || d->rope_pairing == SOL_ROPE_HALF, SOL_ERR_INVALID_ARGUMENT,
+          "rope_pairing %d is not a sol_rope_pairing", (int)d->rope_pairing);
+    const int e16 = elems16(d->dt);
+    if (d->rope_pairing == SOL_ROPE_HALF)
+        for (int c = 0; c < 3; ++c)
+            CHECK(d->rope->dims[c] % (2 * e16) == 0, SOL_ERR_UNSUPPORTED,
+                  "rotate-half pairing needs chunk widths that are multiples of %d (chunk %d is %d)", 2 * e16, c,
+                  (int)d->rope->dims[c]);
+    const int64_t ts = d->out_token_stride, hs = d->out_head_stride, ss = d->out_sample_stride;
+    CHECK(ts > 0 && hs > 0 && ss >= 0, SOL_ERR_INVALID_ARGUMENT, "output strides must be positive");
+    CHECK(ts % e16 == 0 && hs % e16 == 0 && ss % e16 == 0, SOL_ERR_MISALIGNED,
+          "output strides must be multiples of %d elements", e16);
+    if (d->n_tokens == 0) return SOL_OK;  // nothing to do; empty tensors may be NULL
+    const int64_t hd = (int64_t)d->n_heads * d->head_dim;
+    TRY(check_tensor("q", d->q, d->ld_q, hd, d->dt, true));
+    TRY(check_tensor("k", d->k, d->ld_k, hd, d->dt, true));
+    CHECK(d->q_out && d->k_out, SOL_ERR_INVALID_ARGUMENT, "q_out or k_out is NULL");
+    CHECK(aligned16(d->q_out) && aligned16(d->k_out), SOL_ERR_MISALIGNED, "q_out or k_out is not 16-byte aligned");
+    // extent of an output: the farthest element it addresses, plus one
+    const int64_t tps = d->tokens_per_sample > 0 ? d->tokens_per_sample : d->n_tokens;
+    const int64_t n_samples = (d->n_tokens + tps - 1) / tps;
+    const int64_t last_local = d->n_tokens <= tps ? d->n_tokens - 1 : tps - 1;
+    const int64_t extent = (n_samples - 1) * ss + last_local * ts + (int64_t)(d->n_heads - 1) * hs + d->head_dim;
+    const size_t es = esize(d->dt);
+    auto range_overlap = [&](const void* a, int64_t na, const void* b, int64_t nb) {
+        const char* a0 = (const char*)a;
+        const char* b0 = (const char*)b;
+        return a0 < b0 + nb * (int64_t)es && b0 < a0 + na * (int64_t)es;
+    };
+    const int64_t in_q = (d->n_tokens - 1) * d->ld_q + hd, in_k = (d->n_tokens - 1) * d->ld_k + hd;
+    const bool token_major_q = ts == d->ld_q && hs == d->head_dim && (ss == tps * d->ld_q || n_samples == 1);
+    const bool token_major_k = ts == d->ld_k && hs == d->head_dim && (ss == tps * d->ld_k || n_samples == 1);
+    CHECK(d->q_out == d->q ? token_major_q : !range_overlap(d->q_out, extent, d->q, in_q) && !range_overlap(d->q_out, extent, d->k, in_k),
+          SOL_ERR_INVALID_ARGUMENT, "q_out overlaps the inputs other than as q itself with q's layout");
+    CHECK(d->k_out == d->k ? token_major_k : !range_overlap(d->k_out, extent, d->k, in_k) && !range_overlap(d->k_out, extent, d->q, in_q),
+          SOL_ERR_INVALID_ARGUMENT, "k_out overlaps the inputs other than as k itself with k's layout");
+    CHECK(!range_overlap(d->q_out, extent, d->k_out, extent) || (d->q_out == d->q && d->k_out == d->k),
+          SOL_ERR_INVALID_ARGUMENT, "q_out and k_out overlap");
+    const sol::QkOutStrides os{ts, hs, ss};
+    return cuda_status(sol::launch_qk_ex(d->dt, d->norm_span == SOL_NORM_ACROSS_HEADS,
+                                         d->rope_pairing == SOL_ROPE_HALF, d->q_out, d->k_out, os, d->q, d->k,
+                                         d->ld_q, d->ld_k, d->wq, d->wk, d->pos, d->grid_H, d->grid_W,
+                                         d->tokens_per_sample, d->rope->view, d->n_tokens, d->n_heads,
+                                         d->head_dim, d->eps, (cudaStream_t)stream),
+                       "sol_qk_rmsnorm_rope3d_ex launch");
+}
+
 sol_status sol_dit_prologue(void* x_out, void* h, const void* x, const void* y,
                             const void* gate, const void* shift, const void* scale, int64_t ld,
                             int64_t ld_mod, sol_modsel sel, int64_t n_tokens, int64_t d,

@@ -35,6 +35,20 @@ class ModSel(ctypes.Structure):
 
 
 _P, _I64, _I32, _F, _D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_double
+
+
+class QkDesc(ctypes.Structure):
+    """sol_qk_desc (include/sol.h)."""
+    _fields_ = [("q_out", _P), ("k_out", _P), ("out_token_stride", _I64), ("out_head_stride", _I64),
+                ("out_sample_stride", _I64), ("q", _P), ("k", _P), ("ld_q", _I64), ("ld_k", _I64),
+                ("wq", _P), ("wk", _P), ("pos", _P), ("grid_T", _I32), ("grid_H", _I32), ("grid_W", _I32),
+                ("tokens_per_sample", _I64), ("rope", _P), ("n_tokens", _I64), ("n_heads", _I32),
+                ("head_dim", _I32), ("eps", _F), ("norm_span", _I32), ("rope_pairing", _I32),
+                ("dt", ctypes.c_int)]
+
+
+NORM_PER_HEAD, NORM_ACROSS_HEADS = 0, 1
+ROPE_INTERLEAVED, ROPE_HALF = 0, 1
 _E = ctypes.c_int  # enums
 
 # argument types per exported function, in header order
@@ -56,6 +70,7 @@ SIGNATURES = {
     "sol_dit_epilogue": ([_P, _I64, _P, _P, _P, _I32, _I32, _I32, _I64, _P, _I64, _I32, _I32, _F,
                           _E, _P], _E),
     "sol_subblock_count": ([_I64, _I64, _I32], _I64),
+    "sol_qk_rmsnorm_rope3d_ex": ([ctypes.POINTER(QkDesc), _P], _E),
     "sol_dit_epilogue_pool": ([_P, _I64, _P, _P, _P, _I32, _I32, _I32, _I64, _P, _I64, _I32, _I32, _F,
                                _P, _P, _I64, _I32, _E, _P], _E),
     "sol_qk_rmsnorm_rope3d_noalloc": ([_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _P, _P, _I32, _I32,
@@ -315,3 +330,23 @@ def dit_epilogue_pool(qkv, pooled_q, pooled_k, rope: Rope3D, *, n_heads, head_di
         int(tokens_per_sample), rope.handle, qkv.shape[0], int(n_heads), int(head_dim), eps,
         _ptr(pooled_q), _ptr(pooled_k), _ld(pooled_q), int(block_tokens), _dtype(qkv), _stream(stream)),
         "sol_dit_epilogue_pool")
+
+
+def qk_rmsnorm_rope3d_ex(q_out, k_out, q, k, rope: Rope3D, *, n_heads, head_dim, wq=None, wk=None, pos=None,
+                         grid=(0, 0, 0), tokens_per_sample=0, eps=1e-6, norm_span=NORM_PER_HEAD,
+                         pairing=ROPE_INTERLEAVED, out_strides=None, stream=None):
+    """sol_qk_rmsnorm_rope3d_ex.  out_strides = (token, head, sample) element strides of
+    q_out and k_out (default: token-major rows like q_out's).  q_out / k_out are passed as
+    base pointers (tensors of any shape)."""
+    if pos is not None and (pos.dtype != torch.int32 or not pos.is_contiguous()):
+        raise TypeError("pos must be a contiguous int32 [N, 3] tensor")
+    n = q.shape[0]
+    if out_strides is None:
+        ld = _ld(q_out)
+        tps = tokens_per_sample if tokens_per_sample > 0 else n
+        out_strides = (ld, head_dim, tps * ld)
+    d = QkDesc(_ptr(q_out), _ptr(k_out), int(out_strides[0]), int(out_strides[1]), int(out_strides[2]),
+               _ptr(q), _ptr(k), _ld(q), _ld(k), _ptr(wq), _ptr(wk), _ptr(pos), int(grid[0]), int(grid[1]),
+               int(grid[2]), int(tokens_per_sample), rope.handle, n, int(n_heads), int(head_dim), float(eps),
+               int(norm_span), int(pairing), _dtype(q))
+    _check(lib().sol_qk_rmsnorm_rope3d_ex(ctypes.byref(d), _stream(stream)), "sol_qk_rmsnorm_rope3d_ex")

@@ -188,6 +188,50 @@ sol_status sol_qk_rmsnorm_rope3d(void* q_out, void* k_out, int64_t ld_qo, int64_
                                  int64_t n_tokens, int32_t n_heads, int32_t head_dim,
                                  float eps, sol_dtype dt, sol_stream_t stream);
 
+/* QK RMSNorm + 3D RoPE in the other conventions the pages leave open, and with outputs
+ * at any (token, head, sample) strides -- e.g. straight into an attention-friendly
+ * [sample, head, token, dim] layout.
+ *   norm_span     SOL_NORM_PER_HEAD: RMS over each head vector, weights [head_dim] (as
+ *                 sol_qk_rmsnorm_rope3d);  SOL_NORM_ACROSS_HEADS: RMS over all
+ *                 n_heads * head_dim elements of the row, weights [n_heads * head_dim].
+ *   rope_pairing  SOL_ROPE_INTERLEAVED: pairs (2j, 2j+1) inside each axis chunk (as
+ *                 sol_qk_rmsnorm_rope3d);  SOL_ROPE_HALF: pairs (j, j + D_c/2), angle
+ *                 p_c * theta^(-2j/D_c); needs every chunk width to be a multiple of 16
+ *                 (bf16) or 8 (f32).
+ *   Outputs       element (token n, head h, dim i) of q (k) goes to
+ *                     q_out[s * out_sample_stride + (n - s * tokens_per_sample) * out_token_stride
+ *                           + h * out_head_stride + i],   s = n / tokens_per_sample
+ *                 (s = 0 when tokens_per_sample is 0).  Strides are in elements, multiples
+ *                 of 8 (bf16) / 4 (f32).  Token-major rows: token = ld, head = head_dim,
+ *                 sample = tokens_per_sample * ld.  Head-major [S, H, N, D]: token =
+ *                 head_dim, head = N * head_dim, sample = H * N * head_dim.  An output may
+ *                 equal its input only with the input's own token-major strides; otherwise
+ *                 outputs must not overlap the inputs.
+ *   Other fields as in sol_qk_rmsnorm_rope3d. */
+typedef enum { SOL_NORM_PER_HEAD = 0, SOL_NORM_ACROSS_HEADS = 1 } sol_norm_span;
+typedef enum { SOL_ROPE_INTERLEAVED = 0, SOL_ROPE_HALF = 1 } sol_rope_pairing;
+typedef struct {
+    void* q_out;
+    void* k_out;
+    int64_t out_token_stride, out_head_stride, out_sample_stride;
+    const void* q;
+    const void* k;
+    int64_t ld_q, ld_k;
+    const void* wq;
+    const void* wk;
+    const int32_t* pos;
+    int32_t grid_T, grid_H, grid_W;
+    int64_t tokens_per_sample;
+    const sol_rope3d* rope;
+    int64_t n_tokens;
+    int32_t n_heads, head_dim;
+    float eps;
+    int32_t norm_span;    /* sol_norm_span */
+    int32_t rope_pairing; /* sol_rope_pairing */
+    sol_dtype dt;
+} sol_qk_desc;
+sol_status sol_qk_rmsnorm_rope3d_ex(const sol_qk_desc* desc, sol_stream_t stream);
+
 /* Fused block prologue [STM-RES: one pass instead of two, same math]:
  *     x'_i = x_i + gate[r]_i * y_i             (skipped when y == NULL: x' = x)
  *     h_i  = AdaLN(x')_i  as in sol_adaln_modulate, on the UNROUNDED fp32 x'.

@@ -54,6 +54,9 @@ def _load():
         lib.oracle_gated_residual_cache_diff.argtypes = [P, P, P, I64, P, I64, P, I64, I, P, I64, I,
                                                          P, I64, I, P, I32, I64, P, I64, I64]
         lib.oracle_gated_residual_cache_diff.restype = None
+        lib.oracle_qk_rmsnorm_rope3d_ex.argtypes = [P, P, P, P, I64, I64, I, P, P, I, P, I32, I32, I32,
+                                                    I64, I32, I32, I32, D, P, I64, I32, I32, D, I, I]
+        lib.oracle_qk_rmsnorm_rope3d_ex.restype = I
         lib.oracle_block_mean.argtypes = [P, P, I64, I64, I64, I64]
         lib.oracle_block_mean.restype = I64
         lib.oracle_swiglu.argtypes = [P, I64, P, P, I64, I, I64, I64]
@@ -269,3 +272,31 @@ def block_mean(v, *, tokens_per_sample=0, block=64):
     got = _load().oracle_block_mean(out.ctypes.data, v.ctypes.data, n, width, int(tokens_per_sample),
                                     int(block))
     return out[:got]
+
+
+NORM_PER_HEAD, NORM_ACROSS_HEADS = 0, 1
+ROPE_INTERLEAVED, ROPE_HALF = 0, 1
+
+
+def qk_rmsnorm_rope3d_ex(q, k, wq=None, wk=None, *, n_heads, head_dim, pos=None, grid=(0, 0, 0),
+                         tokens_per_sample=0, dims=(32, 48, 48), theta=10000.0, eps=1e-6, rows=None,
+                         norm_span=NORM_PER_HEAD, pairing=ROPE_INTERLEAVED):
+    """QK RMSNorm + 3D RoPE with a choice of norm span (per head, or across all heads with
+    weights [n_heads*head_dim]) and rotary pairing (interleaved, or rotate-half).  Returns
+    token-major (q_out, k_out) float64 arrays."""
+    src = q if q is not None else k
+    n = src.shape[0]
+    hd = n_heads * head_dim
+    qo = np.empty((n, hd), np.float64) if q is not None else None
+    ko = np.empty((n, hd), np.float64) if k is not None else None
+    w = wq if wq is not None else wk
+    pos_arr, pos_p = _pos_ptr(pos)
+    rw = _rows(rows, n)
+    rc = _load().oracle_qk_rmsnorm_rope3d_ex(
+        _ptr(qo), _ptr(ko), _ptr(q), _ptr(k), _ld(q) if q is not None else 0, _ld(k) if k is not None else 0,
+        _code(src), _ptr(wq), _ptr(wk), _code(w), pos_p, int(grid[0]), int(grid[1]), int(grid[2]),
+        int(tokens_per_sample), int(dims[0]), int(dims[1]), int(dims[2]), float(theta), _ptr(rw), n,
+        int(n_heads), int(head_dim), float(eps), int(norm_span), int(pairing))
+    if rc != 0:
+        raise ValueError("RoPE split does not fit head_dim (dims must be even and sum to it)")
+    return qo, ko

@@ -340,3 +340,86 @@ int64_t oracle_block_mean(double* pooled, const double* v, int64_t n_tokens, int
     }
     return written;
 }
+
+/* Convention variants of QK RMSNorm + 3D RoPE (the pages fix neither the norm span nor
+ * the rotary pairing; these are the other plausible readings).
+ *   norm_span 0: RMS over each head vector, weights [head_dim] (oracle_qk_rmsnorm_rope3d);
+ *   norm_span 1: RMS over all n_heads * head_dim elements of the row, weights
+ *                [n_heads * head_dim].
+ *   pairing 0: interleaved pairs (2j, 2j+1) inside each axis chunk;
+ *   pairing 1: rotate-half pairs (j, j + D_c/2) inside each axis chunk, turned by
+ *              phi = p_c * theta^(-2j / D_c), j < D_c / 2.
+ * Outputs are token-major [n_tokens, n_heads * head_dim]. */
+static void norm_rope_row_ex(double* out, const void* in, int64_t in_off, int dt, const void* w,
+                             int dt_w, int32_t n_heads, int32_t head_dim, double eps,
+                             const int64_t p[3], const int32_t dims[3], double theta,
+                             int norm_span, int pairing)
+{
+    const int64_t hd = (int64_t)n_heads * head_dim;
+    double full_inv = 0.0;
+    if (norm_span == 1) {
+        double ms = 0.0;
+        for (int64_t i = 0; i < hd; ++i) {
+            const double v = load(in, dt, in_off + i);
+            ms += v * v;
+        }
+        full_inv = 1.0 / sqrt(ms / (double)hd + eps);
+    }
+    double vn[1024];
+    for (int32_t h = 0; h < n_heads; ++h) {
+        const int64_t base = (int64_t)h * head_dim;
+        double inv = full_inv;
+        if (norm_span == 0) {
+            double ms = 0.0;
+            for (int32_t i = 0; i < head_dim; ++i) {
+                const double v = load(in, dt, in_off + base + i);
+                ms += v * v;
+            }
+            inv = 1.0 / sqrt(ms / (double)head_dim + eps);
+        }
+        for (int32_t i = 0; i < head_dim; ++i) {
+            const int64_t wi = norm_span == 1 ? base + i : i;
+            vn[i] = load(in, dt, in_off + base + i) * inv * (w ? load(w, dt_w, wi) : 1.0);
+        }
+        int32_t off = 0;
+        for (int c = 0; c < 3; ++c) {
+            const int32_t D = dims[c];
+            for (int32_t j = 0; j < D / 2; ++j) {
+                const double phi = (double)p[c] * pow(theta, -2.0 * (double)j / (double)D);
+                const double cs = cos(phi), sn = sin(phi);
+                const int32_t a = pairing == 1 ? off + j : off + 2 * j;
+                const int32_t b = pairing == 1 ? off + j + D / 2 : off + 2 * j + 1;
+                const double u = vn[a], v = vn[b];
+                out[base + a] = u * cs - v * sn;
+                out[base + b] = u * sn + v * cs;
+            }
+            off += D;
+        }
+    }
+}
+
+int oracle_qk_rmsnorm_rope3d_ex(double* q_out, double* k_out, const void* q, const void* k,
+                                int64_t ld_q, int64_t ld_k, int dt, const void* wq, const void* wk,
+                                int dt_w, const int32_t* pos, int32_t grid_T, int32_t grid_H,
+                                int32_t grid_W, int64_t tokens_per_sample, int32_t dim_t,
+                                int32_t dim_h, int32_t dim_w, double theta, const int64_t* rows,
+                                int64_t n_tokens, int32_t n_heads, int32_t head_dim, double eps,
+                                int norm_span, int pairing)
+{
+    const int32_t dims[3] = {dim_t, dim_h, dim_w};
+    if (dim_t + dim_h + dim_w != head_dim || (dim_t | dim_h | dim_w) & 1 || head_dim > 1024)
+        return -1;
+    const int64_t hd = (int64_t)n_heads * head_dim;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < n_tokens; ++n) {
+        int64_t p[3];
+        token_position(rows ? rows[n] : n, pos, grid_T, grid_H, grid_W, tokens_per_sample, p);
+        if (q)
+            norm_rope_row_ex(q_out + n * hd, q, n * ld_q, dt, wq, dt_w, n_heads, head_dim, eps, p, dims,
+                             theta, norm_span, pairing);
+        if (k)
+            norm_rope_row_ex(k_out + n * hd, k, n * ld_k, dt, wk, dt_w, n_heads, head_dim, eps, p, dims,
+                             theta, norm_span, pairing);
+    }
+    return 0;
+}

@@ -231,3 +231,77 @@ def test_epilogue_pool_full_workload(orc):
         assert_close(to_f64(pq[b:b + 1]), seg[:, :hd].mean(axis=0, keepdims=True), BF, f"pooled q {b}")
         assert_close(to_f64(pk[b:b + 1]), seg[:, hd:].mean(axis=0, keepdims=True), BF, f"pooled k {b}")
     rope.close()
+
+
+# ------------------------------------------------- convention variants and output layouts
+
+EX_CASES = [  # dtype, head_dim, dims, n_heads, grid, samples
+    (BF, 128, (32, 48, 48), 40, (3, 4, 5), 2),
+    (BF, 64, (16, 16, 32), 5, (4, 3, 3), 3),
+    (torch.float32, 128, (32, 48, 48), 3, (2, 4, 4), 1),
+    (torch.float32, 32, (8, 8, 16), 7, (3, 3, 3), 2),
+]
+
+
+@pytest.mark.parametrize("dtype,head_dim,dims,Hh,grid,B", EX_CASES)
+@pytest.mark.parametrize("span", [sol.NORM_PER_HEAD, sol.NORM_ACROSS_HEADS])
+@pytest.mark.parametrize("pairing", [sol.ROPE_INTERLEAVED, sol.ROPE_HALF])
+def test_qk_ex_conventions_and_layouts(orc, dtype, head_dim, dims, Hh, grid, B, span, pairing):
+    T, H, W = grid
+    tps = T * H * W
+    n, hd = B * tps, Hh * head_dim
+    qkv = randn((n, 3 * hd), dtype, 31, std=1.5)
+    wlen = hd if span == sol.NORM_ACROSS_HEADS else head_dim
+    wq = randn((wlen,), dtype, 32, std=0.02, mean=1.0)
+    wk = randn((wlen,), dtype, 33, std=0.02, mean=1.0)
+    rope = sol.Rope3D(dims, 10000.0, (T + 1, H + 2, W))
+    q, k = qkv[:, :hd], qkv[:, hd:2 * hd]
+    common = dict(n_heads=Hh, head_dim=head_dim, wq=wq, wk=wk, grid=grid, tokens_per_sample=tps,
+                  norm_span=span, pairing=pairing)
+    # token-major, out of place
+    qo, ko = torch.empty((n, hd), dtype=dtype, device=DEV), torch.empty((n, hd), dtype=dtype, device=DEV)
+    sol.qk_rmsnorm_rope3d_ex(qo, ko, q, k, rope, **common)
+    # head-major [B, Hh, N, D] for attention
+    qh = torch.empty((B, Hh, tps, head_dim), dtype=dtype, device=DEV)
+    kh = torch.empty_like(qh)
+    sol.qk_rmsnorm_rope3d_ex(qh, kh, q, k, rope, out_strides=(head_dim, tps * head_dim, Hh * tps * head_dim),
+                             **common)
+    # token-major in place on the packed row
+    inplace = qkv.clone()
+    sol.qk_rmsnorm_rope3d_ex(inplace[:, :hd], inplace[:, hd:2 * hd], inplace[:, :hd], inplace[:, hd:2 * hd],
+                             rope, **common)
+    torch.cuda.synchronize()
+    wq_o, wk_o = orc.qk_rmsnorm_rope3d_ex(to_oracle(q.contiguous()), to_oracle(k.contiguous()), to_oracle(wq),
+                                          to_oracle(wk), n_heads=Hh, head_dim=head_dim, grid=grid,
+                                          tokens_per_sample=tps, dims=dims, norm_span=span, pairing=pairing)
+    assert_close(to_f64(qo), wq_o, dtype, "q")
+    assert_close(to_f64(ko), wk_o, dtype, "k")
+    assert torch.equal(qh.permute(0, 2, 1, 3).reshape(n, hd), qo)
+    assert torch.equal(kh.permute(0, 2, 1, 3).reshape(n, hd), ko)
+    assert torch.equal(inplace[:, :hd], qo) and torch.equal(inplace[:, hd:2 * hd], ko)
+    assert torch.equal(inplace[:, 2 * hd:], qkv[:, 2 * hd:])
+    if span == sol.NORM_PER_HEAD and pairing == sol.ROPE_INTERLEAVED:
+        q2, k2 = torch.empty_like(qo), torch.empty_like(ko)
+        sol.qk_rmsnorm_rope3d(q2, k2, q, k, rope, n_heads=Hh, head_dim=head_dim, wq=wq, wk=wk, grid=grid,
+                              tokens_per_sample=tps)
+        torch.cuda.synchronize()
+        assert torch.equal(q2, qo) and torch.equal(k2, ko)
+    rope.close()
+
+
+def test_qk_ex_rejects_bad_layouts():
+    rope = sol.Rope3D((32, 48, 48), 10000.0, (4, 4, 4))
+    q = randn((8, 128), BF, 1)
+    with pytest.raises(sol.SolError) as e:  # rotate-half needs chunks that are multiples of 16
+        r2 = sol.Rope3D((40, 40, 48), 10000.0, (4, 4, 4))
+        try:
+            sol.qk_rmsnorm_rope3d_ex(torch.empty_like(q), torch.empty_like(q), q, q.clone(), r2, n_heads=1,
+                                     head_dim=128, grid=(2, 2, 2), tokens_per_sample=8, pairing=sol.ROPE_HALF)
+        finally:
+            r2.close()
+    assert e.value.status == sol.ERR_UNSUPPORTED
+    with pytest.raises(sol.SolError) as e:  # an output overlapping the inputs in another layout
+        sol.qk_rmsnorm_rope3d_ex(q, torch.empty_like(q), q, q.clone(), rope, n_heads=1, head_dim=128,
+                                 grid=(2, 2, 2), tokens_per_sample=8, out_strides=(256, 128, 0))
+    assert e.value.status == sol.ERR_INVALID_ARGUMENT
+    rope.close()

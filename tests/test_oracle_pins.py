@@ -531,3 +531,79 @@ def test_block_mean_constant_blocks_and_linearity(oracle_mod):
     np.testing.assert_allclose(oracle_mod.block_mean(2 * a - b, block=64),
                                2 * oracle_mod.block_mean(a, block=64) - oracle_mod.block_mean(b, block=64),
                                rtol=1e-13, atol=1e-14)
+
+
+# ------------------------------------------------- convention variants (norm span, pairing)
+
+
+def _qkx(oracle_mod, v, w=None, pos=None, eps=1e-6, n_heads=1, head_dim=128, **kw):
+    qo, _ = oracle_mod.qk_rmsnorm_rope3d_ex(v, None, w, None, n_heads=n_heads, head_dim=head_dim, pos=pos,
+                                            eps=eps, **kw)
+    return qo
+
+
+def test_ex_defaults_equal_the_base_oracle(oracle_mod):
+    v = RNG.standard_normal((5, 3 * 128)); w = 1 + 0.02 * RNG.standard_normal(128)
+    pos = RNG.integers(0, 40, size=(5, 3)).astype(np.int32)
+    np.testing.assert_array_equal(_qkx(oracle_mod, v, w, pos, n_heads=3), _qk(oracle_mod, v, w, pos, n_heads=3))
+
+
+def test_rope_half_golden_angles(oracle_mod):
+    g = read_golden("rope3d_half_angles.txt")
+    axis_of = {"t": 0, "h": 1, "w": 2}
+    for axis, off, D, j, p, angle in g[None]:
+        off, D, j, p, angle = int(off), int(D), int(j), int(p), float(angle)
+        v = np.zeros((1, 128)); v[0, off + j] = 1.0
+        pos = np.zeros((1, 3), np.int32); pos[0, axis_of[axis]] = p
+        out = _qkx(oracle_mod, v, None, pos, eps=0.0, pairing=oracle_mod.ROPE_HALF)[0]
+        r = math.sqrt(128.0)
+        assert abs(out[off + j] - r * math.cos(angle)) < 1e-12
+        assert abs(out[off + j + D // 2] - r * math.sin(angle)) < 1e-12
+        assert np.all(np.delete(out, [off + j, off + j + D // 2]) == 0.0)
+
+
+def _half_to_interleaved_perm(dims=(32, 48, 48)):
+    """Index map: interleaved position 2j (2j+1) of a chunk holds rotate-half element j (j+D/2)."""
+    perm = []
+    off = 0
+    for D in dims:
+        for j in range(D // 2):
+            perm += [off + j, off + j + D // 2]
+        off += D
+    return np.array(perm)
+
+
+def test_rope_half_is_interleaved_in_permuted_coordinates(oracle_mod):
+    """rotate-half(x) = P^T interleaved(P x), P the permutation pairing (j, j + D/2) as (2j, 2j+1)."""
+    perm = _half_to_interleaved_perm()
+    v = RNG.standard_normal((7, 128))
+    pos = RNG.integers(0, 60, size=(7, 3)).astype(np.int32)
+    half = _qkx(oracle_mod, v, None, pos, eps=0.0, pairing=oracle_mod.ROPE_HALF)
+    inter = _qkx(oracle_mod, np.ascontiguousarray(v[:, perm]), None, pos, eps=0.0)
+    back = np.empty_like(inter); back[:, perm] = inter
+    np.testing.assert_allclose(half, back, rtol=1e-13, atol=1e-13)
+
+
+def test_rope_half_relative_positions(oracle_mod):
+    q = RNG.standard_normal((1, 128)); k = RNG.standard_normal((1, 128))
+    m = np.array([[4, 9, 2]], np.int32); nn = np.array([[1, 3, 30]], np.int32)
+    f = lambda v, p: _qkx(oracle_mod, v, None, p, eps=0.0, pairing=oracle_mod.ROPE_HALF)
+    ref = (f(q, m) @ f(k, nn).T).item()
+    for c in ([0, 0, 7], [11, 0, 0], [5, 6, 40]):
+        c = np.array([c], np.int32)
+        assert abs((f(q, m + c) @ f(k, nn + c).T).item() - ref) < 1e-11
+
+
+def test_norm_across_heads_is_torch_rms_norm_over_the_row(oracle_mod):
+    n, Hh, Dh = 4, 3, 128
+    v = RNG.standard_normal((n, Hh * Dh)) * np.array([[0.5], [1], [3], [20]])
+    w = 1 + 0.02 * RNG.standard_normal(Hh * Dh)
+    out = _qkx(oracle_mod, v, w, np.zeros((n, 3), np.int32), n_heads=Hh,
+               norm_span=oracle_mod.NORM_ACROSS_HEADS)
+    ref = F.rms_norm(torch.from_numpy(v), (Hh * Dh,), weight=torch.from_numpy(w), eps=1e-6).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    # and it differs from the per-head span when heads have different scales
+    v2 = v.copy(); v2[:, :Dh] *= 10
+    a = _qkx(oracle_mod, v2, None, np.zeros((n, 3), np.int32), n_heads=Hh, norm_span=oracle_mod.NORM_ACROSS_HEADS)
+    b = _qkx(oracle_mod, v2, None, np.zeros((n, 3), np.int32), n_heads=Hh)
+    assert not np.allclose(a, b)
