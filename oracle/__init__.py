@@ -4,13 +4,16 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU baseline and
 reference arm may import this package.  The product library (``dit_block_b200``)
 never imports it and shares no code with it.
 
-The arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP over rows); this module
-only marshals numpy arrays into it.  Inputs are numpy arrays of ``float32``,
+The per-token arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP over rows); this
+module marshals numpy arrays into it, and composes it with fp64 numpy matmuls for the
+linear-layer fusions at its end.  Inputs are numpy arrays of ``float32``,
 ``float64`` or ``uint16`` (the raw bits of bf16 values); every output is ``float64``.
 Each function names the operator it computes; the definitions and the page passages
 they follow are in the header of ``oracle.c``.
 
-Parity status: every function is pinned by ``tests/test_oracle_pins.py``.
+Parity status: every function is pinned: the per-token operators by
+``tests/test_oracle_pins.py``, the linear-layer compositions at the end of this module
+by ``tests/test_oracle_linear_pins.py``.
 """
 from __future__ import annotations
 
@@ -300,3 +303,84 @@ def qk_rmsnorm_rope3d_ex(q, k, wq=None, wk=None, *, n_heads, head_dim, pos=None,
     if rc != 0:
         raise ValueError("RoPE split does not fit head_dim (dims must be even and sum to it)")
     return qo, ko
+
+
+# ---------------------------------------------------------------------------------------
+# The per-token operators fused into the block's linear layers.
+#
+# [STM-RES] (section "Resultado principal") credits the fused kernels with cutting
+# memory traffic, intermediate tensors and launches without changing the math.  The
+# per-token operators sit between the DiT block's linear layers: AdaLN feeds the QKV
+# projection, QK RMSNorm + 3D RoPE follows it, the gated residual follows the output
+# projection and the MLP down projection, and SwiGLU follows the MLP up projection.
+# Each function below is the composition, in fp64 with no intermediate rounding, of
+# a linear layer y = a . W^T (W stored [out_features, in_features], the usual linear-
+# layer layout; no bias) with the oracle operator on its input or output side.  The
+# product a . W^T is one numpy fp64 matmul (a library primitive used as one step).
+# ---------------------------------------------------------------------------------------
+
+def to_f64(a: np.ndarray) -> np.ndarray:
+    """Exact widening of float32 / float64 / uint16 (bf16 bits) to float64."""
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if a.dtype in (np.float32, np.float64):
+        return a.astype(np.float64)
+    raise TypeError(f"oracle inputs are float32, float64 or uint16 (bf16 bits), got {a.dtype}")
+
+
+def linear(a, w):
+    """y = a . W^T: a [N, K], W [out, K] -> [N, out] float64."""
+    a64, w64 = to_f64(a), to_f64(w)
+    assert a64.shape[1] == w64.shape[1], "a and W must share the inner dimension"
+    return a64 @ w64.T
+
+
+def linear_magnitude(a, w):
+    """|a| . |W|^T: the sum of |a_k W_jk| behind each output of linear(a, W) (an error-
+    bound helper: rounding the operands or the partial sums moves y by at most a small
+    multiple of this)."""
+    return np.abs(to_f64(a)) @ np.abs(to_f64(w)).T
+
+
+def linear_gated_residual(x, a, w, gate=None, *, stream_id=None, n_streams=1,
+                          tokens_per_sample=0, rows=None):
+    """out = x + gate[r] * (a . W^T): the gated residual on the output projection (or the
+    MLP down projection)."""
+    y = np.ascontiguousarray(linear(a, w))
+    return gated_residual(to_f64(x), y, gate, stream_id=stream_id, n_streams=n_streams,
+                          tokens_per_sample=tokens_per_sample, rows=rows)
+
+
+def linear_swiglu(a, w, inner=None):
+    """out = silu(a . W1^T) * (a . W2^T) with W = [W1; W2] ([2*inner, K]): SwiGLU on the MLP
+    up projection, whose first `inner` outputs are the gated half."""
+    u = np.ascontiguousarray(linear(a, w))
+    return swiglu(u, inner)
+
+
+def adaln_linear(x, w, shift=None, scale=None, *, eps=1e-6, stream_id=None, n_streams=1,
+                 tokens_per_sample=0, rows=None):
+    """y = AdaLN(x) . W^T, AdaLN(x) = LN(x) * (1 + scale[r]) + shift[r].  Returns (y, h) with
+    h = AdaLN(x) in float64 (the exact operand of the product)."""
+    h = adaln_modulate(x, shift, scale, eps=eps, stream_id=stream_id, n_streams=n_streams,
+                       tokens_per_sample=tokens_per_sample, rows=rows)
+    return linear(h, w), h
+
+
+def adaln_qkv_rope(x, w, shift=None, scale=None, wq=None, wk=None, *, n_heads, head_dim,
+                   pos=None, grid=(0, 0, 0), tokens_per_sample=0, dims=(32, 48, 48),
+                   theta=10000.0, eps=1e-6, stream_id=None, n_streams=1, rows=None):
+    """The attention input of a block: qkv = AdaLN(x) . W^T ([N, 3*n_heads*head_dim], q | k | v),
+    then QK RMSNorm + 3D RoPE on q and k (v as projected).  Returns (qkv_out, qkv_pre, h):
+    the result, the projection before the norm, and the AdaLN output."""
+    y, h = adaln_linear(x, w, shift, scale, eps=eps, stream_id=stream_id, n_streams=n_streams,
+                        tokens_per_sample=tokens_per_sample, rows=rows)
+    hd = n_heads * head_dim
+    assert y.shape[1] == 3 * hd, "W must have 3 * n_heads * head_dim rows"
+    y = np.ascontiguousarray(y)
+    qk = dit_epilogue(y, wq, wk, n_heads=n_heads, head_dim=head_dim, pos=pos, grid=grid,
+                      tokens_per_sample=tokens_per_sample, dims=dims, theta=theta, eps=eps,
+                      rows=rows)
+    out = y.copy()
+    out[:, :2 * hd] = qk
+    return out, y, h
