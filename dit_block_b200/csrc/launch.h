@@ -81,6 +81,40 @@ size_t qk_pool_smem_limit();
 // wait on a bulk copy gave up); optionally cleared.  Synchronous.
 uint32_t rows_device_error(bool clear);
 
+// Linear layers on the tensor cores (k_gemm.cu): out = epilogue(A . W^T), bf16 only.
+enum LinearEpi { LINEAR_STORE = 0, LINEAR_GATED = 1, LINEAR_SWIGLU = 2, LINEAR_QKROPE = 3 };
+struct LinearLaunch {
+    int64_t M;          // rows of A (tokens), < 2^31
+    int32_t K;          // inner dimension, multiple of 64
+    int32_t N;          // rows of W: output columns (SwiGLU: 2 * inner), multiple of 256
+    const void* a;      // A [M, K] (row stride ld_a); x for the AdaLN variant
+    int64_t ld_a;
+    const void* w;      // W [N, K] (row stride ld_w)
+    int64_t ld_w;
+    void* out;
+    int64_t ld_out;
+    const void* x;      // gated residual input [M, N]
+    int64_t ld_x;
+    const void* gate;
+    void* stats;        // AdaLN: [M] float2 workspace (mean, rstd)
+    const void* shift;
+    const void* scale;
+    int64_t ld_mod;
+    const ModSel* sel;
+    const void* wq;     // QK norm weights [128]
+    const void* wk;
+    const int32_t* pos;
+    int32_t grid_H, grid_W;
+    int64_t tps;
+    RopeDev rope;
+    int32_t qk_cols;    // columns of q and k (2 * n_heads * 128)
+    float eps;
+};
+cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cudaStream_t s);
+size_t linear_smem_bytes();
+// Error flags raised by the linear kernels' bounded waits; optionally cleared.  Synchronous.
+uint32_t gemm_device_error(bool clear);
+
 // Store a one-line reason for sol_last_error() on this host thread.
 void record_error(const char* msg);
 

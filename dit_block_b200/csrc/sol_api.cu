@@ -2,6 +2,7 @@
 // the RoPE table handle, launch bookkeeping, and dispatch to the kernel launchers.
 // Every check runs on the host before anything is launched, so a rejected call has no
 // side effect on the device.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -201,8 +202,9 @@ sol_status sol_device_errors(uint32_t* flags, int32_t clear)
     CHECK(flags, SOL_ERR_INVALID_ARGUMENT, "flags is NULL");
     const cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_status(e, "sol_device_errors");
-    *flags = sol::rows_device_error(clear != 0);
-    CHECK(*flags != 0xffffffffu, SOL_ERR_CUDA, "reading the device error flags failed");
+    const uint32_t rows = sol::rows_device_error(clear != 0);
+    CHECK(rows != 0xffffffffu, SOL_ERR_CUDA, "reading the device error flags failed");
+    *flags = rows | ((sol::gemm_device_error(clear != 0) & 0xffu) << 8);
     return SOL_OK;
 }
 
@@ -595,6 +597,211 @@ sol_status sol_dit_epilogue(void* qkv, int64_t ld_qkv, const void* wq, const voi
                                                      tokens_per_sample, rope->view, n_tokens,
                                                      n_heads, head_dim, eps, (cudaStream_t)stream),
                        "sol_dit_epilogue launch");
+}
+
+}  // extern "C"
+
+// Shared checks of the linear-layer calls: bf16 only, k a multiple of 64, n_out a
+// multiple of 256, n_tokens below 2^31 (tensor-copy coordinates are 32-bit).
+static sol_status check_linear_shape(int64_t n_tokens, int64_t n_out, int64_t k, sol_dtype dt,
+                                     int64_t n_multiple)
+{
+    CHECK(dt == SOL_DTYPE_BF16, SOL_ERR_UNSUPPORTED, "the linear-layer calls take bf16 only");
+    CHECK(n_tokens >= 0, SOL_ERR_INVALID_ARGUMENT, "n_tokens (%lld) is negative", (long long)n_tokens);
+    CHECK(n_tokens < ((int64_t)1 << 31), SOL_ERR_UNSUPPORTED, "n_tokens (%lld) must be below 2^31",
+          (long long)n_tokens);
+    CHECK(k >= 64 && n_out >= 1, SOL_ERR_INVALID_ARGUMENT, "k (%lld) and the output width (%lld) must be positive, k >= 64",
+          (long long)k, (long long)n_out);
+    CHECK(k % 64 == 0 && k < ((int64_t)1 << 30), SOL_ERR_UNSUPPORTED, "k (%lld) must be a multiple of 64",
+          (long long)k);
+    CHECK(n_out % n_multiple == 0 && n_out < ((int64_t)1 << 30), SOL_ERR_UNSUPPORTED,
+          "output width %lld must be a multiple of %lld", (long long)n_out, (long long)n_multiple);
+    return SOL_OK;
+}
+
+// Byte-range overlap of two row-strided tensors of different shapes.
+// Element sizes: esz_a for a, esz_b for b.
+static bool spans_overlap(const void* a, int64_t rows_a, int64_t ld_a, int64_t w_a, size_t esz_a, const void* b,
+                          int64_t rows_b, int64_t ld_b, int64_t w_b, size_t esz_b)
+{
+    if (!a || !b || rows_a == 0 || rows_b == 0) return false;
+    const char* a0 = (const char*)a;
+    const char* b0 = (const char*)b;
+    const char* a1 = a0 + (size_t)((rows_a - 1) * ld_a + w_a) * esz_a;
+    const char* b1 = b0 + (size_t)((rows_b - 1) * ld_b + w_b) * esz_b;
+    return a0 < b1 && b0 < a1;
+}
+
+static sol_status check_stats(const float* row_stats, int64_t n_tokens)
+{
+    CHECK(row_stats, SOL_ERR_INVALID_ARGUMENT, "row_stats is NULL");
+    CHECK(aligned16(row_stats), SOL_ERR_MISALIGNED, "row_stats is not 16-byte aligned");
+    (void)n_tokens;
+    return SOL_OK;
+}
+
+static sol::LinearLaunch linear_base(void* out, int64_t ld_out, const void* a, int64_t ld_a, const void* w,
+                                     int64_t ld_w, int64_t n_tokens, int64_t n_w_rows, int64_t k)
+{
+    sol::LinearLaunch L{};
+    L.M = n_tokens;
+    L.K = (int32_t)k;
+    L.N = (int32_t)n_w_rows;
+    L.a = a;
+    L.ld_a = ld_a;
+    L.w = w;
+    L.ld_w = ld_w;
+    L.out = out;
+    L.ld_out = ld_out;
+    L.eps = 0.f;
+    return L;
+}
+
+extern "C" {
+
+sol_status sol_linear(void* out, int64_t ld_out, const void* a, int64_t ld_a, const void* w,
+                      int64_t ld_w, int64_t n_tokens, int64_t n_out, int64_t k, sol_dtype dt,
+                      sol_stream_t stream)
+{
+    TRY(check_linear_shape(n_tokens, n_out, k, dt, 256));
+    TRY(check_tensor("w", w, ld_w, k, dt, true));
+    if (n_tokens == 0) return SOL_OK;
+    TRY(check_tensor("out", out, ld_out, n_out, dt, true));
+    TRY(check_tensor("a", a, ld_a, k, dt, true));
+    CHECK(!spans_overlap(out, n_tokens, ld_out, n_out, 2, a, n_tokens, ld_a, k, 2) &&
+              !spans_overlap(out, n_tokens, ld_out, n_out, 2, w, n_out, ld_w, k, 2),
+          SOL_ERR_INVALID_ARGUMENT, "out overlaps an input");
+    const sol::LinearLaunch L = linear_base(out, ld_out, a, ld_a, w, ld_w, n_tokens, n_out, k);
+    return cuda_status(sol::launch_linear(sol::LINEAR_STORE, false, L, (cudaStream_t)stream), "sol_linear launch");
+}
+
+sol_status sol_linear_gated_residual(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                                     const void* a, int64_t ld_a, const void* w, int64_t ld_w,
+                                     const void* gate, int64_t ld_mod, sol_modsel sel,
+                                     int64_t n_tokens, int64_t d, int64_t k, sol_dtype dt,
+                                     sol_stream_t stream)
+{
+    TRY(check_linear_shape(n_tokens, d, k, dt, 256));
+    TRY(check_modsel(sel));
+    TRY(check_tensor("w", w, ld_w, k, dt, true));
+    TRY(check_tensor("gate", gate, ld_mod, d, dt, false));
+    if (n_tokens == 0) return SOL_OK;
+    TRY(check_tensor("out", out, ld_out, d, dt, true));
+    TRY(check_tensor("x", x, ld_x, d, dt, true));
+    TRY(check_tensor("a", a, ld_a, k, dt, true));
+    CHECK(out == x ? ld_out == ld_x : !overlap(out, ld_out, x, ld_x, n_tokens, d, 2), SOL_ERR_INVALID_ARGUMENT,
+          "out overlaps x without being the same tensor");
+    CHECK(!spans_overlap(out, n_tokens, ld_out, d, 2, a, n_tokens, ld_a, k, 2) &&
+              !spans_overlap(out, n_tokens, ld_out, d, 2, w, d, ld_w, k, 2),
+          SOL_ERR_INVALID_ARGUMENT, "out overlaps a or w");
+    sol::LinearLaunch L = linear_base(out, ld_out, a, ld_a, w, ld_w, n_tokens, d, k);
+    const sol::ModSel ms = to_dev(sel, n_tokens);
+    L.x = x;
+    L.ld_x = ld_x;
+    L.gate = gate;
+    L.ld_mod = ld_mod;
+    L.sel = &ms;
+    return cuda_status(sol::launch_linear(sol::LINEAR_GATED, false, L, (cudaStream_t)stream),
+                       "sol_linear_gated_residual launch");
+}
+
+sol_status sol_linear_swiglu(void* out, int64_t ld_out, const void* a, int64_t ld_a, const void* w,
+                             int64_t ld_w, int64_t n_tokens, int64_t inner, int64_t k, sol_dtype dt,
+                             sol_stream_t stream)
+{
+    TRY(check_linear_shape(n_tokens, 2 * inner, k, dt, 256));
+    TRY(check_tensor("w", w, ld_w, k, dt, true));
+    if (n_tokens == 0) return SOL_OK;
+    TRY(check_tensor("out", out, ld_out, inner, dt, true));
+    TRY(check_tensor("a", a, ld_a, k, dt, true));
+    CHECK(!spans_overlap(out, n_tokens, ld_out, inner, 2, a, n_tokens, ld_a, k, 2) &&
+              !spans_overlap(out, n_tokens, ld_out, inner, 2, w, 2 * inner, ld_w, k, 2),
+          SOL_ERR_INVALID_ARGUMENT, "out overlaps a or w");
+    const sol::LinearLaunch L = linear_base(out, ld_out, a, ld_a, w, ld_w, n_tokens, 2 * inner, k);
+    return cuda_status(sol::launch_linear(sol::LINEAR_SWIGLU, false, L, (cudaStream_t)stream),
+                       "sol_linear_swiglu launch");
+}
+
+sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                            const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
+                            const void* w, int64_t ld_w, float* row_stats, int64_t n_tokens,
+                            int64_t n_out, int64_t d, float eps, sol_dtype dt, sol_stream_t stream)
+{
+    TRY(check_linear_shape(n_tokens, n_out, d, dt, 256));
+    TRY(check_modsel(sel));
+    CHECK(std::isfinite(eps) && eps >= 0.f, SOL_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
+    TRY(check_tensor("w", w, ld_w, d, dt, true));
+    TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
+    TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
+    if (n_tokens == 0) return SOL_OK;
+    TRY(check_stats(row_stats, n_tokens));
+    TRY(check_tensor("out", out, ld_out, n_out, dt, true));
+    TRY(check_tensor("x", x, ld_x, d, dt, true));
+    CHECK(!spans_overlap(out, n_tokens, ld_out, n_out, 2, x, n_tokens, ld_x, d, 2) &&
+              !spans_overlap(out, n_tokens, ld_out, n_out, 2, w, n_out, ld_w, d, 2) &&
+              !spans_overlap(out, n_tokens, ld_out, n_out, 2, row_stats, n_tokens, 2, 2, 4) &&
+              !spans_overlap(x, n_tokens, ld_x, d, 2, row_stats, n_tokens, 2, 2, 4),
+          SOL_ERR_INVALID_ARGUMENT, "out or x overlaps another argument");
+    sol::LinearLaunch L = linear_base(out, ld_out, x, ld_x, w, ld_w, n_tokens, n_out, d);
+    const sol::ModSel ms = to_dev(sel, n_tokens);
+    L.stats = row_stats;
+    L.shift = shift;
+    L.scale = scale;
+    L.ld_mod = ld_mod;
+    L.sel = &ms;
+    L.eps = eps;
+    return cuda_status(sol::launch_linear(sol::LINEAR_STORE, true, L, (cudaStream_t)stream),
+                       "sol_adaln_linear launch");
+}
+
+sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t ld_x,
+                              const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
+                              const void* w, int64_t ld_w, float* row_stats, const void* wq,
+                              const void* wk, const int32_t* pos, int32_t grid_T, int32_t grid_H,
+                              int32_t grid_W, const sol_rope3d* rope, int64_t n_tokens,
+                              int32_t n_heads, int32_t head_dim, int64_t d, float eps, sol_dtype dt,
+                              sol_stream_t stream)
+{
+    CHECK(dt == SOL_DTYPE_BF16, SOL_ERR_UNSUPPORTED, "the linear-layer calls take bf16 only");
+    CHECK(head_dim == 128, SOL_ERR_UNSUPPORTED, "sol_adaln_qkv_rope is built for head_dim 128 (got %d)",
+          (int)head_dim);
+    CHECK(n_heads >= 2 && n_heads % 2 == 0, SOL_ERR_UNSUPPORTED,
+          "sol_adaln_qkv_rope needs an even n_heads (two heads per 256-column tile), got %d", (int)n_heads);
+    TRY(check_modsel(sel));
+    TRY(check_qk_common(rope, pos, grid_T, grid_H, grid_W, sel.tokens_per_sample, n_tokens, n_heads, head_dim,
+                        eps, dt, wq, wk));
+    const int64_t n_out = 3 * (int64_t)n_heads * head_dim;
+    TRY(check_linear_shape(n_tokens, n_out, d, dt, 256));
+    TRY(check_tensor("w", w, ld_w, d, dt, true));
+    TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
+    TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
+    if (n_tokens == 0) return SOL_OK;
+    TRY(check_stats(row_stats, n_tokens));
+    TRY(check_tensor("qkv", qkv, ld_qkv, n_out, dt, true));
+    TRY(check_tensor("x", x, ld_x, d, dt, true));
+    CHECK(!spans_overlap(qkv, n_tokens, ld_qkv, n_out, 2, x, n_tokens, ld_x, d, 2) &&
+              !spans_overlap(qkv, n_tokens, ld_qkv, n_out, 2, w, n_out, ld_w, d, 2) &&
+              !spans_overlap(qkv, n_tokens, ld_qkv, n_out, 2, row_stats, n_tokens, 2, 2, 4) &&
+              !spans_overlap(x, n_tokens, ld_x, d, 2, row_stats, n_tokens, 2, 2, 4),
+          SOL_ERR_INVALID_ARGUMENT, "qkv or x overlaps another argument");
+    sol::LinearLaunch L = linear_base(qkv, ld_qkv, x, ld_x, w, ld_w, n_tokens, n_out, d);
+    const sol::ModSel ms = to_dev(sel, n_tokens);
+    L.stats = row_stats;
+    L.shift = shift;
+    L.scale = scale;
+    L.ld_mod = ld_mod;
+    L.sel = &ms;
+    L.eps = eps;
+    L.wq = wq;
+    L.wk = wk;
+    L.pos = pos;
+    L.grid_H = grid_H;
+    L.grid_W = grid_W;
+    L.tps = sel.tokens_per_sample;
+    L.rope = rope->view;
+    L.qk_cols = 2 * n_heads * head_dim;
+    return cuda_status(sol::launch_linear(sol::LINEAR_QKROPE, true, L, (cudaStream_t)stream),
+                       "sol_adaln_qkv_rope launch");
 }
 
 }  // extern "C"

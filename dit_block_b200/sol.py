@@ -76,6 +76,14 @@ SIGNATURES = {
     "sol_qk_rmsnorm_rope3d_noalloc": ([_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _P, _P, _I32, _I32,
                                        _I32, _I64, _I32, _I32, _I32, _D, _I32, _I32, _I32, _I64,
                                        _I32, _I32, _F, _E, _P], _E),
+    "sol_linear": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _E, _P], _E),
+    "sol_linear_gated_residual": ([_P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _I64, ModSel, _I64, _I64,
+                                   _I64, _E, _P], _E),
+    "sol_linear_swiglu": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _E, _P], _E),
+    "sol_adaln_linear": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, _I64, _I64, _I64, _F,
+                          _E, _P], _E),
+    "sol_adaln_qkv_rope": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, _P, _P, _P, _I32, _I32,
+                            _I32, _P, _I64, _I32, _I32, _I64, _F, _E, _P], _E),
 }
 
 _lib = None
@@ -350,3 +358,57 @@ def qk_rmsnorm_rope3d_ex(q_out, k_out, q, k, rope: Rope3D, *, n_heads, head_dim,
                int(grid[2]), int(tokens_per_sample), rope.handle, n, int(n_heads), int(head_dim), float(eps),
                int(norm_span), int(pairing), _dtype(q))
     _check(lib().sol_qk_rmsnorm_rope3d_ex(ctypes.byref(d), _stream(stream)), "sol_qk_rmsnorm_rope3d_ex")
+
+
+# ------------------------------------------------------- linear layers with fused operators
+
+def linear(out, a, w, *, stream=None):
+    """out = a . W^T on the tensor cores (sol_linear); W is [n_out, k]."""
+    _check(lib().sol_linear(_ptr(out), _ld(out), _ptr(a), _ld(a), _ptr(w), _ld(w), a.shape[0], w.shape[0],
+                            a.shape[1], _dtype(a), _stream(stream)), "sol_linear")
+    return out
+
+
+def linear_gated_residual(out, x, a, w, gate=None, *, stream_id=None, n_streams=1, tokens_per_sample=0,
+                          stream=None):
+    """out = x + gate[r] * (a . W^T)  (sol_linear_gated_residual); out may be x."""
+    _check(lib().sol_linear_gated_residual(
+        _ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(a), _ld(a), _ptr(w), _ld(w), _ptr(gate), _mod_ld(gate),
+        _sel(stream_id, n_streams, tokens_per_sample), a.shape[0], w.shape[0], a.shape[1], _dtype(a),
+        _stream(stream)), "sol_linear_gated_residual")
+    return out
+
+
+def linear_swiglu(out, a, w, *, stream=None):
+    """out = silu(a . W1^T) * (a . W2^T) with W = [W1; W2] of [2*inner, k]  (sol_linear_swiglu)."""
+    _check(lib().sol_linear_swiglu(_ptr(out), _ld(out), _ptr(a), _ld(a), _ptr(w), _ld(w), a.shape[0],
+                                   w.shape[0] // 2, a.shape[1], _dtype(a), _stream(stream)),
+           "sol_linear_swiglu")
+    return out
+
+
+def row_stats_workspace(n_tokens: int, device=None) -> torch.Tensor:
+    """A row-statistics workspace for the sol_adaln_* calls: [n_tokens, 2] float32."""
+    return torch.empty((max(int(n_tokens), 1), 2), dtype=torch.float32, device=device or "cuda")
+
+
+def adaln_linear(out, x, w, shift=None, scale=None, *, row_stats, eps=1e-6, stream_id=None, n_streams=1,
+                 tokens_per_sample=0, stream=None):
+    """out = AdaLN(x) . W^T with AdaLN in the operand load  (sol_adaln_linear)."""
+    _check(lib().sol_adaln_linear(
+        _ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
+        _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(row_stats), x.shape[0],
+        w.shape[0], x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_linear")
+    return out
+
+
+def adaln_qkv_rope(qkv, x, w, rope: Rope3D, shift=None, scale=None, *, row_stats, n_heads, head_dim=128,
+                   wq=None, wk=None, pos=None, grid=(0, 0, 0), eps=1e-6, stream_id=None, n_streams=1,
+                   tokens_per_sample=0, stream=None):
+    """qkv = AdaLN(x) . W^T, then QK RMSNorm + 3D RoPE on q and k  (sol_adaln_qkv_rope)."""
+    _check(lib().sol_adaln_qkv_rope(
+        _ptr(qkv), _ld(qkv), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
+        _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(row_stats), _ptr(wq), _ptr(wk),
+        _ptr(pos), int(grid[0]), int(grid[1]), int(grid[2]), rope.handle, x.shape[0], n_heads, head_dim,
+        x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_qkv_rope")
+    return qkv

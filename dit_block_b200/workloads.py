@@ -94,7 +94,9 @@ WORKLOADS = {
 # tensor ids (seed = 1000 * workload.index + id)
 TID = {"x": 1, "y_attn": 2, "y_mlp": 3, "u": 4, "qkv": 5,
        "shift_msa": 10, "scale_msa": 11, "gate_msa": 12,
-       "shift_mlp": 13, "scale_mlp": 14, "gate_mlp": 15, "wq": 20, "wk": 21}
+       "shift_mlp": 13, "scale_mlp": 14, "gate_mlp": 15, "wq": 20, "wk": 21,
+       # linear-layer weights and the activations that feed them
+       "w_qkv": 30, "w_o": 31, "w_up": 32, "w_down": 33, "attn": 34, "act": 35}
 
 _CHUNK_ELEMS = 1 << 26  # draw at most 64M fp32 values at a time (bounded temporaries)
 
@@ -145,6 +147,13 @@ def modulation(w: Workload, name: str, device="cpu") -> torch.Tensor:
 def norm_weight(w: Workload, name: str, device="cpu") -> torch.Tensor:
     t = torch.empty((1, w.head_dim), dtype=w.dtype, device=device)
     return fill_normal_(t, 1000 * w.index + TID[name], 1.0, 0.02).view(w.head_dim)
+
+
+def linear_weight(w: Workload, name: str, out_features: int, in_features: int, device="cpu") -> torch.Tensor:
+    """Linear-layer weight [out_features, in_features] ~ N(0, 1/in_features), so a product
+    with unit-variance activations has unit variance."""
+    t = torch.empty((out_features, in_features), dtype=w.dtype, device=device)
+    return fill_normal_(t, 1000 * w.index + TID[name], 0.0, in_features ** -0.5)
 
 
 def token_layout(w: Workload):

@@ -86,9 +86,12 @@ const char* sol_last_error(void);
 int32_t sol_abi_version(void);
 
 /* Error flags raised on the current device by libsol kernels since the last clear:
- * bit 0 = a kernel's bounded wait on its own asynchronous copy gave up (the kernel
- * recorded it, stopped early and left its outputs incomplete).  Synchronises the current
- * device first; clear != 0 resets the flags.  Never set in normal operation. */
+ * bit 0 = a per-token kernel's bounded wait on its own asynchronous copy gave up;
+ * bits 8..15 = a linear-layer kernel (sol_linear*, sol_adaln_*) gave up a bounded wait
+ * in its copy / MMA / epilogue / transform pipeline.  The kernel recorded it, drained
+ * its own copies and MMAs, stopped early and left its outputs incomplete.  Synchronises
+ * the current device first; clear != 0 resets the flags.  Never set in normal
+ * operation. */
 sol_status sol_device_errors(uint32_t* flags, int32_t clear);
 
 /* AdaLN modulation [XHH-QA, STM-GAN]:
@@ -308,6 +311,84 @@ sol_status sol_qk_rmsnorm_rope3d_noalloc(void* q_out, void* k_out, int64_t ld_qo
                                          int32_t max_h, int32_t max_w, int64_t n_tokens,
                                          int32_t n_heads, int32_t head_dim, float eps,
                                          sol_dtype dt, sol_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Linear layers with the per-token operators fused in.
+ *
+ * [STM-RES] credits the fused kernels with cutting memory traffic, intermediate
+ * tensors and launches without changing the math.  In the DiT block the per-token
+ * operators sit around its linear layers: AdaLN feeds the QKV projection and QK
+ * RMSNorm + 3D RoPE follows it; the gated residual follows the attention output
+ * projection and the MLP down projection; SwiGLU follows the MLP up projection.  The
+ * calls below run each linear layer on the tensor cores and apply the operator to the
+ * operand tile on its way in or to the accumulator on its way out, so the operator's
+ * input or output never makes its own trip through HBM.
+ *
+ * Common rules (in addition to the conventions at the top of this file):
+ *   dt must be SOL_DTYPE_BF16 (the tensor cores take bf16 operands; SOL_ERR_UNSUPPORTED
+ *   otherwise).  W is [n_out, k] with row stride ld_w: the usual linear-layer layout,
+ *   y = a . W^T, no bias.  k must be a multiple of 64 and n_out a multiple of 256
+ *   (SOL_ERR_UNSUPPORTED otherwise); n_tokens < 2^31.  Accumulation is fp32; the
+ *   operand the tensor cores read is bf16 (the AdaLN output is rounded to bf16 in
+ *   shared memory, exactly where the unfused path rounds it when storing h); every
+ *   output element is rounded once, when stored.  No output may overlap an input
+ *   except where stated.  Each call launches one kernel (two for the sol_adaln_*
+ *   calls: a row-statistics pass, then the linear layer).
+ * ------------------------------------------------------------------------------------ */
+
+/* out = a . W^T: a [n_tokens, k], W [n_out, k], out [n_tokens, n_out]. */
+sol_status sol_linear(void* out, int64_t ld_out, const void* a, int64_t ld_a, const void* w,
+                      int64_t ld_w, int64_t n_tokens, int64_t n_out, int64_t k, sol_dtype dt,
+                      sol_stream_t stream);
+
+/* Output / down projection with the gated residual in its epilogue:
+ *     out = x + gate[r] * (a . W^T)
+ * a [n_tokens, k], W [d, k], x and out [n_tokens, d]; gate [B*n_streams, ld_mod] chosen
+ * per token by `sel` as in sol_gated_residual (NULL = zero: out = x).  The product is
+ * not rounded before the residual.  out may be x (same pointer and ld). */
+sol_status sol_linear_gated_residual(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                                     const void* a, int64_t ld_a, const void* w, int64_t ld_w,
+                                     const void* gate, int64_t ld_mod, sol_modsel sel,
+                                     int64_t n_tokens, int64_t d, int64_t k, sol_dtype dt,
+                                     sol_stream_t stream);
+
+/* MLP up projection with SwiGLU in its epilogue:
+ *     out[:, j] = silu((a . W1^T)[:, j]) * (a . W2^T)[:, j],   W = [W1; W2]
+ * W [2*inner, k] holds the gated half W1 in rows [0, inner) and the multiplying half W2
+ * in rows [inner, 2*inner) (the two halves of the packed up projection, in the order
+ * sol_swiglu takes them); out [n_tokens, inner]; inner a multiple of 128.  Neither
+ * half is rounded before the product. */
+sol_status sol_linear_swiglu(void* out, int64_t ld_out, const void* a, int64_t ld_a, const void* w,
+                             int64_t ld_w, int64_t n_tokens, int64_t inner, int64_t k, sol_dtype dt,
+                             sol_stream_t stream);
+
+/* AdaLN fused into the operand load of a linear layer:
+ *     out = h . W^T,   h = LN(x) * (1 + scale[r]) + shift[r]   (as sol_adaln_modulate)
+ * x [n_tokens, d], W [n_out, d], out [n_tokens, n_out]; d a multiple of 64.
+ * row_stats: caller-owned device workspace of n_tokens (mean, 1/sqrt(var + eps)) float
+ * pairs (8 bytes per token, 16-byte aligned), written by the call's first kernel and
+ * read by its second; it must not overlap any other argument.  h is never stored. */
+sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                            const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
+                            const void* w, int64_t ld_w, float* row_stats, int64_t n_tokens,
+                            int64_t n_out, int64_t d, float eps, sol_dtype dt, sol_stream_t stream);
+
+/* The attention input of a block in one pass: AdaLN into the QKV projection, QK RMSNorm
+ * + 3D RoPE in its epilogue:
+ *     qkv = h . W^T  ([n_tokens, 3*n_heads*head_dim] = q | k | v),  h as in
+ *     sol_adaln_linear; then every q and k head vector as sol_dit_epilogue does it
+ *     (RMSNorm with wq / wk, interleaved 3D RoPE from `rope`); v as projected.
+ * head_dim must be 128 and n_heads even.  Positions: pos [n_tokens, 3] int32, or NULL
+ * for the row-major grid (grid_T, grid_H, grid_W) of each sample, samples of
+ * sel.tokens_per_sample tokens (0 = one sample), as in sol_qk_rmsnorm_rope3d.
+ * row_stats as in sol_adaln_linear.  The projection is not rounded before the norm. */
+sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t ld_x,
+                              const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
+                              const void* w, int64_t ld_w, float* row_stats, const void* wq,
+                              const void* wk, const int32_t* pos, int32_t grid_T, int32_t grid_H,
+                              int32_t grid_W, const sol_rope3d* rope, int64_t n_tokens,
+                              int32_t n_heads, int32_t head_dim, int64_t d, float eps, sol_dtype dt,
+                              sol_stream_t stream);
 
 #ifdef __cplusplus
 }

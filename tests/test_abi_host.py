@@ -28,7 +28,7 @@ def last(L):
 
 def test_exports_every_declared_symbol(L):
     names = sol.header_functions()
-    assert len(names) == 17
+    assert len(names) == 22
     for n in names:
         assert hasattr(L, n), f"libsol.so does not export {n}"
         assert n in sol.SIGNATURES, f"binding has no signature for {n}"
@@ -136,3 +136,55 @@ def test_subblock_count(L):
     assert L.sol_subblock_count(100, 0, 64) == 2
     assert L.sol_subblock_count(0, 0, 64) == 0
     assert L.sol_subblock_count(10, 0, 0) == 0
+
+
+def test_linear_validation(L):
+    n, k, d = 300, 512, 768
+    # bf16 only
+    assert L.sol_linear(FAKE, d, FAKE, k, FAKE, k, n, d, k, sol.F32, None) == sol.ERR_UNSUPPORTED
+    assert "bf16" in last(L)
+    # k a multiple of 64, output width a multiple of 256
+    assert L.sol_linear(FAKE, d, FAKE, 520, FAKE, 520, n, d, 520, sol.BF16, None) == sol.ERR_UNSUPPORTED
+    assert L.sol_linear(FAKE, 640, FAKE, k, FAKE, k, n, 640, k, sol.BF16, None) == sol.ERR_UNSUPPORTED
+    assert L.sol_linear(FAKE, d, FAKE, k, FAKE, k, 1 << 31, d, k, sol.BF16, None) == sol.ERR_UNSUPPORTED
+    assert L.sol_linear(FAKE, d, FAKE, k, FAKE, k, -1, d, k, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_linear(FAKE, d, FAKE, k, None, k, n, d, k, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_linear(FAKE, d, FAKE + 8, k, FAKE, k, n, d, k, sol.BF16, None) == sol.ERR_MISALIGNED
+    # out overlapping a
+    assert L.sol_linear(FAKE + 64, d, FAKE, k, FAKE << 4, k, n, d, k, sol.BF16, None) \
+        == sol.ERR_INVALID_ARGUMENT
+    assert "overlaps" in last(L)
+    # n_tokens == 0: valid, nothing launched
+    assert L.sol_linear(None, d, None, k, FAKE, k, 0, d, k, sol.BF16, None) == sol.OK
+
+
+def test_linear_epilogue_variants_validation(L):
+    n, k, d = 300, 512, 768
+    x, a, w, out = FAKE, FAKE << 2, FAKE << 3, FAKE << 4
+    # gated residual: out may be x itself but not partially overlap it
+    assert L.sol_linear_gated_residual(x + 64, d, x, d, a, k, w, k, None, 0, SEL, n, d, k, sol.BF16, None) \
+        == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_linear_gated_residual(out, d, x, d, a, k, w, k, None, 0, sol.ModSel(None, 0, 0), n, d, k,
+                                       sol.BF16, None) == sol.ERR_INVALID_ARGUMENT  # n_streams 0
+    assert L.sol_linear_gated_residual(out, d, x, d, a, k, w, k, None, 0, SEL, n, 640, k, sol.BF16, None) \
+        == sol.ERR_UNSUPPORTED
+    # SwiGLU: W has 2*inner rows, inner a multiple of 128
+    assert L.sol_linear_swiglu(out, 192, a, k, w, k, n, 192, k, sol.BF16, None) == sol.ERR_UNSUPPORTED
+    assert L.sol_linear_swiglu(out, 256, a, k, w, k, n, 256, k, sol.F32, None) == sol.ERR_UNSUPPORTED
+    # AdaLN variants need the row-statistics workspace
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, None, n, d, k, 1e-6, sol.BF16,
+                              None) == sol.ERR_INVALID_ARGUMENT
+    assert "row_stats" in last(L)
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, FAKE << 5, n, d, k, float("inf"),
+                              sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    # row_stats inside x
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, x + 1024, n, d, k, 1e-6,
+                              sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    # the QKV call is built for head_dim 128 and an even head count
+    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, FAKE << 5, None, None, None,
+                                2, 4, 4, None, n, 4, 64, k, 1e-6, sol.BF16, None) == sol.ERR_UNSUPPORTED
+    assert L.sol_adaln_qkv_rope(out, 1152, x, k, None, None, 0, SEL, w, k, FAKE << 5, None, None, None,
+                                2, 4, 4, None, n, 3, 128, k, 1e-6, sol.BF16, None) == sol.ERR_UNSUPPORTED
+    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, FAKE << 5, None, None, None,
+                                2, 4, 4, None, n, 2, 128, k, 1e-6, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    assert "rope is NULL" in last(L)
