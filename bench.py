@@ -43,6 +43,7 @@ from dit_block_b200 import workloads  # noqa: E402
 
 METRIC = "fused DiT-op HBM GB/s & tokens/s at 125k/246k tokens; % of B200 HBM peak"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 SPEC_HBM_GBS = 8000.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_swiglu_fullres_10s.md")
 OPS = ("adaln_modulate", "dit_epilogue", "dit_prologue", "swiglu", "gated_residual")
@@ -123,6 +124,15 @@ def measured_peak():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_peak():
+    """Dense bf16 TFLOP/s of a cuBLAS GEMM timed alone on this machine's B200s (burst)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def source_digest() -> str:
@@ -315,6 +325,7 @@ def run_ours(args, w):
 
     # ---- ops beyond the block pass, each timed alone on the same workload
     next_ops = {} if args.no_next else time_next_ops(bufs, dev, args)
+    linear_ops = {} if (args.no_next or args.linear_tokens <= 0) else time_linear_ops(bufs, dev, args)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -351,6 +362,7 @@ def run_ours(args, w):
                      "algorithmic_bytes": dom_bytes},
         "clocks": clk,
         "next_ops": next_ops,
+        "linear_ops": linear_ops,
         "gpu_launches": len(OPS) * args.steps,
         "e2e": e2e,
     }
@@ -436,6 +448,82 @@ def time_next_ops(bufs, dev, args) -> dict:
     return out
 
 
+def time_linear_ops(bufs, dev, args) -> dict:
+    """The block's linear layers with the per-token operators fused in (tcgen05 GEMMs),
+    each timed alone on the first `linear_tokens` tokens of the workload (median of 10
+    launches), beside the same work unfused: a cuBLAS GEMM (torch.matmul) plus the
+    libsol per-token kernel, and the bare cuBLAS GEMM."""
+    from dit_block_b200 import sol, workloads as wl
+    w, i = bufs.w, bufs.inp
+    if w.dtype != torch.bfloat16 or w.head_dim != 128:
+        return {}
+    m = min(int(args.linear_tokens), bufs.n_tokens)
+    peak, src = measured_bf16_peak()
+    stream = torch.cuda.current_stream(dev)
+    x = i["x"][:m]
+    hd, d, inner = w.hd, w.d, w.inner
+    # ops on one sample's tokens: modulation rows of sample 0, positions from its grid
+    sel = dict(n_streams=1, tokens_per_sample=0)
+    out = {"tokens": m, "peak_tflops": peak, "peak_source": src + " (burst cuBLAS bf16)"}
+
+    def entry(name, flops, fused, unfused, cublas, plain, saved_bytes):
+        tf = _time(fused, 10, stream)
+        tu = _time(unfused, 10, stream)
+        tcb = _time(cublas, 10, stream)
+        tp = _time(plain, 10, stream)
+        ach = flops / (tf * 1e-3) / 1e12
+        out[name] = {"ms": round(tf, 4), "TFLOP_s": round(ach, 1), "frac_of_bf16_peak": round(ach / peak, 4),
+                     "unfused_ms": round(tu, 4), "cublas_gemm_ms": round(tcb, 4),
+                     "libsol_plain_gemm_ms": round(tp, 4), "speedup_vs_unfused": round(tu / tf, 3),
+                     "hbm_bytes_saved_per_token": saved_bytes}
+
+    stats = sol.row_stats_workspace(m, dev)
+    Wqkv = wl.linear_weight(w, "w_qkv", 3 * hd, d, dev)
+    qkv = torch.empty((m, 3 * hd), dtype=w.dtype, device=dev)
+    h = torch.empty_like(x)
+    sh, sc = i["shift_msa"][:1], i["scale_msa"][:1]
+    fused = lambda: sol.adaln_qkv_rope(qkv, x, Wqkv, bufs.rope, sh, sc, row_stats=stats, n_heads=w.n_heads,
+                                       wq=i["wq"], wk=i["wk"], grid=w.grid, eps=w.eps, **sel)
+
+    def unfused():
+        sol.adaln_modulate(h, x, sh, sc, eps=w.eps, **sel)
+        torch.matmul(h, Wqkv.t(), out=qkv)
+        sol.dit_epilogue(qkv, bufs.rope, n_heads=w.n_heads, head_dim=w.head_dim, wq=i["wq"], wk=i["wk"],
+                         grid=w.grid, eps=w.eps)
+    entry("adaln_qkv_rope", 2.0 * m * d * 3 * hd, fused, unfused, lambda: torch.matmul(x, Wqkv.t(), out=qkv),
+          lambda: sol.linear(qkv, x, Wqkv), 2 * d * 2 + 2 * (2 * hd) * 2)
+    del Wqkv, qkv, h, stats
+
+    for name, K, wname, gate in (("o_proj_gated_residual", d, "w_o", "gate_msa"),
+                                 ("down_proj_gated_residual", inner, "w_down", "gate_mlp")):
+        a = i["y_attn"][:m] if K == d else wl.activation(w, "act", m, K, dev)
+        W = wl.linear_weight(w, wname, d, K, dev)
+        o = torch.empty_like(x)
+        y = torch.empty_like(x)
+        g = i[gate][:1]
+        fused = lambda: sol.linear_gated_residual(o, x, a, W, g, **sel)
+
+        def unfused():
+            torch.matmul(a, W.t(), out=y)
+            sol.gated_residual(o, x, y, g, **sel)
+        entry(name, 2.0 * m * K * d, fused, unfused, lambda: torch.matmul(a, W.t(), out=y),
+              lambda: sol.linear(y, a, W), 2 * d * 2)
+        del a, W, o, y
+
+    Wup = wl.linear_weight(w, "w_up", 2 * inner, d, dev)
+    act = torch.empty((m, inner), dtype=w.dtype, device=dev)
+    u = torch.empty((m, 2 * inner), dtype=w.dtype, device=dev)
+    fused = lambda: sol.linear_swiglu(act, x, Wup)
+
+    def unfused():
+        torch.matmul(x, Wup.t(), out=u)
+        sol.swiglu(act, u, inner=inner)
+    entry("up_proj_swiglu", 2.0 * m * d * 2 * inner, fused, unfused, lambda: torch.matmul(x, Wup.t(), out=u),
+          lambda: sol.linear(u, x, Wup), 2 * (2 * inner) * 2)
+    del Wup, act, u
+    return out
+
+
 def run_e2e(args, bufs, dev, world, step_bytes):
     """The pass through the public host-buffer API (dit_block_b200.pipeline): pinned host
     inputs in, five launches per chunk, pinned host outputs back; every copy is inside
@@ -499,6 +587,8 @@ def main(argv=None):
     p.add_argument("--e2e-chunk", type=int, default=8192, help="tokens per pipelined chunk")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-next", action="store_true", help="skip timing the ops outside the block pass")
+    p.add_argument("--linear-tokens", type=int, default=32768,
+                   help="tokens of the fused linear-layer timings (0 skips them)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-tokens", type=int, default=256, help="oracle token sample per reference step")

@@ -8,20 +8,33 @@
 // "Resultado principal": fused kernels cut memory traffic, intermediate tensors and
 // launches without changing the math.
 //
-// Design (one persistent CTA per SM, 128 x 256 output tiles, K in steps of 64):
-//   warp 0        tensor-copy producer: A tile 128 x 64 and B tile 256 x 64 (bf16,
-//                 128-byte swizzle) per stage into a 4-stage shared-memory ring;
-//   warp 1        MMA issuer: four 128 x 256 x 16 tcgen05.mma per stage into one of two
-//                 TMEM accumulators (2 x 256 fp32 columns), so the epilogue of tile i
+// Design: persistent CTAs, output tiles of 256 accumulator columns, K in steps of 64
+// (one 128-byte swizzle row of bf16).  Two shapes of the same kernel:
+//   single  one CTA per SM, 128 x 256 tiles, 4-stage ring of A 128x64 + B 256x64;
+//   pair    a cluster of two CTAs on two SMs, 256 x 256 tiles computed by 256-row
+//           tcgen05.mma (cta_group::2) issued by the leader CTA; each CTA loads half
+//           of A (its 128 rows) and half of B (128 of the 256 columns) into a 6-stage
+//           ring of 32 KiB stages and holds its 128 accumulator rows in its own TMEM.
+//           Per SM the copies per MMA drop by a third and the ring is half as deep
+//           again, which hides the copy latency.  The variant with the AdaLN operand
+//           transform runs single (see use_pair()).
+// Warp roles:
+//   warp 0        tensor-copy producer (one thread);
+//   warp 1        MMA issuer (one thread; the leader CTA only in a pair) into one of two
+//                 TMEM accumulators of 256 fp32 columns, so the epilogue of tile i
 //                 overlaps the main loop of tile i+1; owns the TMEM allocation;
 //   warps 2..5    epilogue: each thread owns one accumulator row (TMEM lane), reads it
 //                 32 columns at a time and applies the fused operator;
-//   warps 6..9    (AdaLN variant only) operand transform: rewrite each landed x tile in
-//                 shared memory as h = (x - mean) * rstd * (1 + scale) + shift in bf16
-//                 before the MMA reads it.
-// Every wait on an mbarrier is bounded; a wait that gives up raises an error flag and
-// the CTA drains its in-flight copies and MMAs, frees its TMEM and returns.
+//   warps 6..13   (AdaLN variant only) operand transform, two groups on alternate
+//                 stages: rewrite each landed x tile in shared memory as
+//                 h = (x - mean) * rstd * (1 + scale) + shift in bf16 before the MMA
+//                 reads it.
+// No copy uses multicast: the leader commits to its own and to the peer's barriers one
+// at a time.  Every wait on an mbarrier is bounded; a wait that gives up raises an error
+// flag and the CTA drains its in-flight copies and MMAs, frees its TMEM and returns.
 #include <algorithm>
+#include <cstdlib>
+#include <string>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -34,34 +47,48 @@
 namespace sol {
 namespace gemm {
 
-constexpr int BM = 128;                   // rows of a tile (TMEM lanes)
+constexpr int BM = 128;                   // accumulator rows per CTA (TMEM lanes)
 constexpr int BN = 256;                   // accumulator columns of a tile
-constexpr int BK = 64;                    // K per stage: one 128-byte swizzle row of bf16
+constexpr int BK = 64;                    // K per stage
 constexpr int UK = 16;                    // K of one tcgen05.mma (kind::f16)
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;      // 16 KiB
-constexpr int B_BYTES = BN * BK * 2;      // 32 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int A_BYTES = BM * BK * 2;      // 16 KiB: this CTA's rows of A per stage
 constexpr int TMEM_COLS = 2 * BN;         // two accumulators
 constexpr int GROUP_M = 16;               // m-blocks per raster group (L2 reuse)
+constexpr int MAX_STAGES = 6;
 constexpr int PRODUCER_WARP = 0, MMA_WARP = 1, XFORM_WARP0 = 6;  // epilogue: warps 2..5
 constexpr uint32_t kWaitLimit = 4096;     // polls of <= ~1 ms each
 
+template <bool PAIR> struct Shape {
+    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr int B_ROWS = PAIR ? BN / 2 : BN;   // rows of B (output columns) this CTA loads
+    static constexpr int B_BYTES = B_ROWS * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TILE_M = PAIR ? 2 * BM : BM;   // rows of one output tile
+};
+
 enum Epi : int { EPI_STORE = 0, EPI_GATED = 1, EPI_SWIGLU = 2, EPI_QKROPE = 3 };
 
-// Shared-memory bookkeeping after the (1024-byte aligned) stage ring.
+// Shared-memory bookkeeping after the (1024-byte aligned) stage ring.  The barriers the
+// MMA waits on live in the leader: full (the copies of both CTAs of a pair, armed by the
+// leader alone), ready (transforms of both CTAs), acc_empty (epilogues of both CTAs).
+// With the AdaLN transform each CTA's copies complete on its own full[s], which its
+// transform warps wait for.
 struct Bars {
-    uint64_t full[STAGES];    // copy landed (tx count)
-    uint64_t ready[STAGES];   // operand transformed (AdaLN variant), 128 arrivals
-    uint64_t empty[STAGES];   // MMAs reading the stage finished (tcgen05.commit)
-    uint64_t acc_full[2];     // accumulator complete (tcgen05.commit)
-    uint64_t acc_empty[2];    // accumulator drained by the epilogue, 128 arrivals
-    uint64_t drain;           // every MMA of this CTA finished (teardown)
+    uint64_t full[MAX_STAGES];       // copies landed (tx count)
+    uint64_t ready[MAX_STAGES];      // A rewritten by the transform, one arrival per warp
+    uint64_t empty[MAX_STAGES];      // MMAs reading the stage finished (tcgen05.commit)
+    uint64_t acc_full[2];            // accumulator complete (tcgen05.commit)
+    uint64_t acc_empty[2];           // accumulator drained, one arrival per epilogue warp
+    uint64_t drain;                  // every MMA issued by this CTA finished (teardown)
+    int32_t peer_last[MAX_STAGES];   // pair leader: phase of the peer's last copy per stage (-1: none)
     uint32_t tmem_base;
     volatile int32_t abort;
 };
 
-constexpr size_t smem_bytes() { return 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Bars); }
+template <bool PAIR> constexpr size_t smem_bytes()
+{
+    return 1024 /*alignment slack*/ + (size_t)Shape<PAIR>::STAGES * Shape<PAIR>::STAGE_BYTES + sizeof(Bars);
+}
 
 __device__ uint32_t g_gemm_error;
 
@@ -95,9 +122,28 @@ struct Params {
     float eps;
 };
 
+// Where this CTA sits: its rank in the pair (0 when single), the index of its pair (or
+// CTA) among the persistent workers, and how many workers there are.
+struct Where {
+    uint32_t rank;
+    int64_t worker, n_workers;
+};
+
+template <bool PAIR> __device__ __forceinline__ Where where()
+{
+    Where w;
+    w.rank = PAIR ? tc::cluster_rank() : 0u;
+    w.worker = PAIR ? blockIdx.x / 2 : blockIdx.x;
+    w.n_workers = PAIR ? gridDim.x / 2 : gridDim.x;
+    return w;
+}
+
+// Tile t -> (m-block of TILE_M rows, n-block of 256 columns), rastered in groups of
+// GROUP_M m-blocks so concurrent tiles share A rows and B columns in L2.
+template <bool PAIR>
 __device__ __forceinline__ void tile_coords(int64_t t, const Params& p, int64_t& m_blk, int32_t& n_blk)
 {
-    const int64_t num_m = (p.M + BM - 1) / BM;
+    const int64_t num_m = (p.M + Shape<PAIR>::TILE_M - 1) / Shape<PAIR>::TILE_M;
     const int64_t per_group = (int64_t)GROUP_M * p.n_tiles_n;
     const int64_t g = t / per_group;
     const int64_t first_m = g * GROUP_M;
@@ -108,11 +154,27 @@ __device__ __forceinline__ void tile_coords(int64_t t, const Params& p, int64_t&
 }
 
 // Bounded wait that also gives up as soon as another role of the CTA has aborted.
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, Bars* b)
+// Pair barriers are waited with acquire at cluster scope (the peer arrives on them).
+// SOL_GEMM_PAIR_POLL 1: pair waits poll with the hardware's own short time limit (no
+// suspend-time hint), giving up after kWaitLimitPoll polls.
+#ifndef SOL_GEMM_PAIR_POLL
+#define SOL_GEMM_PAIR_POLL 1
+#endif
+constexpr uint32_t kWaitLimitPoll = 1u << 26;
+
+template <bool PAIR> __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, Bars* b)
 {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (b->abort) return false;
+    const uint32_t limit = (PAIR && SOL_GEMM_PAIR_POLL) ? kWaitLimitPoll : kWaitLimit;
+    for (uint32_t i = 0; i < limit; ++i) {
+        bool ok;
+        if (!PAIR)
+            ok = mbar_try_wait(bar, parity);
+        else if (SOL_GEMM_PAIR_POLL)
+            ok = tc::mbar_poll_cluster(bar, parity);
+        else
+            ok = tc::mbar_try_wait_cluster(bar, parity, 1000000u);
+        if (ok) return true;
+        if ((i & 15u) == 15u && b->abort) return false;
     }
     return false;
 }
@@ -124,69 +186,99 @@ __device__ __forceinline__ void raise_abort(Bars* b, uint32_t code)
 }
 
 // ---------------------------------------------------------------------------------
-// Producer: one thread streams the A and B tiles of every (tile, k-block) into the ring.
-// B rows of a tile: [n0, n0+128) and [n1, n1+128); for SwiGLU n0 = 128*n_blk (gated
-// half) and n1 = inner + 128*n_blk (multiplying half), otherwise n0 = 256*n_blk and
-// n1 = n0 + 128.  Rows of A past M read as zeros (tensor-map bounds).
-template <int EPI>
+// Producer (one thread per CTA): for every (tile, k-block) wait until the stage slot is
+// free, then copy this CTA's 128 rows of A and its rows of B into it.  B rows of a tile:
+// [n0, n0+128) and [n1, n1+128), with n0 = 128*n_blk (gated half) and n1 = inner +
+// 128*n_blk (multiplying half) for SwiGLU, else n0 = 256*n_blk and n1 = n0 + 128; a single
+// CTA loads both, CTA r of a pair loads n_r.  Rows of A past M read as zeros (tensor-map
+// bounds).  The copies complete on this CTA's full[s], except those of a pair's peer
+// without the transform, which complete on the leader's full[s]: the leader arms it for
+// the bytes of both CTAs (the peer's copies may land before the leader arms the phase;
+// the phase cannot complete before the leader's arrival), so the peer makes no remote
+// arrival, whose cluster-scope release would cost more than the copy issue itself.
+template <int EPI, bool PRO, bool PAIR>
 __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const Params& p, uint8_t* ring,
-                             Bars* b)
+                             Bars* b, const Where& w)
 {
+    using S = Shape<PAIR>;
+    const bool remote = PAIR && !PRO && w.rank == 1;  // this CTA's copies complete on the leader
     const int kblocks = p.K / BK;
     int s = 0;
     uint32_t phase = 0;
-    int32_t last_parity[STAGES];
+    int32_t last_parity[MAX_STAGES];
 #pragma unroll
-    for (int i = 0; i < STAGES; ++i) last_parity[i] = -1;
+    for (int i = 0; i < MAX_STAGES; ++i) last_parity[i] = -1;
 
-    for (int64_t t = blockIdx.x; t < p.num_tiles && !b->abort; t += gridDim.x) {
+    for (int64_t t = w.worker; t < p.num_tiles && !b->abort; t += w.n_workers) {
         int64_t m_blk;
         int32_t n_blk;
-        tile_coords(t, p, m_blk, n_blk);
-        const int32_t y_a = (int32_t)(m_blk * BM);
+        tile_coords<PAIR>(t, p, m_blk, n_blk);
+        const int32_t y_a = (int32_t)(m_blk * S::TILE_M + (int64_t)w.rank * BM);
         const int32_t n0 = EPI == EPI_SWIGLU ? n_blk * (BN / 2) : n_blk * BN;
         const int32_t n1 = EPI == EPI_SWIGLU ? p.inner + n_blk * (BN / 2) : n0 + BN / 2;
         for (int kb = 0; kb < kblocks; ++kb) {
-            if (!wait_or_abort(smem_u32(&b->empty[s]), phase ^ 1u, b)) {
+            if (!wait_or_abort<PAIR>(smem_u32(&b->empty[s]), phase ^ 1u, b)) {
                 raise_abort(b, 1u);
                 break;
             }
-            const uint32_t full = smem_u32(&b->full[s]);
-            const uint32_t dst = smem_u32(ring + (size_t)s * STAGE_BYTES);
-            mbar_arrive_expect_tx(full, STAGE_BYTES);
-            tc::tma_load_2d(dst, tmA, kb * BK, y_a, full);
-            tc::tma_load_2d(dst + A_BYTES, tmB, kb * BK, n0, full);
-            tc::tma_load_2d(dst + A_BYTES + B_BYTES / 2, tmB, kb * BK, n1, full);
+            const uint32_t dst = smem_u32(ring + (size_t)s * S::STAGE_BYTES);
+            if (remote) {
+                // no arrival from the peer: the leader armed full[s] for both CTAs' bytes
+                const uint32_t bar = tc::mapa(smem_u32(&b->full[s]), 0);
+                tc::tma_load_2d_pair(dst, tmA, kb * BK, y_a, bar);
+                tc::tma_load_2d_pair(dst + A_BYTES, tmB, kb * BK, n1, bar);
+            } else {
+                const uint32_t full = smem_u32(&b->full[s]);
+                mbar_arrive_expect_tx(full, (PAIR && !PRO) ? 2 * S::STAGE_BYTES : S::STAGE_BYTES);
+                tc::tma_load_2d(dst, tmA, kb * BK, y_a, full);
+                if (PAIR) {
+                    tc::tma_load_2d(dst + A_BYTES, tmB, kb * BK, w.rank == 0 ? n0 : n1, full);
+                } else {
+                    tc::tma_load_2d(dst + A_BYTES, tmB, kb * BK, n0, full);
+                    tc::tma_load_2d(dst + A_BYTES + S::B_BYTES / 2, tmB, kb * BK, n1, full);
+                }
+            }
             last_parity[s] = (int32_t)phase;
-            if (++s == STAGES) {
+            if (++s == S::STAGES) {
                 s = 0;
                 phase ^= 1u;
             }
         }
     }
-    // Teardown: every copy issued must have landed before the CTA may exit.
+    // Teardown: every copy issued must have landed before the CTA may exit.  A peer whose
+    // copies complete on the leader hands its last phase per stage to the leader, which
+    // waits for them between two cluster barriers at the end of the kernel.
+    if (remote) {
 #pragma unroll
-    for (int i = 0; i < STAGES; ++i)
+        for (int i = 0; i < MAX_STAGES; ++i)
+            tc::st_cluster_u32(tc::mapa(smem_u32(&b->peer_last[i]), 0), (uint32_t)last_parity[i]);
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < MAX_STAGES; ++i)
         if (last_parity[i] >= 0 && !mbar_wait_bounded(smem_u32(&b->full[i]), (uint32_t)last_parity[i], kWaitLimit))
             atomicOr(&g_gemm_error, 2u);
 }
 
 // ---------------------------------------------------------------------------------
-// MMA issuer: one thread.  Stage s is consumed once its copy landed (or, with the AdaLN
-// transform, once the transform warps rewrote it); its slot is released by a commit
-// when the four MMAs reading it finish.
-template <bool PRO>
-__device__ void run_mma(const Params& p, uint8_t* ring, Bars* b)
+// MMA issuer: one thread (of the leader, in a pair).  Stage s is consumed once its copies
+// landed (full[s], counting both CTAs' copies in a pair) or, with the AdaLN
+// transform, once the transform warps (of both CTAs) rewrote it (ready[s]).  The slot is
+// released by a commit to empty[s] of each CTA when the four MMAs reading it finish; a
+// finished accumulator is announced by a commit to acc_full of each CTA.
+template <bool PRO, bool PAIR>
+__device__ void run_mma(const Params& p, uint8_t* ring, Bars* b, const Where& w)
 {
+    using S = Shape<PAIR>;
     const int kblocks = p.K / BK;
-    const uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
+    const uint32_t idesc = tc::idesc_bf16_f32(S::TILE_M, BN);
     int s = 0;
     uint32_t phase = 0;
     int64_t it = 0;
-    for (int64_t t = blockIdx.x; t < p.num_tiles && !b->abort; t += gridDim.x, ++it) {
+    for (int64_t t = w.worker; t < p.num_tiles && !b->abort; t += w.n_workers, ++it) {
         const int ab = (int)(it & 1);
         const uint32_t acc_phase = (uint32_t)((it >> 1) & 1);
-        if (!wait_or_abort(smem_u32(&b->acc_empty[ab]), acc_phase ^ 1u, b)) {
+        if (!wait_or_abort<PAIR>(smem_u32(&b->acc_empty[ab]), acc_phase ^ 1u, b)) {
             raise_abort(b, 4u);
             break;
         }
@@ -194,33 +286,56 @@ __device__ void run_mma(const Params& p, uint8_t* ring, Bars* b)
         const uint32_t d_tmem = b->tmem_base + (uint32_t)(ab * BN);
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb) {
-            const uint32_t bar = PRO ? smem_u32(&b->ready[s]) : smem_u32(&b->full[s]);
-            if (!wait_or_abort(bar, phase, b)) {
+            bool got;
+            if (PRO)
+                got = wait_or_abort<PAIR>(smem_u32(&b->ready[s]), phase, b);
+            else
+                got = wait_or_abort<PAIR>(smem_u32(&b->full[s]), phase, b);
+            if (!got) {
                 raise_abort(b, 8u);
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
-            const uint32_t a_addr = smem_u32(ring + (size_t)s * STAGE_BYTES);
+            const uint32_t a_addr = smem_u32(ring + (size_t)s * S::STAGE_BYTES);
             const uint64_t a_desc = tc::smem_desc_sw128(a_addr);
             const uint64_t b_desc = tc::smem_desc_sw128(a_addr + A_BYTES);
 #pragma unroll
             for (int kk = 0; kk < BK / UK; ++kk) {
                 // advance K by 16 elements = 32 bytes inside the swizzle row (field >> 4)
-                tc::mma_bf16(d_tmem, a_desc + (uint64_t)(kk * 2), b_desc + (uint64_t)(kk * 2), idesc,
-                             (kb | kk) != 0 ? 1u : 0u);
+                const uint64_t da = a_desc + (uint64_t)(kk * 2), db = b_desc + (uint64_t)(kk * 2);
+                const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+                if (PAIR)
+                    tc::mma_bf16_pair(d_tmem, da, db, idesc, acc);
+                else
+                    tc::mma_bf16(d_tmem, da, db, idesc, acc);
             }
-            tc::commit(smem_u32(&b->empty[s]));
-            if (++s == STAGES) {
+            const uint32_t e = smem_u32(&b->empty[s]);
+            if (PAIR) {
+                tc::commit_pair(e);
+                tc::commit_pair(tc::mapa(e, 1));
+            } else {
+                tc::commit(e);
+            }
+            if (++s == S::STAGES) {
                 s = 0;
                 phase ^= 1u;
             }
         }
         if (!ok) break;
-        tc::commit(smem_u32(&b->acc_full[ab]));
+        const uint32_t f = smem_u32(&b->acc_full[ab]);
+        if (PAIR) {
+            tc::commit_pair(f);
+            tc::commit_pair(tc::mapa(f, 1));
+        } else {
+            tc::commit(f);
+        }
     }
     // Teardown: wait for every MMA this thread issued.
-    tc::commit(smem_u32(&b->drain));
+    if (PAIR)
+        tc::commit_pair(smem_u32(&b->drain));
+    else
+        tc::commit(smem_u32(&b->drain));
     if (!mbar_wait_bounded(smem_u32(&b->drain), 0u, kWaitLimit)) atomicOr(&g_gemm_error, 16u);
 }
 
@@ -307,18 +422,19 @@ __device__ __forceinline__ void qk_head(uint32_t taddr, bool live, const bf16* w
     }
 }
 
-// Epilogue warps 2..5: thread (warp w, lane l) owns accumulator row 32*(w % 4) + l, the
-// TMEM lane quarter warp w may access.
-template <int EPI>
-__device__ void run_epilogue(const Params& p, Bars* b)
+// Epilogue warps 2..5: thread (warp w, lane l) owns accumulator row 32*(w % 4) + l of this
+// CTA's 128 rows, the TMEM lane quarter warp w may access.  A drained accumulator is
+// announced to the leader's acc_empty (one arrival per warp of each CTA).
+template <int EPI, bool PAIR>
+__device__ void run_epilogue(const Params& p, Bars* b, const Where& w)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3;
     int64_t it = 0;
-    for (int64_t t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++it) {
+    for (int64_t t = w.worker; t < p.num_tiles; t += w.n_workers, ++it) {
         const int ab = (int)(it & 1);
         const uint32_t acc_phase = (uint32_t)((it >> 1) & 1);
-        const bool got = wait_or_abort(smem_u32(&b->acc_full[ab]), acc_phase, b);
+        const bool got = wait_or_abort<PAIR>(smem_u32(&b->acc_full[ab]), acc_phase, b);
         if (!__all_sync(0xffffffffu, got)) {
             raise_abort(b, 32u);
             break;
@@ -326,8 +442,8 @@ __device__ void run_epilogue(const Params& p, Bars* b)
         tc::fence_after_sync();
         int64_t m_blk;
         int32_t n_blk;
-        tile_coords(t, p, m_blk, n_blk);
-        const int64_t row = m_blk * BM + quarter * 32 + lane;
+        tile_coords<PAIR>(t, p, m_blk, n_blk);
+        const int64_t row = m_blk * Shape<PAIR>::TILE_M + (int64_t)w.rank * BM + quarter * 32 + lane;
         const bool live = row < p.M;
         const uint32_t tbase = b->tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * BN);
         float v[32];
@@ -394,141 +510,254 @@ __device__ void run_epilogue(const Params& p, Bars* b)
             }
         }
         tc::fence_before_sync();
-        tc::mbar_arrive(smem_u32(&b->acc_empty[ab]));
+        __syncwarp();
+        if (lane == 0) {
+            // the leader's acc_empty (this CTA's own when single)
+            const uint32_t e = smem_u32(&b->acc_empty[ab]);
+            if (PAIR)
+                tc::mbar_arrive_cluster(tc::mapa(e, 0));
+            else
+                tc::mbar_arrive(e);
+        }
     }
 }
 
+
 // ---------------------------------------------------------------------------------
-// AdaLN operand transform (warps 6..9): thread m rewrites row m of every landed A tile
-// in place.  In the 128-byte swizzle a row is eight 16-byte chunks; physical chunk c of
-// row m holds logical chunk c ^ (m % 8), i.e. columns 8*(c ^ (m % 8)) .. +7 of the
-// k-block.  Thread m visits its chunks starting at chunk m % 8, so the eight threads of
-// a quarter-warp touch eight different bank groups.  Rows past M stay zero (never
-// stored).  Each thread fences its generic-proxy writes before arriving, so the
-// tensor core (async proxy) reads the rewritten tile.
-__device__ void run_transform(const Params& p, uint8_t* ring, Bars* b)
+// AdaLN operand transform (warps 6 and up: XFORM_GROUPS groups of four warps taking
+// alternate k-blocks, so a group has XFORM_GROUPS MMA stage times per k-block).  The
+// tensor copy lands the x tile (bf16, 128-byte swizzle) in the stage's A slot; the group
+// rewrites it in place as
+//     h = fma(fma(x, rstd, -mean * rstd), 1 + scale, shift)       (fp32, stored bf16)
+// and arrives on the leader's ready[s], which the MMA waits for instead of full[s] (the
+// transform itself waits for this CTA's full[s]).
+// Mapping: lane L of warp w (of the group) handles row m = 4w + L/8 + 16j, j = 0..7, and
+// logical 16-byte chunk kc = (L % 8) ^ (4 * (L / 16)) of each row (columns 8*kc ..
+// 8*kc+7 of the k-block).  Logical chunk kc of row m sits at physical chunk kc ^ (m % 8),
+// which is the same for all j (16j = 0 mod 8), so a thread's chunk position is fixed.
+// The eight lanes of a quarter-warp (L/8 fixed) hit eight different chunks, and so do
+// lanes {0-3, 16-19} (and the other such pairs: their chunk sets differ by the xor with
+// 4 ^ 2), so a 128-bit shared access is conflict-free under either lane grouping.  When
+// its rows share one modulation row (a tile inside one sample and one stream) the thread
+// holds that row's 1 + scale and shift for its eight columns, fetched one k-block ahead;
+// otherwise each row loads its own.  Rows past M stay zero (never stored).  Each thread
+// fences its generic-proxy stores before its warp arrives, so the tensor core (async
+// proxy) reads the rewritten tile.
+#ifndef SOL_GEMM_XFORM_GROUPS
+#define SOL_GEMM_XFORM_GROUPS 2
+#endif
+constexpr int XFORM_GROUPS = SOL_GEMM_XFORM_GROUPS;
+constexpr int XFORM_WARPS = 4;
+constexpr int XFORM_THREADS = 32 * XFORM_WARPS * XFORM_GROUPS;
+// every stage must always belong to the same group (XFORM_WARPS arrivals per CTA and use)
+static_assert(Shape<false>::STAGES % XFORM_GROUPS == 0 && Shape<true>::STAGES % XFORM_GROUPS == 0,
+              "the transform groups must divide the stage count");
+
+__device__ __forceinline__ uint4 lds128(uint32_t a)
 {
-    const int m = threadIdx.x - XFORM_WARP0 * 32;
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, const uint4& v)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void load_mod8(const Params& p, int64_t r, int k0, float2* g, float2* sh)
+{
+    if (p.scale) {
+        unpack2<bf16>(ld_cached(p.scale + r * p.ld_mod + k0), g);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) g[e] = make_float2(0.f, 0.f);
+    }
+    if (p.shift) {
+        unpack2<bf16>(ld_cached(p.shift + r * p.ld_mod + k0), sh);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sh[e] = make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) g[e] = __fadd2_rn(make_float2(1.f, 1.f), g[e]);
+}
+
+template <bool PAIR>
+__device__ void run_transform(const Params& p, uint8_t* ring, Bars* b, const Where& w)
+{
+    using S = Shape<PAIR>;
+    const int tg = threadIdx.x - XFORM_WARP0 * 32;
+    const int lane = threadIdx.x & 31;
+    const int group = tg / (32 * XFORM_WARPS);
+    const int wg = (tg % (32 * XFORM_WARPS)) >> 5;  // warp within the group
+    const int r8 = 4 * wg + (lane >> 3);            // first row, 0..15
+    const int kc = (lane & 7) ^ (4 * (lane >> 4));
+    const int phys = kc ^ (r8 & 7);
     const int kblocks = p.K / BK;
-    int s = 0;
-    uint32_t phase = 0;
-    for (int64_t t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+    const uint32_t ring_s = smem_u32(ring);
+    int64_t kglob = 0;                              // k-blocks of earlier tiles: ring position
+    for (int64_t tile = w.worker; tile < p.num_tiles; tile += w.n_workers) {
         int64_t m_blk;
         int32_t n_blk;
-        tile_coords(t, p, m_blk, n_blk);
-        const int64_t row = m_blk * BM + m;
-        const bool live = row < p.M;
-        float mu = 0.f, rs = 0.f;
-        const bf16 *sc = nullptr, *sh = nullptr;
-        if (live) {
-            const float2 st = __ldg(p.stats + row);
-            mu = st.x;
-            rs = st.y;
-            const int64_t r = mod_row(row, p.sel);
-            if (p.scale) sc = p.scale + r * p.ld_mod;
-            if (p.shift) sh = p.shift + r * p.ld_mod;
+        tile_coords<PAIR>(tile, p, m_blk, n_blk);
+        const int64_t row0 = m_blk * S::TILE_M + (int64_t)w.rank * BM + r8;
+        float2 ac[8];                                // (rstd, -mean * rstd) per row
+        uint32_t live = 0;
+        bool uniform = true;
+        int64_t rmod0 = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int64_t row = row0 + 16 * j;
+            ac[j] = make_float2(0.f, 0.f);
+            if (row < p.M) {
+                const float2 st = __ldg(p.stats + row);
+                ac[j] = make_float2(st.y, -st.x * st.y);
+                const int64_t r = mod_row(row, p.sel);
+                if (j == 0) rmod0 = r;
+                else if (r != rmod0) uniform = false;
+                live |= 1u << j;
+            }
         }
+        int kb = (int)(((group - kglob % XFORM_GROUPS) % XFORM_GROUPS + XFORM_GROUPS) % XFORM_GROUPS);
+        float2 g[4], sh[4], gn[4], shn[4];
+        if (uniform && kb < kblocks) load_mod8(p, rmod0, kb * BK + 8 * kc, g, sh);
         bool ok = true;
-        for (int kb = 0; kb < kblocks; ++kb) {
-            if (!wait_or_abort(smem_u32(&b->full[s]), phase, b)) {
+        for (; kb < kblocks; kb += XFORM_GROUPS) {
+            const int64_t kg = kglob + kb;
+            const int s = (int)(kg % S::STAGES);
+            const uint32_t phase = (uint32_t)((kg / S::STAGES) & 1);
+            const int k0 = kb * BK + 8 * kc;
+            if (uniform && kb + XFORM_GROUPS < kblocks) load_mod8(p, rmod0, k0 + XFORM_GROUPS * BK, gn, shn);
+            if (!wait_or_abort<PAIR>(smem_u32(&b->full[s]), phase, b)) {
                 raise_abort(b, 64u);
                 ok = false;
                 break;
             }
-            if (live) {
-                uint8_t* base = ring + (size_t)s * STAGE_BYTES + (size_t)m * 128;
-#pragma unroll 2
-                for (int i = 0; i < 8; ++i) {
-                    const int c = (i + m) & 7;
-                    const int k0 = kb * BK + 8 * (c ^ (m & 7));
-                    uint4* cell = reinterpret_cast<uint4*>(base + 16 * c);
-                    float2 f[4], g[4], h[4];
-                    unpack2<bf16>(*cell, f);
-                    if (sc) {
-                        unpack2<bf16>(ld_cached(sc + k0), g);
-                    } else {
+            const uint32_t base = ring_s + (uint32_t)(s * S::STAGE_BYTES + 16 * phys + r8 * 128);
+            uint4 cell[8];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) g[e] = make_float2(0.f, 0.f);
-                    }
-                    if (sh) {
-                        unpack2<bf16>(ld_cached(sh + k0), h);
-                    } else {
+            for (int j = 0; j < 8; ++j)
+                if (live >> j & 1u) cell[j] = lds128(base + 16 * 128 * j);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) h[e] = make_float2(0.f, 0.f);
-                    }
-                    const float2 mu2 = make_float2(mu, mu), rs2 = make_float2(rs, rs), one = make_float2(1.f, 1.f);
+            for (int j = 0; j < 8; ++j) {
+                if (!(live >> j & 1u)) continue;
+                if (!uniform) load_mod8(p, mod_row(row0 + 16 * j, p.sel), k0, g, sh);
+                float2 f[4], h[4];
+                unpack2<bf16>(cell[j], f);
+                const float2 a2 = make_float2(ac[j].x, ac[j].x), c2 = make_float2(ac[j].y, ac[j].y);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 nrm = __fmul2_rn(__fadd2_rn(f[e], make_float2(-mu2.x, -mu2.y)), rs2);
-                        h[e] = __ffma2_rn(nrm, __fadd2_rn(one, g[e]), h[e]);
-                    }
-                    *cell = pack2<bf16>(h);
-                }
+                for (int e = 0; e < 4; ++e) h[e] = __ffma2_rn(__ffma2_rn(f[e], a2, c2), g[e], sh[e]);
+                sts128(base + 16 * 128 * j, pack2<bf16>(h));
             }
             fence_proxy_async_smem();
-            tc::mbar_arrive(smem_u32(&b->ready[s]));
-            if (++s == STAGES) {
-                s = 0;
-                phase ^= 1u;
+            __syncwarp();
+            if (lane == 0) {
+                // the leader's ready[s] (this CTA's own when single)
+                const uint32_t r = smem_u32(&b->ready[s]);
+                if (PAIR)
+                    tc::mbar_arrive_cluster(tc::mapa(r, 0));
+                else
+                    tc::mbar_arrive(r);
+            }
+            if (uniform) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    g[e] = gn[e];
+                    sh[e] = shn[e];
+                }
             }
         }
         if (!ok) break;
+        kglob += kblocks;
     }
 }
 
+
 // ---------------------------------------------------------------------------------
 // The kernel: roles by warp (see the file header).
-template <int EPI, bool PRO>
-__global__ void __launch_bounds__(PRO ? 320 : 192, 1)
+template <int EPI, bool PRO, bool PAIR>
+__global__ void __launch_bounds__(PRO ? 192 + XFORM_THREADS : 192, 1)
     k_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
              const __grid_constant__ Params p)
 {
+    using S = Shape<PAIR>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Bars* b = reinterpret_cast<Bars*>(ring + (size_t)STAGES * STAGE_BYTES);
+    uint8_t* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Bars* b = reinterpret_cast<Bars*>(ring + (size_t)S::STAGES * S::STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Where w = where<PAIR>();
 
     if (threadIdx.x == 0) {
 #pragma unroll
-        for (int i = 0; i < STAGES; ++i) {
+        for (int i = 0; i < S::STAGES; ++i) {
             mbar_init(smem_u32(&b->full[i]), 1);
-            mbar_init(smem_u32(&b->ready[i]), 128);
+            mbar_init(smem_u32(&b->ready[i]), (PAIR ? 2 : 1) * XFORM_WARPS);  // one per warp of each CTA
             mbar_init(smem_u32(&b->empty[i]), 1);
         }
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&b->acc_full[i]), 1);
-            mbar_init(smem_u32(&b->acc_empty[i]), 128);
+            mbar_init(smem_u32(&b->acc_empty[i]), (PAIR ? 2 : 1) * 4);  // one per epilogue warp of each CTA
         }
         mbar_init(smem_u32(&b->drain), 1);
+#pragma unroll
+        for (int i = 0; i < MAX_STAGES; ++i) b->peer_last[i] = -1;
         b->abort = 0;
         mbar_fence_init();
         tc::prefetch_tmap(&tmA);
         tc::prefetch_tmap(&tmB);
     }
     if (warp == MMA_WARP) {
-        tc::tmem_alloc(smem_u32(&b->tmem_base), TMEM_COLS);
-        tc::tmem_relinquish();
+        if constexpr (PAIR) {
+            tc::tmem_alloc_pair(smem_u32(&b->tmem_base), TMEM_COLS);
+            tc::tmem_relinquish_pair();
+        } else {
+            tc::tmem_alloc(smem_u32(&b->tmem_base), TMEM_COLS);
+            tc::tmem_relinquish();
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
+    if constexpr (PAIR) tc::cluster_sync();  // both CTAs' barriers exist before any remote arrival
     tc::fence_after_sync();
 
     if (warp == PRODUCER_WARP) {
-        if (lane == 0) run_producer<EPI>(&tmA, &tmB, p, ring, b);
+        if (lane == 0) run_producer<EPI, PRO, PAIR>(&tmA, &tmB, p, ring, b, w);
     } else if (warp == MMA_WARP) {
-        if (lane == 0) run_mma<PRO>(p, ring, b);
+        if (lane == 0) {
+            if (!PAIR || w.rank == 0) run_mma<PRO, PAIR>(p, ring, b, w);
+        }
     } else if (warp < XFORM_WARP0) {
-        run_epilogue<EPI>(p, b);
+        run_epilogue<EPI, PAIR>(p, b, w);
     } else if (PRO) {
-        run_transform(p, ring, b);
+        run_transform<PAIR>(p, ring, b, w);
     }
 
     tc::fence_before_sync();
     __syncthreads();
+    if constexpr (PAIR) {
+        // the leader's MMAs into this CTA's TMEM have drained; the peer's last copy phases
+        // are in the leader's peer_last
+        tc::cluster_sync();
+        if constexpr (!PRO) {
+            if (w.rank == 0 && threadIdx.x == 0) {
+#pragma unroll
+                for (int i = 0; i < MAX_STAGES; ++i) {
+                    const int32_t ph = b->peer_last[i];
+                    if (ph >= 0 && !mbar_wait_bounded(smem_u32(&b->full[i]), (uint32_t)ph, kWaitLimit))
+                        atomicOr(&g_gemm_error, 2u);
+                }
+            }
+        }
+        tc::cluster_sync();  // every copy into either CTA has landed
+    }
     if (warp == MMA_WARP) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(b->tmem_base, TMEM_COLS);
+        if constexpr (PAIR)
+            tc::tmem_dealloc_pair(b->tmem_base, TMEM_COLS);
+        else
+            tc::tmem_dealloc(b->tmem_base, TMEM_COLS);
     }
 }
 
@@ -597,28 +826,81 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
     if (!fn) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {ld * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)gemm::BK, (cuuint32_t)(gemm::BM)};
+    const cuuint32_t box[2] = {(cuuint32_t)gemm::BK, (cuuint32_t)gemm::BM};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI, bool PRO>
+// Tile shape per variant.  Measured on B200: CTA pairs are faster for the plain and
+// epilogue-fused GEMMs (the copies per MMA drop by a third); with the AdaLN operand
+// transform the single shape is faster (in a pair every transformed stage of the peer
+// must be announced to the leader with a cluster-scope release, which costs more than the
+// deeper ring saves).  SOL_LINEAR_SHAPE=single / pair overrides the choice.
+bool use_pair(bool transform)
+{
+    static const int forced = [] {
+        const char* e = std::getenv("SOL_LINEAR_SHAPE");
+        if (e && std::string(e) == "single") return 0;
+        if (e && std::string(e) == "pair") return 1;
+        return -1;
+    }();
+    return forced >= 0 ? forced == 1 : !transform;
+}
+
+template <int EPI, bool PRO, bool PAIR>
 cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const gemm::Params& p, cudaStream_t s)
 {
-    auto kern = gemm::k_linear<EPI, PRO>;
-    const size_t smem = gemm::smem_bytes();
+    auto kern = gemm::k_linear<EPI, PRO, PAIR>;
+    const size_t smem = gemm::smem_bytes<PAIR>();
+    const int threads = PRO ? 192 + gemm::XFORM_THREADS : 192;
     static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
-    const int64_t grid = std::min<int64_t>(p.num_tiles, (int64_t)sm_count());
-    kern<<<(unsigned)grid, PRO ? 320 : 192, smem, s>>>(ma, mb, p);
-    return cudaGetLastError();
+    if constexpr (!PAIR) {
+        const int64_t grid = std::min<int64_t>(p.num_tiles, (int64_t)sm_count());
+        kern<<<(unsigned)grid, threads, smem, s>>>(ma, mb, p);
+        return cudaGetLastError();
+    } else {
+        cudaLaunchAttribute la[1];
+        la[0].id = cudaLaunchAttributeClusterDimension;
+        la[0].val.clusterDim.x = 2;
+        la[0].val.clusterDim.y = 1;
+        la[0].val.clusterDim.z = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cfg.attrs = la;
+        cfg.numAttrs = 1;
+        // as many pairs as can be resident at once (persistent workers)
+        static int max_pairs = [&] {
+            cudaLaunchConfig_t q = cfg;
+            q.gridDim = dim3(2 * (sm_count() / 2));
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n < 1) n = sm_count() / 2;
+            return n;
+        }();
+        const int64_t pairs = std::min<int64_t>(p.num_tiles, (int64_t)max_pairs);
+        cfg.gridDim = dim3((unsigned)(2 * pairs));
+        return cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
+    }
+}
+
+template <int EPI, bool PRO>
+cudaError_t launch_shape(const CUtensorMap& ma, const CUtensorMap& mb, gemm::Params& p, int64_t M, cudaStream_t s)
+{
+    if (use_pair(PRO)) {
+        p.num_tiles = (M + gemm::Shape<true>::TILE_M - 1) / gemm::Shape<true>::TILE_M * (int64_t)p.n_tiles_n;
+        return launch_kernel<EPI, PRO, true>(ma, mb, p, s);
+    }
+    p.num_tiles = (M + gemm::Shape<false>::TILE_M - 1) / gemm::Shape<false>::TILE_M * (int64_t)p.n_tiles_n;
+    return launch_kernel<EPI, PRO, false>(ma, mb, p, s);
 }
 
 }  // namespace
 
-size_t linear_smem_bytes() { return gemm::smem_bytes(); }
+size_t linear_smem_bytes() { return gemm::smem_bytes<true>(); }
 
 cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cudaStream_t s)
 {
@@ -634,7 +916,6 @@ cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cuda
     p.K = a.K;
     p.n_tiles_n = a.N / gemm::BN;  // SwiGLU: inner / 128 pair tiles of 256 columns
     p.inner = a.N / 2;
-    p.num_tiles = (a.M + gemm::BM - 1) / gemm::BM * (int64_t)p.n_tiles_n;
     p.out = static_cast<bf16*>(a.out);
     p.ld_out = a.ld_out;
     p.x = static_cast<const bf16*>(a.x);
@@ -664,14 +945,15 @@ cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cuda
     }
     switch (epi) {
     case LINEAR_STORE:
-        return adaln ? launch_kernel<gemm::EPI_STORE, true>(ma, mb, p, s) : launch_kernel<gemm::EPI_STORE, false>(ma, mb, p, s);
+        return adaln ? launch_shape<gemm::EPI_STORE, true>(ma, mb, p, a.M, s)
+                     : launch_shape<gemm::EPI_STORE, false>(ma, mb, p, a.M, s);
     case LINEAR_GATED:
-        return launch_kernel<gemm::EPI_GATED, false>(ma, mb, p, s);
+        return launch_shape<gemm::EPI_GATED, false>(ma, mb, p, a.M, s);
     case LINEAR_SWIGLU:
-        return launch_kernel<gemm::EPI_SWIGLU, false>(ma, mb, p, s);
+        return launch_shape<gemm::EPI_SWIGLU, false>(ma, mb, p, a.M, s);
     case LINEAR_QKROPE:
-        return adaln ? launch_kernel<gemm::EPI_QKROPE, true>(ma, mb, p, s)
-                     : launch_kernel<gemm::EPI_QKROPE, false>(ma, mb, p, s);
+        return adaln ? launch_shape<gemm::EPI_QKROPE, true>(ma, mb, p, a.M, s)
+                     : launch_shape<gemm::EPI_QKROPE, false>(ma, mb, p, a.M, s);
     }
     return cudaErrorInvalidValue;
 }
