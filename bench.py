@@ -477,12 +477,12 @@ def time_linear_ops(bufs, dev, args) -> dict:
                      "libsol_plain_gemm_ms": round(tp, 4), "speedup_vs_unfused": round(tu / tf, 3),
                      "hbm_bytes_saved_per_token": saved_bytes}
 
-    stats = sol.row_stats_workspace(m, dev)
+    ws = sol.adaln_workspace(m, 3 * hd, d, device=dev)
     Wqkv = wl.linear_weight(w, "w_qkv", 3 * hd, d, dev)
     qkv = torch.empty((m, 3 * hd), dtype=w.dtype, device=dev)
     h = torch.empty_like(x)
     sh, sc = i["shift_msa"][:1], i["scale_msa"][:1]
-    fused = lambda: sol.adaln_qkv_rope(qkv, x, Wqkv, bufs.rope, sh, sc, row_stats=stats, n_heads=w.n_heads,
+    fused = lambda: sol.adaln_qkv_rope(qkv, x, Wqkv, bufs.rope, sh, sc, workspace=ws, n_heads=w.n_heads,
                                        wq=i["wq"], wk=i["wk"], grid=w.grid, eps=w.eps, **sel)
 
     def unfused():
@@ -492,7 +492,7 @@ def time_linear_ops(bufs, dev, args) -> dict:
                          grid=w.grid, eps=w.eps)
     entry("adaln_qkv_rope", 2.0 * m * d * 3 * hd, fused, unfused, lambda: torch.matmul(x, Wqkv.t(), out=qkv),
           lambda: sol.linear(qkv, x, Wqkv), 2 * d * 2 + 2 * (2 * hd) * 2)
-    del Wqkv, qkv, h, stats
+    del Wqkv, qkv, h, ws
 
     for name, K, wname, gate in (("o_proj_gated_residual", d, "w_o", "gate_msa"),
                                  ("down_proj_gated_residual", inner, "w_down", "gate_mlp")):

@@ -55,7 +55,10 @@ constexpr int A_BYTES = BM * BK * 2;      // 16 KiB: this CTA's rows of A per st
 constexpr int TMEM_COLS = 2 * BN;         // two accumulators
 constexpr int GROUP_M = 16;               // m-blocks per raster group (L2 reuse)
 constexpr int MAX_STAGES = 6;
-constexpr int PRODUCER_WARP = 0, MMA_WARP = 1, XFORM_WARP0 = 6;  // epilogue: warps 2..5
+constexpr int PRODUCER_WARP = 0, MMA_WARP = 1, EPI_WARP0 = 2, XFORM_WARP0 = 6;
+// Epilogue warps: 8 (two per TMEM lane quarter, each taking half of the 256 columns), or
+// 4 beside the AdaLN transform warps (the register file holds no more).
+template <bool PRO> __host__ __device__ constexpr int epi_warps() { return PRO ? 4 : 8; }
 constexpr uint32_t kWaitLimit = 4096;     // polls of <= ~1 ms each
 
 template <bool PAIR> struct Shape {
@@ -120,6 +123,11 @@ struct Params {
     RopeDev rope;
     int32_t qk_cols;      // 2 * n_heads * head_dim: columns that get norm + RoPE
     float eps;
+    // AdaLN folded into the weights: y = rstd * (x . V_r^T - mean * c_r) + b_r
+    const uint32_t* rmask;  // [ceil(M / 128)]: bit r set if a row of the 128-row block uses row r
+    const float* fold_c;    // [R, n_w]: column sums of the folded weights V_r
+    const float* fold_b;    // [R, n_w]: shift_r . W^T
+    int32_t n_w;            // output columns (rows of W) per modulation row
 };
 
 // Where this CTA sits: its rank in the pair (0 when single), the index of its pair (or
@@ -151,6 +159,46 @@ __device__ __forceinline__ void tile_coords(int64_t t, const Params& p, int64_t&
     const int64_t local = t - g * per_group;
     m_blk = first_m + local % gm;
     n_blk = (int32_t)(local / gm);
+}
+
+// Modulation rows used by the rows of m-block m_blk (AdaLN fold), else one pass.
+template <bool PAIR, bool FOLD>
+__device__ __forceinline__ uint32_t tile_rows_mask(const Params& p, int64_t m_blk)
+{
+    if (!FOLD) return 1u;
+    const int64_t b0 = m_blk * (Shape<PAIR>::TILE_M / BM);
+    uint32_t m = __ldg(p.rmask + b0);
+    if (PAIR && (b0 + 1) * BM < p.M) m |= __ldg(p.rmask + b0 + 1);
+    return m;
+}
+
+// One unit of work: a tile or, with the AdaLN fold, a tile and one modulation row present
+// in its rows (computed with that row's folded weights; the epilogue stores only the rows
+// that use it).  Every role walks the same sequence of passes.
+struct Pass {
+    int64_t t;
+    int64_t m_blk;
+    int32_t n_blk;
+    uint32_t rm;  // modulation rows of this tile still to do
+    int32_t r;    // modulation row of this pass
+};
+
+__device__ __forceinline__ Pass pass_begin() { return Pass{-1, 0, 0, 0u, 0}; }
+
+template <bool PAIR, bool FOLD>
+__device__ __forceinline__ bool next_pass(Pass& q, const Params& p, const Where& w)
+{
+    while (true) {
+        if (q.rm) {
+            q.r = __ffs(q.rm) - 1;
+            q.rm &= q.rm - 1;
+            return true;
+        }
+        q.t = q.t < 0 ? w.worker : q.t + w.n_workers;
+        if (q.t >= p.num_tiles) return false;
+        tile_coords<PAIR>(q.t, p, q.m_blk, q.n_blk);
+        q.rm = tile_rows_mask<PAIR, FOLD>(p, q.m_blk);
+    }
 }
 
 // Bounded wait that also gives up as soon as another role of the CTA has aborted.
@@ -196,7 +244,7 @@ __device__ __forceinline__ void raise_abort(Bars* b, uint32_t code)
 // the bytes of both CTAs (the peer's copies may land before the leader arms the phase;
 // the phase cannot complete before the leader's arrival), so the peer makes no remote
 // arrival, whose cluster-scope release would cost more than the copy issue itself.
-template <int EPI, bool PRO, bool PAIR>
+template <int EPI, bool PRO, bool FOLD, bool PAIR>
 __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const Params& p, uint8_t* ring,
                              Bars* b, const Where& w)
 {
@@ -209,12 +257,14 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
 #pragma unroll
     for (int i = 0; i < MAX_STAGES; ++i) last_parity[i] = -1;
 
-    for (int64_t t = w.worker; t < p.num_tiles && !b->abort; t += w.n_workers) {
-        int64_t m_blk;
-        int32_t n_blk;
-        tile_coords<PAIR>(t, p, m_blk, n_blk);
+    Pass q = pass_begin();
+    while (!b->abort && next_pass<PAIR, FOLD>(q, p, w)) {
+        const int64_t m_blk = q.m_blk;
+        const int32_t n_blk = q.n_blk;
         const int32_t y_a = (int32_t)(m_blk * S::TILE_M + (int64_t)w.rank * BM);
-        const int32_t n0 = EPI == EPI_SWIGLU ? n_blk * (BN / 2) : n_blk * BN;
+        // with the fold, B is this pass's modulation row's block of folded weights
+        const int32_t nr = FOLD ? q.r * p.n_w : 0;
+        const int32_t n0 = EPI == EPI_SWIGLU ? n_blk * (BN / 2) : nr + n_blk * BN;
         const int32_t n1 = EPI == EPI_SWIGLU ? p.inner + n_blk * (BN / 2) : n0 + BN / 2;
         for (int kb = 0; kb < kblocks; ++kb) {
             if (!wait_or_abort<PAIR>(smem_u32(&b->empty[s]), phase ^ 1u, b)) {
@@ -266,7 +316,7 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
 // transform, once the transform warps (of both CTAs) rewrote it (ready[s]).  The slot is
 // released by a commit to empty[s] of each CTA when the four MMAs reading it finish; a
 // finished accumulator is announced by a commit to acc_full of each CTA.
-template <bool PRO, bool PAIR>
+template <bool PRO, bool FOLD, bool PAIR>
 __device__ void run_mma(const Params& p, uint8_t* ring, Bars* b, const Where& w)
 {
     using S = Shape<PAIR>;
@@ -275,7 +325,8 @@ __device__ void run_mma(const Params& p, uint8_t* ring, Bars* b, const Where& w)
     int s = 0;
     uint32_t phase = 0;
     int64_t it = 0;
-    for (int64_t t = w.worker; t < p.num_tiles && !b->abort; t += w.n_workers, ++it) {
+    Pass q = pass_begin();
+    for (; !b->abort && next_pass<PAIR, FOLD>(q, p, w); ++it) {
         const int ab = (int)(it & 1);
         const uint32_t acc_phase = (uint32_t)((it >> 1) & 1);
         if (!wait_or_abort<PAIR>(smem_u32(&b->acc_empty[ab]), acc_phase ^ 1u, b)) {
@@ -374,16 +425,41 @@ __device__ __forceinline__ void token_pos(int64_t row, const Params& p, int& p0,
     }
 }
 
+// AdaLN folded into the weights: the accumulator row holds x . V_r^T; the projection of
+// h = (x - mean) * rstd * (1 + scale_r) + shift_r is rstd * (acc - mean * c_r) + b_r.
+struct FoldRow {
+    float mu, rs;
+    const float* c;  // c_r + the tile's first column
+    const float* b;  // b_r + the tile's first column
+};
+
+template <bool FOLD> __device__ __forceinline__ void fold32(float* v, const FoldRow& f, int col)
+{
+    if constexpr (FOLD) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 c4 = __ldg(reinterpret_cast<const float4*>(f.c + col) + j);
+            const float4 b4 = __ldg(reinterpret_cast<const float4*>(f.b + col) + j);
+            v[4 * j + 0] = fmaf(f.rs, fmaf(-f.mu, c4.x, v[4 * j + 0]), b4.x);
+            v[4 * j + 1] = fmaf(f.rs, fmaf(-f.mu, c4.y, v[4 * j + 1]), b4.y);
+            v[4 * j + 2] = fmaf(f.rs, fmaf(-f.mu, c4.z, v[4 * j + 2]), b4.z);
+            v[4 * j + 3] = fmaf(f.rs, fmaf(-f.mu, c4.w, v[4 * j + 3]), b4.w);
+        }
+    }
+}
+
 // One 128-wide head vector of the accumulator row (TMEM columns taddr .. +127):
 // v / sqrt(mean(v^2) + eps) * w, then the interleaved 3D rotation, stored to dst.
+template <bool FOLD>
 __device__ __forceinline__ void qk_head(uint32_t taddr, bool live, const bf16* w, const Params& p, int p0, int p1,
-                                        int p2, bf16* dst)
+                                        int p2, bf16* dst, const FoldRow& fr, int col)
 {
     float v[32];
     float ss = 0.f;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
         tc::ld32(taddr + 32 * c, v);
+        if (live) fold32<FOLD>(v, fr, col + 32 * c);
 #pragma unroll
         for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
     }
@@ -393,6 +469,7 @@ __device__ __forceinline__ void qk_head(uint32_t taddr, bool live, const bf16* w
     for (int c = 0; c < 4; ++c) {
         tc::ld32(taddr + 32 * c, v);
         if (!live) continue;
+        fold32<FOLD>(v, fr, col + 32 * c);
         float fw[32];
         if (w) {
 #pragma unroll
@@ -422,16 +499,21 @@ __device__ __forceinline__ void qk_head(uint32_t taddr, bool live, const bf16* w
     }
 }
 
-// Epilogue warps 2..5: thread (warp w, lane l) owns accumulator row 32*(w % 4) + l of this
-// CTA's 128 rows, the TMEM lane quarter warp w may access.  A drained accumulator is
-// announced to the leader's acc_empty (one arrival per warp of each CTA).
-template <int EPI, bool PAIR>
+// Epilogue warps 2 .. 2+EW-1: thread (warp w, lane l) owns accumulator row 32*(w % 4) + l
+// of this CTA's 128 rows (the TMEM lane quarter warp w may access) and, with EW = 8, half
+// of its 256 columns ((w - 2) / 4 picks the half; a half is one head of the QKV epilogue).
+// A drained accumulator is announced to the leader's acc_empty (one arrival per warp of
+// each CTA).
+template <int EPI, bool FOLD, bool PAIR, int EW>
 __device__ void run_epilogue(const Params& p, Bars* b, const Where& w)
 {
+    constexpr int H = EW / 4;  // column parts per accumulator row
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3;
+    const int part = (warp - EPI_WARP0) / 4;  // this thread's part of the 256 columns
     int64_t it = 0;
-    for (int64_t t = w.worker; t < p.num_tiles; t += w.n_workers, ++it) {
+    Pass q = pass_begin();
+    for (; next_pass<PAIR, FOLD>(q, p, w); ++it) {
         const int ab = (int)(it & 1);
         const uint32_t acc_phase = (uint32_t)((it >> 1) & 1);
         const bool got = wait_or_abort<PAIR>(smem_u32(&b->acc_full[ab]), acc_phase, b);
@@ -440,20 +522,33 @@ __device__ void run_epilogue(const Params& p, Bars* b, const Where& w)
             break;
         }
         tc::fence_after_sync();
-        int64_t m_blk;
-        int32_t n_blk;
-        tile_coords<PAIR>(t, p, m_blk, n_blk);
+        const int64_t m_blk = q.m_blk;
+        const int32_t n_blk = q.n_blk;
         const int64_t row = m_blk * Shape<PAIR>::TILE_M + (int64_t)w.rank * BM + quarter * 32 + lane;
-        const bool live = row < p.M;
+        bool live = row < p.M;
+        FoldRow fr{0.f, 0.f, nullptr, nullptr};
+        if constexpr (FOLD) {
+            // rows of another modulation row are stored by that row's pass
+            if (live) live = mod_row(row, p.sel) == q.r;
+            if (live) {
+                const float2 st = __ldg(p.stats + row);
+                fr.mu = st.x;
+                fr.rs = st.y;
+            }
+            fr.c = p.fold_c + (int64_t)q.r * p.n_w;
+            fr.b = p.fold_b + (int64_t)q.r * p.n_w;
+        }
         const uint32_t tbase = b->tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * BN);
         float v[32];
 
         if constexpr (EPI == EPI_STORE) {
             bf16* dst = p.out + row * p.ld_out + (int64_t)n_blk * BN;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = part * (8 / H); c < (part + 1) * (8 / H); ++c) {
                 tc::ld32(tbase + 32 * c, v);
-                        if (live) store32(dst + 32 * c, v);
+                if (!live) continue;
+                fold32<FOLD>(v, fr, n_blk * BN + 32 * c);
+                store32(dst + 32 * c, v);
             }
         } else if constexpr (EPI == EPI_GATED) {
             const int64_t col0 = (int64_t)n_blk * BN;
@@ -462,9 +557,9 @@ __device__ void run_epilogue(const Params& p, Bars* b, const Where& w)
             if (live && p.gate) gr = p.gate + mod_row(row, p.sel) * p.ld_mod + col0;
             bf16* dst = p.out + row * p.ld_out + col0;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = part * (8 / H); c < (part + 1) * (8 / H); ++c) {
                 tc::ld32(tbase + 32 * c, v);
-                        if (!live) continue;
+                if (!live) continue;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     float fx[8], fg[8];
@@ -484,10 +579,10 @@ __device__ void run_epilogue(const Params& p, Bars* b, const Where& w)
             bf16* dst = p.out + row * p.ld_out + (int64_t)n_blk * (BN / 2);
             float u[32];
 #pragma unroll 1
-            for (int c = 0; c < BN / 64; ++c) {
+            for (int c = part * (4 / H); c < (part + 1) * (4 / H); ++c) {
                 tc::ld32(tbase + 32 * c, v);
                 tc::ld32(tbase + BN / 2 + 32 * c, u);
-                        if (!live) continue;
+                if (!live) continue;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = silu_mul_fast(v[i], u[i]);
                 store32(dst + 32 * c, v);
@@ -497,16 +592,19 @@ __device__ void run_epilogue(const Params& p, Bars* b, const Where& w)
             bf16* dst = p.out + row * p.ld_out + col0;
             if (col0 >= p.qk_cols) {  // v heads: as projected
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
+                for (int c = part * (8 / H); c < (part + 1) * (8 / H); ++c) {
                     tc::ld32(tbase + 32 * c, v);
-                                if (live) store32(dst + 32 * c, v);
+                    if (!live) continue;
+                    fold32<FOLD>(v, fr, col0 + 32 * c);
+                    store32(dst + 32 * c, v);
                 }
             } else {
                 int p0 = 0, p1 = 0, p2 = 0;
                 if (live) token_pos(row, p, p0, p1, p2);
                 const bf16* w = col0 < p.qk_cols / 2 ? p.wq : p.wk;
-                qk_head(tbase, live, w, p, p0, p1, p2, dst);
-                qk_head(tbase + 128, live, w, p, p0, p1, p2, dst + 128);
+#pragma unroll 1
+                for (int hh = part * (2 / H); hh < (part + 1) * (2 / H); ++hh)
+                    qk_head<FOLD>(tbase + 128 * hh, live, w, p, p0, p1, p2, dst + 128 * hh, fr, col0 + 128 * hh);
             }
         }
         tc::fence_before_sync();
@@ -676,8 +774,13 @@ __device__ void run_transform(const Params& p, uint8_t* ring, Bars* b, const Whe
 
 // ---------------------------------------------------------------------------------
 // The kernel: roles by warp (see the file header).
-template <int EPI, bool PRO, bool PAIR>
-__global__ void __launch_bounds__(PRO ? 192 + XFORM_THREADS : 192, 1)
+template <bool PRO> __host__ __device__ constexpr int block_threads()
+{
+    return PRO ? 192 + XFORM_THREADS : 64 + 32 * epi_warps<false>();
+}
+
+template <int EPI, bool PRO, bool FOLD, bool PAIR>
+__global__ void __launch_bounds__(block_threads<PRO>(), 1)
     k_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
              const __grid_constant__ Params p)
 {
@@ -698,7 +801,7 @@ __global__ void __launch_bounds__(PRO ? 192 + XFORM_THREADS : 192, 1)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&b->acc_full[i]), 1);
-            mbar_init(smem_u32(&b->acc_empty[i]), (PAIR ? 2 : 1) * 4);  // one per epilogue warp of each CTA
+            mbar_init(smem_u32(&b->acc_empty[i]), (PAIR ? 2 : 1) * epi_warps<PRO>());  // per epilogue warp, each CTA
         }
         mbar_init(smem_u32(&b->drain), 1);
 #pragma unroll
@@ -723,13 +826,13 @@ __global__ void __launch_bounds__(PRO ? 192 + XFORM_THREADS : 192, 1)
     tc::fence_after_sync();
 
     if (warp == PRODUCER_WARP) {
-        if (lane == 0) run_producer<EPI, PRO, PAIR>(&tmA, &tmB, p, ring, b, w);
+        if (lane == 0) run_producer<EPI, PRO, FOLD, PAIR>(&tmA, &tmB, p, ring, b, w);
     } else if (warp == MMA_WARP) {
         if (lane == 0) {
-            if (!PAIR || w.rank == 0) run_mma<PRO, PAIR>(p, ring, b, w);
+            if (!PAIR || w.rank == 0) run_mma<PRO, FOLD, PAIR>(p, ring, b, w);
         }
-    } else if (warp < XFORM_WARP0) {
-        run_epilogue<EPI, PAIR>(p, b, w);
+    } else if (warp < EPI_WARP0 + epi_warps<PRO>()) {
+        run_epilogue<EPI, FOLD, PAIR, epi_warps<PRO>()>(p, b, w);
     } else if (PRO) {
         run_transform<PAIR>(p, ring, b, w);
     }
@@ -762,11 +865,11 @@ __global__ void __launch_bounds__(PRO ? 192 + XFORM_THREADS : 192, 1)
 }
 
 // ---------------------------------------------------------------------------------
-// Row statistics for the AdaLN operand transform: (mean, 1/sqrt(var + eps)) of each row
-// of x, biased variance by two passes (the second re-reads the row from L1/L2).  One
-// warp per row.
-__global__ void __launch_bounds__(256) k_row_stats(float2* stats, const bf16* x, int64_t ld_x, int64_t M, int32_t d,
-                                                   float eps)
+// Row statistics for the AdaLN variants: (mean, 1/sqrt(var + eps)) of each row of x,
+// biased variance by two passes (the second re-reads the row from L1/L2).  One warp per
+// row.  With rmask, also the set of modulation rows each 128-row block uses (bit r).
+__global__ void __launch_bounds__(256) k_row_stats(float2* stats, uint32_t* rmask, ModSel sel, const bf16* x,
+                                                   int64_t ld_x, int64_t M, int32_t d, float eps)
 {
     const int lane = threadIdx.x & 31;
     const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -793,7 +896,66 @@ __global__ void __launch_bounds__(256) k_row_stats(float2* stats, const bf16* x,
             }
         }
         const float var = warp_sum(q) / (float)d;
-        if (lane == 0) stats[row] = make_float2(mu, rsqrtf(var + eps));
+        if (lane == 0) {
+            stats[row] = make_float2(mu, rsqrtf(var + eps));
+            if (rmask) atomicOr(rmask + (row >> 7), 1u << (uint32_t)mod_row(row, sel));
+        }
+    }
+}
+
+// AdaLN folded into a linear layer's weights, per modulation row r and output column j:
+//     V_r[j, k] = bf16(W[j, k] * (1 + scale_r[k]))       (the folded weights)
+//     c_r[j]    = sum_k V_r[j, k]                         (fp32, of the rounded V)
+//     b_r[j]    = sum_k shift_r[k] * W[j, k]              (fp32)
+// so that LN-modulated rows project as rstd * (x . V_r^T - mean * c_r) + b_r.  One warp
+// per (r, j); V is [R * n_w, K] with row stride K.
+__global__ void __launch_bounds__(256) k_fold_weights(bf16* V, float* c, float* bsum, const bf16* W, int64_t ld_w,
+                                                      int32_t n_w, int32_t K, const bf16* scale, const bf16* shift,
+                                                      int64_t ld_mod, int32_t R)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t wstep = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t total = (int64_t)R * n_w;
+    for (int64_t idx = w0; idx < total; idx += wstep) {
+        const int64_t r = idx / n_w, j = idx - r * n_w;
+        const bf16* wr = W + j * ld_w;
+        bf16* vr = V + idx * (int64_t)K;
+        float cs = 0.f, bs = 0.f;
+        for (int v = lane; v < K / 8; v += 32) {
+            float fw[8], fg[8], fs[8];
+            unpack<bf16>(ld_cached(wr + 8 * v), fw);
+            if (scale) {
+                unpack<bf16>(ld_cached(scale + r * ld_mod + 8 * v), fg);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) fg[e] = 0.f;
+            }
+            if (shift) {
+                unpack<bf16>(ld_cached(shift + r * ld_mod + 8 * v), fs);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) fs[e] = 0.f;
+            }
+            float fv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                fv[e] = fw[e] * (1.f + fg[e]);
+                bs = fmaf(fs[e], fw[e], bs);
+            }
+            const uint4 pv = pack<bf16>(fv);
+            *reinterpret_cast<uint4*>(vr + 8 * v) = pv;
+            float rv[8];
+            unpack<bf16>(pv, rv);  // the rounded values the tensor cores will read
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cs += rv[e];
+        }
+        cs = warp_sum(cs);
+        bs = warp_sum(bs);
+        if (lane == 0) {
+            c[idx] = cs;
+            bsum[idx] = bs;
+        }
     }
 }
 
@@ -849,12 +1011,12 @@ bool use_pair(bool transform)
     return forced >= 0 ? forced == 1 : !transform;
 }
 
-template <int EPI, bool PRO, bool PAIR>
+template <int EPI, bool PRO, bool FOLD, bool PAIR>
 cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const gemm::Params& p, cudaStream_t s)
 {
-    auto kern = gemm::k_linear<EPI, PRO, PAIR>;
+    auto kern = gemm::k_linear<EPI, PRO, FOLD, PAIR>;
     const size_t smem = gemm::smem_bytes<PAIR>();
-    const int threads = PRO ? 192 + gemm::XFORM_THREADS : 192;
+    const int threads = gemm::block_threads<PRO>();
     static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
     if constexpr (!PAIR) {
@@ -887,15 +1049,25 @@ cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const ge
     }
 }
 
-template <int EPI, bool PRO>
+template <int EPI, bool PRO, bool FOLD = false>
 cudaError_t launch_shape(const CUtensorMap& ma, const CUtensorMap& mb, gemm::Params& p, int64_t M, cudaStream_t s)
 {
     if (use_pair(PRO)) {
         p.num_tiles = (M + gemm::Shape<true>::TILE_M - 1) / gemm::Shape<true>::TILE_M * (int64_t)p.n_tiles_n;
-        return launch_kernel<EPI, PRO, true>(ma, mb, p, s);
+        return launch_kernel<EPI, PRO, FOLD, true>(ma, mb, p, s);
     }
     p.num_tiles = (M + gemm::Shape<false>::TILE_M - 1) / gemm::Shape<false>::TILE_M * (int64_t)p.n_tiles_n;
-    return launch_kernel<EPI, PRO, false>(ma, mb, p, s);
+    return launch_kernel<EPI, PRO, FOLD, false>(ma, mb, p, s);
+}
+
+// AdaLN strategy: fold (default) or the operand transform; SOL_ADALN_STRATEGY overrides.
+bool adaln_fold()
+{
+    static const bool fold = [] {
+        const char* e = std::getenv("SOL_ADALN_STRATEGY");
+        return !(e && std::string(e) == "transform");
+    }();
+    return fold;
 }
 
 }  // namespace
@@ -936,12 +1108,41 @@ cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cuda
     p.qk_cols = a.qk_cols;
     p.eps = a.eps;
 
+    const bool fold = adaln && adaln_fold();
     if (adaln) {
         const int64_t blocks = std::min<int64_t>((a.M + 7) / 8, (int64_t)sm_count() * 16);
-        gemm::k_row_stats<<<(unsigned)blocks, 256, 0, s>>>(static_cast<float2*>(a.stats),
-                                                           static_cast<const bf16*>(a.a), a.ld_a, a.M, a.K, a.eps);
+        const ModSel sel = a.sel ? *a.sel : ModSel{};
+        if (fold) {
+            cudaError_t e = cudaMemsetAsync(a.rmask, 0, (size_t)((a.M + gemm::BM - 1) / gemm::BM) * 4, s);
+            if (e != cudaSuccess) return e;
+        }
+        gemm::k_row_stats<<<(unsigned)blocks, 256, 0, s>>>(static_cast<float2*>(a.stats), fold ? a.rmask : nullptr,
+                                                           sel, static_cast<const bf16*>(a.a), a.ld_a, a.M, a.K,
+                                                           a.eps);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
+    }
+    if (fold) {
+        // fold the modulation into the weights, then a plain GEMM on x with the correction
+        // rstd * (acc - mean * c_r) + b_r in its epilogue
+        const int64_t rows = (int64_t)a.n_mod_rows * a.N;
+        const int64_t blocks = std::min<int64_t>((rows + 7) / 8, (int64_t)sm_count() * 16);
+        gemm::k_fold_weights<<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<bf16*>(a.fold_v), a.fold_c, a.fold_b, static_cast<const bf16*>(a.w), a.ld_w, a.N, a.K,
+            static_cast<const bf16*>(a.scale), static_cast<const bf16*>(a.shift), a.ld_mod, a.n_mod_rows);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        if (!make_map(&mb, a.fold_v, (uint64_t)rows, (uint64_t)a.K, (uint64_t)a.K)) {
+            record_error("tensor map encoding failed for the folded weights");
+            return cudaErrorInvalidValue;
+        }
+        p.rmask = a.rmask;
+        p.fold_c = a.fold_c;
+        p.fold_b = a.fold_b;
+        p.n_w = a.N;
+        if (epi == LINEAR_STORE) return launch_shape<gemm::EPI_STORE, false, true>(ma, mb, p, a.M, s);
+        if (epi == LINEAR_QKROPE) return launch_shape<gemm::EPI_QKROPE, false, true>(ma, mb, p, a.M, s);
+        return cudaErrorInvalidValue;
     }
     switch (epi) {
     case LINEAR_STORE:

@@ -109,6 +109,12 @@ struct LinearLaunch {
     RopeDev rope;
     int32_t qk_cols;    // columns of q and k (2 * n_heads * 128)
     float eps;
+    // AdaLN folded into the weights (workspace regions)
+    uint32_t* rmask;    // [ceil(M / 128)] modulation rows per 128-row block
+    void* fold_v;       // [n_mod_rows * N, K] bf16 folded weights
+    float* fold_c;      // [n_mod_rows, N]
+    float* fold_b;      // [n_mod_rows, N]
+    int32_t n_mod_rows; // modulation rows the call may use (<= 32)
 };
 cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cudaStream_t s);
 size_t linear_smem_bytes();

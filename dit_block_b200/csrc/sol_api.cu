@@ -632,12 +632,56 @@ static bool spans_overlap(const void* a, int64_t rows_a, int64_t ld_a, int64_t w
     return a0 < b1 && b0 < a1;
 }
 
-static sol_status check_stats(const float* row_stats, int64_t n_tokens)
+// Modulation rows a call may use: ceil(n_tokens / tokens_per_sample) * n_streams, or
+// n_streams for one sample.
+static int64_t mod_rows(int64_t n_tokens, const sol_modsel& sel)
 {
-    CHECK(row_stats, SOL_ERR_INVALID_ARGUMENT, "row_stats is NULL");
-    CHECK(aligned16(row_stats), SOL_ERR_MISALIGNED, "row_stats is not 16-byte aligned");
-    (void)n_tokens;
+    const int64_t samples = sel.tokens_per_sample > 0 ? (n_tokens + sel.tokens_per_sample - 1) / sel.tokens_per_sample : 1;
+    return std::max<int64_t>(samples, 1) * sel.n_streams;
+}
+
+// Workspace of the sol_adaln_* calls: row statistics, per-128-row modulation-row sets,
+// folded-weight column sums and shift projections, then the folded weights; every region
+// 256-byte aligned.
+struct AdalnWorkspace {
+    size_t stats, rmask, c, b, v, total;
+};
+
+static AdalnWorkspace adaln_layout(int64_t n_tokens, int64_t n_out, int64_t d, int64_t R)
+{
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    AdalnWorkspace w{};
+    w.stats = 0;
+    w.rmask = up(w.stats + (size_t)n_tokens * 8);
+    w.c = up(w.rmask + (size_t)((n_tokens + 127) / 128) * 4);
+    w.b = up(w.c + (size_t)(R * n_out) * 4);
+    w.v = up(w.b + (size_t)(R * n_out) * 4);
+    w.total = up(w.v + (size_t)(R * n_out) * (size_t)d * 2);
+    return w;
+}
+
+static sol_status check_workspace(const void* ws, size_t bytes, int64_t n_tokens, int64_t n_out, int64_t d,
+                                  const sol_modsel& sel, AdalnWorkspace* lay, int64_t* R)
+{
+    *R = mod_rows(n_tokens, sel);
+    CHECK(*R <= 32, SOL_ERR_UNSUPPORTED, "%lld modulation rows (more than 32)", (long long)*R);
+    *lay = adaln_layout(n_tokens, n_out, d, *R);
+    CHECK(ws, SOL_ERR_INVALID_ARGUMENT, "workspace is NULL");
+    CHECK((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, SOL_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    CHECK(bytes >= lay->total, SOL_ERR_INVALID_ARGUMENT, "workspace of %zu bytes is below the %zu needed", bytes,
+          lay->total);
     return SOL_OK;
+}
+
+static void set_workspace(sol::LinearLaunch& L, void* ws, const AdalnWorkspace& lay, int64_t R)
+{
+    char* base = static_cast<char*>(ws);
+    L.stats = base + lay.stats;
+    L.rmask = reinterpret_cast<uint32_t*>(base + lay.rmask);
+    L.fold_c = reinterpret_cast<float*>(base + lay.c);
+    L.fold_b = reinterpret_cast<float*>(base + lay.b);
+    L.fold_v = base + lay.v;
+    L.n_mod_rows = (int32_t)R;
 }
 
 static sol::LinearLaunch linear_base(void* out, int64_t ld_out, const void* a, int64_t ld_a, const void* w,
@@ -722,10 +766,19 @@ sol_status sol_linear_swiglu(void* out, int64_t ld_out, const void* a, int64_t l
                        "sol_linear_swiglu launch");
 }
 
+size_t sol_adaln_workspace_bytes(int64_t n_tokens, int64_t n_out, int64_t d, sol_modsel sel)
+{
+    if (n_tokens < 0 || n_out < 1 || d < 1 || sel.n_streams < 1 || sel.tokens_per_sample < 0) return 0;
+    const int64_t R = mod_rows(n_tokens, sel);
+    if (R > 32) return 0;
+    return adaln_layout(n_tokens, n_out, d, R).total;
+}
+
 sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld_x,
                             const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
-                            const void* w, int64_t ld_w, float* row_stats, int64_t n_tokens,
-                            int64_t n_out, int64_t d, float eps, sol_dtype dt, sol_stream_t stream)
+                            const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,
+                            int64_t n_tokens, int64_t n_out, int64_t d, float eps, sol_dtype dt,
+                            sol_stream_t stream)
 {
     TRY(check_linear_shape(n_tokens, n_out, d, dt, 256));
     TRY(check_modsel(sel));
@@ -734,17 +787,20 @@ sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld
     TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
     TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
     if (n_tokens == 0) return SOL_OK;
-    TRY(check_stats(row_stats, n_tokens));
+    AdalnWorkspace lay;
+    int64_t R = 0;
+    TRY(check_workspace(workspace, workspace_bytes, n_tokens, n_out, d, sel, &lay, &R));
     TRY(check_tensor("out", out, ld_out, n_out, dt, true));
     TRY(check_tensor("x", x, ld_x, d, dt, true));
     CHECK(!spans_overlap(out, n_tokens, ld_out, n_out, 2, x, n_tokens, ld_x, d, 2) &&
               !spans_overlap(out, n_tokens, ld_out, n_out, 2, w, n_out, ld_w, d, 2) &&
-              !spans_overlap(out, n_tokens, ld_out, n_out, 2, row_stats, n_tokens, 2, 2, 4) &&
-              !spans_overlap(x, n_tokens, ld_x, d, 2, row_stats, n_tokens, 2, 2, 4),
-          SOL_ERR_INVALID_ARGUMENT, "out or x overlaps another argument");
+              !spans_overlap(out, n_tokens, ld_out, n_out, 2, workspace, 1, 0, (int64_t)lay.total, 1) &&
+              !spans_overlap(x, n_tokens, ld_x, d, 2, workspace, 1, 0, (int64_t)lay.total, 1) &&
+              !spans_overlap(w, n_out, ld_w, d, 2, workspace, 1, 0, (int64_t)lay.total, 1),
+          SOL_ERR_INVALID_ARGUMENT, "out, x or w overlaps another argument");
     sol::LinearLaunch L = linear_base(out, ld_out, x, ld_x, w, ld_w, n_tokens, n_out, d);
     const sol::ModSel ms = to_dev(sel, n_tokens);
-    L.stats = row_stats;
+    set_workspace(L, workspace, lay, R);
     L.shift = shift;
     L.scale = scale;
     L.ld_mod = ld_mod;
@@ -756,8 +812,8 @@ sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld
 
 sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t ld_x,
                               const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
-                              const void* w, int64_t ld_w, float* row_stats, const void* wq,
-                              const void* wk, const int32_t* pos, int32_t grid_T, int32_t grid_H,
+                              const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,
+                              const void* wq, const void* wk, const int32_t* pos, int32_t grid_T, int32_t grid_H,
                               int32_t grid_W, const sol_rope3d* rope, int64_t n_tokens,
                               int32_t n_heads, int32_t head_dim, int64_t d, float eps, sol_dtype dt,
                               sol_stream_t stream)
@@ -776,17 +832,20 @@ sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t 
     TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
     TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
     if (n_tokens == 0) return SOL_OK;
-    TRY(check_stats(row_stats, n_tokens));
+    AdalnWorkspace lay;
+    int64_t R = 0;
+    TRY(check_workspace(workspace, workspace_bytes, n_tokens, n_out, d, sel, &lay, &R));
     TRY(check_tensor("qkv", qkv, ld_qkv, n_out, dt, true));
     TRY(check_tensor("x", x, ld_x, d, dt, true));
     CHECK(!spans_overlap(qkv, n_tokens, ld_qkv, n_out, 2, x, n_tokens, ld_x, d, 2) &&
               !spans_overlap(qkv, n_tokens, ld_qkv, n_out, 2, w, n_out, ld_w, d, 2) &&
-              !spans_overlap(qkv, n_tokens, ld_qkv, n_out, 2, row_stats, n_tokens, 2, 2, 4) &&
-              !spans_overlap(x, n_tokens, ld_x, d, 2, row_stats, n_tokens, 2, 2, 4),
-          SOL_ERR_INVALID_ARGUMENT, "qkv or x overlaps another argument");
+              !spans_overlap(qkv, n_tokens, ld_qkv, n_out, 2, workspace, 1, 0, (int64_t)lay.total, 1) &&
+              !spans_overlap(x, n_tokens, ld_x, d, 2, workspace, 1, 0, (int64_t)lay.total, 1) &&
+              !spans_overlap(w, n_out, ld_w, d, 2, workspace, 1, 0, (int64_t)lay.total, 1),
+          SOL_ERR_INVALID_ARGUMENT, "qkv, x or w overlaps another argument");
     sol::LinearLaunch L = linear_base(qkv, ld_qkv, x, ld_x, w, ld_w, n_tokens, n_out, d);
     const sol::ModSel ms = to_dev(sel, n_tokens);
-    L.stats = row_stats;
+    set_workspace(L, workspace, lay, R);
     L.shift = shift;
     L.scale = scale;
     L.ld_mod = ld_mod;

@@ -80,10 +80,11 @@ SIGNATURES = {
     "sol_linear_gated_residual": ([_P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _I64, ModSel, _I64, _I64,
                                    _I64, _E, _P], _E),
     "sol_linear_swiglu": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _E, _P], _E),
-    "sol_adaln_linear": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, _I64, _I64, _I64, _F,
-                          _E, _P], _E),
-    "sol_adaln_qkv_rope": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, _P, _P, _P, _I32, _I32,
-                            _I32, _P, _I64, _I32, _I32, _I64, _F, _E, _P], _E),
+    "sol_adaln_workspace_bytes": ([_I64, _I64, _I64, ModSel], ctypes.c_size_t),
+    "sol_adaln_linear": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _I64, _I64,
+                          _I64, _F, _E, _P], _E),
+    "sol_adaln_qkv_rope": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _P, _P, _P,
+                            _I32, _I32, _I32, _P, _I64, _I32, _I32, _I64, _F, _E, _P], _E),
 }
 
 _lib = None
@@ -387,28 +388,40 @@ def linear_swiglu(out, a, w, *, stream=None):
     return out
 
 
-def row_stats_workspace(n_tokens: int, device=None) -> torch.Tensor:
-    """A row-statistics workspace for the sol_adaln_* calls: [n_tokens, 2] float32."""
-    return torch.empty((max(int(n_tokens), 1), 2), dtype=torch.float32, device=device or "cuda")
+def adaln_workspace_bytes(n_tokens: int, n_out: int, d: int, *, n_streams=1, tokens_per_sample=0) -> int:
+    """Bytes of workspace the sol_adaln_* calls need (sol_adaln_workspace_bytes)."""
+    return int(lib().sol_adaln_workspace_bytes(int(n_tokens), int(n_out), int(d),
+                                               ModSel(None, int(n_streams), int(tokens_per_sample))))
 
 
-def adaln_linear(out, x, w, shift=None, scale=None, *, row_stats, eps=1e-6, stream_id=None, n_streams=1,
+def adaln_workspace(n_tokens: int, n_out: int, d: int, *, n_streams=1, tokens_per_sample=0,
+                    device=None) -> torch.Tensor:
+    """A workspace for the sol_adaln_* calls (uint8 device tensor; torch allocations are
+    256-byte aligned)."""
+    nb = adaln_workspace_bytes(n_tokens, n_out, d, n_streams=n_streams, tokens_per_sample=tokens_per_sample)
+    if nb == 0:
+        raise ValueError("no workspace size for these arguments (more than 32 modulation rows?)")
+    return torch.empty((nb,), dtype=torch.uint8, device=device or "cuda")
+
+
+def adaln_linear(out, x, w, shift=None, scale=None, *, workspace, eps=1e-6, stream_id=None, n_streams=1,
                  tokens_per_sample=0, stream=None):
-    """out = AdaLN(x) . W^T with AdaLN in the operand load  (sol_adaln_linear)."""
+    """out = AdaLN(x) . W^T with the modulation folded into the weights  (sol_adaln_linear)."""
     _check(lib().sol_adaln_linear(
         _ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
-        _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(row_stats), x.shape[0],
-        w.shape[0], x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_linear")
+        _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(workspace), workspace.numel(),
+        x.shape[0], w.shape[0], x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_linear")
     return out
 
 
-def adaln_qkv_rope(qkv, x, w, rope: Rope3D, shift=None, scale=None, *, row_stats, n_heads, head_dim=128,
+def adaln_qkv_rope(qkv, x, w, rope: Rope3D, shift=None, scale=None, *, workspace, n_heads, head_dim=128,
                    wq=None, wk=None, pos=None, grid=(0, 0, 0), eps=1e-6, stream_id=None, n_streams=1,
                    tokens_per_sample=0, stream=None):
     """qkv = AdaLN(x) . W^T, then QK RMSNorm + 3D RoPE on q and k  (sol_adaln_qkv_rope)."""
     _check(lib().sol_adaln_qkv_rope(
         _ptr(qkv), _ld(qkv), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
-        _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(row_stats), _ptr(wq), _ptr(wk),
+        _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(workspace), workspace.numel(),
+        _ptr(wq), _ptr(wk),
         _ptr(pos), int(grid[0]), int(grid[1]), int(grid[2]), rope.handle, x.shape[0], n_heads, head_dim,
         x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_qkv_rope")
     return qkv

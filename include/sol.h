@@ -41,6 +41,7 @@
 #ifndef SOL_H
 #define SOL_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -328,12 +329,11 @@ sol_status sol_qk_rmsnorm_rope3d_noalloc(void* q_out, void* k_out, int64_t ld_qo
  *   dt must be SOL_DTYPE_BF16 (the tensor cores take bf16 operands; SOL_ERR_UNSUPPORTED
  *   otherwise).  W is [n_out, k] with row stride ld_w: the usual linear-layer layout,
  *   y = a . W^T, no bias.  k must be a multiple of 64 and n_out a multiple of 256
- *   (SOL_ERR_UNSUPPORTED otherwise); n_tokens < 2^31.  Accumulation is fp32; the
- *   operand the tensor cores read is bf16 (the AdaLN output is rounded to bf16 in
- *   shared memory, exactly where the unfused path rounds it when storing h); every
- *   output element is rounded once, when stored.  No output may overlap an input
- *   except where stated.  Each call launches one kernel (two for the sol_adaln_*
- *   calls: a row-statistics pass, then the linear layer).
+ *   (SOL_ERR_UNSUPPORTED otherwise); n_tokens < 2^31.  The tensor cores read bf16
+ *   operands and accumulate in fp32; every output element is rounded once, when
+ *   stored.  No output may overlap an input
+ *   except where stated.  Each call launches one kernel (the sol_adaln_* calls three:
+ *   row statistics, the weight fold, then the linear layer).
  * ------------------------------------------------------------------------------------ */
 
 /* out = a . W^T: a [n_tokens, k], W [n_out, k], out [n_tokens, n_out]. */
@@ -362,16 +362,32 @@ sol_status sol_linear_swiglu(void* out, int64_t ld_out, const void* a, int64_t l
                              int64_t ld_w, int64_t n_tokens, int64_t inner, int64_t k, sol_dtype dt,
                              sol_stream_t stream);
 
-/* AdaLN fused into the operand load of a linear layer:
+/* Device workspace, in bytes, that sol_adaln_linear and sol_adaln_qkv_rope need for
+ * n_tokens tokens, n_out output columns and d input columns, with the modulation rows
+ * `sel` implies (R = ceil(n_tokens / tokens_per_sample) * n_streams, or n_streams when
+ * tokens_per_sample is 0): per token 8 bytes of row statistics, per 128 tokens 4 bytes
+ * of modulation-row sets, and per modulation row the folded weights (n_out * d bf16)
+ * plus two fp32 vectors of n_out.  Returns 0 for invalid sizes or R > 32. */
+size_t sol_adaln_workspace_bytes(int64_t n_tokens, int64_t n_out, int64_t d, sol_modsel sel);
+
+/* AdaLN fused into a linear layer:
  *     out = h . W^T,   h = LN(x) * (1 + scale[r]) + shift[r]   (as sol_adaln_modulate)
- * x [n_tokens, d], W [n_out, d], out [n_tokens, n_out]; d a multiple of 64.
- * row_stats: caller-owned device workspace of n_tokens (mean, 1/sqrt(var + eps)) float
- * pairs (8 bytes per token, 16-byte aligned), written by the call's first kernel and
- * read by its second; it must not overlap any other argument.  h is never stored. */
+ * x [n_tokens, d], W [n_out, d], out [n_tokens, n_out]; d a multiple of 64; at most 32
+ * modulation rows (SOL_ERR_UNSUPPORTED otherwise).  h is never stored.  The modulation is
+ * folded into the weights: per modulation row r the call writes V_r = bf16(W * (1 +
+ * scale_r)) (column-wise), c_r = sum_k V_r[:, k] and b_r = shift_r . W^T into the
+ * workspace, computes mean and 1/sqrt(var + eps) of every row of x, and runs one GEMM of
+ * x against V_r whose epilogue forms rstd * (acc - mean * c_r) + b_r: the same value as
+ * projecting h, computed from the unrounded LN output (the only rounding of an operand
+ * is that of the folded weights, of the same size as rounding h to bf16).  A tile whose
+ * rows use several modulation rows is computed once per row used.
+ * workspace: caller-owned device memory of at least sol_adaln_workspace_bytes(...)
+ * bytes, 256-byte aligned, overlapping no other argument; its contents are scratch. */
 sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld_x,
                             const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
-                            const void* w, int64_t ld_w, float* row_stats, int64_t n_tokens,
-                            int64_t n_out, int64_t d, float eps, sol_dtype dt, sol_stream_t stream);
+                            const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,
+                            int64_t n_tokens, int64_t n_out, int64_t d, float eps, sol_dtype dt,
+                            sol_stream_t stream);
 
 /* The attention input of a block in one pass: AdaLN into the QKV projection, QK RMSNorm
  * + 3D RoPE in its epilogue:
@@ -381,10 +397,12 @@ sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld
  * head_dim must be 128 and n_heads even.  Positions: pos [n_tokens, 3] int32, or NULL
  * for the row-major grid (grid_T, grid_H, grid_W) of each sample, samples of
  * sel.tokens_per_sample tokens (0 = one sample), as in sol_qk_rmsnorm_rope3d.
- * row_stats as in sol_adaln_linear.  The projection is not rounded before the norm. */
+ * workspace as in sol_adaln_linear (with n_out = 3 * n_heads * head_dim).  The
+ * projection is not rounded before the norm. */
 sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t ld_x,
                               const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
-                              const void* w, int64_t ld_w, float* row_stats, const void* wq,
+                              const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,
+                              const void* wq,
                               const void* wk, const int32_t* pos, int32_t grid_T, int32_t grid_H,
                               int32_t grid_W, const sol_rope3d* rope, int64_t n_tokens,
                               int32_t n_heads, int32_t head_dim, int64_t d, float eps, sol_dtype dt,

@@ -28,7 +28,7 @@ def last(L):
 
 def test_exports_every_declared_symbol(L):
     names = sol.header_functions()
-    assert len(names) == 22
+    assert len(names) == 23
     for n in names:
         assert hasattr(L, n), f"libsol.so does not export {n}"
         assert n in sol.SIGNATURES, f"binding has no signature for {n}"
@@ -171,20 +171,32 @@ def test_linear_epilogue_variants_validation(L):
     # SwiGLU: W has 2*inner rows, inner a multiple of 128
     assert L.sol_linear_swiglu(out, 192, a, k, w, k, n, 192, k, sol.BF16, None) == sol.ERR_UNSUPPORTED
     assert L.sol_linear_swiglu(out, 256, a, k, w, k, n, 256, k, sol.F32, None) == sol.ERR_UNSUPPORTED
-    # AdaLN variants need the row-statistics workspace
-    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, None, n, d, k, 1e-6, sol.BF16,
+    # AdaLN variants need a workspace of sol_adaln_workspace_bytes
+    need = L.sol_adaln_workspace_bytes(n, d, k, SEL)
+    assert need >= n * 8 + d * k * 2
+    ws = FAKE << 6
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, None, need, n, d, k, 1e-6, sol.BF16,
                               None) == sol.ERR_INVALID_ARGUMENT
-    assert "row_stats" in last(L)
-    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, FAKE << 5, n, d, k, float("inf"),
+    assert "workspace" in last(L)
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws, need - 1, n, d, k, 1e-6, sol.BF16,
+                              None) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws + 16, need, n, d, k, 1e-6, sol.BF16,
+                              None) == sol.ERR_MISALIGNED
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws, need, n, d, k, float("inf"),
                               sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
-    # row_stats inside x
-    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, x + 1024, n, d, k, 1e-6,
-                              sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    # workspace overlapping x
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, x + 1024, need, n, d, k, 1e-6,
+                              sol.BF16, None) in (sol.ERR_INVALID_ARGUMENT, sol.ERR_MISALIGNED)
+    # at most 32 modulation rows: 33 samples of 10 tokens
+    many = sol.ModSel(None, 1, 10)
+    assert L.sol_adaln_workspace_bytes(330, d, k, many) == 0
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, many, w, k, ws, need, 330, d, k, 1e-6, sol.BF16,
+                              None) == sol.ERR_UNSUPPORTED
     # the QKV call is built for head_dim 128 and an even head count
-    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, FAKE << 5, None, None, None,
+    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, ws, need, None, None, None,
                                 2, 4, 4, None, n, 4, 64, k, 1e-6, sol.BF16, None) == sol.ERR_UNSUPPORTED
-    assert L.sol_adaln_qkv_rope(out, 1152, x, k, None, None, 0, SEL, w, k, FAKE << 5, None, None, None,
+    assert L.sol_adaln_qkv_rope(out, 1152, x, k, None, None, 0, SEL, w, k, ws, need, None, None, None,
                                 2, 4, 4, None, n, 3, 128, k, 1e-6, sol.BF16, None) == sol.ERR_UNSUPPORTED
-    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, FAKE << 5, None, None, None,
+    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, ws, need, None, None, None,
                                 2, 4, 4, None, n, 2, 128, k, 1e-6, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
     assert "rope is NULL" in last(L)

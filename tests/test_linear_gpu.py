@@ -159,6 +159,34 @@ def test_linear_swiglu(oracle_mod, m):
     check(out, want, bound, f"linear_swiglu m={m}")
 
 
+def modulation_rows(n, stream_id, n_streams, tokens_per_sample):
+    """Modulation row of each token (the selection rule of sol_modsel)."""
+    tok = np.arange(n)
+    sample = tok // tokens_per_sample if tokens_per_sample > 0 else np.zeros(n, np.int64)
+    sid = np.zeros(n, np.int64) if stream_id is None else np.minimum(stream_id.astype(np.int64), n_streams - 1)
+    return sample * n_streams + sid
+
+
+def adaln_projection_bound(oracle_mod, x, W, shift, scale, h, rows_r, eps):
+    """Error bound of AdaLN(x) . W^T as the library computes it, for either strategy:
+    * operand transform: h rounded to bf16 (2^-9 |h|) plus fp32 accumulation -> ACC * S;
+    * weight fold: V = bf16(W (1 + scale_r)) rounded (2^-9 |(x - mean) rstd g W| <= 2^-9
+      (|h| + |shift|) |W|), plus fp32 accumulation of x . V^T and of c_r = sum_k V, both
+      multiplied by rstd (K 2^-23 rstd (|x| |g| + |mean| |g|) . |W|^T).
+    Returns the larger of the two, elementwise."""
+    X = oracle_mod.to_f64(x)
+    Wf = np.abs(oracle_mod.to_f64(W))
+    n, K = X.shape
+    mu = X.mean(1)
+    rs = 1.0 / np.sqrt(((X - mu[:, None]) ** 2).mean(1) + eps)
+    G = np.abs(1.0 + oracle_mod.to_f64(scale)[rows_r]) if scale is not None else np.ones_like(X)
+    Sh = np.abs(oracle_mod.to_f64(shift)[rows_r]) if shift is not None else np.zeros_like(X)
+    S = np.abs(h) @ Wf.T
+    fold = 2.0 ** -9 * ((np.abs(h) + Sh) @ Wf.T)
+    fold += K * 2.0 ** -23 * rs[:, None] * (((np.abs(X) + np.abs(mu)[:, None]) * G) @ Wf.T)
+    return np.maximum(ACC * S, fold)
+
+
 def adaln_inputs(w, m):
     pos, sid, kw = sel_kwargs(w)
     x = wl.activation(w, "x", m, w.d, "cuda")
@@ -175,23 +203,26 @@ def test_adaln_linear(oracle_mod, w):
     x, shift, scale, sid, _, kw = adaln_inputs(w, m)
     W = wl.linear_weight(w, "w_qkv", 768, w.d, "cuda")
     out = torch.empty((m, 768), dtype=torch.bfloat16, device="cuda")
-    stats = sol.row_stats_workspace(m)
-    sol.adaln_linear(out, x, W, shift, scale, row_stats=stats, eps=w.eps, stream_id=sid, **kw)
+    ws = sol.adaln_workspace(m, 768, w.d, **kw)
+    sol.adaln_linear(out, x, W, shift, scale, workspace=ws, eps=w.eps, stream_id=sid, **kw)
     torch.cuda.synchronize()
     y, h = oracle_mod.adaln_linear(to_oracle(x), to_oracle(W), to_oracle(shift), to_oracle(scale), eps=w.eps,
                                    stream_id=to_oracle(sid), **kw)
-    check(out, y, ACC * oracle_mod.linear_magnitude(h, to_oracle(W)), f"adaln_linear {w.name}")
-    # the workspace holds each row's mean and 1/sqrt(var + eps)
+    rr = modulation_rows(m, to_oracle(sid), w.n_streams, kw["tokens_per_sample"])
+    bound = adaln_projection_bound(oracle_mod, to_oracle(x), to_oracle(W), to_oracle(shift), to_oracle(scale), h,
+                                   rr, w.eps)
+    check(out, y, bound, f"adaln_linear {w.name}")
+    # the workspace starts with each row's mean and 1/sqrt(var + eps)
     xf = f64(x)
     mu = xf.mean(1)
     rs = 1 / np.sqrt(((xf - mu[:, None]) ** 2).mean(1) + w.eps)
-    st = stats.cpu().double().numpy()
+    st = ws[:8 * m].view(torch.float32).view(m, 2).cpu().double().numpy()
     np.testing.assert_allclose(st[:, 0], mu, rtol=1e-4, atol=1e-5)
     np.testing.assert_allclose(st[:, 1], rs, rtol=1e-4)
 
 
-def qk_bound(pre, S, wq, wk, n_heads, eps):
-    """Error bound of q|k after RMSNorm + RoPE given the bound ACC * S on the projection:
+def qk_bound(pre, E, wq, wk, n_heads, eps):
+    """Error bound of q|k after RMSNorm + RoPE given the bound E on the projection:
     with e_j <= E_j on a head vector v, r' = sqrt(mean v'^2 + eps) moves by at most
     rms(E), so each normalised element moves by at most |w_j| E_j / r' + |v_j w_j| rms(E) /
     (r r'), and a rotation of a pair moves an element by at most sqrt(2) times the larger
@@ -199,7 +230,7 @@ def qk_bound(pre, S, wq, wk, n_heads, eps):
     n = pre.shape[0]
     hd = pre.shape[1] // 2
     v = pre.reshape(n, 2 * n_heads, 128)
-    E = (ACC * S).reshape(n, 2 * n_heads, 128)
+    E = E.reshape(n, 2 * n_heads, 128)
     w = np.concatenate([np.broadcast_to(wq, (n_heads, 128)), np.broadcast_to(wk, (n_heads, 128))])[None]
     r = np.sqrt((v ** 2).mean(-1, keepdims=True) + eps)
     rms_e = np.sqrt((E ** 2).mean(-1, keepdims=True))
@@ -217,10 +248,10 @@ def test_adaln_qkv_rope(oracle_mod, w):
     W = wl.linear_weight(w, "w_qkv", 3 * hd, w.d, "cuda")
     wq, wk = wl.norm_weight(w, "wq", "cuda"), wl.norm_weight(w, "wk", "cuda")
     qkv = torch.empty((m, 3 * hd), dtype=torch.bfloat16, device="cuda")
-    stats = sol.row_stats_workspace(m)
+    ws = sol.adaln_workspace(m, 3 * hd, w.d, **kw)
     grid = w.grid
     with sol.Rope3D(w.rope_dims, w.theta, w.max_pos) as rope:
-        sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, row_stats=stats, n_heads=w.n_heads, wq=wq, wk=wk,
+        sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, workspace=ws, n_heads=w.n_heads, wq=wq, wk=wk,
                            pos=pos, grid=grid, eps=w.eps, stream_id=sid, **kw)
         torch.cuda.synchronize()
     Wh = to_oracle(W)
@@ -228,10 +259,11 @@ def test_adaln_qkv_rope(oracle_mod, w):
         to_oracle(x), Wh, to_oracle(shift), to_oracle(scale), to_oracle(wq), to_oracle(wk), n_heads=w.n_heads,
         head_dim=128, pos=to_oracle(pos), grid=grid, tokens_per_sample=kw["tokens_per_sample"],
         dims=w.rope_dims, theta=w.theta, eps=w.eps, stream_id=to_oracle(sid), n_streams=w.n_streams)
-    S = oracle_mod.linear_magnitude(h, Wh)
-    bq = qk_bound(pre[:, :2 * hd], S[:, :2 * hd], f64(wq), f64(wk), w.n_heads, w.eps)
+    rr = modulation_rows(m, to_oracle(sid), w.n_streams, kw["tokens_per_sample"])
+    E = adaln_projection_bound(oracle_mod, to_oracle(x), Wh, to_oracle(shift), to_oracle(scale), h, rr, w.eps)
+    bq = qk_bound(pre[:, :2 * hd], E[:, :2 * hd], f64(wq), f64(wk), w.n_heads, w.eps)
     check(qkv[:, :2 * hd], want[:, :2 * hd], bq, f"adaln_qkv_rope q|k {w.name}")
-    check(qkv[:, 2 * hd:], want[:, 2 * hd:], ACC * S[:, 2 * hd:], f"adaln_qkv_rope v {w.name}")
+    check(qkv[:, 2 * hd:], want[:, 2 * hd:], E[:, 2 * hd:], f"adaln_qkv_rope v {w.name}")
 
 
 # ----------------------------------------------------- the block's layer shapes (d 5120)
@@ -295,17 +327,18 @@ def test_full_shape_adaln_qkv_rope(oracle_mod):
     W = wl.linear_weight(w, "w_qkv", 3 * w.hd, w.d, "cuda")
     wq, wk = wl.norm_weight(w, "wq", "cuda"), wl.norm_weight(w, "wk", "cuda")
     qkv = torch.empty((m, 3 * w.hd), dtype=torch.bfloat16, device="cuda")
-    stats = sol.row_stats_workspace(m)
+    ws = sol.adaln_workspace(m, 3 * w.hd, w.d)
     with sol.Rope3D(w.rope_dims, w.theta, w.max_pos) as rope:
-        sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, row_stats=stats, n_heads=w.n_heads, wq=wq, wk=wk,
+        sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, workspace=ws, n_heads=w.n_heads, wq=wq, wk=wk,
                            grid=w.grid, eps=w.eps)
         torch.cuda.synchronize()
     Wh = to_oracle(W)
     want, pre, h = oracle_mod.adaln_qkv_rope(
         to_oracle(x), Wh, to_oracle(shift), to_oracle(scale), to_oracle(wq), to_oracle(wk), n_heads=w.n_heads,
         head_dim=128, grid=w.grid, dims=w.rope_dims, theta=w.theta, eps=w.eps)
-    S = oracle_mod.linear_magnitude(h, Wh)
     hd = w.hd
-    bq = qk_bound(pre[:, :2 * hd], S[:, :2 * hd], f64(wq), f64(wk), w.n_heads, w.eps)
+    E = adaln_projection_bound(oracle_mod, to_oracle(x), Wh, to_oracle(shift), to_oracle(scale), h,
+                               np.zeros(m, np.int64), w.eps)
+    bq = qk_bound(pre[:, :2 * hd], E[:, :2 * hd], f64(wq), f64(wk), w.n_heads, w.eps)
     check(qkv[:, :2 * hd], want[:, :2 * hd], bq, "AdaLN -> QKV -> QK norm + RoPE, q|k")
-    check(qkv[:, 2 * hd:], want[:, 2 * hd:], ACC * S[:, 2 * hd:], "AdaLN -> QKV, v")
+    check(qkv[:, 2 * hd:], want[:, 2 * hd:], E[:, 2 * hd:], "AdaLN -> QKV, v")
