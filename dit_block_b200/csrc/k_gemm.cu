@@ -13,7 +13,7 @@
 //   single  one CTA per SM, 128 x 256 tiles, 4-stage ring of A 128x64 + B 256x64;
 //   pair    a cluster of two CTAs on two SMs, 256 x 256 tiles computed by 256-row
 //           tcgen05.mma (cta_group::2) issued by the leader CTA; each CTA loads half
-//           of A (its 128 rows) and half of B (128 of the 256 columns) into a 6-stage
+//           of A (its 128 rows) and half of B (128 of the 256 columns) into a 7-stage
 //           ring of 32 KiB stages and holds its 128 accumulator rows in its own TMEM.
 //           Per SM the copies per MMA drop by a third and the ring is half as deep
 //           again, which hides the copy latency.  The variant with the AdaLN operand
@@ -53,8 +53,14 @@ constexpr int BK = 64;                    // K per stage
 constexpr int UK = 16;                    // K of one tcgen05.mma (kind::f16)
 constexpr int A_BYTES = BM * BK * 2;      // 16 KiB: this CTA's rows of A per stage
 constexpr int TMEM_COLS = 2 * BN;         // two accumulators
-constexpr int GROUP_M = 16;               // m-blocks per raster group (L2 reuse)
-constexpr int MAX_STAGES = 6;
+#ifndef SOL_GEMM_GROUP_M
+#define SOL_GEMM_GROUP_M 16
+#endif
+#ifndef SOL_GEMM_PAIR_STAGES
+#define SOL_GEMM_PAIR_STAGES 7
+#endif
+constexpr int GROUP_M = SOL_GEMM_GROUP_M;  // m-blocks per raster group (L2 reuse)
+constexpr int MAX_STAGES = SOL_GEMM_PAIR_STAGES > 4 ? SOL_GEMM_PAIR_STAGES : 4;
 constexpr int PRODUCER_WARP = 0, MMA_WARP = 1, EPI_WARP0 = 2, XFORM_WARP0 = 6;
 // Epilogue warps: 8 (two per TMEM lane quarter, each taking half of the 256 columns), or
 // 4 beside the AdaLN transform warps (the register file holds no more).
@@ -62,7 +68,7 @@ template <bool PRO> __host__ __device__ constexpr int epi_warps() { return PRO ?
 constexpr uint32_t kWaitLimit = 4096;     // polls of <= ~1 ms each
 
 template <bool PAIR> struct Shape {
-    static constexpr int STAGES = PAIR ? 6 : 4;
+    static constexpr int STAGES = PAIR ? SOL_GEMM_PAIR_STAGES : 4;
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;   // rows of B (output columns) this CTA loads
     static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -648,8 +654,9 @@ constexpr int XFORM_GROUPS = SOL_GEMM_XFORM_GROUPS;
 constexpr int XFORM_WARPS = 4;
 constexpr int XFORM_THREADS = 32 * XFORM_WARPS * XFORM_GROUPS;
 // every stage must always belong to the same group (XFORM_WARPS arrivals per CTA and use)
-static_assert(Shape<false>::STAGES % XFORM_GROUPS == 0 && Shape<true>::STAGES % XFORM_GROUPS == 0,
-              "the transform groups must divide the stage count");
+static_assert(Shape<false>::STAGES % XFORM_GROUPS == 0, "the transform groups must divide the stage count");
+// pairs take the transform only when the groups divide their ring too
+constexpr bool kPairTransform = Shape<true>::STAGES % XFORM_GROUPS == 0;
 
 __device__ __forceinline__ uint4 lds128(uint32_t a)
 {
@@ -1052,9 +1059,11 @@ cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const ge
 template <int EPI, bool PRO, bool FOLD = false>
 cudaError_t launch_shape(const CUtensorMap& ma, const CUtensorMap& mb, gemm::Params& p, int64_t M, cudaStream_t s)
 {
-    if (use_pair(PRO)) {
-        p.num_tiles = (M + gemm::Shape<true>::TILE_M - 1) / gemm::Shape<true>::TILE_M * (int64_t)p.n_tiles_n;
-        return launch_kernel<EPI, PRO, FOLD, true>(ma, mb, p, s);
+    if constexpr (!PRO || gemm::kPairTransform) {
+        if (use_pair(PRO)) {
+            p.num_tiles = (M + gemm::Shape<true>::TILE_M - 1) / gemm::Shape<true>::TILE_M * (int64_t)p.n_tiles_n;
+            return launch_kernel<EPI, PRO, FOLD, true>(ma, mb, p, s);
+        }
     }
     p.num_tiles = (M + gemm::Shape<false>::TILE_M - 1) / gemm::Shape<false>::TILE_M * (int64_t)p.n_tiles_n;
     return launch_kernel<EPI, PRO, FOLD, false>(ma, mb, p, s);
