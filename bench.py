@@ -391,6 +391,24 @@ def _time(fn, reps: int, stream) -> float:
     return statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(reps))
 
 
+def _time_interleaved(fns, reps: int, stream) -> list[float]:
+    """Median milliseconds of each of `fns`, timed in turn within every repetition (CUDA
+    events on `stream`)."""
+    for fn in fns:
+        for _ in range(3):
+            fn()
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+          for _ in fns]
+    for r in range(reps):
+        for i, fn in enumerate(fns):
+            ev[i][r][0].record(stream)
+            fn()
+            ev[i][r][1].record(stream)
+    torch.cuda.synchronize()
+    return [statistics.median(a.elapsed_time(b) for a, b in ev[i]) for i in range(len(fns))]
+
+
 def time_next_ops(bufs, dev, args) -> dict:
     """Each op outside the block pass, timed alone at the workload's size (median of
     20 launches), with its algorithmic bytes per token."""
@@ -467,10 +485,9 @@ def time_linear_ops(bufs, dev, args) -> dict:
     out = {"tokens": m, "peak_tflops": peak, "peak_source": src + " (burst cuBLAS bf16)"}
 
     def entry(name, flops, fused, unfused, cublas, plain, saved_bytes):
-        tf = _time(fused, 10, stream)
-        tu = _time(unfused, 10, stream)
-        tcb = _time(cublas, 10, stream)
-        tp = _time(plain, 10, stream)
+        # the four arms alternate launch by launch, so clock drift under the power cap
+        # affects them alike
+        tf, tu, tcb, tp = _time_interleaved([fused, unfused, cublas, plain], 10, stream)
         ach = flops / (tf * 1e-3) / 1e12
         out[name] = {"ms": round(tf, 4), "TFLOP_s": round(ach, 1), "frac_of_bf16_peak": round(ach / peak, 4),
                      "unfused_ms": round(tu, 4), "cublas_gemm_ms": round(tcb, 4),

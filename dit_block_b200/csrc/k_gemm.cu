@@ -455,39 +455,38 @@ template <bool FOLD> __device__ __forceinline__ void fold32(float* v, const Fold
 }
 
 // One 128-wide head vector of the accumulator row (TMEM columns taddr .. +127):
-// v / sqrt(mean(v^2) + eps) * w, then the interleaved 3D rotation, stored to dst.
+// v / sqrt(mean(v^2) + eps) * w, then the interleaved 3D rotation, stored to dst.  The
+// vector is read from TMEM once and held in registers (a second read would compete with
+// the MMAs writing the other accumulator).
 template <bool FOLD>
 __device__ __forceinline__ void qk_head(uint32_t taddr, bool live, const bf16* w, const Params& p, int p0, int p1,
                                         int p2, bf16* dst, const FoldRow& fr, int col)
 {
-    float v[32];
-    float ss = 0.f;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-        tc::ld32(taddr + 32 * c, v);
-        if (live) fold32<FOLD>(v, fr, col + 32 * c);
+    // the whole head vector in registers: one read of its 128 TMEM columns
+    float v[128];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
-    }
+    for (int c = 0; c < 4; ++c) tc::ld32(taddr + 32 * c, v + 32 * c);
+    if (!live) return;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) fold32<FOLD>(v + 32 * c, fr, col + 32 * c);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 128; ++i) ss = fmaf(v[i], v[i], ss);
     const float r = rsqrtf(ss * (1.f / 128.f) + p.eps);
     const int h0 = p.rope.half[0], h01 = p.rope.half[0] + p.rope.half[1];
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-        tc::ld32(taddr + 32 * c, v);
-        if (!live) continue;
-        fold32<FOLD>(v, fr, col + 32 * c);
-        float fw[32];
-        if (w) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) unpack<bf16>(ld_cached(w + 32 * c + 8 * j), fw + 8 * j);
+    for (int c = 0; c < 16; ++c) {  // 8 elements (4 pairs) at a time
+        float fw[8];
+        if (w) {
+            unpack<bf16>(ld_cached(w + 8 * c), fw);
         } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) fw[i] = 1.f;
+            for (int e = 0; e < 8; ++e) fw[e] = 1.f;
         }
-        float o[32];
+        float o[8];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const int pi = 16 * c + m;  // pair index inside the head
+        for (int m = 0; m < 4; ++m) {
+            const int pi = 4 * c + m;  // pair index inside the head
             const float2* tab;
             if (pi < h0)
                 tab = p.rope.tab[0] + pi + (int64_t)p0 * p.rope.half[0];
@@ -496,12 +495,12 @@ __device__ __forceinline__ void qk_head(uint32_t taddr, bool live, const bf16* w
             else
                 tab = p.rope.tab[2] + (pi - h01) + (int64_t)p2 * p.rope.half[2];
             const float2 cs = __ldg(tab);
-            const float a = v[2 * m] * r * fw[2 * m];
-            const float b = v[2 * m + 1] * r * fw[2 * m + 1];
+            const float a = v[8 * c + 2 * m] * r * fw[2 * m];
+            const float b = v[8 * c + 2 * m + 1] * r * fw[2 * m + 1];
             o[2 * m] = a * cs.x - b * cs.y;
             o[2 * m + 1] = a * cs.y + b * cs.x;
         }
-        store32(dst + 32 * c, o);
+        *reinterpret_cast<uint4*>(dst + 8 * c) = pack<bf16>(o);
     }
 }
 
