@@ -325,7 +325,7 @@ def run_ours(args, w):
 
     # ---- ops beyond the block pass, each timed alone on the same workload
     next_ops = {} if args.no_next else time_next_ops(bufs, dev, args)
-    linear_ops = {} if (args.no_next or args.linear_tokens <= 0) else time_linear_ops(bufs, dev, args)
+    linear_ops = {} if (args.no_next or args.linear_tokens <= 0) else time_linear_ops(w, dev, args.linear_tokens)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -466,19 +466,24 @@ def time_next_ops(bufs, dev, args) -> dict:
     return out
 
 
-def time_linear_ops(bufs, dev, args) -> dict:
+def time_linear_ops(w, dev, m: int) -> dict:
     """The block's linear layers with the per-token operators fused in (tcgen05 GEMMs),
-    each timed alone on the first `linear_tokens` tokens of the workload (median of 10
-    launches), beside the same work unfused: a cuBLAS GEMM (torch.matmul) plus the
-    libsol per-token kernel, and the bare cuBLAS GEMM."""
+    each timed alone on `m` tokens of the workload's first sample (seeded inputs of its
+    shapes, weights ~ N(0, 1/in_features); median of 10 launches), beside the same work
+    unfused: a cuBLAS GEMM (torch.matmul) plus the libsol per-token kernel, the bare
+    cuBLAS GEMM and the bare libsol GEMM."""
     from dit_block_b200 import sol, workloads as wl
-    w, i = bufs.w, bufs.inp
     if w.dtype != torch.bfloat16 or w.head_dim != 128:
         return {}
-    m = min(int(args.linear_tokens), bufs.n_tokens)
+    m = min(int(m), w.tokens_per_sample)
     peak, src = measured_bf16_peak()
     stream = torch.cuda.current_stream(dev)
-    x = i["x"][:m]
+    i = {"x": wl.activation(w, "x", m, w.d, dev), "y_attn": wl.activation(w, "y_attn", m, w.d, dev),
+         "wq": wl.norm_weight(w, "wq", dev), "wk": wl.norm_weight(w, "wk", dev)}
+    for k in ("shift_msa", "scale_msa", "gate_msa", "gate_mlp"):
+        i[k] = wl.modulation(w, k, dev)
+    rope = sol.Rope3D(w.rope_dims, w.theta, w.max_pos)
+    x = i["x"]
     hd, d, inner = w.hd, w.d, w.inner
     # ops on one sample's tokens: modulation rows of sample 0, positions from its grid
     sel = dict(n_streams=1, tokens_per_sample=0)
@@ -499,13 +504,13 @@ def time_linear_ops(bufs, dev, args) -> dict:
     qkv = torch.empty((m, 3 * hd), dtype=w.dtype, device=dev)
     h = torch.empty_like(x)
     sh, sc = i["shift_msa"][:1], i["scale_msa"][:1]
-    fused = lambda: sol.adaln_qkv_rope(qkv, x, Wqkv, bufs.rope, sh, sc, workspace=ws, n_heads=w.n_heads,
+    fused = lambda: sol.adaln_qkv_rope(qkv, x, Wqkv, rope, sh, sc, workspace=ws, n_heads=w.n_heads,
                                        wq=i["wq"], wk=i["wk"], grid=w.grid, eps=w.eps, **sel)
 
     def unfused():
         sol.adaln_modulate(h, x, sh, sc, eps=w.eps, **sel)
         torch.matmul(h, Wqkv.t(), out=qkv)
-        sol.dit_epilogue(qkv, bufs.rope, n_heads=w.n_heads, head_dim=w.head_dim, wq=i["wq"], wk=i["wk"],
+        sol.dit_epilogue(qkv, rope, n_heads=w.n_heads, head_dim=w.head_dim, wq=i["wq"], wk=i["wk"],
                          grid=w.grid, eps=w.eps)
     entry("adaln_qkv_rope", 2.0 * m * d * 3 * hd, fused, unfused, lambda: torch.matmul(x, Wqkv.t(), out=qkv),
           lambda: sol.linear(qkv, x, Wqkv), 2 * d * 2 + 2 * (2 * hd) * 2)
@@ -513,7 +518,7 @@ def time_linear_ops(bufs, dev, args) -> dict:
 
     for name, K, wname, gate in (("o_proj_gated_residual", d, "w_o", "gate_msa"),
                                  ("down_proj_gated_residual", inner, "w_down", "gate_mlp")):
-        a = i["y_attn"][:m] if K == d else wl.activation(w, "act", m, K, dev)
+        a = i["y_attn"] if K == d else wl.activation(w, "act", m, K, dev)
         W = wl.linear_weight(w, wname, d, K, dev)
         o = torch.empty_like(x)
         y = torch.empty_like(x)
@@ -538,7 +543,20 @@ def time_linear_ops(bufs, dev, args) -> dict:
     entry("up_proj_swiglu", 2.0 * m * d * 2 * inner, fused, unfused, lambda: torch.matmul(x, Wup.t(), out=u),
           lambda: sol.linear(u, x, Wup), 2 * (2 * inner) * 2)
     del Wup, act, u
+    rope.close()
     return out
+
+
+def run_linear_only(args, w):
+    """--linear-only: the fused linear-layer timings alone, one JSON line."""
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    from dit_block_b200 import sol
+    sol.lib()
+    res = time_linear_ops(w, dev, args.linear_tokens)
+    torch.cuda.synchronize(dev)
+    print(json.dumps({"workload": w.name, "linear_ops": res, "device_errors": sol.device_errors()}), flush=True)
+    return 0
 
 
 def run_e2e(args, bufs, dev, world, step_bytes):
@@ -606,6 +624,8 @@ def main(argv=None):
     p.add_argument("--no-next", action="store_true", help="skip timing the ops outside the block pass")
     p.add_argument("--linear-tokens", type=int, default=32768,
                    help="tokens of the fused linear-layer timings (0 skips them)")
+    p.add_argument("--linear-only", action="store_true",
+                   help="time only the fused linear layers (prints their own JSON line)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-tokens", type=int, default=256, help="oracle token sample per reference step")
@@ -615,6 +635,8 @@ def main(argv=None):
     w = workloads.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.linear_only:
+        return run_linear_only(args, w)
     return run_ours(args, w)
 
 
