@@ -1008,13 +1008,10 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 // deeper ring saves).  SOL_LINEAR_SHAPE=single / pair overrides the choice.
 bool use_pair(bool transform)
 {
-    static const int forced = [] {
-        const char* e = std::getenv("SOL_LINEAR_SHAPE");
-        if (e && std::string(e) == "single") return 0;
-        if (e && std::string(e) == "pair") return 1;
-        return -1;
-    }();
-    return forced >= 0 ? forced == 1 : !transform;
+    const char* e = std::getenv("SOL_LINEAR_SHAPE");  // read per call (cheap beside a GEMM)
+    if (e && std::string(e) == "single") return false;
+    if (e && std::string(e) == "pair") return true;
+    return !transform;
 }
 
 template <int EPI, bool PRO, bool FOLD, bool PAIR>
@@ -1068,14 +1065,12 @@ cudaError_t launch_shape(const CUtensorMap& ma, const CUtensorMap& mb, gemm::Par
     return launch_kernel<EPI, PRO, FOLD, false>(ma, mb, p, s);
 }
 
-// AdaLN strategy: fold (default) or the operand transform; SOL_ADALN_STRATEGY overrides.
+// AdaLN strategy: fold (default) or the operand transform; SOL_ADALN_STRATEGY overrides
+// (read per call).
 bool adaln_fold()
 {
-    static const bool fold = [] {
-        const char* e = std::getenv("SOL_ADALN_STRATEGY");
-        return !(e && std::string(e) == "transform");
-    }();
-    return fold;
+    const char* e = std::getenv("SOL_ADALN_STRATEGY");
+    return !(e && std::string(e) == "transform");
 }
 
 }  // namespace

@@ -342,3 +342,118 @@ def test_full_shape_adaln_qkv_rope(oracle_mod):
     bq = qk_bound(pre[:, :2 * hd], E[:, :2 * hd], f64(wq), f64(wk), w.n_heads, w.eps)
     check(qkv[:, :2 * hd], want[:, :2 * hd], bq, "AdaLN -> QKV -> QK norm + RoPE, q|k")
     check(qkv[:, 2 * hd:], want[:, 2 * hd:], E[:, 2 * hd:], "AdaLN -> QKV, v")
+
+
+# ------------------------------------------- the other shapes and strategies of the kernel
+
+@pytest.mark.parametrize("env", [{"SOL_LINEAR_SHAPE": "single"}, {"SOL_ADALN_STRATEGY": "transform"},
+                                 {"SOL_LINEAR_SHAPE": "single", "SOL_ADALN_STRATEGY": "transform"},
+                                 {"SOL_LINEAR_SHAPE": "pair", "SOL_ADALN_STRATEGY": "transform"}],
+                         ids=lambda e: ",".join(f"{k}={v}" for k, v in e.items()))
+def test_alternative_shapes_and_strategies(oracle_mod, monkeypatch, env):
+    """Single-CTA tiles and the AdaLN operand transform (selected per call by the library's
+    environment switches) compute the same results under the same bounds."""
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    w = PACKED
+    m = w.n_tokens
+    x, shift, scale, sid, pos, kw = adaln_inputs(w, m)
+    hd = w.hd
+    W = wl.linear_weight(w, "w_qkv", 3 * hd, w.d, "cuda")
+    wq, wk = wl.norm_weight(w, "wq", "cuda"), wl.norm_weight(w, "wk", "cuda")
+    qkv = torch.empty((m, 3 * hd), dtype=torch.bfloat16, device="cuda")
+    ws = sol.adaln_workspace(m, 3 * hd, w.d, **kw)
+    with sol.Rope3D(w.rope_dims, w.theta, w.max_pos) as rope:
+        sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, workspace=ws, n_heads=w.n_heads, wq=wq, wk=wk,
+                           pos=pos, grid=w.grid, eps=w.eps, stream_id=sid, **kw)
+        torch.cuda.synchronize()
+    Wh = to_oracle(W)
+    want, pre, h = oracle_mod.adaln_qkv_rope(
+        to_oracle(x), Wh, to_oracle(shift), to_oracle(scale), to_oracle(wq), to_oracle(wk), n_heads=w.n_heads,
+        head_dim=128, pos=to_oracle(pos), grid=w.grid, tokens_per_sample=kw["tokens_per_sample"],
+        dims=w.rope_dims, theta=w.theta, eps=w.eps, stream_id=to_oracle(sid), n_streams=w.n_streams)
+    rr = modulation_rows(m, to_oracle(sid), w.n_streams, kw["tokens_per_sample"])
+    E = adaln_projection_bound(oracle_mod, to_oracle(x), Wh, to_oracle(shift), to_oracle(scale), h, rr, w.eps)
+    bq = qk_bound(pre[:, :2 * hd], E[:, :2 * hd], f64(wq), f64(wk), w.n_heads, w.eps)
+    check(qkv[:, :2 * hd], want[:, :2 * hd], bq, f"adaln_qkv_rope q|k {env}")
+    check(qkv[:, 2 * hd:], want[:, 2 * hd:], E[:, 2 * hd:], f"adaln_qkv_rope v {env}")
+    # the plain epilogues in the forced shape too
+    a = wl.activation(w, "attn", m, w.d, "cuda")
+    Wup = wl.linear_weight(w, "w_up", 2 * w.inner, w.d, "cuda")
+    out = torch.empty((m, w.inner), dtype=torch.bfloat16, device="cuda")
+    sol.linear_swiglu(out, a, Wup)
+    torch.cuda.synchronize()
+    A, Wu = to_oracle(a), to_oracle(Wup)
+    u = oracle_mod.linear(A, Wu)
+    S = oracle_mod.linear_magnitude(A, Wu)
+    ga, up = u[:, :w.inner], u[:, w.inner:]
+    ea, eb = ACC * S[:, :w.inner], ACC * S[:, w.inner:]
+    bound = 1.1 * ea * (np.abs(up) + eb) + np.abs(ga / (1 + np.exp(-ga))) * eb
+    check(out, oracle_mod.swiglu(np.ascontiguousarray(u), w.inner), bound, f"linear_swiglu {env}")
+
+
+# ------------------------------------ the size bench.py times (--linear-tokens), sampled rows
+
+BENCH_M = 32768
+
+
+def sample_rows(m, n=48, seed=7):
+    rng = np.random.default_rng(seed)
+    rows = np.concatenate([[0, 1, 127, 128, 255, 256, m - 1], rng.choice(m, n - 7, replace=False)])
+    return np.unique(rows)
+
+
+def test_bench_size_adaln_qkv_rope_sampled(oracle_mod):
+    w = FULL
+    m = BENCH_M
+    x = wl.activation(w, "x", m, w.d, "cuda")
+    shift, scale = wl.modulation(w, "shift_msa", "cuda"), wl.modulation(w, "scale_msa", "cuda")
+    W = wl.linear_weight(w, "w_qkv", 3 * w.hd, w.d, "cuda")
+    wq, wk = wl.norm_weight(w, "wq", "cuda"), wl.norm_weight(w, "wk", "cuda")
+    qkv = torch.empty((m, 3 * w.hd), dtype=torch.bfloat16, device="cuda")
+    ws = sol.adaln_workspace(m, 3 * w.hd, w.d)
+    with sol.Rope3D(w.rope_dims, w.theta, w.max_pos) as rope:
+        sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, workspace=ws, n_heads=w.n_heads, wq=wq, wk=wk,
+                           grid=w.grid, eps=w.eps)
+        torch.cuda.synchronize()
+    rows = sample_rows(m)
+    xs = to_oracle(x[torch.from_numpy(rows).cuda()])
+    Wh = to_oracle(W)
+    want, pre, h = oracle_mod.adaln_qkv_rope(
+        xs, Wh, to_oracle(shift), to_oracle(scale), to_oracle(wq), to_oracle(wk), n_heads=w.n_heads, head_dim=128,
+        grid=w.grid, dims=w.rope_dims, theta=w.theta, eps=w.eps, rows=rows)
+    hd = w.hd
+    E = adaln_projection_bound(oracle_mod, xs, Wh, to_oracle(shift), to_oracle(scale), h,
+                               np.zeros(len(rows), np.int64), w.eps)
+    got = qkv[torch.from_numpy(rows).cuda()]
+    bq = qk_bound(pre[:, :2 * hd], E[:, :2 * hd], f64(wq), f64(wk), w.n_heads, w.eps)
+    check(got[:, :2 * hd], want[:, :2 * hd], bq, "AdaLN -> QKV -> QK norm + RoPE at 32,768 tokens, q|k")
+    check(got[:, 2 * hd:], want[:, 2 * hd:], E[:, 2 * hd:], "AdaLN -> QKV at 32,768 tokens, v")
+
+
+def test_bench_size_mlp_sampled(oracle_mod):
+    w = FULL
+    m = BENCH_M
+    x = wl.activation(w, "x", m, w.d, "cuda")
+    act = wl.activation(w, "act", m, w.inner, "cuda")
+    Wup = wl.linear_weight(w, "w_up", 2 * w.inner, w.d, "cuda")
+    Wdn = wl.linear_weight(w, "w_down", w.d, w.inner, "cuda")
+    gate = wl.modulation(w, "gate_mlp", "cuda")
+    up = torch.empty((m, w.inner), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(x)
+    sol.linear_swiglu(up, x, Wup)
+    sol.linear_gated_residual(out, x, act, Wdn, gate)
+    torch.cuda.synchronize()
+    rows = sample_rows(m, seed=11)
+    ri = torch.from_numpy(rows).cuda()
+    xs, As = to_oracle(x[ri]), to_oracle(act[ri])
+    Wu, Wd, G = to_oracle(Wup), to_oracle(Wdn), to_oracle(gate)
+    u = oracle_mod.linear(xs, Wu)
+    S = oracle_mod.linear_magnitude(xs, Wu)
+    ga, b_ = u[:, :w.inner], u[:, w.inner:]
+    ea, eb = ACC * S[:, :w.inner], ACC * S[:, w.inner:]
+    bound = 1.1 * ea * (np.abs(b_) + eb) + np.abs(ga / (1 + np.exp(-ga))) * eb
+    check(up[ri], oracle_mod.swiglu(np.ascontiguousarray(u), w.inner), bound, "up + SwiGLU at 32,768 tokens")
+    want = oracle_mod.linear_gated_residual(xs, As, Wd, G)
+    bound = ACC * np.abs(oracle_mod.to_f64(G))[0][None, :] * oracle_mod.linear_magnitude(As, Wd)
+    check(out[ri], want, bound, "down + gated residual at 32,768 tokens")
