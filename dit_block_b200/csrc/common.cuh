@@ -182,7 +182,7 @@ __device__ __forceinline__ float block_sum(float v, float* buf)
 }  // namespace sol
 
 // ---------------------------------------------------------------------------------
-// Bulk asynchronous copies (global -> shared, no multicast) completed on an mbarrier.
+// Bulk asynchronous copies (global -> this CTA's shared memory) completed on an mbarrier.
 namespace sol {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
@@ -207,7 +207,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
-// One non-multicast bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned)
+// One bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned)
 // from global memory into this CTA's shared memory, counted on mbarrier `bar`.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
 {

@@ -29,8 +29,8 @@
 //                 stages: rewrite each landed x tile in shared memory as
 //                 h = (x - mean) * rstd * (1 + scale) + shift in bf16 before the MMA
 //                 reads it.
-// No copy uses multicast: the leader commits to its own and to the peer's barriers one
-// at a time.  Every wait on an mbarrier is bounded; a wait that gives up raises an error
+// Every copy lands in the shared memory of the one CTA that issued it, and the leader
+// commits to its own and to the peer's barriers one at a time.  Every wait on an mbarrier is bounded; a wait that gives up raises an error
 // flag and the CTA drains its in-flight copies and MMAs, frees its TMEM and returns.
 #include <algorithm>
 #include <cstdlib>

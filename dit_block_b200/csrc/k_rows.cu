@@ -1,7 +1,7 @@
 // k_rows.cu -- AdaLN modulation and the fused block prologue (gated residual -> AdaLN).
 //
 // Main kernel, k_adaln_bulk: a persistent CTA streams its rows (x, and y for the
-// prologue) into a ring of `stages` shared-memory buffers with non-multicast 1-D bulk
+// prologue) into a ring of `stages` shared-memory buffers with single-CTA 1-D bulk
 // async copies completed on one mbarrier per buffer.  While a row is reduced, the next
 // stages-1 rows of the CTA are already in flight, so HBM never waits on the reductions.
 // A buffer is refilled as soon as every thread has copied its slice of the row into

@@ -1,6 +1,7 @@
 // tcgen05.cuh -- thin wrappers over the sm_100a tensor-core (tcgen05), tensor-memory
 // and tensor-copy (TMA) instructions used by the linear-layer kernels, plus the two
-// descriptor encoders they need.  Inline PTX only; no multicast form of any copy.
+// descriptor encoders they need.  Inline PTX only; every copy fills the issuing CTA's
+// own shared memory.
 #pragma once
 
 #include <stdint.h>
@@ -108,7 +109,7 @@ __device__ __forceinline__ void ld32(uint32_t taddr, float* v)
 }
 
 // ---------------------------------------------------------------------------------
-// Tensor copies (TMA), global -> this CTA's shared memory, no multicast.
+// Tensor copies (TMA), global -> this CTA's own shared memory.
 
 // Load the box at (x = inner coordinate, y = row) of the 2-D tensor map `tmap` (a
 // __grid_constant__ kernel parameter) into `dst`, counted on mbarrier `bar`.  x must be
@@ -198,7 +199,8 @@ __device__ __forceinline__ void commit_pair(uint32_t bar)
 }
 
 // Tensor copy into this CTA's shared memory whose completion is counted on an mbarrier
-// that may live in the peer CTA (`bar` a shared::cluster address).  No multicast.
+// that may live in the peer CTA (`bar` a shared::cluster address).  The data lands in
+// this CTA only.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, int32_t x, int32_t y,
                                                  uint32_t bar)
 {
