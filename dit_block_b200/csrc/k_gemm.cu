@@ -34,6 +34,7 @@
 // flag and the CTA drains its in-flight copies and MMAs, frees its TMEM and returns.
 #include <algorithm>
 #include <cstdlib>
+#include <mutex>
 #include <string>
 
 #include <cuda.h>
@@ -1020,9 +1021,23 @@ cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const ge
     auto kern = gemm::k_linear<EPI, PRO, FOLD, PAIR>;
     const size_t smem = gemm::smem_bytes<PAIR>();
     const int threads = gemm::block_threads<PRO>();
-    static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (attr != cudaSuccess) return attr;
+    // per device: the shared-memory attribute and the resident pair count
+    constexpr int kMaxDevices = 64;
+    static int attr_set[kMaxDevices] = {};
+    static int max_pairs_dev[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::unique_lock<std::mutex> lk(mu);
+    if (!attr_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = 1;
+    }
     if constexpr (!PAIR) {
+        lk.unlock();
         const int64_t grid = std::min<int64_t>(p.num_tiles, (int64_t)sm_count());
         kern<<<(unsigned)grid, threads, smem, s>>>(ma, mb, p);
         return cudaGetLastError();
@@ -1039,14 +1054,15 @@ cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const ge
         cfg.attrs = la;
         cfg.numAttrs = 1;
         // as many pairs as can be resident at once (persistent workers)
-        static int max_pairs = [&] {
+        if (!max_pairs_dev[dev]) {
             cudaLaunchConfig_t q = cfg;
             q.gridDim = dim3(2 * (sm_count() / 2));
             int n = 0;
             if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n < 1) n = sm_count() / 2;
-            return n;
-        }();
-        const int64_t pairs = std::min<int64_t>(p.num_tiles, (int64_t)max_pairs);
+            max_pairs_dev[dev] = n;
+        }
+        const int64_t pairs = std::min<int64_t>(p.num_tiles, (int64_t)max_pairs_dev[dev]);
+        lk.unlock();
         cfg.gridDim = dim3((unsigned)(2 * pairs));
         return cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
     }
