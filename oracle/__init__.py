@@ -384,3 +384,13 @@ def adaln_qkv_rope(x, w, shift=None, scale=None, wq=None, wk=None, *, n_heads, h
     out = y.copy()
     out[:, :2 * hd] = qk
     return out, y, h
+
+
+def adaln_linear_swiglu(x, w, shift=None, scale=None, inner=None, *, eps=1e-6, stream_id=None, n_streams=1,
+                        tokens_per_sample=0, rows=None):
+    """The MLP input of a block: u = AdaLN(x) . W^T with W = [W1; W2] ([2*inner, d]), then
+    SwiGLU silu(u[:, :inner]) * u[:, inner:].  Returns (out, u, h)."""
+    u, h = adaln_linear(x, w, shift, scale, eps=eps, stream_id=stream_id, n_streams=n_streams,
+                        tokens_per_sample=tokens_per_sample, rows=rows)
+    u = np.ascontiguousarray(u)
+    return swiglu(u, inner), u, h

@@ -178,3 +178,19 @@ def test_adaln_qkv_rope_wiring(oracle_mod):
     pre_q = pre[:, :hd].reshape(n, n_heads, head_dim)
     expect = np.sqrt(((pre_q * wq) ** 2).mean(-1) / ((pre_q ** 2).mean(-1) + 1e-6))
     np.testing.assert_allclose(rms_q, expect, rtol=1e-12)
+
+
+def test_adaln_linear_swiglu_by_permutation(oracle_mod):
+    n, d, inner = 6, 16, 8
+    x = RNG.standard_normal((n, d)) * 2 - 0.5
+    shift = RNG.standard_normal((1, d)) * 0.1
+    scale = RNG.standard_normal((1, d)) * 0.1
+    p1, p2 = cyclic(d, 3)[:inner], cyclic(d, 11)[inner:]
+    w = np.concatenate([perm_matrix(cyclic(d, 3))[:inner], perm_matrix(cyclic(d, 11))[inner:]])
+    out, u, h = oracle_mod.adaln_linear_swiglu(x, w, shift, scale, inner, eps=1e-6)
+    th = torch.from_numpy(h)
+    np.testing.assert_allclose(out, (F.silu(th[:, p1]) * th[:, p2]).numpy(), rtol=1e-13, atol=1e-14)
+    np.testing.assert_array_equal(u, np.concatenate([h[:, p1], h[:, p2]], axis=1))
+    ref_h = (F.layer_norm(torch.from_numpy(x), (d,), eps=1e-6) * (1 + torch.from_numpy(scale))
+             + torch.from_numpy(shift)).numpy()
+    np.testing.assert_allclose(h, ref_h, rtol=1e-12, atol=1e-13)
