@@ -542,7 +542,19 @@ def time_linear_ops(w, dev, m: int) -> dict:
         sol.swiglu(act, u, inner=inner)
     entry("up_proj_swiglu", 2.0 * m * d * 2 * inner, fused, unfused, lambda: torch.matmul(x, Wup.t(), out=u),
           lambda: sol.linear(u, x, Wup), 2 * (2 * inner) * 2)
-    del Wup, act, u
+    # the MLP input in one pass: AdaLN -> up projection -> SwiGLU
+    ws2 = sol.adaln_workspace(m, 2 * inner, d, device=dev)
+    fused = lambda: sol.adaln_linear_swiglu(act, x, Wup, i["shift_msa"][:1], i["scale_msa"][:1], workspace=ws2,
+                                            eps=w.eps, **sel)
+    h2 = torch.empty_like(x)
+
+    def unfused():
+        sol.adaln_modulate(h2, x, i["shift_msa"][:1], i["scale_msa"][:1], eps=w.eps, **sel)
+        torch.matmul(h2, Wup.t(), out=u)
+        sol.swiglu(act, u, inner=inner)
+    entry("adaln_up_proj_swiglu", 2.0 * m * d * 2 * inner, fused, unfused, lambda: torch.matmul(x, Wup.t(), out=u),
+          lambda: sol.linear(u, x, Wup), 2 * d * 2 + 2 * (2 * inner) * 2)
+    del Wup, act, u, ws2, h2
     rope.close()
     return out
 

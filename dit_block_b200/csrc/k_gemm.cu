@@ -271,8 +271,8 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
         const int32_t y_a = (int32_t)(m_blk * S::TILE_M + (int64_t)w.rank * BM);
         // with the fold, B is this pass's modulation row's block of folded weights
         const int32_t nr = FOLD ? q.r * p.n_w : 0;
-        const int32_t n0 = EPI == EPI_SWIGLU ? n_blk * (BN / 2) : nr + n_blk * BN;
-        const int32_t n1 = EPI == EPI_SWIGLU ? p.inner + n_blk * (BN / 2) : n0 + BN / 2;
+        const int32_t n0 = nr + (EPI == EPI_SWIGLU ? n_blk * (BN / 2) : n_blk * BN);
+        const int32_t n1 = EPI == EPI_SWIGLU ? nr + p.inner + n_blk * (BN / 2) : n0 + BN / 2;
         for (int kb = 0; kb < kblocks; ++kb) {
             if (!wait_or_abort<PAIR>(smem_u32(&b->empty[s]), phase ^ 1u, b)) {
                 raise_abort(b, 1u);
@@ -589,6 +589,8 @@ __device__ void run_epilogue(const Params& p, Bars* b, const Where& w)
                 tc::ld32(tbase + 32 * c, v);
                 tc::ld32(tbase + BN / 2 + 32 * c, u);
                 if (!live) continue;
+                fold32<FOLD>(v, fr, n_blk * (BN / 2) + 32 * c);
+                fold32<FOLD>(u, fr, p.inner + n_blk * (BN / 2) + 32 * c);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = silu_mul_fast(v[i], u[i]);
                 store32(dst + 32 * c, v);
@@ -1161,6 +1163,7 @@ cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cuda
         p.n_w = a.N;
         if (epi == LINEAR_STORE) return launch_shape<gemm::EPI_STORE, false, true>(ma, mb, p, a.M, s);
         if (epi == LINEAR_QKROPE) return launch_shape<gemm::EPI_QKROPE, false, true>(ma, mb, p, a.M, s);
+        if (epi == LINEAR_SWIGLU) return launch_shape<gemm::EPI_SWIGLU, false, true>(ma, mb, p, a.M, s);
         return cudaErrorInvalidValue;
     }
     switch (epi) {
@@ -1170,7 +1173,8 @@ cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cuda
     case LINEAR_GATED:
         return launch_shape<gemm::EPI_GATED, false>(ma, mb, p, a.M, s);
     case LINEAR_SWIGLU:
-        return launch_shape<gemm::EPI_SWIGLU, false>(ma, mb, p, a.M, s);
+        return adaln ? launch_shape<gemm::EPI_SWIGLU, true>(ma, mb, p, a.M, s)
+                     : launch_shape<gemm::EPI_SWIGLU, false>(ma, mb, p, a.M, s);
     case LINEAR_QKROPE:
         return adaln ? launch_shape<gemm::EPI_QKROPE, true>(ma, mb, p, a.M, s)
                      : launch_shape<gemm::EPI_QKROPE, false>(ma, mb, p, a.M, s);

@@ -810,6 +810,43 @@ sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld
                        "sol_adaln_linear launch");
 }
 
+sol_status sol_adaln_linear_swiglu(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                                   const void* shift, const void* scale, int64_t ld_mod,
+                                   sol_modsel sel, const void* w, int64_t ld_w, void* workspace,
+                                   size_t workspace_bytes, int64_t n_tokens, int64_t inner,
+                                   int64_t d, float eps, sol_dtype dt, sol_stream_t stream)
+{
+    const int64_t n_out = 2 * inner;
+    TRY(check_linear_shape(n_tokens, n_out, d, dt, 256));
+    TRY(check_modsel(sel));
+    CHECK(std::isfinite(eps) && eps >= 0.f, SOL_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
+    TRY(check_tensor("w", w, ld_w, d, dt, true));
+    TRY(check_tensor("shift", shift, ld_mod, d, dt, false));
+    TRY(check_tensor("scale", scale, ld_mod, d, dt, false));
+    if (n_tokens == 0) return SOL_OK;
+    AdalnWorkspace lay;
+    int64_t R = 0;
+    TRY(check_workspace(workspace, workspace_bytes, n_tokens, n_out, d, sel, &lay, &R));
+    TRY(check_tensor("out", out, ld_out, inner, dt, true));
+    TRY(check_tensor("x", x, ld_x, d, dt, true));
+    CHECK(!spans_overlap(out, n_tokens, ld_out, inner, 2, x, n_tokens, ld_x, d, 2) &&
+              !spans_overlap(out, n_tokens, ld_out, inner, 2, w, n_out, ld_w, d, 2) &&
+              !spans_overlap(out, n_tokens, ld_out, inner, 2, workspace, 1, 0, (int64_t)lay.total, 1) &&
+              !spans_overlap(x, n_tokens, ld_x, d, 2, workspace, 1, 0, (int64_t)lay.total, 1) &&
+              !spans_overlap(w, n_out, ld_w, d, 2, workspace, 1, 0, (int64_t)lay.total, 1),
+          SOL_ERR_INVALID_ARGUMENT, "out, x or w overlaps another argument");
+    sol::LinearLaunch L = linear_base(out, ld_out, x, ld_x, w, ld_w, n_tokens, n_out, d);
+    const sol::ModSel ms = to_dev(sel, n_tokens);
+    set_workspace(L, workspace, lay, R);
+    L.shift = shift;
+    L.scale = scale;
+    L.ld_mod = ld_mod;
+    L.sel = &ms;
+    L.eps = eps;
+    return cuda_status(sol::launch_linear(sol::LINEAR_SWIGLU, true, L, (cudaStream_t)stream),
+                       "sol_adaln_linear_swiglu launch");
+}
+
 sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t ld_x,
                               const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
                               const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,

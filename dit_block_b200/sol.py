@@ -83,6 +83,8 @@ SIGNATURES = {
     "sol_adaln_workspace_bytes": ([_I64, _I64, _I64, ModSel], ctypes.c_size_t),
     "sol_adaln_linear": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _I64, _I64,
                           _I64, _F, _E, _P], _E),
+    "sol_adaln_linear_swiglu": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _I64,
+                                 _I64, _I64, _F, _E, _P], _E),
     "sol_adaln_qkv_rope": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _P, _P, _P,
                             _I32, _I32, _I32, _P, _I64, _I32, _I32, _I64, _F, _E, _P], _E),
 }
@@ -411,6 +413,16 @@ def adaln_linear(out, x, w, shift=None, scale=None, *, workspace, eps=1e-6, stre
         _ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
         _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(workspace), workspace.numel(),
         x.shape[0], w.shape[0], x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_linear")
+    return out
+
+
+def adaln_linear_swiglu(out, x, w, shift=None, scale=None, *, workspace, eps=1e-6, stream_id=None,
+                        n_streams=1, tokens_per_sample=0, stream=None):
+    """out = silu(h . W1^T) * (h . W2^T), h = AdaLN(x), W = [W1; W2]  (sol_adaln_linear_swiglu)."""
+    _check(lib().sol_adaln_linear_swiglu(
+        _ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
+        _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(workspace), workspace.numel(),
+        x.shape[0], w.shape[0] // 2, x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_linear_swiglu")
     return out
 
 

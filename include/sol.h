@@ -389,6 +389,19 @@ sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld
                             int64_t n_tokens, int64_t n_out, int64_t d, float eps, sol_dtype dt,
                             sol_stream_t stream);
 
+/* The MLP input of a block in one pass: AdaLN into the up projection, SwiGLU in its
+ * epilogue:
+ *     out[:, j] = silu((h . W1^T)[:, j]) * (h . W2^T)[:, j],   W = [W1; W2],
+ *     h = LN(x) * (1 + scale[r]) + shift[r]   (as sol_adaln_linear)
+ * x [n_tokens, d], W [2*inner, d] (gated half first, as sol_linear_swiglu), out
+ * [n_tokens, inner]; inner a multiple of 128; workspace as in sol_adaln_linear with
+ * n_out = 2 * inner.  Neither h nor the projection is stored or rounded. */
+sol_status sol_adaln_linear_swiglu(void* out, int64_t ld_out, const void* x, int64_t ld_x,
+                                   const void* shift, const void* scale, int64_t ld_mod,
+                                   sol_modsel sel, const void* w, int64_t ld_w, void* workspace,
+                                   size_t workspace_bytes, int64_t n_tokens, int64_t inner,
+                                   int64_t d, float eps, sol_dtype dt, sol_stream_t stream);
+
 /* The attention input of a block in one pass: AdaLN into the QKV projection, QK RMSNorm
  * + 3D RoPE in its epilogue:
  *     qkv = h . W^T  ([n_tokens, 3*n_heads*head_dim] = q | k | v),  h as in

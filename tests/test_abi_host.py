@@ -28,7 +28,7 @@ def last(L):
 
 def test_exports_every_declared_symbol(L):
     names = sol.header_functions()
-    assert len(names) == 23
+    assert len(names) == 24
     for n in names:
         assert hasattr(L, n), f"libsol.so does not export {n}"
         assert n in sol.SIGNATURES, f"binding has no signature for {n}"
@@ -200,3 +200,20 @@ def test_linear_epilogue_variants_validation(L):
     assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, ws, need, None, None, None,
                                 2, 4, 4, None, n, 2, 128, k, 1e-6, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
     assert "rope is NULL" in last(L)
+
+
+def test_adaln_linear_swiglu_validation(L):
+    n, k, inner = 300, 512, 384
+    x, w, out = FAKE, FAKE << 3, FAKE << 4
+    need = L.sol_adaln_workspace_bytes(n, 2 * inner, k, SEL)
+    ws = FAKE << 6
+    assert L.sol_adaln_linear_swiglu(out, inner, x, k, None, None, 0, SEL, w, k, ws, need, n, inner, k, 1e-6,
+                                     sol.F32, None) == sol.ERR_UNSUPPORTED
+    assert L.sol_adaln_linear_swiglu(out, 192, x, k, None, None, 0, SEL, w, k, ws, need, n, 192, k, 1e-6,
+                                     sol.BF16, None) == sol.ERR_UNSUPPORTED  # inner not a multiple of 128
+    assert L.sol_adaln_linear_swiglu(out, inner, x, k, None, None, 0, SEL, w, k, None, need, n, inner, k, 1e-6,
+                                     sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_adaln_linear_swiglu(out, inner, x, k, None, None, 0, SEL, w, k, ws, need - 256, n, inner, k,
+                                     1e-6, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_adaln_linear_swiglu(None, inner, None, k, None, None, 0, SEL, w, k, None, 0, 0, inner, k, 1e-6,
+                                     sol.BF16, None) == sol.OK

@@ -457,3 +457,23 @@ def test_bench_size_mlp_sampled(oracle_mod):
     want = oracle_mod.linear_gated_residual(xs, As, Wd, G)
     bound = ACC * np.abs(oracle_mod.to_f64(G))[0][None, :] * oracle_mod.linear_magnitude(As, Wd)
     check(out[ri], want, bound, "down + gated residual at 32,768 tokens")
+
+
+@pytest.mark.parametrize("w", [SMALL, PACKED], ids=lambda w: w.name)
+def test_adaln_linear_swiglu(oracle_mod, w):
+    m = w.n_tokens
+    x, shift, scale, sid, _, kw = adaln_inputs(w, m)
+    W = wl.linear_weight(w, "w_up", 2 * w.inner, w.d, "cuda")
+    out = torch.empty((m, w.inner), dtype=torch.bfloat16, device="cuda")
+    ws = sol.adaln_workspace(m, 2 * w.inner, w.d, **kw)
+    sol.adaln_linear_swiglu(out, x, W, shift, scale, workspace=ws, eps=w.eps, stream_id=sid, **kw)
+    torch.cuda.synchronize()
+    Wh = to_oracle(W)
+    want, u, h = oracle_mod.adaln_linear_swiglu(to_oracle(x), Wh, to_oracle(shift), to_oracle(scale), w.inner,
+                                                eps=w.eps, stream_id=to_oracle(sid), **kw)
+    rr = modulation_rows(m, to_oracle(sid), w.n_streams, kw["tokens_per_sample"])
+    E = adaln_projection_bound(oracle_mod, to_oracle(x), Wh, to_oracle(shift), to_oracle(scale), h, rr, w.eps)
+    ga, up = u[:, :w.inner], u[:, w.inner:]
+    ea, eb = E[:, :w.inner], E[:, w.inner:]
+    bound = 1.1 * ea * (np.abs(up) + eb) + np.abs(ga / (1 + np.exp(-ga))) * eb
+    check(out, want, bound, f"adaln_linear_swiglu {w.name}")
