@@ -390,6 +390,17 @@ def test_alternative_shapes_and_strategies(oracle_mod, monkeypatch, env):
     ea, eb = ACC * S[:, :w.inner], ACC * S[:, w.inner:]
     bound = 1.1 * ea * (np.abs(up) + eb) + np.abs(ga / (1 + np.exp(-ga))) * eb
     check(out, oracle_mod.swiglu(np.ascontiguousarray(u), w.inner), bound, f"linear_swiglu {env}")
+    # AdaLN into the up projection with SwiGLU, in the forced shape / strategy
+    ws2 = sol.adaln_workspace(m, 2 * w.inner, w.d, **kw)
+    sol.adaln_linear_swiglu(out, x, Wup, shift, scale, workspace=ws2, eps=w.eps, stream_id=sid, **kw)
+    torch.cuda.synchronize()
+    want, u2, h2 = oracle_mod.adaln_linear_swiglu(to_oracle(x), Wu, to_oracle(shift), to_oracle(scale), w.inner,
+                                                  eps=w.eps, stream_id=to_oracle(sid), **kw)
+    E2 = adaln_projection_bound(oracle_mod, to_oracle(x), Wu, to_oracle(shift), to_oracle(scale), h2, rr, w.eps)
+    ga, up = u2[:, :w.inner], u2[:, w.inner:]
+    ea, eb = E2[:, :w.inner], E2[:, w.inner:]
+    bound = 1.1 * ea * (np.abs(up) + eb) + np.abs(ga / (1 + np.exp(-ga))) * eb
+    check(out, want, bound, f"adaln_linear_swiglu {env}")
 
 
 # ------------------------------------ the size bench.py times (--linear-tokens), sampled rows
