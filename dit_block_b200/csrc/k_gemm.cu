@@ -1,7 +1,8 @@
 // k_gemm.cu -- the block's linear layers y = a . W^T on the fifth-generation tensor
-// cores, with the per-token operators fused into the operand load or the epilogue, so
-// that their inputs and outputs never make an extra trip through HBM:
-//   AdaLN -> QKV projection -> QK RMSNorm + 3D RoPE   (operand transform + epilogue)
+// cores, with the per-token operators fused in, so that their inputs and outputs never
+// make an extra trip through HBM:
+//   AdaLN -> QKV projection -> QK RMSNorm + 3D RoPE   (weight fold + epilogue)
+//   AdaLN -> MLP up projection -> SwiGLU              (weight fold + epilogue)
 //   MLP up projection -> SwiGLU                        (epilogue)
 //   output / MLP down projection -> gated residual     (epilogue)
 // [STM-RES] "SGLang acelera video do MiniMax-H3 em ate 6,2x em GPUs H200", section
@@ -18,20 +19,23 @@
 //           Per SM the copies per MMA drop by a third and the ring is half as deep
 //           again, which hides the copy latency.  The variant with the AdaLN operand
 //           transform runs single (see use_pair()).
+// AdaLN, two ways: the default folds (1 + scale) into a per-call copy of the weights and
+// corrects each accumulator row as rstd * (acc - mean * c_r) + b_r in the epilogue (a
+// plain GEMM on the raw tokens; see k_fold_weights); the alternative rewrites each landed
+// x tile in shared memory as h before the MMA reads it (the operand transform).
 // Warp roles:
 //   warp 0        tensor-copy producer (one thread);
 //   warp 1        MMA issuer (one thread; the leader CTA only in a pair) into one of two
 //                 TMEM accumulators of 256 fp32 columns, so the epilogue of tile i
 //                 overlaps the main loop of tile i+1; owns the TMEM allocation;
-//   warps 2..5    epilogue: each thread owns one accumulator row (TMEM lane), reads it
-//                 32 columns at a time and applies the fused operator;
-//   warps 6..13   (AdaLN variant only) operand transform, two groups on alternate
-//                 stages: rewrite each landed x tile in shared memory as
-//                 h = (x - mean) * rstd * (1 + scale) + shift in bf16 before the MMA
-//                 reads it.
+//   warps 2..9    epilogue (2..5 beside the transform): each thread owns one
+//                 accumulator row (TMEM lane) and half of its columns (all of them with
+//                 four warps), reads them 32 columns at a time and applies the operator;
+//   warps 6..13   (operand-transform variant only) two groups on alternate stages.
 // Every copy lands in the shared memory of the one CTA that issued it, and the leader
-// commits to its own and to the peer's barriers one at a time.  Every wait on an mbarrier is bounded; a wait that gives up raises an error
-// flag and the CTA drains its in-flight copies and MMAs, frees its TMEM and returns.
+// commits to its own and to the peer's barriers one at a time.  Every wait on an mbarrier
+// is bounded; a wait that gives up raises an error flag and the CTA drains its in-flight
+// copies and MMAs, frees its TMEM and returns.
 #include <algorithm>
 #include <cstdlib>
 #include <mutex>
@@ -115,7 +119,7 @@ struct Params {
     const bf16* x;
     int64_t ld_x;
     const bf16* gate;
-    // AdaLN operand transform
+    // AdaLN (both strategies)
     const float2* stats;  // [M] (mean, rstd)
     const bf16* shift;
     const bf16* scale;
