@@ -1,0 +1,148 @@
+// k_adaln_warp.cu -- AdaLN modulation (bf16) with one warp per token row, the whole row
+// held in registers.
+//
+// [XHH-QA] "8xH200 上的 MiniMax-H3" (xhh.club), Q&A on the fused kernels: AdaLN
+// modulation.  Per row: mean, biased variance by a second pass over the registers (no
+// cancellation from outliers), then h = (x - mean) * rstd * (1 + scale[r]) + shift[r].
+//
+// Lane l holds 16-byte vectors l, l + 32, ..., so every warp-wide load and store covers
+// 512 contiguous bytes; the reductions are warp shuffles only (no shared memory, no
+// barrier).  With VPL vectors per lane a row is 256 * VPL elements (d = 5120: VPL = 20,
+// 80 registers of packed bf16).  Arithmetic is f32x2; the row is widened from its
+// packed form in each of the three passes instead of being kept in fp32 (which would
+// double the registers and halve the rows in flight).  h may be x itself: a row is read
+// completely before any of it is written.  Used for bf16 AdaLN with d a multiple of 256
+// (up to 6144); the bulk-copy ring kernel (k_rows.cu) takes fp32, other widths and the
+// prologue.
+#include <algorithm>
+#include <cstdlib>
+#include <string>
+
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+// Launch shape, from a sweep on B200 at 245,952 x 5120 tokens (alone, full clock): blocks
+// of 64 threads, >= 4 per SM (the row needs ~226 registers per lane unspilled): 6.39-6.48
+// TB/s; 256 x 1: 6.25-6.46; 128 x 3 (capped at 168 registers, spilling): 5.99-6.13.
+#ifndef SOL_ADALN_WARP_BLOCK
+#define SOL_ADALN_WARP_BLOCK 64
+#endif
+#ifndef SOL_ADALN_WARP_MINB
+#define SOL_ADALN_WARP_MINB 4
+#endif
+
+namespace sol {
+
+template <int VPL>
+__global__ void __launch_bounds__(SOL_ADALN_WARP_BLOCK, SOL_ADALN_WARP_MINB) k_adaln_warp(bf16* h, int64_t ld_h, const bf16* x, int64_t ld_x,
+                                                    const bf16* shift, const bf16* scale, int64_t ld_mod,
+                                                    ModSel sel, int64_t n_tokens, float eps)
+{
+    constexpr int D = 256 * VPL;
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t wstep = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t row = w0; row < n_tokens; row += wstep) {
+        uint4 xv[VPL];
+        const bf16* xr = x + row * ld_x + 8 * lane;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) xv[i] = ld_stream(xr + 256 * i);
+
+        float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            float2 f[4];
+            unpack2<bf16>(xv[i], f);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s2 = __fadd2_rn(s2, f[e]);
+        }
+        const float mu = warp_sum(s2.x + s2.y) * (1.f / D);
+        const float2 mu2 = make_float2(-mu, -mu);
+        float2 q2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            float2 f[4];
+            unpack2<bf16>(xv[i], f);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 c = __fadd2_rn(f[e], mu2);
+                q2 = __ffma2_rn(c, c, q2);
+            }
+        }
+        const float rs = rsqrtf(warp_sum(q2.x + q2.y) * (1.f / D) + eps);
+        const float2 a2 = make_float2(rs, rs), c2 = make_float2(-mu * rs, -mu * rs);
+
+        const int64_t r = mod_row(row, sel);
+        const bf16* sc = scale ? scale + r * ld_mod + 8 * lane : nullptr;
+        const bf16* sh = shift ? shift + r * ld_mod + 8 * lane : nullptr;
+        bf16* hr = h + row * ld_h + 8 * lane;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            float2 f[4], g[4], b[4], o[4];
+            unpack2<bf16>(xv[i], f);
+            if (sc) {
+                unpack2<bf16>(ld_cached(sc + 256 * i), g);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) g[e] = make_float2(0.f, 0.f);
+            }
+            if (sh) {
+                unpack2<bf16>(ld_cached(sh + 256 * i), b);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) b[e] = make_float2(0.f, 0.f);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                o[e] = __ffma2_rn(__ffma2_rn(f[e], a2, c2), __fadd2_rn(make_float2(1.f, 1.f), g[e]), b[e]);
+            st_stream(hr + 256 * i, pack2<bf16>(o));
+        }
+    }
+}
+
+namespace {
+
+template <int VPL>
+cudaError_t launch_vpl(void* h, int64_t ld_h, const void* x, int64_t ld_x, const void* shift, const void* scale,
+                       int64_t ld_mod, const ModSel& sel, int64_t n_tokens, float eps, cudaStream_t s)
+{
+    auto kern = k_adaln_warp<VPL>;
+    constexpr int block = SOL_ADALN_WARP_BLOCK;
+    const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), block, 0);
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t rows_per_cta = block / 32;
+    const int64_t grid = std::min<int64_t>((int64_t)per_sm * sm_count(), (n_tokens + rows_per_cta - 1) / rows_per_cta);
+    kern<<<(unsigned)grid, block, 0, s>>>(static_cast<bf16*>(h), ld_h, static_cast<const bf16*>(x), ld_x,
+                                        static_cast<const bf16*>(shift), static_cast<const bf16*>(scale), ld_mod,
+                                        sel, n_tokens, eps);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool adaln_warp_fits(sol_dtype dt, int64_t d)
+{
+    if (!(dt == SOL_DTYPE_BF16 && d % 256 == 0 && d / 256 >= 1 && d / 256 <= 24)) return false;
+    const char* e = std::getenv("SOL_ADALN_KERNEL");  // "bulk" selects the ring kernel (read per call)
+    return !(e && std::string(e) == "bulk");
+}
+
+cudaError_t launch_adaln_warp(void* h, int64_t ld_h, const void* x, int64_t ld_x, const void* shift,
+                              const void* scale, int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
+                              float eps, cudaStream_t s)
+{
+    switch (d / 256) {
+#define SOL_ADALN_VPL(v) \
+    case v: return launch_vpl<v>(h, ld_h, x, ld_x, shift, scale, ld_mod, sel, n_tokens, eps, s);
+        SOL_ADALN_VPL(1) SOL_ADALN_VPL(2) SOL_ADALN_VPL(3) SOL_ADALN_VPL(4) SOL_ADALN_VPL(5) SOL_ADALN_VPL(6)
+        SOL_ADALN_VPL(7) SOL_ADALN_VPL(8) SOL_ADALN_VPL(9) SOL_ADALN_VPL(10) SOL_ADALN_VPL(11) SOL_ADALN_VPL(12)
+        SOL_ADALN_VPL(13) SOL_ADALN_VPL(14) SOL_ADALN_VPL(15) SOL_ADALN_VPL(16) SOL_ADALN_VPL(17) SOL_ADALN_VPL(18)
+        SOL_ADALN_VPL(19) SOL_ADALN_VPL(20) SOL_ADALN_VPL(21) SOL_ADALN_VPL(22) SOL_ADALN_VPL(23) SOL_ADALN_VPL(24)
+#undef SOL_ADALN_VPL
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace sol

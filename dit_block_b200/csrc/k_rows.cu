@@ -575,6 +575,8 @@ cudaError_t launch_adaln_rows(sol_dtype dt, void* x_out, int64_t ld_xo, void* h,
                               int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
                               float eps, cudaStream_t s)
 {
+    if (!y && adaln_warp_fits(dt, d))
+        return launch_adaln_warp(h, ld_h, x, ld_x, shift, scale, ld_mod, sel, n_tokens, d, eps, s);
     const int64_t vpr = d / (dt == SOL_DTYPE_BF16 ? 8 : 4);
     const bool resid = y != nullptr;
     const bool bulk_fits =

@@ -124,6 +124,13 @@ uint32_t gemm_device_error(bool clear);
 // Store a one-line reason for sol_last_error() on this host thread.
 void record_error(const char* msg);
 
+// AdaLN with one warp per row held in registers (k_adaln_warp.cu): whether it takes this
+// call, and its launcher.
+bool adaln_warp_fits(sol_dtype dt, int64_t d);
+cudaError_t launch_adaln_warp(void* h, int64_t ld_h, const void* x, int64_t ld_x, const void* shift,
+                              const void* scale, int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
+                              float eps, cudaStream_t s);
+
 // Whether a row of `vpr` 16-byte vectors fits the register-resident AdaLN kernel.
 bool adaln_row_fits(int64_t vpr);
 
