@@ -32,6 +32,15 @@
 #ifndef SOL_ADALN_WARP_MINB
 #define SOL_ADALN_WARP_MINB 4
 #endif
+// Fused prologue, from the same sweep (x, y at 245,952 x 5120): 4 warps per row, >= 4 CTAs
+// per SM (126 registers): 6.40-6.54 TB/s; 2 warps per row (222 registers): 6.06-6.10;
+// 4 warps with 3 or 5 CTAs per SM: 6.18-6.27 / 6.05-6.06; the ring kernel: 5.92-6.31.
+#ifndef SOL_PROLOGUE_REGS_MINB
+#define SOL_PROLOGUE_REGS_MINB 4
+#endif
+#ifndef SOL_PROLOGUE_REGS_WPR
+#define SOL_PROLOGUE_REGS_WPR 4  // warps per row of the fused prologue
+#endif
 
 namespace sol {
 
@@ -102,6 +111,108 @@ __global__ void __launch_bounds__(SOL_ADALN_WARP_BLOCK, SOL_ADALN_WARP_MINB) k_a
     }
 }
 
+// Fused prologue x' = x + gate[r] * y, h = AdaLN(x') (bf16) with one CTA of WPR warps per
+// row: each warp holds its 1/WPR of the row -- x, y and the gate row, VPH 16-byte vectors
+// of each per lane (d = 256 * VPH * WPR; d = 5120 with four warps: 60 registers) -- and
+// x' is recomputed in fp32 from them in each pass (never rounded before the norm).  The
+// warps' sums meet in shared memory, one barrier per reduction.  x_out (x' rounded) and h are
+// written in the last pass; x_out may be x (a row is read completely first).
+template <int VPH, int WPR>
+__global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
+    k_prologue_regs(bf16* x_out, int64_t ld_xo, bf16* h, int64_t ld_h, const bf16* x, int64_t ld_x, const bf16* y,
+                    int64_t ld_y, const bf16* gate, const bf16* shift, const bf16* scale, int64_t ld_mod,
+                    ModSel sel, int64_t n_tokens, float eps)
+{
+    constexpr int D = 256 * VPH * WPR;
+    __shared__ float red[2][WPR];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int col = warp * (256 * VPH) + 8 * lane;  // this lane's first element; vector i at + 256 i
+    for (int64_t row = blockIdx.x; row < n_tokens; row += gridDim.x) {
+        const int64_t r = mod_row(row, sel);
+        uint4 xv[VPH], yv[VPH], gv[VPH];
+        const bf16* xr = x + row * ld_x + col;
+        const bf16* yr = y + row * ld_y + col;
+#pragma unroll
+        for (int i = 0; i < VPH; ++i) {
+            xv[i] = ld_stream(xr + 256 * i);
+            yv[i] = ld_stream(yr + 256 * i);
+        }
+        const bf16* gr = gate ? gate + r * ld_mod + col : nullptr;
+#pragma unroll
+        for (int i = 0; i < VPH; ++i) gv[i] = gr ? ld_cached(gr + 256 * i) : make_uint4(0u, 0u, 0u, 0u);
+
+        float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < VPH; ++i) {
+            float2 fx[4], fy[4], fg[4];
+            unpack2<bf16>(xv[i], fx);
+            unpack2<bf16>(yv[i], fy);
+            unpack2<bf16>(gv[i], fg);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s2 = __fadd2_rn(s2, __ffma2_rn(fg[e], fy[e], fx[e]));
+        }
+        float t = warp_sum(s2.x + s2.y);
+        if (lane == 0) red[0][warp] = t;
+        __syncthreads();
+        float tot = 0.f;
+#pragma unroll
+        for (int k = 0; k < WPR; ++k) tot += red[0][k];
+        const float mu = tot * (1.f / D);
+        const float2 mu2 = make_float2(-mu, -mu);
+        float2 q2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < VPH; ++i) {
+            float2 fx[4], fy[4], fg[4];
+            unpack2<bf16>(xv[i], fx);
+            unpack2<bf16>(yv[i], fy);
+            unpack2<bf16>(gv[i], fg);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 c = __fadd2_rn(__ffma2_rn(fg[e], fy[e], fx[e]), mu2);
+                q2 = __ffma2_rn(c, c, q2);
+            }
+        }
+        t = warp_sum(q2.x + q2.y);
+        if (lane == 0) red[1][warp] = t;
+        __syncthreads();
+        tot = 0.f;
+#pragma unroll
+        for (int k = 0; k < WPR; ++k) tot += red[1][k];
+        const float rs = rsqrtf(tot * (1.f / D) + eps);
+        const float2 a2 = make_float2(rs, rs), c2 = make_float2(-mu * rs, -mu * rs);
+        const bf16* sc = scale ? scale + r * ld_mod + col : nullptr;
+        const bf16* sh = shift ? shift + r * ld_mod + col : nullptr;
+        bf16* xo = x_out + row * ld_xo + col;
+        bf16* hr = h + row * ld_h + col;
+#pragma unroll
+        for (int i = 0; i < VPH; ++i) {
+            float2 fx[4], fy[4], fg[4], xp[4], m1[4], m0[4], o[4];
+            unpack2<bf16>(xv[i], fx);
+            unpack2<bf16>(yv[i], fy);
+            unpack2<bf16>(gv[i], fg);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) xp[e] = __ffma2_rn(fg[e], fy[e], fx[e]);
+            st_stream(xo + 256 * i, pack2<bf16>(xp));
+            if (sc) {
+                unpack2<bf16>(ld_cached(sc + 256 * i), m1);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) m1[e] = make_float2(0.f, 0.f);
+            }
+            if (sh) {
+                unpack2<bf16>(ld_cached(sh + 256 * i), m0);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) m0[e] = make_float2(0.f, 0.f);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                o[e] = __ffma2_rn(__ffma2_rn(xp[e], a2, c2), __fadd2_rn(make_float2(1.f, 1.f), m1[e]), m0[e]);
+            st_stream(hr + 256 * i, pack2<bf16>(o));
+        }
+    }
+}
+
 namespace {
 
 template <int VPL>
@@ -120,6 +231,22 @@ cudaError_t launch_vpl(void* h, int64_t ld_h, const void* x, int64_t ld_x, const
     return cudaGetLastError();
 }
 
+template <int VPH, int WPR>
+cudaError_t launch_pro_vph(void* x_out, void* h, const void* x, const void* y, const void* gate, const void* shift,
+                           const void* scale, int64_t ld, int64_t ld_mod, const ModSel& sel, int64_t n_tokens,
+                           float eps, cudaStream_t s)
+{
+    auto kern = k_prologue_regs<VPH, WPR>;
+    const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), 32 * WPR, 0);
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t grid = std::min<int64_t>((int64_t)per_sm * sm_count(), n_tokens);
+    kern<<<(unsigned)grid, 32 * WPR, 0, s>>>(static_cast<bf16*>(x_out), ld, static_cast<bf16*>(h), ld,
+                                       static_cast<const bf16*>(x), ld, static_cast<const bf16*>(y), ld,
+                                       static_cast<const bf16*>(gate), static_cast<const bf16*>(shift),
+                                       static_cast<const bf16*>(scale), ld_mod, sel, n_tokens, eps);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool adaln_warp_fits(sol_dtype dt, int64_t d)
@@ -127,6 +254,32 @@ bool adaln_warp_fits(sol_dtype dt, int64_t d)
     if (!(dt == SOL_DTYPE_BF16 && d % 256 == 0 && d / 256 >= 1 && d / 256 <= 24)) return false;
     const char* e = std::getenv("SOL_ADALN_KERNEL");  // "bulk" selects the ring kernel (read per call)
     return !(e && std::string(e) == "bulk");
+}
+
+bool prologue_regs_fits(sol_dtype dt, int64_t d)
+{
+    constexpr int W = SOL_PROLOGUE_REGS_WPR;
+    if (!(dt == SOL_DTYPE_BF16 && d % (256 * W) == 0 && d / (256 * W) >= 1 && d / (256 * W) <= 24 / W)) return false;
+    const char* e = std::getenv("SOL_ADALN_KERNEL");  // "bulk" selects the ring kernel (read per call)
+    return !(e && std::string(e) == "bulk");
+}
+
+cudaError_t launch_prologue_regs(void* x_out, void* h, const void* x, const void* y, const void* gate,
+                                 const void* shift, const void* scale, int64_t ld, int64_t ld_mod, const ModSel& sel,
+                                 int64_t n_tokens, int64_t d, float eps, cudaStream_t s)
+{
+    constexpr int W = SOL_PROLOGUE_REGS_WPR;
+    switch (d / (256 * W)) {
+#define SOL_PRO_VPH(v)                                                                                           \
+    case v:                                                                                                      \
+        if constexpr (v * W <= 24)                                                                               \
+            return launch_pro_vph<v, W>(x_out, h, x, y, gate, shift, scale, ld, ld_mod, sel, n_tokens, eps, s); \
+        break;
+        SOL_PRO_VPH(1) SOL_PRO_VPH(2) SOL_PRO_VPH(3) SOL_PRO_VPH(4) SOL_PRO_VPH(5) SOL_PRO_VPH(6)
+        SOL_PRO_VPH(7) SOL_PRO_VPH(8) SOL_PRO_VPH(9) SOL_PRO_VPH(10) SOL_PRO_VPH(11) SOL_PRO_VPH(12)
+#undef SOL_PRO_VPH
+    }
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_adaln_warp(void* h, int64_t ld_h, const void* x, int64_t ld_x, const void* shift,

@@ -577,6 +577,8 @@ cudaError_t launch_adaln_rows(sol_dtype dt, void* x_out, int64_t ld_xo, void* h,
 {
     if (!y && adaln_warp_fits(dt, d))
         return launch_adaln_warp(h, ld_h, x, ld_x, shift, scale, ld_mod, sel, n_tokens, d, eps, s);
+    if (y && x_out && ld_xo == ld_h && ld_x == ld_h && ld_y == ld_h && prologue_regs_fits(dt, d))
+        return launch_prologue_regs(x_out, h, x, y, gate, shift, scale, ld_h, ld_mod, sel, n_tokens, d, eps, s);
     const int64_t vpr = d / (dt == SOL_DTYPE_BF16 ? 8 : 4);
     const bool resid = y != nullptr;
     const bool bulk_fits =

@@ -131,6 +131,12 @@ cudaError_t launch_adaln_warp(void* h, int64_t ld_h, const void* x, int64_t ld_x
                               const void* scale, int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
                               float eps, cudaStream_t s);
 
+// Fused prologue with the row in registers (two warps per row, k_adaln_warp.cu).
+bool prologue_regs_fits(sol_dtype dt, int64_t d);
+cudaError_t launch_prologue_regs(void* x_out, void* h, const void* x, const void* y, const void* gate,
+                                 const void* shift, const void* scale, int64_t ld, int64_t ld_mod, const ModSel& sel,
+                                 int64_t n_tokens, int64_t d, float eps, cudaStream_t s);
+
 // Whether a row of `vpr` 16-byte vectors fits the register-resident AdaLN kernel.
 bool adaln_row_fits(int64_t vpr);
 
