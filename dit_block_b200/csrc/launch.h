@@ -59,6 +59,14 @@ cudaError_t launch_qk_rmsnorm_rope3d(sol_dtype dt, void* q_out, void* k_out, int
                                      const RopeDev& rope, int64_t n_tokens, int32_t n_heads,
                                      int32_t head_dim, float eps, cudaStream_t s);
 
+// QK RMSNorm + 3D RoPE with one warp per (token, q or k) row in registers (k_qk_regs.cu):
+// bf16, head_dim 128, an even number of heads.
+bool qk_regs_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim);
+cudaError_t launch_qk_regs(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, const void* q, const void* k,
+                           int64_t ld_q, int64_t ld_k, const void* wq, const void* wk, const int32_t* pos,
+                           int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope, int64_t n_tokens,
+                           int32_t n_heads, float eps, cudaStream_t s);
+
 // QK RMSNorm + 3D RoPE, convention variants (k_qk_ex.cu): `across` = RMS over all heads
 // with weights [n_heads * head_dim]; `half` = rotate-half pairs; any output strides.
 cudaError_t launch_qk_ex(sol_dtype dt, bool across, bool half, void* q_out, void* k_out,
