@@ -13,7 +13,12 @@
 // double the registers and halve the rows in flight).  h may be x itself: a row is read
 // completely before any of it is written.  Used for bf16 AdaLN with d a multiple of 256
 // (up to 6144); the bulk-copy ring kernel (k_rows.cu) takes fp32, other widths and the
-// prologue.
+// prologues that are not register-resident.
+//
+// Both kernels here launch one CTA per row (or per block of rows) instead of a persistent
+// grid: SMs are refilled as CTAs retire, which at 245,952 x 5120 measured AdaLN 6.30 ->
+// 6.43 TB/s and the prologue 6.33 -> 6.73 TB/s on B200 (the launch shapes below were
+// swept under the persistent grid).
 #include <algorithm>
 #include <cstdlib>
 #include <string>
@@ -23,17 +28,20 @@
 #include "common.cuh"
 #include "launch.h"
 
-// Launch shape, from a sweep on B200 at 245,952 x 5120 tokens (alone, full clock): blocks
-// of 64 threads, >= 4 per SM (the row needs ~226 registers per lane unspilled): 6.39-6.48
-// TB/s; 256 x 1: 6.25-6.46; 128 x 3 (capped at 168 registers, spilling): 5.99-6.13.
+// Launch shape, from sweeps on B200 at 245,952 x 5120 tokens (alone, full clock).  With
+// one CTA per row block: one warp per CTA, >= 8 per SM: 6.56 TB/s; 64 x 4: 6.49-6.50;
+// 128 x 2: 6.42.  (Under the earlier persistent grid: 64 x 4: 6.39-6.48; 256 x 1:
+// 6.25-6.46; 128 x 3, capped at 168 registers and spilling: 5.99-6.13.)  The row needs
+// ~226 registers per lane unspilled.
 #ifndef SOL_ADALN_WARP_BLOCK
-#define SOL_ADALN_WARP_BLOCK 64
+#define SOL_ADALN_WARP_BLOCK 32
 #endif
 #ifndef SOL_ADALN_WARP_MINB
-#define SOL_ADALN_WARP_MINB 4
+#define SOL_ADALN_WARP_MINB 8
 #endif
-// Fused prologue, from the same sweep (x, y at 245,952 x 5120): 4 warps per row, >= 4 CTAs
-// per SM (126 registers): 6.40-6.54 TB/s; 2 warps per row (222 registers): 6.06-6.10;
+// Fused prologue, from the same sweeps (x, y at 245,952 x 5120): 4 warps per row, >= 4
+// CTAs per SM (126 registers); one CTA per row: 6.71-6.78 TB/s (5 per SM: 6.76-6.78, 3 per
+// SM: 6.05-6.13).  Persistent grid: 6.40-6.54; 2 warps per row (222 registers): 6.06-6.10;
 // 4 warps with 3 or 5 CTAs per SM: 6.18-6.27 / 6.05-6.06; the ring kernel: 5.92-6.31.
 #ifndef SOL_PROLOGUE_REGS_MINB
 #define SOL_PROLOGUE_REGS_MINB 4
@@ -224,7 +232,9 @@ cudaError_t launch_vpl(void* h, int64_t ld_h, const void* x, int64_t ld_x, const
     const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), block, 0);
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t rows_per_cta = block / 32;
-    const int64_t grid = std::min<int64_t>((int64_t)per_sm * sm_count(), (n_tokens + rows_per_cta - 1) / rows_per_cta);
+    // one CTA per rows_per_cta rows (the row loop covers what the grid limit leaves): the
+    // hardware refills SMs as CTAs retire, which streams faster than a persistent grid
+    const int64_t grid = std::min<int64_t>(0x7fffffffLL, (n_tokens + rows_per_cta - 1) / rows_per_cta);
     kern<<<(unsigned)grid, block, 0, s>>>(static_cast<bf16*>(h), ld_h, static_cast<const bf16*>(x), ld_x,
                                         static_cast<const bf16*>(shift), static_cast<const bf16*>(scale), ld_mod,
                                         sel, n_tokens, eps);
@@ -239,7 +249,7 @@ cudaError_t launch_pro_vph(void* x_out, void* h, const void* x, const void* y, c
     auto kern = k_prologue_regs<VPH, WPR>;
     const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), 32 * WPR, 0);
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const int64_t grid = std::min<int64_t>((int64_t)per_sm * sm_count(), n_tokens);
+    const int64_t grid = std::min<int64_t>(0x7fffffffLL, n_tokens);  // one CTA per row, as above
     kern<<<(unsigned)grid, 32 * WPR, 0, s>>>(static_cast<bf16*>(x_out), ld, static_cast<bf16*>(h), ld,
                                        static_cast<const bf16*>(x), ld, static_cast<const bf16*>(y), ld,
                                        static_cast<const bf16*>(gate), static_cast<const bf16*>(shift),

@@ -2,9 +2,13 @@
 // activation.  Both are pure HBM streams (2 reads : 1 write per element), so the design
 // is about bytes in flight and coalescing, not arithmetic:
 //   * every access is a 16-byte vector; consecutive threads touch consecutive vectors;
-//   * a CTA owns one fixed column chunk (blockDim.x * U vectors) of a row and walks rows
-//     with a grid stride; the grid is (resident CTAs per SM * SMs) rounded to a multiple
-//     of the chunks per row, so a CTA never changes columns;
+//   * a CTA owns one fixed column chunk (blockDim.x * U vectors) of a row and never
+//     changes columns.  The gated residual and SwiGLU launch one CTA per (row, chunk), so
+//     the hardware refills each SM as CTAs retire; at 245,952 tokens this streams 16-22%
+//     faster on B200 than a persistent grid walking rows with a stride (SwiGLU 5.8 -> 7.1
+//     TB/s, gated residual 6.1 -> 7.05 TB/s).  The Cache-DiT variant keeps the persistent
+//     grid (resident CTAs per SM * SMs, a multiple of the chunks per row), so that its
+//     per-sample fp64 sums cost a few atomics per CTA rather than per row;
 //   * each thread issues all U x inputs loads before the first use (U * 32 bytes in
 //     flight per thread); inputs nothing in the kernel writes come through the
 //     read-only path, outputs are stored without L1 allocation;
@@ -12,8 +16,15 @@
 #include "common.cuh"
 #include "launch.h"
 
+// First choice of 16-byte vectors per thread and input (U), per kernel, from a sweep on
+// B200 at 245,952 tokens: the gated residual (d 5120) streams 7.17-7.18 TB/s with U = 2
+// against 7.05-7.06 with U = 4 or 8; SwiGLU (d 13,824) 7.13-7.14 with U = 4..8 against
+// 6.45-6.48 with U = 2.
+#ifndef SOL_GATED_UPREF_FIRST
+#define SOL_GATED_UPREF_FIRST 2
+#endif
 #ifndef SOL_STREAM_UPREF_FIRST
-#define SOL_STREAM_UPREF_FIRST 4  // first choice of 16-byte vectors per thread and input
+#define SOL_STREAM_UPREF_FIRST 4  // SwiGLU and the Cache-DiT variant
 #endif
 
 namespace sol {
@@ -175,8 +186,9 @@ template <> __device__ __forceinline__ float silu_mul<float>(float a, float b)
 }
 
 // SwiGLU [XHH-QA, STM-GAN]: out_j = silu(a_j) * b_j.  MAXT / MINB: launch bounds; blocks of
-// at most 288 threads are compiled for three resident CTAs per SM (75 registers), which
-// keeps a third row in flight (bf16 d 13,824: +2.3% at 245,952 tokens).
+// at most 288 threads are compiled for three resident CTAs per SM (72 registers instead of
+// 76, which allow two), keeping a third row in flight (bf16 d 13,824, 245,952 tokens:
+// +2.3% under the persistent grid this kernel used to run on).
 template <typename T, int U, int MAXT, int MINB>
 __global__ void __launch_bounds__(MAXT, MINB)
 k_swiglu(T* __restrict__ out, int64_t ld_out, const T* __restrict__ a, const T* __restrict__ b,
@@ -236,14 +248,14 @@ struct StreamShape {
 };
 
 // Column chunking of a row of `vpr` vectors: the fewest idle lanes, then U in the
-// preference order below, then blockDim nearest 256.
-StreamShape choose_stream_shape(int64_t vpr)
+// preference order below (first_u moved to the front), then blockDim nearest 256.
+StreamShape choose_stream_shape(int64_t vpr, int first_u)
 {
     int kU[] = {4, 6, 8, 3, 2, 1};
-    for (int i = 0; i < 6; ++i)  // move the configured first choice to the front
-        if (kU[i] == SOL_STREAM_UPREF_FIRST) {
+    for (int i = 0; i < 6; ++i)
+        if (kU[i] == first_u) {
             for (int j = i; j > 0; --j) kU[j] = kU[j - 1];
-            kU[0] = SOL_STREAM_UPREF_FIRST;
+            kU[0] = first_u;
         }
     StreamShape best{0, 0, 0};
     int64_t best_waste = -1;
@@ -268,6 +280,15 @@ StreamShape choose_stream_shape(int64_t vpr)
     return best;
 }
 
+// One CTA per row chunk (capped at the grid limit; the kernels' row loop covers the rest).
+// The hardware then refills each SM as its CTAs retire, which streams measurably faster on
+// B200 than a persistent grid whose CTAs walk rows with a stride.
+int64_t flat_grid(const StreamShape& sh, int64_t n_tokens)
+{
+    const int64_t max_rows = 0x7fffffffLL / sh.cpr;
+    return (n_tokens < max_rows ? n_tokens : max_rows) * sh.cpr;
+}
+
 int64_t stream_grid(const void* kernel, const StreamShape& sh, int64_t n_tokens)
 {
     const int64_t resident = (int64_t)ctas_per_sm(kernel, sh.threads, 0) * sm_count();
@@ -282,8 +303,7 @@ cudaError_t run_gated_ro(void* out, int64_t ld_out, const void* x, int64_t ld_x,
                          int64_t ld_y, const void* gate, int64_t ld_mod, const ModSel& sel,
                          int64_t n_tokens, int64_t vpr, const StreamShape& sh, cudaStream_t s)
 {
-    const void* kfn = (const void*)k_gated_residual<T, U, RO>;
-    const int64_t grid = stream_grid(kfn, sh, n_tokens);
+    const int64_t grid = flat_grid(sh, n_tokens);
     k_gated_residual<T, U, RO><<<(unsigned)grid, sh.threads, 0, s>>>(
         (T*)out, ld_out, (const T*)x, ld_x, (const T*)y, ld_y, (const T*)gate, ld_mod, sel,
         n_tokens, (int32_t)vpr, sh.cpr);
@@ -306,8 +326,7 @@ template <typename T, int U, int MAXT, int MINB>
 cudaError_t run_swiglu_bounds(void* out, int64_t ld_out, const void* a, const void* b, int64_t ld_in,
                               int64_t n_tokens, int64_t vpr, const StreamShape& sh, cudaStream_t s)
 {
-    const void* kfn = (const void*)k_swiglu<T, U, MAXT, MINB>;
-    const int64_t grid = stream_grid(kfn, sh, n_tokens);
+    const int64_t grid = flat_grid(sh, n_tokens);
     k_swiglu<T, U, MAXT, MINB><<<(unsigned)grid, sh.threads, 0, s>>>((T*)out, ld_out, (const T*)a,
                                                                       (const T*)b, ld_in, n_tokens,
                                                                       (int32_t)vpr, sh.cpr);
@@ -342,7 +361,7 @@ cudaError_t launch_gated_residual(sol_dtype dt, void* out, int64_t ld_out, const
                                   cudaStream_t s)
 {
     const int64_t vpr = d / (dt == SOL_DTYPE_BF16 ? 8 : 4);
-    const StreamShape sh = choose_stream_shape(vpr);
+    const StreamShape sh = choose_stream_shape(vpr, SOL_GATED_UPREF_FIRST);
 #define CALL_B(U) run_gated<bf16, U>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, sel, n_tokens, vpr, sh, s)
 #define CALL_F(U) run_gated<float, U>(out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, sel, n_tokens, vpr, sh, s)
     if (dt == SOL_DTYPE_BF16) {
@@ -389,7 +408,7 @@ cudaError_t launch_gated_residual_diff(sol_dtype dt, void* out, int64_t ld_out, 
                                        cudaStream_t s)
 {
     const int64_t vpr = d / (dt == SOL_DTYPE_BF16 ? 8 : 4);
-    const StreamShape sh = choose_stream_shape(vpr);
+    const StreamShape sh = choose_stream_shape(vpr, SOL_STREAM_UPREF_FIRST);
 #define CALL_B(U) run_diff_r<bf16, U>(refresh, out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, cache, ld_c, sums, sel, n_tokens, vpr, sh, s)
 #define CALL_F(U) run_diff_r<float, U>(refresh, out, ld_out, x, ld_x, y, ld_y, gate, ld_mod, cache, ld_c, sums, sel, n_tokens, vpr, sh, s)
     if (dt == SOL_DTYPE_BF16) {
@@ -404,7 +423,7 @@ cudaError_t launch_swiglu(sol_dtype dt, void* out, int64_t ld_out, const void* a
                           int64_t ld_in, int64_t n_tokens, int64_t inner, cudaStream_t s)
 {
     const int64_t vpr = inner / (dt == SOL_DTYPE_BF16 ? 8 : 4);
-    const StreamShape sh = choose_stream_shape(vpr);
+    const StreamShape sh = choose_stream_shape(vpr, SOL_STREAM_UPREF_FIRST);
 #define CALL_B(U) run_swiglu<bf16, U>(out, ld_out, a, b, ld_in, n_tokens, vpr, sh, s)
 #define CALL_F(U) run_swiglu<float, U>(out, ld_out, a, b, ld_in, n_tokens, vpr, sh, s)
     if (dt == SOL_DTYPE_BF16) {
