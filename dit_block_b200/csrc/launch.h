@@ -66,6 +66,13 @@ cudaError_t launch_qk_regs(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_k
                            int64_t ld_q, int64_t ld_k, const void* wq, const void* wk, const int32_t* pos,
                            int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope, int64_t n_tokens,
                            int32_t n_heads, float eps, cudaStream_t s);
+// The same kernel for the convention variants (norm across heads, rotate-half pairs, strided
+// outputs): bf16, head_dim 128, a multiple of 8 heads up to 48.
+bool qk_regs_ex_fits(sol_dtype dt, bool half, int32_t n_heads, int32_t head_dim, const RopeDev& rope);
+cudaError_t launch_qk_regs_ex(bool across, bool half, void* q_out, void* k_out, const QkOutStrides& os, const void* q,
+                              const void* k, int64_t ld_q, int64_t ld_k, const void* wq, const void* wk,
+                              const int32_t* pos, int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope,
+                              int64_t n_tokens, int32_t n_heads, float eps, cudaStream_t s);
 
 // QK RMSNorm + 3D RoPE, convention variants (k_qk_ex.cu): `across` = RMS over all heads
 // with weights [n_heads * head_dim]; `half` = rotate-half pairs; any output strides.
