@@ -6,9 +6,9 @@
 //     changes columns.  The gated residual and SwiGLU launch one CTA per (row, chunk), so
 //     the hardware refills each SM as CTAs retire; at 245,952 tokens this streams 16-22%
 //     faster on B200 than a persistent grid walking rows with a stride (SwiGLU 5.8 -> 7.1
-//     TB/s, gated residual 6.1 -> 7.05 TB/s).  The Cache-DiT variant keeps the persistent
-//     grid (resident CTAs per SM * SMs, a multiple of the chunks per row), so that its
-//     per-sample fp64 sums cost a few atomics per CTA rather than per row;
+//     TB/s, gated residual 6.1 -> 7.05 TB/s).  The Cache-DiT variant gives each CTA a
+//     contiguous run of 8 rows, so that its per-sample fp64 sums cost one atomic per warp
+//     and sum per run rather than per row;
 //   * each thread issues all U x inputs loads before the first use (U * 32 bytes in
 //     flight per thread); inputs nothing in the kernel writes come through the
 //     read-only path, outputs are stored without L1 allocation;
@@ -22,6 +22,12 @@
 // 6.45-6.48 with U = 2.
 #ifndef SOL_GATED_UPREF_FIRST
 #define SOL_GATED_UPREF_FIRST 2
+#endif
+// Rows per CTA of the Cache-DiT variant, from a sweep on B200 (245,952 x 5120, refresh):
+// 8: 1.92 ms; 32: 1.98; a persistent-sized run (0): 2.11; 2: 3.80 (the per-warp fp64
+// atomics then contend).
+#ifndef SOL_DIFF_ROWS_PER_CTA
+#define SOL_DIFF_ROWS_PER_CTA 8
 #endif
 #ifndef SOL_STREAM_UPREF_FIRST
 #define SOL_STREAM_UPREF_FIRST 4  // SwiGLU and the Cache-DiT variant
@@ -78,19 +84,21 @@ k_gated_residual(T* __restrict__ out, int64_t ld_out, const T* x, int64_t ld_x,
 // in k_gated_residual; r = gate*y is compared with the cached residual of the previous
 // step, sums[s] += (sum |r - cache|, sum |cache|) over sample s, and with REFRESH the
 // cache is overwritten by r.  Each thread keeps fp32 partials per row and folds them into
-// fp64 accumulators; when a CTA moves to another sample (and at the end) every warp adds
-// its fp64 totals with one atomicAdd per sum, so no block barrier is needed.
+// fp64 accumulators; a CTA walks a contiguous run of rows_per_cta rows, and when it moves
+// to another sample (and at the end) every warp adds its fp64 totals with one atomicAdd
+// per sum, so no block barrier is needed.
 template <typename T, int U, bool REFRESH>
 __global__ void __launch_bounds__(512)
 k_gated_residual_diff(T* __restrict__ out, int64_t ld_out, const T* x, int64_t ld_x,
                       const T* __restrict__ y, int64_t ld_y, const T* __restrict__ gate,
                       int64_t ld_mod, T* cache, int64_t ld_c, double* __restrict__ sums,
-                      ModSel sel, int64_t n_tokens, int32_t vpr, int32_t cpr)
+                      ModSel sel, int64_t n_tokens, int32_t vpr, int32_t cpr, int64_t rows_per_cta)
 {
     constexpr int E = Vec<T>::N;
     const int chunk = blockIdx.x % cpr;
-    const int64_t row_step = gridDim.x / cpr;
     const int col0 = chunk * blockDim.x * U + threadIdx.x;
+    const int64_t row0 = (int64_t)(blockIdx.x / cpr) * rows_per_cta;
+    const int64_t row1 = row0 + rows_per_cta < n_tokens ? row0 + rows_per_cta : n_tokens;
     double acc_d = 0.0, acc_c = 0.0;
     int64_t cur = -1;
     auto flush = [&]() {
@@ -107,7 +115,7 @@ k_gated_residual_diff(T* __restrict__ out, int64_t ld_out, const T* x, int64_t l
         acc_d = 0.0;
         acc_c = 0.0;
     };
-    for (int64_t row = blockIdx.x / cpr; row < n_tokens; row += row_step) {
+    for (int64_t row = row0; row < row1; ++row) {  // a contiguous run of rows per CTA
         const int64_t mr = mod_row(row, sel);
         const int64_t sample = sample_of(row, sel);
         if (sample != cur) {  // uniform across the CTA
@@ -379,11 +387,20 @@ cudaError_t run_diff(void* out, int64_t ld_out, const void* x, int64_t ld_x, con
                      double* sums, const ModSel& sel, int64_t n_tokens, int64_t vpr,
                      const StreamShape& sh, cudaStream_t s)
 {
-    const void* kfn = (const void*)k_gated_residual_diff<T, U, REFRESH>;
-    const int64_t grid = stream_grid(kfn, sh, n_tokens);
+    if (n_tokens <= 0) return cudaSuccess;
+    // Rows per CTA: SOL_DIFF_ROWS_PER_CTA, or (0) as many as a grid of resident CTAs needs.
+    int64_t rows = SOL_DIFF_ROWS_PER_CTA;
+    if (rows <= 0) {
+        const void* kfn = (const void*)k_gated_residual_diff<T, U, REFRESH>;
+        const int64_t groups = stream_grid(kfn, sh, n_tokens) / sh.cpr;
+        rows = (n_tokens + groups - 1) / groups;
+    }
+    const int64_t max_groups = 0x7fffffffLL / sh.cpr;
+    if ((n_tokens + rows - 1) / rows > max_groups) rows = (n_tokens + max_groups - 1) / max_groups;
+    const int64_t grid = (n_tokens + rows - 1) / rows * sh.cpr;
     k_gated_residual_diff<T, U, REFRESH><<<(unsigned)grid, sh.threads, 0, s>>>(
         (T*)out, ld_out, (const T*)x, ld_x, (const T*)y, ld_y, (const T*)gate, ld_mod, (T*)cache, ld_c,
-        sums, sel, n_tokens, (int32_t)vpr, sh.cpr);
+        sums, sel, n_tokens, (int32_t)vpr, sh.cpr, rows);
     return cudaGetLastError();
 }
 

@@ -166,6 +166,8 @@ POOL_CASES = [  # dtype, head_dim, dims, n_heads, grid, samples, audio tokens pe
     (BF, 128, (32, 48, 48), 40, (2, 3, 4), 2, 5, 64),    # packed video+audio, explicit positions
     (torch.float32, 128, (32, 48, 48), 2, (2, 4, 4), 1, 0, 64),
     (torch.float32, 32, (8, 12, 12), 7, (3, 3, 3), 2, 0, 5),
+    (BF, 128, (32, 48, 48), 8, (3, 3, 5), 2, 3, 7),      # register kernel, 1 slot per warp, odd blocks
+    (BF, 128, (32, 48, 48), 48, (2, 2, 3), 1, 0, 5),     # register kernel, 6 slots per warp
 ]
 
 
@@ -240,6 +242,7 @@ EX_CASES = [  # dtype, head_dim, dims, n_heads, grid, samples
     (BF, 64, (16, 16, 32), 5, (4, 3, 3), 3),
     (torch.float32, 128, (32, 48, 48), 3, (2, 4, 4), 1),
     (torch.float32, 32, (8, 8, 16), 7, (3, 3, 3), 2),
+    (BF, 128, (32, 48, 48), 8, (2, 3, 5), 3),   # register kernel, 4 slots per lane
 ]
 
 
