@@ -62,6 +62,9 @@ __global__ void __launch_bounds__(SOL_ADALN_WARP_BLOCK, SOL_ADALN_WARP_MINB) k_a
     const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t wstep = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t row = w0; row < n_tokens; row += wstep) {
+        // the modulation row first: with per-token stream ids its load is then in flight
+        // with the row's, not on the critical path after the reductions
+        const int64_t r = mod_row(row, sel);
         uint4 xv[VPL];
         const bf16* xr = x + row * ld_x + 8 * lane;
 #pragma unroll
@@ -91,7 +94,6 @@ __global__ void __launch_bounds__(SOL_ADALN_WARP_BLOCK, SOL_ADALN_WARP_MINB) k_a
         const float rs = rsqrtf(warp_sum(q2.x + q2.y) * (1.f / D) + eps);
         const float2 a2 = make_float2(rs, rs), c2 = make_float2(-mu * rs, -mu * rs);
 
-        const int64_t r = mod_row(row, sel);
         const bf16* sc = scale ? scale + r * ld_mod + 8 * lane : nullptr;
         const bf16* sh = shift ? shift + r * ld_mod + 8 * lane : nullptr;
         bf16* hr = h + row * ld_h + 8 * lane;
