@@ -46,7 +46,8 @@ def randn(shape, dtype, seed, std=1.0, mean=0.0):
 # --------------------------------------------------------------------------- small cases
 
 SHAPES = [  # (n_tokens, d): several rows per CTA wave, ragged widths, a single row
-    (1, 8), (37, 256), (301, 5120), (67, 5128), (129, 1000), (5, 16384), (2049, 64)]
+    (1, 8), (37, 256), (301, 5120), (67, 5128), (129, 1000), (5, 16384), (2049, 64),
+    (19, 6144), (23, 1024)]  # the widest register-resident rows; the narrowest 4-warp prologue
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, BF])
@@ -118,6 +119,8 @@ QK_CASES = [  # dtype, head_dim, dims, n_heads, grid (T,H,W), samples
     (torch.float32, 128, (32, 48, 48), 2, (2, 4, 4), 1),
     (torch.float32, 64, (16, 24, 24), 3, (5, 2, 3), 2),
     (torch.float32, 32, (8, 12, 12), 7, (3, 3, 3), 1),
+    (BF, 128, (32, 48, 48), 48, (2, 3, 4), 2),   # register kernel, 24 slots per lane (the most)
+    (BF, 128, (32, 48, 48), 2, (3, 3, 3), 1),    # register kernel, 1 slot per lane
 ]
 
 
