@@ -39,12 +39,15 @@
 #ifndef SOL_ADALN_WARP_MINB
 #define SOL_ADALN_WARP_MINB 8
 #endif
-// Fused prologue, from the same sweeps (x, y at 245,952 x 5120): 4 warps per row, >= 4
-// CTAs per SM (126 registers); one CTA per row: 6.71-6.78 TB/s (5 per SM: 6.76-6.78, 3 per
-// SM: 6.05-6.13).  Persistent grid: 6.40-6.54; 2 warps per row (222 registers): 6.06-6.10;
-// 4 warps with 3 or 5 CTAs per SM: 6.18-6.27 / 6.05-6.06; the ring kernel: 5.92-6.31.
+// Fused prologue, from the same sweeps (x, y at 245,952 x 5120): 4 warps per row, one CTA
+// per row, x' kept in fp32 registers, >= 6 CTAs per SM (80 registers): 1.48 ms alone, 1.50
+// ms inside 100 back-to-back block passes under the power cap (~1.6 GHz).  The same with 5
+// CTAs per SM: 1.48 / 1.52; with 4 (120 registers): 1.80 under the cap.  x' re-formed
+// from the packed inputs in every pass (126 registers, 4 per SM): 1.49-1.50 / 1.57.
+// Earlier, persistent grid: 6.40-6.54 TB/s; 2 warps per row (222 registers): 6.06-6.10;
+// the ring kernel: 5.92-6.31.
 #ifndef SOL_PROLOGUE_REGS_MINB
-#define SOL_PROLOGUE_REGS_MINB 4
+#define SOL_PROLOGUE_REGS_MINB 6
 #endif
 #ifndef SOL_PROLOGUE_REGS_WPR
 #define SOL_PROLOGUE_REGS_WPR 4  // warps per row of the fused prologue
@@ -122,11 +125,12 @@ __global__ void __launch_bounds__(SOL_ADALN_WARP_BLOCK, SOL_ADALN_WARP_MINB) k_a
 }
 
 // Fused prologue x' = x + gate[r] * y, h = AdaLN(x') (bf16) with one CTA of WPR warps per
-// row: each warp holds its 1/WPR of the row -- x, y and the gate row, VPH 16-byte vectors
-// of each per lane (d = 256 * VPH * WPR; d = 5120 with four warps: 60 registers) -- and
-// x' is recomputed in fp32 from them in each pass (never rounded before the norm).  The
-// warps' sums meet in shared memory, one barrier per reduction.  x_out (x' rounded) and h are
-// written in the last pass; x_out may be x (a row is read completely first).
+// row: each warp loads its 1/WPR of the row -- x, y and the gate row, VPH 16-byte vectors
+// of each per lane (d = 256 * VPH * WPR) -- forms x' once in fp32 registers (d = 5120 with
+// four warps: 40 registers; never rounded before the norm) and reads it in the two later
+// passes.  x_out (x' rounded) is written in the first pass, h in the last; x_out may be x
+// (a lane overwrites only elements it has already read).  The warps' sums meet in shared
+// memory, one barrier per reduction.
 template <int VPH, int WPR>
 __global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
     k_prologue_regs(bf16* x_out, int64_t ld_xo, bf16* h, int64_t ld_h, const bf16* x, int64_t ld_x, const bf16* y,
@@ -151,6 +155,10 @@ __global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
 #pragma unroll
         for (int i = 0; i < VPH; ++i) gv[i] = gr ? ld_cached(gr + 256 * i) : make_uint4(0u, 0u, 0u, 0u);
 
+        // x' = x + gate * y once, kept in fp32 (never rounded before the norm); x_out gets
+        // its rounding at once -- a lane overwrites only what it has already read
+        bf16* xo = x_out + row * ld_xo + col;
+        float2 xp[VPH][4];
         float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < VPH; ++i) {
@@ -159,7 +167,11 @@ __global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
             unpack2<bf16>(yv[i], fy);
             unpack2<bf16>(gv[i], fg);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) s2 = __fadd2_rn(s2, __ffma2_rn(fg[e], fy[e], fx[e]));
+            for (int e = 0; e < 4; ++e) {
+                xp[i][e] = __ffma2_rn(fg[e], fy[e], fx[e]);
+                s2 = __fadd2_rn(s2, xp[i][e]);
+            }
+            st_stream(xo + 256 * i, pack2<bf16>(xp[i]));
         }
         float t = warp_sum(s2.x + s2.y);
         if (lane == 0) red[0][warp] = t;
@@ -172,13 +184,9 @@ __global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
         float2 q2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < VPH; ++i) {
-            float2 fx[4], fy[4], fg[4];
-            unpack2<bf16>(xv[i], fx);
-            unpack2<bf16>(yv[i], fy);
-            unpack2<bf16>(gv[i], fg);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 c = __fadd2_rn(__ffma2_rn(fg[e], fy[e], fx[e]), mu2);
+                const float2 c = __fadd2_rn(xp[i][e], mu2);
                 q2 = __ffma2_rn(c, c, q2);
             }
         }
@@ -192,17 +200,10 @@ __global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
         const float2 a2 = make_float2(rs, rs), c2 = make_float2(-mu * rs, -mu * rs);
         const bf16* sc = scale ? scale + r * ld_mod + col : nullptr;
         const bf16* sh = shift ? shift + r * ld_mod + col : nullptr;
-        bf16* xo = x_out + row * ld_xo + col;
         bf16* hr = h + row * ld_h + col;
 #pragma unroll
         for (int i = 0; i < VPH; ++i) {
-            float2 fx[4], fy[4], fg[4], xp[4], m1[4], m0[4], o[4];
-            unpack2<bf16>(xv[i], fx);
-            unpack2<bf16>(yv[i], fy);
-            unpack2<bf16>(gv[i], fg);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) xp[e] = __ffma2_rn(fg[e], fy[e], fx[e]);
-            st_stream(xo + 256 * i, pack2<bf16>(xp));
+            float2 m1[4], m0[4], o[4];
             if (sc) {
                 unpack2<bf16>(ld_cached(sc + 256 * i), m1);
             } else {
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                o[e] = __ffma2_rn(__ffma2_rn(xp[e], a2, c2), __fadd2_rn(make_float2(1.f, 1.f), m1[e]), m0[e]);
+                o[e] = __ffma2_rn(__ffma2_rn(xp[i][e], a2, c2), __fadd2_rn(make_float2(1.f, 1.f), m1[e]), m0[e]);
             st_stream(hr + 256 * i, pack2<bf16>(o));
         }
     }
