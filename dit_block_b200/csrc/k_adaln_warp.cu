@@ -12,8 +12,15 @@
 // packed form in each of the three passes instead of being kept in fp32 (which would
 // double the registers and halve the rows in flight).  h may be x itself: a row is read
 // completely before any of it is written.  Used for bf16 AdaLN with d a multiple of 256
-// (up to 6144); the bulk-copy ring kernel (k_rows.cu) takes fp32, other widths and the
-// prologues that are not register-resident.
+// (up to 6144) that the four-warp kernel below does not take; the bulk-copy ring kernel
+// (k_rows.cu) takes fp32, other widths and the prologues that are not register-resident.
+//
+// The four-warp kernel (k_prologue_regs) serves the fused prologue and, without its
+// residual, plain AdaLN too (d a multiple of 1024 up to 6144, h and x with one row
+// stride): a quarter row per warp fits in fp32 registers, so x is widened once instead of
+// in each of three passes, and 64 registers allow 8 CTAs (32 warps) per SM.  At 245,952 x
+// 5120: 0.740 ms (6.81 TB/s) alone against 0.777 for the one-warp kernel, and 0.815 vs
+// 0.854 ms inside 100 back-to-back block passes under the power cap.
 //
 // Both kernels here launch one CTA per row (or per block of rows) instead of a persistent
 // grid: SMs are refilled as CTAs retire, which at 245,952 x 5120 measured AdaLN 6.30 ->
@@ -48,6 +55,9 @@
 // the ring kernel: 5.92-6.31.
 #ifndef SOL_PROLOGUE_REGS_MINB
 #define SOL_PROLOGUE_REGS_MINB 6
+#endif
+#ifndef SOL_ADALN4_MINB
+#define SOL_ADALN4_MINB 8  // the same kernel without the residual (plain AdaLN); 10 or 12 spill: 3.0-3.7 TB/s
 #endif
 #ifndef SOL_PROLOGUE_REGS_WPR
 #define SOL_PROLOGUE_REGS_WPR 4  // warps per row of the fused prologue
@@ -131,8 +141,9 @@ __global__ void __launch_bounds__(SOL_ADALN_WARP_BLOCK, SOL_ADALN_WARP_MINB) k_a
 // passes.  x_out (x' rounded) is written in the first pass, h in the last; x_out may be x
 // (a lane overwrites only elements it has already read).  The warps' sums meet in shared
 // memory, one barrier per reduction.
-template <int VPH, int WPR>
-__global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
+// RES = false: plain AdaLN of x (no residual, no x_out) in the same four-warp form.
+template <int VPH, int WPR, bool RES>
+__global__ void __launch_bounds__(32 * WPR, RES ? SOL_PROLOGUE_REGS_MINB : SOL_ADALN4_MINB)
     k_prologue_regs(bf16* x_out, int64_t ld_xo, bf16* h, int64_t ld_h, const bf16* x, int64_t ld_x, const bf16* y,
                     int64_t ld_y, const bf16* gate, const bf16* shift, const bf16* scale, int64_t ld_mod,
                     ModSel sel, int64_t n_tokens, float eps)
@@ -149,9 +160,9 @@ __global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
 #pragma unroll
         for (int i = 0; i < VPH; ++i) {
             xv[i] = ld_stream(xr + 256 * i);
-            yv[i] = ld_stream(yr + 256 * i);
+            if (RES) yv[i] = ld_stream(yr + 256 * i);
         }
-        const bf16* gr = gate ? gate + r * ld_mod + col : nullptr;
+        const bf16* gr = RES && gate ? gate + r * ld_mod + col : nullptr;
 #pragma unroll
         for (int i = 0; i < VPH; ++i) gv[i] = gr ? ld_cached(gr + 256 * i) : make_uint4(0u, 0u, 0u, 0u);
 
@@ -162,16 +173,21 @@ __global__ void __launch_bounds__(32 * WPR, SOL_PROLOGUE_REGS_MINB)
         float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < VPH; ++i) {
-            float2 fx[4], fy[4], fg[4];
+            float2 fx[4];
             unpack2<bf16>(xv[i], fx);
-            unpack2<bf16>(yv[i], fy);
-            unpack2<bf16>(gv[i], fg);
+            if constexpr (RES) {
+                float2 fy[4], fg[4];
+                unpack2<bf16>(yv[i], fy);
+                unpack2<bf16>(gv[i], fg);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                xp[i][e] = __ffma2_rn(fg[e], fy[e], fx[e]);
-                s2 = __fadd2_rn(s2, xp[i][e]);
+                for (int e = 0; e < 4; ++e) xp[i][e] = __ffma2_rn(fg[e], fy[e], fx[e]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xp[i][e] = fx[e];
             }
-            st_stream(xo + 256 * i, pack2<bf16>(xp[i]));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s2 = __fadd2_rn(s2, xp[i][e]);
+            if (RES) st_stream(xo + 256 * i, pack2<bf16>(xp[i]));
         }
         float t = warp_sum(s2.x + s2.y);
         if (lane == 0) red[0][warp] = t;
@@ -244,12 +260,12 @@ cudaError_t launch_vpl(void* h, int64_t ld_h, const void* x, int64_t ld_x, const
     return cudaGetLastError();
 }
 
-template <int VPH, int WPR>
+template <int VPH, int WPR, bool RES>
 cudaError_t launch_pro_vph(void* x_out, void* h, const void* x, const void* y, const void* gate, const void* shift,
                            const void* scale, int64_t ld, int64_t ld_mod, const ModSel& sel, int64_t n_tokens,
                            float eps, cudaStream_t s)
 {
-    auto kern = k_prologue_regs<VPH, WPR>;
+    auto kern = k_prologue_regs<VPH, WPR, RES>;
     const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), 32 * WPR, 0);
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t grid = std::min<int64_t>(0x7fffffffLL, n_tokens);  // one CTA per row, as above
@@ -285,8 +301,13 @@ cudaError_t launch_prologue_regs(void* x_out, void* h, const void* x, const void
     switch (d / (256 * W)) {
 #define SOL_PRO_VPH(v)                                                                                           \
     case v:                                                                                                      \
-        if constexpr (v * W <= 24)                                                                               \
-            return launch_pro_vph<v, W>(x_out, h, x, y, gate, shift, scale, ld, ld_mod, sel, n_tokens, eps, s); \
+        if constexpr (v * W <= 24) {                                                                             \
+            if (y)                                                                                               \
+                return launch_pro_vph<v, W, true>(x_out, h, x, y, gate, shift, scale, ld, ld_mod, sel, n_tokens, \
+                                                  eps, s);                                                       \
+            return launch_pro_vph<v, W, false>(x_out, h, x, y, gate, shift, scale, ld, ld_mod, sel, n_tokens,    \
+                                               eps, s);                                                          \
+        }                                                                                                        \
         break;
         SOL_PRO_VPH(1) SOL_PRO_VPH(2) SOL_PRO_VPH(3) SOL_PRO_VPH(4) SOL_PRO_VPH(5) SOL_PRO_VPH(6)
         SOL_PRO_VPH(7) SOL_PRO_VPH(8) SOL_PRO_VPH(9) SOL_PRO_VPH(10) SOL_PRO_VPH(11) SOL_PRO_VPH(12)

@@ -20,6 +20,10 @@
 #include "common.cuh"
 #include "launch.h"
 
+#ifndef SOL_ADALN_FOUR_WARPS
+#define SOL_ADALN_FOUR_WARPS 1  // plain AdaLN on the four-warp prologue kernel (no residual); 0: one warp per row
+#endif
+
 namespace sol {
 
 template <typename T, int U, bool RESID>
@@ -575,6 +579,9 @@ cudaError_t launch_adaln_rows(sol_dtype dt, void* x_out, int64_t ld_xo, void* h,
                               int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
                               float eps, cudaStream_t s)
 {
+    if (!y && SOL_ADALN_FOUR_WARPS && ld_x == ld_h && prologue_regs_fits(dt, d))
+        return launch_prologue_regs(nullptr, h, x, nullptr, nullptr, shift, scale, ld_h, ld_mod, sel, n_tokens, d,
+                                    eps, s);
     if (!y && adaln_warp_fits(dt, d))
         return launch_adaln_warp(h, ld_h, x, ld_x, shift, scale, ld_mod, sel, n_tokens, d, eps, s);
     if (y && x_out && ld_xo == ld_h && ld_x == ld_h && ld_y == ld_h && prologue_regs_fits(dt, d))
