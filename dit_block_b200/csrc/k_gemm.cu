@@ -28,9 +28,10 @@
 //   warp 1        MMA issuer (one thread; the leader CTA only in a pair) into one of two
 //                 TMEM accumulators of 256 fp32 columns, so the epilogue of tile i
 //                 overlaps the main loop of tile i+1; owns the TMEM allocation;
-//   warps 2..9    epilogue (2..5 beside the transform): each thread owns one
-//                 accumulator row (TMEM lane) and half of its columns (all of them with
-//                 four warps), reads them 32 columns at a time and applies the operator;
+//   warps 2..9    epilogue (2..5 for the plain and gated-residual epilogues and beside
+//                 the transform): each thread owns one accumulator row (TMEM lane) and
+//                 half of its columns (all of them with four warps), reads them 32
+//                 columns at a time and applies the operator;
 //   warps 6..13   (operand-transform variant only) two groups on alternate stages.
 // Every copy lands in the shared memory of the one CTA that issued it, and the leader
 // commits to its own and to the peer's barriers one at a time.  Every wait on an mbarrier
