@@ -1,8 +1,8 @@
 // k_gemm.cu -- the block's linear layers y = a . W^T on the fifth-generation tensor
 // cores, with the per-token operators fused in, so that their inputs and outputs never
 // make an extra trip through HBM:
-//   AdaLN -> QKV projection -> QK RMSNorm + 3D RoPE   (weight fold + epilogue)
-//   AdaLN -> MLP up projection -> SwiGLU              (weight fold + epilogue)
+//   AdaLN -> QKV projection -> QK RMSNorm + 3D RoPE   (AdaLN strategy + epilogue)
+//   AdaLN -> MLP up projection -> SwiGLU              (AdaLN strategy + epilogue)
 //   MLP up projection -> SwiGLU                        (epilogue)
 //   output / MLP down projection -> gated residual     (epilogue)
 // [STM-RES] "SGLang acelera video do MiniMax-H3 em ate 6,2x em GPUs H200", section
@@ -19,10 +19,12 @@
 //           Per SM the copies per MMA drop by a third and the ring is half as deep
 //           again, which hides the copy latency.  The variant with the AdaLN operand
 //           transform runs single (see use_pair()).
-// AdaLN, two ways: the default folds (1 + scale) into a per-call copy of the weights and
-// corrects each accumulator row as rstd * (acc - mean * c_r) + b_r in the epilogue (a
-// plain GEMM on the raw tokens; see k_fold_weights); the alternative rewrites each landed
-// x tile in shared memory as h before the MMA reads it (the operand transform).
+// AdaLN, three ways (adaln_strategy()): the default stages h = AdaLN(x) through the
+// workspace with the per-token row kernel and runs the plain GEMM on it (one h round
+// trip, measured fastest); "fold" folds (1 + scale) into a per-call copy of the weights
+// and corrects each accumulator row as rstd * (acc - mean * c_r) + b_r in the epilogue (a
+// plain GEMM on the raw tokens; see k_fold_weights); "transform" rewrites each landed x
+// tile in shared memory as h before the MMA reads it (the operand transform).
 // Warp roles:
 //   warp 0        tensor-copy producer (one thread);
 //   warp 1        MMA issuer (one thread; the leader CTA only in a pair) into one of two
@@ -1098,12 +1100,20 @@ cudaError_t launch_shape(const CUtensorMap& ma, const CUtensorMap& mb, gemm::Par
     return launch_kernel<EPI, PRO, FOLD, false>(ma, mb, p, s);
 }
 
-// AdaLN strategy: fold (default) or the operand transform; SOL_ADALN_STRATEGY overrides
-// (read per call).
-bool adaln_fold()
+// AdaLN strategy (SOL_ADALN_STRATEGY overrides, read per call):
+//   stage (default): the AdaLN row kernel writes h (bf16) into the workspace and the plain
+//     GEMM with the fused epilogue reads it -- one h round trip through HBM, no change to
+//     the GEMM; at 32,768 tokens this is the fastest of the three (AdaLN -> QKV + RoPE
+//     4.17-4.23 ms vs 4.33-4.51 folded; AdaLN -> up + SwiGLU 7.21-7.23 vs 7.63-7.92);
+//   fold: the modulation folded into the weights, corrected in the epilogue (no h);
+//   transform: the x tile rewritten as h in shared memory before the MMA (no h).
+enum AdalnStrategy { ADALN_STAGE, ADALN_FOLD, ADALN_TRANSFORM };
+AdalnStrategy adaln_strategy()
 {
     const char* e = std::getenv("SOL_ADALN_STRATEGY");
-    return !(e && std::string(e) == "transform");
+    if (e && std::string(e) == "transform") return ADALN_TRANSFORM;
+    if (e && std::string(e) == "fold") return ADALN_FOLD;
+    return ADALN_STAGE;
 }
 
 }  // namespace
@@ -1144,7 +1154,20 @@ cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cuda
     p.qk_cols = a.qk_cols;
     p.eps = a.eps;
 
-    const bool fold = adaln && adaln_fold();
+    const AdalnStrategy strategy = adaln ? adaln_strategy() : ADALN_TRANSFORM;
+    if (adaln && strategy == ADALN_STAGE) {
+        // h = AdaLN(x) into the workspace (K elements per row), then the GEMM on h
+        const ModSel sel = a.sel ? *a.sel : ModSel{};
+        cudaError_t e = launch_adaln_rows(SOL_DTYPE_BF16, nullptr, 0, a.fold_v, a.K, a.a, a.ld_a, nullptr, 0, nullptr,
+                                          a.shift, a.scale, a.ld_mod, sel, a.M, a.K, a.eps, s);
+        if (e != cudaSuccess) return e;
+        if (!make_map(&ma, a.fold_v, (uint64_t)a.M, (uint64_t)a.K, (uint64_t)a.K)) {
+            record_error("tensor map encoding failed for the staged AdaLN output");
+            return cudaErrorInvalidValue;
+        }
+        adaln = false;
+    }
+    const bool fold = adaln && strategy == ADALN_FOLD;
     if (adaln) {
         const int64_t blocks = std::min<int64_t>((a.M + 7) / 8, (int64_t)sm_count() * 16);
         const ModSel sel = a.sel ? *a.sel : ModSel{};

@@ -641,8 +641,9 @@ static int64_t mod_rows(int64_t n_tokens, const sol_modsel& sel)
 }
 
 // Workspace of the sol_adaln_* calls: row statistics, per-128-row modulation-row sets,
-// folded-weight column sums and shift projections, then the folded weights; every region
-// 256-byte aligned.
+// folded-weight column sums and shift projections, then one region that holds either the
+// folded weights (fold strategy) or the staged AdaLN output h (stage strategy), whichever
+// is larger; every region 256-byte aligned.
 struct AdalnWorkspace {
     size_t stats, rmask, c, b, v, total;
 };
@@ -656,7 +657,8 @@ static AdalnWorkspace adaln_layout(int64_t n_tokens, int64_t n_out, int64_t d, i
     w.c = up(w.rmask + (size_t)((n_tokens + 127) / 128) * 4);
     w.b = up(w.c + (size_t)(R * n_out) * 4);
     w.v = up(w.b + (size_t)(R * n_out) * 4);
-    w.total = up(w.v + (size_t)(R * n_out) * (size_t)d * 2);
+    const size_t folded = (size_t)(R * n_out) * (size_t)d * 2, staged = (size_t)n_tokens * (size_t)d * 2;
+    w.total = up(w.v + (folded > staged ? folded : staged));
     return w;
 }
 

@@ -362,25 +362,32 @@ sol_status sol_linear_swiglu(void* out, int64_t ld_out, const void* a, int64_t l
                              int64_t ld_w, int64_t n_tokens, int64_t inner, int64_t k, sol_dtype dt,
                              sol_stream_t stream);
 
-/* Device workspace, in bytes, that sol_adaln_linear and sol_adaln_qkv_rope need for
- * n_tokens tokens, n_out output columns and d input columns, with the modulation rows
- * `sel` implies (R = ceil(n_tokens / tokens_per_sample) * n_streams, or n_streams when
- * tokens_per_sample is 0): per token 8 bytes of row statistics, per 128 tokens 4 bytes
- * of modulation-row sets, and per modulation row the folded weights (n_out * d bf16)
- * plus two fp32 vectors of n_out.  Returns 0 for invalid sizes or R > 32. */
+/* Device workspace, in bytes, that sol_adaln_linear, sol_adaln_linear_swiglu and
+ * sol_adaln_qkv_rope need for n_tokens tokens, n_out output columns and d input columns,
+ * with the modulation rows `sel` implies (R = ceil(n_tokens / tokens_per_sample) *
+ * n_streams, or n_streams when tokens_per_sample is 0): per token 8 bytes of row
+ * statistics, per 128 tokens 4 bytes of modulation-row sets, per modulation row two fp32
+ * vectors of n_out, and one region of the larger of the staged h (n_tokens * d bf16) and
+ * the folded weights (R * n_out * d bf16).  Returns 0 for invalid sizes or R > 32. */
 size_t sol_adaln_workspace_bytes(int64_t n_tokens, int64_t n_out, int64_t d, sol_modsel sel);
 
 /* AdaLN fused into a linear layer:
  *     out = h . W^T,   h = LN(x) * (1 + scale[r]) + shift[r]   (as sol_adaln_modulate)
  * x [n_tokens, d], W [n_out, d], out [n_tokens, n_out]; d a multiple of 64; at most 32
- * modulation rows (SOL_ERR_UNSUPPORTED otherwise).  h is never stored.  The modulation is
- * folded into the weights: per modulation row r the call writes V_r = bf16(W * (1 +
- * scale_r)) (column-wise), c_r = sum_k V_r[:, k] and b_r = shift_r . W^T into the
- * workspace, computes mean and 1/sqrt(var + eps) of every row of x, and runs one GEMM of
- * x against V_r whose epilogue forms rstd * (acc - mean * c_r) + b_r: the same value as
- * projecting h, computed from the unrounded LN output (the only rounding of an operand
- * is that of the folded weights, of the same size as rounding h to bf16).  A tile whose
- * rows use several modulation rows is computed once per row used.
+ * modulation rows (SOL_ERR_UNSUPPORTED otherwise).  Three strategies compute it; the
+ * environment variable SOL_ADALN_STRATEGY (read at each call) picks one:
+ *   "stage" (the default, the fastest on B200): h is written once, rounded to bf16, into
+ *     the workspace by the AdaLN row kernel and read back by the GEMM, whose epilogue
+ *     applies the fused operator (the per-token operator's output never goes to HBM);
+ *   "fold": h is never formed -- per modulation row r the call writes V_r = bf16(W * (1 +
+ *     scale_r)) (column-wise), c_r = sum_k V_r[:, k] and b_r = shift_r . W^T into the
+ *     workspace, computes mean and 1/sqrt(var + eps) of every row of x, and runs one
+ *     GEMM of x against V_r whose epilogue forms rstd * (acc - mean * c_r) + b_r (the
+ *     only rounding of an operand is that of the folded weights, of the same size as
+ *     rounding h); a tile whose rows use several modulation rows is computed once per
+ *     row used;
+ *   "transform": h is never stored -- each x tile is rewritten as bf16 h in shared
+ *     memory before the tensor cores read it.
  * workspace: caller-owned device memory of at least sol_adaln_workspace_bytes(...)
  * bytes, 256-byte aligned, overlapping no other argument; its contents are scratch. */
 sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld_x,
@@ -394,8 +401,9 @@ sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld
  *     out[:, j] = silu((h . W1^T)[:, j]) * (h . W2^T)[:, j],   W = [W1; W2],
  *     h = LN(x) * (1 + scale[r]) + shift[r]   (as sol_adaln_linear)
  * x [n_tokens, d], W [2*inner, d] (gated half first, as sol_linear_swiglu), out
- * [n_tokens, inner]; inner a multiple of 128; workspace as in sol_adaln_linear with
- * n_out = 2 * inner.  Neither h nor the projection is stored or rounded. */
+ * [n_tokens, inner]; inner a multiple of 128; workspace and strategies as in
+ * sol_adaln_linear with n_out = 2 * inner.  The projection is neither stored nor rounded
+ * before the SwiGLU. */
 sol_status sol_adaln_linear_swiglu(void* out, int64_t ld_out, const void* x, int64_t ld_x,
                                    const void* shift, const void* scale, int64_t ld_mod,
                                    sol_modsel sel, const void* w, int64_t ld_w, void* workspace,
@@ -410,8 +418,8 @@ sol_status sol_adaln_linear_swiglu(void* out, int64_t ld_out, const void* x, int
  * head_dim must be 128 and n_heads even.  Positions: pos [n_tokens, 3] int32, or NULL
  * for the row-major grid (grid_T, grid_H, grid_W) of each sample, samples of
  * sel.tokens_per_sample tokens (0 = one sample), as in sol_qk_rmsnorm_rope3d.
- * workspace as in sol_adaln_linear (with n_out = 3 * n_heads * head_dim).  The
- * projection is not rounded before the norm. */
+ * workspace and strategies as in sol_adaln_linear (with n_out = 3 * n_heads * head_dim).
+ * The projection is not rounded before the norm. */
 sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t ld_x,
                               const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
                               const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,

@@ -198,7 +198,7 @@ def adaln_inputs(w, m):
 
 
 @pytest.mark.parametrize("w", [SMALL, PACKED], ids=lambda w: w.name)
-def test_adaln_linear(oracle_mod, w):
+def test_adaln_linear(oracle_mod, monkeypatch, w):
     m = w.n_tokens
     x, shift, scale, sid, _, kw = adaln_inputs(w, m)
     W = wl.linear_weight(w, "w_qkv", 768, w.d, "cuda")
@@ -212,7 +212,11 @@ def test_adaln_linear(oracle_mod, w):
     bound = adaln_projection_bound(oracle_mod, to_oracle(x), to_oracle(W), to_oracle(shift), to_oracle(scale), h,
                                    rr, w.eps)
     check(out, y, bound, f"adaln_linear {w.name}")
-    # the workspace starts with each row's mean and 1/sqrt(var + eps)
+    # with the weights folded, the workspace starts with each row's mean and 1/sqrt(var + eps)
+    monkeypatch.setenv("SOL_ADALN_STRATEGY", "fold")
+    sol.adaln_linear(out, x, W, shift, scale, workspace=ws, eps=w.eps, stream_id=sid, **kw)
+    torch.cuda.synchronize()
+    check(out, y, bound, f"adaln_linear {w.name}, weights folded")
     xf = f64(x)
     mu = xf.mean(1)
     rs = 1 / np.sqrt(((xf - mu[:, None]) ** 2).mean(1) + w.eps)
@@ -348,11 +352,14 @@ def test_full_shape_adaln_qkv_rope(oracle_mod):
 
 @pytest.mark.parametrize("env", [{"SOL_LINEAR_SHAPE": "single"}, {"SOL_ADALN_STRATEGY": "transform"},
                                  {"SOL_LINEAR_SHAPE": "single", "SOL_ADALN_STRATEGY": "transform"},
-                                 {"SOL_LINEAR_SHAPE": "pair", "SOL_ADALN_STRATEGY": "transform"}],
+                                 {"SOL_LINEAR_SHAPE": "pair", "SOL_ADALN_STRATEGY": "transform"},
+                                 {"SOL_ADALN_STRATEGY": "fold"}, {"SOL_ADALN_STRATEGY": "stage"},
+                                 {"SOL_LINEAR_SHAPE": "single", "SOL_ADALN_STRATEGY": "stage"}],
                          ids=lambda e: ",".join(f"{k}={v}" for k, v in e.items()))
 def test_alternative_shapes_and_strategies(oracle_mod, monkeypatch, env):
-    """Single-CTA tiles and the AdaLN operand transform (selected per call by the library's
-    environment switches) compute the same results under the same bounds."""
+    """Single-CTA tiles and each AdaLN strategy -- weights folded, operand transformed, h
+    staged through the workspace (selected per call by the library's environment switches)
+    -- compute the same results under the same bounds."""
     for k, v in env.items():
         monkeypatch.setenv(k, v)
     w = PACKED
