@@ -408,7 +408,8 @@ def adaln_workspace(n_tokens: int, n_out: int, d: int, *, n_streams=1, tokens_pe
 
 def adaln_linear(out, x, w, shift=None, scale=None, *, workspace, eps=1e-6, stream_id=None, n_streams=1,
                  tokens_per_sample=0, stream=None):
-    """out = AdaLN(x) . W^T with the modulation folded into the weights  (sol_adaln_linear)."""
+    """out = AdaLN(x) . W^T  (sol_adaln_linear; the library stages h through the workspace,
+    or folds the modulation into the weights, or transforms the operand: SOL_ADALN_STRATEGY)."""
     _check(lib().sol_adaln_linear(
         _ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
         _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(workspace), workspace.numel(),
