@@ -20,6 +20,8 @@
 #include <cstdlib>
 #include <string>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -384,7 +386,7 @@ cudaError_t run_pool(void* q, void* k, int64_t ld_q, int64_t ld_k, void* pq, voi
     const void* kfn = (const void*)k_qk_rope_pool<T, LPH>;
     const size_t smem = qk_pool_smem_bytes(sizeof(T) == 2 ? SOL_DTYPE_BF16 : SOL_DTYPE_F32, n_heads,
                                            LPH * Vec<T>::N);
-    static bool attr_set[64];
+    static std::atomic<bool> attr_set[64];  // per device; a repeated set is harmless
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {

@@ -17,6 +17,8 @@
 // plus one shared-memory exchange.  The residual sum x' = x + gate*y stays unrounded in
 // registers for the norm; only its stored copy is rounded.  Modulation rows come
 // through the read-only path and stay L1/L2 resident across rows of the same sample.
+#include <atomic>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -531,7 +533,7 @@ cudaError_t run_bulk(void* x_out, int64_t ld_xo, void* h, int64_t ld_h, const vo
     }
     if (stages < 2) return cudaErrorInvalidConfiguration;
     const size_t smem = bulk_smem_bytes(vpr, (int)sizeof(T), RESID, MODF32, stages);
-    static bool attr_set[64];  // per instantiation and device
+    static std::atomic<bool> attr_set[64];  // per instantiation and device; a repeated set is harmless
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
