@@ -327,8 +327,8 @@ def run_ours(args, w):
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
     total_ms = start.elapsed_time(end)
-    per_op_ms = {op: sum(ev[s][j].elapsed_time(ev[s][j + 1]) for s in range(args.steps)) / args.steps
-                 for j, op in enumerate(OPS)}
+    op_times = {op: [ev[s][j].elapsed_time(ev[s][j + 1]) for s in range(args.steps)] for j, op in enumerate(OPS)}
+    per_op_ms = {op: sum(t) / len(t) for op, t in op_times.items()}
     total_ms, = max_over_ranks([total_ms], world, dev)
     ms_step = total_ms / args.steps
     value = step_bytes * world * args.steps / (total_ms * 1e-3) / 1e9
@@ -350,6 +350,7 @@ def run_ours(args, w):
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     traffic = ncu_traffic(n)
     per_op = {op: {"ms": round(per_op_ms[op], 4),
+                   "ms_median": round(statistics.median(op_times[op]), 4), "ms_min": round(min(op_times[op]), 4),
                    "GB_s": round(bpt[op] * n / (per_op_ms[op] * 1e-3) / 1e9, 1),
                    "frac_of_measured_peak": round(bpt[op] * n / (per_op_ms[op] * 1e-3) / 1e9 / peak, 4),
                    "bytes_per_token": bpt[op]} for op in OPS}
