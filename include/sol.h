@@ -37,6 +37,15 @@
  *   n_tokens == 0 is valid and launches nothing; tensor pointers may then be NULL.
  *   Aliasing.  Only the aliases each function lists are allowed (every row is read
  *              completely before it is written).  Any other overlap is undefined.
+ *   Kernel choice.  Each op picks its kernel from the shape (the register-resident and
+ *              streaming kernels where they fit, general ones otherwise); every choice
+ *              computes the same values within the stated tolerance.  Environment
+ *              variables, read at each call, force the alternatives (for testing and
+ *              timing): SOL_ADALN_KERNEL=bulk (AdaLN / prologue on the bulk-copy ring
+ *              kernel), SOL_QK_KERNEL=step (QK RMSNorm + RoPE, its variants and the
+ *              pooled epilogue on the general kernels), SOL_LINEAR_SHAPE=single|pair
+ *              (linear layers on one CTA per SM or on CTA pairs), SOL_ADALN_STRATEGY=
+ *              stage|fold|transform (see sol_adaln_linear).
  */
 #ifndef SOL_H
 #define SOL_H
