@@ -421,7 +421,9 @@ def sample_rows(m, n=48, seed=7):
     return np.unique(rows)
 
 
-def test_bench_size_adaln_qkv_rope_sampled(oracle_mod):
+@pytest.mark.parametrize("strategy", ["stage", "fold"])
+def test_bench_size_adaln_qkv_rope_sampled(oracle_mod, monkeypatch, strategy):
+    monkeypatch.setenv("SOL_ADALN_STRATEGY", strategy)
     w = FULL
     m = BENCH_M
     x = wl.activation(w, "x", m, w.d, "cuda")
@@ -495,3 +497,30 @@ def test_adaln_linear_swiglu(oracle_mod, w):
     ea, eb = E[:, :w.inner], E[:, w.inner:]
     bound = 1.1 * ea * (np.abs(up) + eb) + np.abs(ga / (1 + np.exp(-ga))) * eb
     check(out, want, bound, f"adaln_linear_swiglu {w.name}")
+
+
+@pytest.mark.parametrize("strategy", ["stage", "fold"])
+def test_bench_size_adaln_linear_swiglu_sampled(oracle_mod, monkeypatch, strategy):
+    """AdaLN -> up projection + SwiGLU at the size bench.py times, both AdaLN strategies,
+    checked on sampled rows (the first and last tiles included)."""
+    monkeypatch.setenv("SOL_ADALN_STRATEGY", strategy)
+    w = FULL
+    m = BENCH_M
+    x = wl.activation(w, "x", m, w.d, "cuda")
+    shift, scale = wl.modulation(w, "shift_mlp", "cuda"), wl.modulation(w, "scale_mlp", "cuda")
+    W = wl.linear_weight(w, "w_up", 2 * w.inner, w.d, "cuda")
+    out = torch.empty((m, w.inner), dtype=torch.bfloat16, device="cuda")
+    ws = sol.adaln_workspace(m, 2 * w.inner, w.d)
+    sol.adaln_linear_swiglu(out, x, W, shift, scale, workspace=ws, eps=w.eps)
+    torch.cuda.synchronize()
+    rows = sample_rows(m, seed=13)
+    ri = torch.from_numpy(rows).cuda()
+    xs, Wh = to_oracle(x[ri]), to_oracle(W)
+    want, u, h = oracle_mod.adaln_linear_swiglu(xs, Wh, to_oracle(shift), to_oracle(scale), w.inner, eps=w.eps,
+                                                rows=rows)
+    E = adaln_projection_bound(oracle_mod, xs, Wh, to_oracle(shift), to_oracle(scale), h,
+                               np.zeros(len(rows), np.int64), w.eps)
+    ga, up = u[:, :w.inner], u[:, w.inner:]
+    ea, eb = E[:, :w.inner], E[:, w.inner:]
+    bound = 1.1 * ea * (np.abs(up) + eb) + np.abs(ga / (1 + np.exp(-ga))) * eb
+    check(out[ri], want, bound, f"AdaLN -> up + SwiGLU at 32,768 tokens ({strategy})")
