@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(32 * WPR, RES ? SOL_PROLOGUE_REGS_MINB : SOL_A
 
         // x' = x + gate * y once, kept in fp32 (never rounded before the norm); x_out gets
         // its rounding at once -- a lane overwrites only what it has already read
-        bf16* xo = x_out + row * ld_xo + col;
+        bf16* xo = RES ? x_out + row * ld_xo + col : nullptr;  // no x_out without the residual
         float2 xp[VPH][4];
         float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
