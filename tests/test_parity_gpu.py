@@ -385,3 +385,23 @@ def test_adjacent_buffers_are_not_overlaps(orc):
     torch.cuda.synchronize()
     assert_close(to_f64(out), orc.swiglu(to_oracle(u), inner), BF, "adjacent swiglu")
     assert torch.equal(o2, x)
+
+
+@pytest.mark.parametrize("d", [1024, 5120])
+@pytest.mark.parametrize("ld_h_extra,ld_x_extra", [(0, 0), (64, 64), (0, 64), (128, 0)])
+def test_adaln_row_strides_select_kernels(orc, d, ld_h_extra, ld_x_extra):
+    """bf16 AdaLN at widths the four-warp row kernel takes: equal row strides of h and x
+    run it, different strides the one-warp kernel; both match the oracle and leave the
+    padding between rows untouched."""
+    n = 77
+    ld_h, ld_x = d + ld_h_extra, d + ld_x_extra
+    xb, x = _guarded(n, d, ld_x, BF)
+    x.copy_(randn((n, d), BF, 91, std=2.0, mean=0.5))
+    hb, h = _guarded(n, d, ld_h, BF)
+    shift, scale = (randn((2, d), BF, 92 + i, std=0.1) for i in range(2))
+    kw = dict(tokens_per_sample=40)  # rows 0..39 -> sample 0, 40..76 -> sample 1
+    sol.adaln_modulate(h, x, shift, scale, eps=1e-6, **kw)
+    torch.cuda.synchronize()
+    want = orc.adaln_modulate(to_oracle(x.contiguous()), to_oracle(shift), to_oracle(scale), **kw)
+    assert_close(to_f64(h.contiguous()), want, BF, f"adaln d={d} ld_h={ld_h} ld_x={ld_x}")
+    assert _guards_intact(hb, n, d, ld_h)
