@@ -92,5 +92,24 @@ class BlockBuffers:
         for op in OPS:
             self.launch(op, stream)
 
+    def capture(self, steps: int = 1) -> torch.cuda.CUDAGraph:
+        """Record `steps` passes into a CUDA graph; ``graph.replay()`` then issues them as
+        one launch instead of five kernel launches per pass, which matters at small token
+        counts.  One eager pass runs first, outside the capture, so that every kernel's
+        one-time attribute and occupancy setup is done (the op modifies q and k in place,
+        so that pass counts like any other).  The graph reads and writes these buffers: it
+        stays valid while they live, and their contents may change between replays."""
+        dev = self.inp["x"].device
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            self.step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(steps):
+                self.step()
+        return g
+
     def close(self):
         self.rope.close()

@@ -66,3 +66,24 @@ def test_chunks_never_cross_samples():
     assert sum(L for _, L, _ in ch) == w.n_tokens
     for c0, L, b in ch:
         assert c0 // w.tokens_per_sample == b == (c0 + L - 1) // w.tokens_per_sample
+
+
+@pytest.mark.parametrize("w", CASES[:2], ids=lambda w: w.name)
+def test_graph_replay_equals_eager_passes(w):
+    """BlockBuffers.capture: a captured pass replayed is bit-identical to the same passes
+    issued eagerly (capture runs one eager pass first, so both sides run two)."""
+    n = min(w.n_tokens, 3000)
+    eager = block.BlockBuffers.allocate(w, "cuda", n_tokens=n)
+    graph = block.BlockBuffers.allocate(w, "cuda", inputs={k: v.clone() if torch.is_tensor(v) else v
+                                                           for k, v in eager.inp.items()})
+    eager.step()
+    eager.step()
+    g = graph.capture(steps=1)
+    g.replay()
+    torch.cuda.synchronize()
+    for name in ("h1", "x1", "h2", "act", "x2"):
+        assert torch.equal(getattr(eager, name), getattr(graph, name)), name
+    assert torch.equal(eager.inp["qkv"], graph.inp["qkv"])
+    del g
+    eager.close()
+    graph.close()
