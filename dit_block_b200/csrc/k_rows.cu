@@ -1,6 +1,9 @@
-// k_rows.cu -- AdaLN modulation and the fused block prologue (gated residual -> AdaLN).
+// k_rows.cu -- AdaLN modulation and the fused block prologue (gated residual -> AdaLN):
+// the entry point launch_adaln_rows and the general kernels.  bf16 rows of the common
+// widths go to the register-resident kernels of k_adaln_warp.cu (see the dispatch at the
+// end of this file); fp32 and every other width take the kernels below.
 //
-// Main kernel, k_adaln_bulk: a persistent CTA streams its rows (x, and y for the
+// Bulk-copy ring kernel, k_adaln_bulk: a persistent CTA streams its rows (x, and y for the
 // prologue) into a ring of `stages` shared-memory buffers with single-CTA 1-D bulk
 // async copies completed on one mbarrier per buffer.  While a row is reduced, the next
 // stages-1 rows of the CTA are already in flight, so HBM never waits on the reductions.
