@@ -184,6 +184,17 @@ def dist_env():
     return rank, world, local
 
 
+def all_ranks_agree(ok: bool, world: int, device) -> bool:
+    """True only if every rank passes `ok`: a decision that changes which collectives a
+    rank takes next must be the same on every rank."""
+    if world == 1:
+        return bool(ok)
+    import torch.distributed as dist
+    t = torch.tensor([1 if ok else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return bool(t.item())
+
+
 def max_over_ranks(vals: list[float], world: int, device) -> list[float]:
     if world == 1:
         return vals
@@ -624,11 +635,14 @@ def run_e2e(args, bufs, dev, world, step_bytes):
         avail = psutil.virtual_memory().available
     except Exception:
         avail = 0
-    if h2d + d2h > 0.4 * avail:
+    # every rank of the node pins its own buffers; all ranks take the same decision, since
+    # skipping also skips the barrier and the reduction below
+    need = (h2d + d2h) * world
+    if not all_ranks_agree(need <= 0.4 * avail, world, dev):
         pipe.close()
         return {"value": None, "unit": "GB/s",
-                "error": f"skipped: {(h2d + d2h) / 1e9:.1f} GB of pinned host buffers > 40% of the "
-                         f"{avail / 1e9:.1f} GB available host memory"}
+                "error": f"skipped: {need / 1e9:.1f} GB of pinned host buffers over {world} rank(s) > 40% "
+                         f"of the {avail / 1e9:.1f} GB available host memory (on some rank)"}
     host_in, host_out, host_mod = pipeline.host_buffers(w, n)
     for k in pipeline.IN_NAMES:
         host_in[k].copy_(i[k])

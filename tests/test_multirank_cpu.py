@@ -1,5 +1,6 @@
 """Multi-rank host logic on CPU (gloo, world size 2): the max-over-ranks reduction of the
-timing, and bench.py's reference arm under torchrun (rank 0 alone runs and prints).
+timing, the all-ranks agreement on a go / no-go, and bench.py's reference arm under
+torchrun (rank 0 alone runs and prints).
 The data path itself has no collective: every rank runs its own replica."""
 from __future__ import annotations
 
@@ -34,7 +35,10 @@ def _worker(rank, world, port, q):
                             timeout=datetime.timedelta(seconds=60))
     # each rank "measured" a different time; every rank must get the max
     got = bench.max_over_ranks([10.0 + 5 * rank, 1.0 - rank], world, torch.device("cpu"))
-    q.put((rank, got, bench.dist_env()))
+    # a go / no-go that differs between ranks must come out the same everywhere
+    agree = (bench.all_ranks_agree(rank == 0, world, torch.device("cpu")),
+             bench.all_ranks_agree(True, world, torch.device("cpu")))
+    q.put((rank, got, bench.dist_env(), agree))
     dist.destroy_process_group()
 
 
@@ -49,15 +53,17 @@ def test_max_over_ranks_gloo():
     for p in ps:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, got, env in res:
+    for rank, got, env, agree in res:
         assert got == [15.0, 1.0]
         assert env == (rank, 2, 0)
+        assert agree == (False, True)
 
 
 def test_single_rank_max_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks([3.0, 4.0], 1, torch.device("cpu")) == [3.0, 4.0]
+    assert bench.all_ranks_agree(True, 1, torch.device("cpu")) and not bench.all_ranks_agree(False, 1, None)
 
 
 @pytest.mark.timeout(600)
