@@ -126,7 +126,8 @@ struct LinearLaunch {
     float eps;
     // AdaLN folded into the weights (workspace regions)
     uint32_t* rmask;    // [ceil(M / 128)] modulation rows per 128-row block
-    void* fold_v;       // [n_mod_rows * N, K] bf16 folded weights
+    void* fold_v;       // workspace region: [n_mod_rows * N, K] bf16 folded weights (fold strategy)
+                        // or [M, K] bf16 staged h = AdaLN(x) (stage strategy)
     float* fold_c;      // [n_mod_rows, N]
     float* fold_b;      // [n_mod_rows, N]
     int32_t n_mod_rows; // modulation rows the call may use (<= 32)
