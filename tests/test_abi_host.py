@@ -174,6 +174,10 @@ def test_linear_epilogue_variants_validation(L):
     # AdaLN variants need a workspace of sol_adaln_workspace_bytes
     need = L.sol_adaln_workspace_bytes(n, d, k, SEL)
     assert need >= n * 8 + d * k * 2
+    # the shared region holds the larger of the folded weights and the staged h
+    tall = 100_000  # more tokens than output columns: h (n * k) outgrows the folded weights (d * k)
+    assert L.sol_adaln_workspace_bytes(tall, d, k, SEL) >= tall * 8 + tall * k * 2
+    assert L.sol_adaln_workspace_bytes(tall, d, k, SEL) < tall * 8 + tall * k * 2 + d * k * 2
     ws = FAKE << 6
     assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, None, need, n, d, k, 1e-6, sol.BF16,
                               None) == sol.ERR_INVALID_ARGUMENT
