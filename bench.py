@@ -535,7 +535,7 @@ def time_linear_ops(w, dev, m: int) -> dict:
     sus, sus_src = measured_bf16_sustained()
     out = {"tokens": m, "peak_tflops": peak, "peak_source": src + " (burst cuBLAS bf16)",
            "sustained_peak_tflops": sus, "sustained_peak_source": sus_src + " (cuBLAS bf16 under the power cap)",
-           "adaln_strategy": os.environ.get("SOL_ADALN_STRATEGY", "stage")}
+           "adaln_strategy": "stage"}
 
     def entry(name, flops, fused, unfused, cublas, plain, saved_bytes):
         # the four arms alternate launch by launch, so clock drift under the power cap

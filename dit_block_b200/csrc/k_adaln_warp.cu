@@ -27,8 +27,6 @@
 // 6.43 TB/s and the prologue 6.33 -> 6.73 TB/s on B200 (the launch shapes below were
 // swept under the persistent grid).
 #include <algorithm>
-#include <cstdlib>
-#include <string>
 
 #include <cuda_bf16.h>
 
@@ -280,17 +278,13 @@ cudaError_t launch_pro_vph(void* x_out, void* h, const void* x, const void* y, c
 
 bool adaln_warp_fits(sol_dtype dt, int64_t d)
 {
-    if (!(dt == SOL_DTYPE_BF16 && d % 256 == 0 && d / 256 >= 1 && d / 256 <= 24)) return false;
-    const char* e = std::getenv("SOL_ADALN_KERNEL");  // "bulk" selects the ring kernel (read per call)
-    return !(e && std::string(e) == "bulk");
+    return dt == SOL_DTYPE_BF16 && d % 256 == 0 && d / 256 >= 1 && d / 256 <= 24;
 }
 
 bool prologue_regs_fits(sol_dtype dt, int64_t d)
 {
     constexpr int W = SOL_PROLOGUE_REGS_WPR;
-    if (!(dt == SOL_DTYPE_BF16 && d % (256 * W) == 0 && d / (256 * W) >= 1 && d / (256 * W) <= 24 / W)) return false;
-    const char* e = std::getenv("SOL_ADALN_KERNEL");  // "bulk" selects the ring kernel (read per call)
-    return !(e && std::string(e) == "bulk");
+    return dt == SOL_DTYPE_BF16 && d % (256 * W) == 0 && d / (256 * W) >= 1 && d / (256 * W) <= 24 / W;
 }
 
 cudaError_t launch_prologue_regs(void* x_out, void* h, const void* x, const void* y, const void* gate,

@@ -19,7 +19,7 @@
 //           Per SM the copies per MMA drop by a third and the ring is half as deep
 //           again, which hides the copy latency.  The variant with the AdaLN operand
 //           transform runs single (see use_pair()).
-// AdaLN, three ways (adaln_strategy()): the default stages h = AdaLN(x) through the
+// AdaLN, three ways (the caller's sol_adaln_strategy): "stage" stages h = AdaLN(x) through the
 // workspace with the per-token row kernel and runs the plain GEMM on it (one h round
 // trip, measured fastest); "fold" folds (1 + scale) into a per-call copy of the weights
 // and corrects each accumulator row as rstd * (acc - mean * c_r) + b_r in the epilogue (a
@@ -40,9 +40,7 @@
 // is bounded; a wait that gives up raises an error flag and the CTA drains its in-flight
 // copies and MMAs, frees its TMEM and returns.
 #include <algorithm>
-#include <cstdlib>
 #include <mutex>
-#include <string>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -1021,18 +1019,13 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tile shape per variant.  Measured on B200: CTA pairs are faster for the plain and
-// epilogue-fused GEMMs (the copies per MMA drop by a third); with the AdaLN operand
-// transform the single shape is faster (in a pair every transformed stage of the peer
-// must be announced to the leader with a cluster-scope release, which costs more than the
-// deeper ring saves).  SOL_LINEAR_SHAPE=single / pair overrides the choice.
-bool use_pair(bool transform)
-{
-    const char* e = std::getenv("SOL_LINEAR_SHAPE");  // read per call (cheap beside a GEMM)
-    if (e && std::string(e) == "single") return false;
-    if (e && std::string(e) == "pair") return true;
-    return !transform;
-}
+// Tile shape per variant, from the shape alone.  Measured on B200: CTA pairs are faster
+// for the plain and epilogue-fused GEMMs (the copies per MMA drop by a third); with the
+// AdaLN operand transform the single shape is faster (in a pair every transformed stage of
+// the peer must be announced to the leader with a cluster-scope release, which costs more
+// than the deeper ring saves).  A call of at most 128 rows also runs single: a pair's
+// 256-row tile would leave the second CTA's half empty.
+bool use_pair(bool transform, int64_t M) { return !transform && M > gemm::Shape<false>::TILE_M; }
 
 template <int EPI, bool PRO, bool FOLD, bool PAIR>
 cudaError_t launch_kernel(const CUtensorMap& ma, const CUtensorMap& mb, const gemm::Params& p, cudaStream_t s)
@@ -1091,7 +1084,7 @@ template <int EPI, bool PRO, bool FOLD = false>
 cudaError_t launch_shape(const CUtensorMap& ma, const CUtensorMap& mb, gemm::Params& p, int64_t M, cudaStream_t s)
 {
     if constexpr (!PRO || gemm::kPairTransform) {
-        if (use_pair(PRO)) {
+        if (use_pair(PRO, M)) {
             p.num_tiles = (M + gemm::Shape<true>::TILE_M - 1) / gemm::Shape<true>::TILE_M * (int64_t)p.n_tiles_n;
             return launch_kernel<EPI, PRO, FOLD, true>(ma, mb, p, s);
         }
@@ -1100,21 +1093,13 @@ cudaError_t launch_shape(const CUtensorMap& ma, const CUtensorMap& mb, gemm::Par
     return launch_kernel<EPI, PRO, FOLD, false>(ma, mb, p, s);
 }
 
-// AdaLN strategy (SOL_ADALN_STRATEGY overrides, read per call):
-//   stage (default): the AdaLN row kernel writes h (bf16) into the workspace and the plain
-//     GEMM with the fused epilogue reads it -- one h round trip through HBM, no change to
-//     the GEMM; at 32,768 tokens this is the fastest of the three (AdaLN -> QKV + RoPE
-//     4.17-4.23 ms vs 4.33-4.51 folded; AdaLN -> up + SwiGLU 7.21-7.23 vs 7.63-7.92);
+// AdaLN strategy, chosen by the caller (sol_adaln_strategy):
+//   stage (the fastest on B200): the AdaLN row kernel writes h (bf16) into the workspace
+//     and the plain GEMM with the fused epilogue reads it -- one h round trip through
+//     HBM, no change to the GEMM (AdaLN -> QKV + RoPE 4.17-4.23 ms vs 4.33-4.51 folded;
+//     AdaLN -> up + SwiGLU 7.21-7.23 vs 7.63-7.92, at 32,768 tokens);
 //   fold: the modulation folded into the weights, corrected in the epilogue (no h);
 //   transform: the x tile rewritten as h in shared memory before the MMA (no h).
-enum AdalnStrategy { ADALN_STAGE, ADALN_FOLD, ADALN_TRANSFORM };
-AdalnStrategy adaln_strategy()
-{
-    const char* e = std::getenv("SOL_ADALN_STRATEGY");
-    if (e && std::string(e) == "transform") return ADALN_TRANSFORM;
-    if (e && std::string(e) == "fold") return ADALN_FOLD;
-    return ADALN_STAGE;
-}
 
 }  // namespace
 
@@ -1154,8 +1139,8 @@ cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cuda
     p.qk_cols = a.qk_cols;
     p.eps = a.eps;
 
-    const AdalnStrategy strategy = adaln ? adaln_strategy() : ADALN_TRANSFORM;
-    if (adaln && strategy == ADALN_STAGE) {
+    const int32_t strategy = adaln ? a.adaln_strategy : SOL_ADALN_TRANSFORM;
+    if (adaln && strategy == SOL_ADALN_STAGE) {
         // h = AdaLN(x) into the workspace (K elements per row), then the GEMM on h
         const ModSel sel = a.sel ? *a.sel : ModSel{};
         cudaError_t e = launch_adaln_rows(SOL_DTYPE_BF16, nullptr, 0, a.fold_v, a.K, a.a, a.ld_a, nullptr, 0, nullptr,
@@ -1167,7 +1152,7 @@ cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cuda
         }
         adaln = false;
     }
-    const bool fold = adaln && strategy == ADALN_FOLD;
+    const bool fold = adaln && strategy == SOL_ADALN_FOLD;
     if (adaln) {
         const int64_t blocks = std::min<int64_t>((a.M + 7) / 8, (int64_t)sm_count() * 16);
         const ModSel sel = a.sel ? *a.sel : ModSel{};

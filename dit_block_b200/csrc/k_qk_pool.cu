@@ -17,8 +17,6 @@
 // different banks).  After the block, one barrier; the CTA scales the sums by 1/count,
 // stores the pooled q and k rows and clears the accumulator.  Means are taken over the
 // fp32 results before their rounding to the output type.
-#include <cstdlib>
-#include <string>
 
 #include <atomic>
 
@@ -425,11 +423,8 @@ cudaError_t run_pool_regs(void* q, void* k, int64_t ld_q, int64_t ld_k, void* pq
 bool pool_regs_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim)
 {
     constexpr int heads_step = 2 * SOL_POOL_PARTS;
-    if (!(dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads % heads_step == 0 && n_heads >= heads_step &&
-          n_heads <= 48))
-        return false;
-    const char* e = std::getenv("SOL_QK_KERNEL");  // "step" selects k_qk_rope_pool (read per call)
-    return !(e && std::string(e) == "step");
+    return dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads % heads_step == 0 && n_heads >= heads_step &&
+           n_heads <= 48;
 }
 
 }  // namespace

@@ -16,8 +16,6 @@
 // the convention variants of k_qk_ex.cu (norm across all heads, rotate-half pairs, strided
 // outputs) for bf16 with a multiple of 8 heads.
 #include <algorithm>
-#include <cstdlib>
-#include <string>
 
 #include <cuda_bf16.h>
 
@@ -245,19 +243,11 @@ cudaError_t launch_vpl(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, c
     return cudaGetLastError();
 }
 
-bool step_kernel_requested()
-{
-    const char* e = std::getenv("SOL_QK_KERNEL");  // "step" selects k_qk.cu / k_qk_ex.cu (read per call)
-    return e && std::string(e) == "step";
-}
-
 }  // namespace
 
 bool qk_regs_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim)
 {
-    if (!(dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads % 2 == 0 && n_heads >= 2 && n_heads <= 48))
-        return false;
-    return !step_kernel_requested();
+    return dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads % 2 == 0 && n_heads >= 2 && n_heads <= 48;
 }
 
 cudaError_t launch_qk_regs(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, const void* q, const void* k,
@@ -290,7 +280,7 @@ bool qk_regs_ex_fits(sol_dtype dt, bool half, int32_t n_heads, int32_t head_dim,
     if (half)
         for (int c = 0; c < 3; ++c)
             if (rope.half[c] % 8 != 0 || reinterpret_cast<uintptr_t>(rope.tab[c]) % 16 != 0) return false;
-    return !step_kernel_requested();
+    return true;
 }
 
 cudaError_t launch_qk_regs_ex(bool across, bool half, void* q_out, void* k_out, const QkOutStrides& os, const void* q,

@@ -131,6 +131,7 @@ struct LinearLaunch {
     float* fold_c;      // [n_mod_rows, N]
     float* fold_b;      // [n_mod_rows, N]
     int32_t n_mod_rows; // modulation rows the call may use (<= 32)
+    int32_t adaln_strategy;  // sol_adaln_strategy of the sol_adaln_* calls
 };
 cudaError_t launch_linear(LinearEpi epi, bool adaln, const LinearLaunch& a, cudaStream_t s);
 size_t linear_smem_bytes();

@@ -195,7 +195,7 @@ const char* sol_status_string(sol_status status)
 
 const char* sol_last_error(void) { return g_last_error.c_str(); }
 
-int32_t sol_abi_version(void) { return 1; }
+int32_t sol_abi_version(void) { return 2; }
 
 sol_status sol_device_errors(uint32_t* flags, int32_t clear)
 {
@@ -675,6 +675,13 @@ static sol_status check_workspace(const void* ws, size_t bytes, int64_t n_tokens
     return SOL_OK;
 }
 
+static sol_status check_strategy(int32_t strategy)
+{
+    CHECK(strategy == SOL_ADALN_STAGE || strategy == SOL_ADALN_FOLD || strategy == SOL_ADALN_TRANSFORM,
+          SOL_ERR_INVALID_ARGUMENT, "strategy %d is not a sol_adaln_strategy", (int)strategy);
+    return SOL_OK;
+}
+
 static void set_workspace(sol::LinearLaunch& L, void* ws, const AdalnWorkspace& lay, int64_t R)
 {
     char* base = static_cast<char*>(ws);
@@ -779,9 +786,10 @@ size_t sol_adaln_workspace_bytes(int64_t n_tokens, int64_t n_out, int64_t d, sol
 sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld_x,
                             const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
                             const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,
-                            int64_t n_tokens, int64_t n_out, int64_t d, float eps, sol_dtype dt,
-                            sol_stream_t stream)
+                            int32_t strategy, int64_t n_tokens, int64_t n_out, int64_t d, float eps,
+                            sol_dtype dt, sol_stream_t stream)
 {
+    TRY(check_strategy(strategy));
     TRY(check_linear_shape(n_tokens, n_out, d, dt, 256));
     TRY(check_modsel(sel));
     CHECK(std::isfinite(eps) && eps >= 0.f, SOL_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
@@ -808,6 +816,7 @@ sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld
     L.ld_mod = ld_mod;
     L.sel = &ms;
     L.eps = eps;
+    L.adaln_strategy = strategy;
     return cuda_status(sol::launch_linear(sol::LINEAR_STORE, true, L, (cudaStream_t)stream),
                        "sol_adaln_linear launch");
 }
@@ -815,9 +824,10 @@ sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld
 sol_status sol_adaln_linear_swiglu(void* out, int64_t ld_out, const void* x, int64_t ld_x,
                                    const void* shift, const void* scale, int64_t ld_mod,
                                    sol_modsel sel, const void* w, int64_t ld_w, void* workspace,
-                                   size_t workspace_bytes, int64_t n_tokens, int64_t inner,
-                                   int64_t d, float eps, sol_dtype dt, sol_stream_t stream)
+                                   size_t workspace_bytes, int32_t strategy, int64_t n_tokens,
+                                   int64_t inner, int64_t d, float eps, sol_dtype dt, sol_stream_t stream)
 {
+    TRY(check_strategy(strategy));
     const int64_t n_out = 2 * inner;
     TRY(check_linear_shape(n_tokens, n_out, d, dt, 256));
     TRY(check_modsel(sel));
@@ -845,6 +855,7 @@ sol_status sol_adaln_linear_swiglu(void* out, int64_t ld_out, const void* x, int
     L.ld_mod = ld_mod;
     L.sel = &ms;
     L.eps = eps;
+    L.adaln_strategy = strategy;
     return cuda_status(sol::launch_linear(sol::LINEAR_SWIGLU, true, L, (cudaStream_t)stream),
                        "sol_adaln_linear_swiglu launch");
 }
@@ -852,11 +863,12 @@ sol_status sol_adaln_linear_swiglu(void* out, int64_t ld_out, const void* x, int
 sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t ld_x,
                               const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
                               const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,
-                              const void* wq, const void* wk, const int32_t* pos, int32_t grid_T, int32_t grid_H,
-                              int32_t grid_W, const sol_rope3d* rope, int64_t n_tokens,
-                              int32_t n_heads, int32_t head_dim, int64_t d, float eps, sol_dtype dt,
-                              sol_stream_t stream)
+                              int32_t strategy, const void* wq, const void* wk, const int32_t* pos,
+                              int32_t grid_T, int32_t grid_H, int32_t grid_W, const sol_rope3d* rope,
+                              int64_t n_tokens, int32_t n_heads, int32_t head_dim, int64_t d, float eps,
+                              sol_dtype dt, sol_stream_t stream)
 {
+    TRY(check_strategy(strategy));
     CHECK(dt == SOL_DTYPE_BF16, SOL_ERR_UNSUPPORTED, "the linear-layer calls take bf16 only");
     CHECK(head_dim == 128, SOL_ERR_UNSUPPORTED, "sol_adaln_qkv_rope is built for head_dim 128 (got %d)",
           (int)head_dim);
@@ -890,6 +902,7 @@ sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t 
     L.ld_mod = ld_mod;
     L.sel = &ms;
     L.eps = eps;
+    L.adaln_strategy = strategy;
     L.wq = wq;
     L.wk = wk;
     L.pos = pos;

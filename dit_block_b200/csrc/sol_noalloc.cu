@@ -19,7 +19,9 @@
 //
 // Set-up: the device address of the array is looked up once per device with
 // cudaGetSymbolAddress, with that device current, on the first call made on it; that
-// first call should therefore come before any stream capture.
+// first call should therefore come before any stream capture.  The address is kept for
+// the life of the process, so it goes stale if the device's primary context is destroyed
+// (cudaDeviceReset): the entry point is not for use after a reset.
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>

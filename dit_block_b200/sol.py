@@ -48,6 +48,8 @@ class QkDesc(ctypes.Structure):
 
 
 NORM_PER_HEAD, NORM_ACROSS_HEADS = 0, 1
+ADALN_STAGE, ADALN_FOLD, ADALN_TRANSFORM = 0, 1, 2
+_STRATEGIES = {"stage": ADALN_STAGE, "fold": ADALN_FOLD, "transform": ADALN_TRANSFORM}
 ROPE_INTERLEAVED, ROPE_HALF = 0, 1
 _E = ctypes.c_int  # enums
 
@@ -81,12 +83,12 @@ SIGNATURES = {
                                    _I64, _E, _P], _E),
     "sol_linear_swiglu": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _E, _P], _E),
     "sol_adaln_workspace_bytes": ([_I64, _I64, _I64, ModSel], ctypes.c_size_t),
-    "sol_adaln_linear": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _I64, _I64,
-                          _I64, _F, _E, _P], _E),
-    "sol_adaln_linear_swiglu": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _I64,
-                                 _I64, _I64, _F, _E, _P], _E),
-    "sol_adaln_qkv_rope": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _P, _P, _P,
-                            _I32, _I32, _I32, _P, _I64, _I32, _I32, _I64, _F, _E, _P], _E),
+    "sol_adaln_linear": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _I32, _I64,
+                          _I64, _I64, _F, _E, _P], _E),
+    "sol_adaln_linear_swiglu": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _I32,
+                                 _I64, _I64, _I64, _F, _E, _P], _E),
+    "sol_adaln_qkv_rope": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _P, _I64, _P, ctypes.c_size_t, _I32, _P,
+                            _P, _P, _I32, _I32, _I32, _P, _I64, _I32, _I32, _I64, _F, _E, _P], _E),
 }
 
 _lib = None
@@ -406,35 +408,42 @@ def adaln_workspace(n_tokens: int, n_out: int, d: int, *, n_streams=1, tokens_pe
     return torch.empty((nb,), dtype=torch.uint8, device=device or "cuda")
 
 
-def adaln_linear(out, x, w, shift=None, scale=None, *, workspace, eps=1e-6, stream_id=None, n_streams=1,
-                 tokens_per_sample=0, stream=None):
-    """out = AdaLN(x) . W^T  (sol_adaln_linear; the library stages h through the workspace,
-    or folds the modulation into the weights, or transforms the operand: SOL_ADALN_STRATEGY)."""
+def _strategy(strategy) -> int:
+    """A sol_adaln_strategy from its name ("stage", "fold", "transform") or its value."""
+    return _STRATEGIES[strategy] if isinstance(strategy, str) else int(strategy)
+
+
+def adaln_linear(out, x, w, shift=None, scale=None, *, workspace, strategy="stage", eps=1e-6, stream_id=None,
+                 n_streams=1, tokens_per_sample=0, stream=None):
+    """out = AdaLN(x) . W^T  (sol_adaln_linear; `strategy` stages h through the workspace,
+    folds the modulation into the weights or transforms the operand: sol_adaln_strategy)."""
     _check(lib().sol_adaln_linear(
         _ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
         _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(workspace), workspace.numel(),
-        x.shape[0], w.shape[0], x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_linear")
+        _strategy(strategy), x.shape[0], w.shape[0], x.shape[1], eps, _dtype(x), _stream(stream)),
+        "sol_adaln_linear")
     return out
 
 
-def adaln_linear_swiglu(out, x, w, shift=None, scale=None, *, workspace, eps=1e-6, stream_id=None,
-                        n_streams=1, tokens_per_sample=0, stream=None):
+def adaln_linear_swiglu(out, x, w, shift=None, scale=None, *, workspace, strategy="stage", eps=1e-6,
+                        stream_id=None, n_streams=1, tokens_per_sample=0, stream=None):
     """out = silu(h . W1^T) * (h . W2^T), h = AdaLN(x), W = [W1; W2]  (sol_adaln_linear_swiglu)."""
     _check(lib().sol_adaln_linear_swiglu(
         _ptr(out), _ld(out), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
         _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(workspace), workspace.numel(),
-        x.shape[0], w.shape[0] // 2, x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_linear_swiglu")
+        _strategy(strategy), x.shape[0], w.shape[0] // 2, x.shape[1], eps, _dtype(x), _stream(stream)),
+        "sol_adaln_linear_swiglu")
     return out
 
 
 def adaln_qkv_rope(qkv, x, w, rope: Rope3D, shift=None, scale=None, *, workspace, n_heads, head_dim=128,
-                   wq=None, wk=None, pos=None, grid=(0, 0, 0), eps=1e-6, stream_id=None, n_streams=1,
-                   tokens_per_sample=0, stream=None):
+                   wq=None, wk=None, pos=None, grid=(0, 0, 0), strategy="stage", eps=1e-6, stream_id=None,
+                   n_streams=1, tokens_per_sample=0, stream=None):
     """qkv = AdaLN(x) . W^T, then QK RMSNorm + 3D RoPE on q and k  (sol_adaln_qkv_rope)."""
     _check(lib().sol_adaln_qkv_rope(
         _ptr(qkv), _ld(qkv), _ptr(x), _ld(x), _ptr(shift), _ptr(scale), _mod_ld(shift, scale),
         _sel(stream_id, n_streams, tokens_per_sample), _ptr(w), _ld(w), _ptr(workspace), workspace.numel(),
-        _ptr(wq), _ptr(wk),
+        _strategy(strategy), _ptr(wq), _ptr(wk),
         _ptr(pos), int(grid[0]), int(grid[1]), int(grid[2]), rope.handle, x.shape[0], n_heads, head_dim,
         x.shape[1], eps, _dtype(x), _stream(stream)), "sol_adaln_qkv_rope")
     return qkv

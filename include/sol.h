@@ -37,15 +37,10 @@
  *   n_tokens == 0 is valid and launches nothing; tensor pointers may then be NULL.
  *   Aliasing.  Only the aliases each function lists are allowed (every row is read
  *              completely before it is written).  Any other overlap is undefined.
- *   Kernel choice.  Each op picks its kernel from the shape (the register-resident and
- *              streaming kernels where they fit, general ones otherwise); every choice
- *              computes the same values within the stated tolerance.  Environment
- *              variables, read at each call, force the alternatives (for testing and
- *              timing): SOL_ADALN_KERNEL=bulk (AdaLN / prologue on the bulk-copy ring
- *              kernel), SOL_QK_KERNEL=step (QK RMSNorm + RoPE, its variants and the
- *              pooled epilogue on the general kernels), SOL_LINEAR_SHAPE=single|pair
- *              (linear layers on one CTA per SM or on CTA pairs), SOL_ADALN_STRATEGY=
- *              stage|fold|transform (see sol_adaln_linear).
+ *   Kernel choice.  Each op picks its kernel from the shape and dtype of the call alone (the
+ *              register-resident and streaming kernels where they fit, general ones
+ *              otherwise); every choice computes the same values within the stated
+ *              tolerance.  Nothing is read from the process environment.
  */
 #ifndef SOL_H
 #define SOL_H
@@ -268,24 +263,6 @@ sol_status sol_dit_epilogue(void* qkv, int64_t ld_qkv, const void* wq, const voi
                             int32_t n_heads, int32_t head_dim, float eps, sol_dtype dt,
                             sol_stream_t stream);
 
-/* QK RMSNorm + 3D RoPE for callers that cannot allocate device memory.  The pages have
- * no counterpart: this entry point exists for hosts that reserve device memory up front
- * and forbid allocation while they run work (inference engines whose pool already holds
- * nearly all of HBM, plugin execute callbacks, latency-critical loops that cannot afford
- * cudaMalloc's device synchronisation).  sol_qk_rmsnorm_rope3d needs a sol_rope3d handle,
- * and creating one calls cudaMalloc; this function allocates nothing.
- *
- * It computes exactly what sol_qk_rmsnorm_rope3d computes, with the table described by
- * (dim_t, dim_h, dim_w, theta, max_t, max_h, max_w) as in sol_rope3d_create.  The table
- * is rebuilt on `stream` by every call inside a fixed device array of
- * SOL_NOALLOC_MAX_ROPE_ENTRIES (cos, sin) pairs (512 KiB, held by every GPU that loads
- * the library until the process exits); a table needing more entries,
- * max_t*dim_t/2 + max_h*dim_h/2 + max_w*dim_w/2, is rejected with SOL_ERR_UNSUPPORTED.
- * All calls share that array: calls whose kernels overlap on the GPU (other streams,
- * unordered host threads) race on it and must be serialised by the caller.
- * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- * current device); make that first call before any stream capture.
- * Other arguments, layouts, aliasing and errors as in sol_qk_rmsnorm_rope3d. */
 /* Number of SubBlock blocks of `block_tokens` tokens in a packed sequence: blocks
  * restart at every sample boundary, so it is n_samples * ceil(tokens_per_sample /
  * block_tokens) (tokens_per_sample 0 = one sample); 0 for invalid arguments. */
@@ -311,6 +288,27 @@ sol_status sol_dit_epilogue_pool(void* qkv, int64_t ld_qkv, const void* wq, cons
                                  void* pooled_k, int64_t ld_pool, int32_t block_tokens, sol_dtype dt,
                                  sol_stream_t stream);
 
+/* QK RMSNorm + 3D RoPE for callers that cannot allocate device memory.  The pages have
+ * no counterpart: this entry point exists for hosts that reserve device memory up front
+ * and forbid allocation while they run work (inference engines whose pool already holds
+ * nearly all of HBM, plugin execute callbacks, latency-critical loops that cannot afford
+ * cudaMalloc's device synchronisation).  sol_qk_rmsnorm_rope3d needs a sol_rope3d handle,
+ * and creating one calls cudaMalloc; this function allocates nothing.
+ *
+ * It computes exactly what sol_qk_rmsnorm_rope3d computes, with the table described by
+ * (dim_t, dim_h, dim_w, theta, max_t, max_h, max_w) as in sol_rope3d_create.  The table
+ * is rebuilt on `stream` by every call inside a fixed device array of
+ * SOL_NOALLOC_MAX_ROPE_ENTRIES (cos, sin) pairs (512 KiB, held by every GPU that loads
+ * the library until the process exits); a table needing more entries,
+ * max_t*dim_t/2 + max_h*dim_h/2 + max_w*dim_w/2, is rejected with SOL_ERR_UNSUPPORTED.
+ * All calls share that array: calls whose kernels overlap on the GPU (other streams,
+ * unordered host threads) race on it and must be serialised by the caller.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * current device) and keeps it for the life of the process; make that first call before
+ * any stream capture.  The kept address does not survive the device's context: after
+ * cudaDeviceReset (or anything else that destroys the primary context) this entry point
+ * must not be called again in the process.
+ * Other arguments, layouts, aliasing and errors as in sol_qk_rmsnorm_rope3d. */
 #define SOL_NOALLOC_MAX_ROPE_ENTRIES 65536
 sol_status sol_qk_rmsnorm_rope3d_noalloc(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko,
                                          const void* q, const void* k, int64_t ld_q, int64_t ld_k,
@@ -380,44 +378,50 @@ sol_status sol_linear_swiglu(void* out, int64_t ld_out, const void* a, int64_t l
  * the folded weights (R * n_out * d bf16).  Returns 0 for invalid sizes or R > 32. */
 size_t sol_adaln_workspace_bytes(int64_t n_tokens, int64_t n_out, int64_t d, sol_modsel sel);
 
+/* How the sol_adaln_* calls apply AdaLN in front of their linear layer; every strategy
+ * computes the same product within the bf16 bound stated at the top of this section.
+ *   SOL_ADALN_STAGE (the fastest on B200): h is written once, rounded to bf16, into the
+ *     workspace by the AdaLN row kernel and read back by the GEMM, whose epilogue applies
+ *     the fused operator (the per-token operator's output never goes to HBM);
+ *   SOL_ADALN_FOLD: h is never formed -- per modulation row r the call writes V_r =
+ *     bf16(W * (1 + scale_r)) (column-wise), c_r = sum_k V_r[:, k] and b_r = shift_r . W^T
+ *     into the workspace, computes mean and 1/sqrt(var + eps) of every row of x, and runs
+ *     one GEMM of x against V_r whose epilogue forms rstd * (acc - mean * c_r) + b_r (the
+ *     only rounding of an operand is that of the folded weights, of the same size as
+ *     rounding h); a tile whose rows use several modulation rows is computed once per row
+ *     used;
+ *   SOL_ADALN_TRANSFORM: h is never stored -- each x tile is rewritten as bf16 h in
+ *     shared memory before the tensor cores read it. */
+typedef enum { SOL_ADALN_STAGE = 0, SOL_ADALN_FOLD = 1, SOL_ADALN_TRANSFORM = 2 } sol_adaln_strategy;
+
 /* AdaLN fused into a linear layer:
  *     out = h . W^T,   h = LN(x) * (1 + scale[r]) + shift[r]   (as sol_adaln_modulate)
  * x [n_tokens, d], W [n_out, d], out [n_tokens, n_out]; d a multiple of 64; at most 32
- * modulation rows (SOL_ERR_UNSUPPORTED otherwise).  Three strategies compute it; the
- * environment variable SOL_ADALN_STRATEGY (read at each call) picks one:
- *   "stage" (the default, the fastest on B200): h is written once, rounded to bf16, into
- *     the workspace by the AdaLN row kernel and read back by the GEMM, whose epilogue
- *     applies the fused operator (the per-token operator's output never goes to HBM);
- *   "fold": h is never formed -- per modulation row r the call writes V_r = bf16(W * (1 +
- *     scale_r)) (column-wise), c_r = sum_k V_r[:, k] and b_r = shift_r . W^T into the
- *     workspace, computes mean and 1/sqrt(var + eps) of every row of x, and runs one
- *     GEMM of x against V_r whose epilogue forms rstd * (acc - mean * c_r) + b_r (the
- *     only rounding of an operand is that of the folded weights, of the same size as
- *     rounding h); a tile whose rows use several modulation rows is computed once per
- *     row used;
- *   "transform": h is never stored -- each x tile is rewritten as bf16 h in shared
- *     memory before the tensor cores read it.
- * workspace: caller-owned device memory of at least sol_adaln_workspace_bytes(...)
- * bytes, 256-byte aligned, overlapping no other argument; its contents are scratch. */
+ * modulation rows (SOL_ERR_UNSUPPORTED otherwise).
+ *   strategy       a sol_adaln_strategy (SOL_ERR_INVALID_ARGUMENT otherwise).
+ *   workspace      caller-owned device memory of at least sol_adaln_workspace_bytes(...)
+ *                  bytes, 256-byte aligned, overlapping no other argument; its contents
+ *                  are scratch. */
 sol_status sol_adaln_linear(void* out, int64_t ld_out, const void* x, int64_t ld_x,
                             const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
                             const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,
-                            int64_t n_tokens, int64_t n_out, int64_t d, float eps, sol_dtype dt,
-                            sol_stream_t stream);
+                            int32_t strategy, int64_t n_tokens, int64_t n_out, int64_t d, float eps,
+                            sol_dtype dt, sol_stream_t stream);
 
 /* The MLP input of a block in one pass: AdaLN into the up projection, SwiGLU in its
  * epilogue:
  *     out[:, j] = silu((h . W1^T)[:, j]) * (h . W2^T)[:, j],   W = [W1; W2],
  *     h = LN(x) * (1 + scale[r]) + shift[r]   (as sol_adaln_linear)
  * x [n_tokens, d], W [2*inner, d] (gated half first, as sol_linear_swiglu), out
- * [n_tokens, inner]; inner a multiple of 128; workspace and strategies as in
+ * [n_tokens, inner]; inner a multiple of 128; workspace and strategy as in
  * sol_adaln_linear with n_out = 2 * inner.  The projection is neither stored nor rounded
  * before the SwiGLU. */
 sol_status sol_adaln_linear_swiglu(void* out, int64_t ld_out, const void* x, int64_t ld_x,
                                    const void* shift, const void* scale, int64_t ld_mod,
                                    sol_modsel sel, const void* w, int64_t ld_w, void* workspace,
-                                   size_t workspace_bytes, int64_t n_tokens, int64_t inner,
-                                   int64_t d, float eps, sol_dtype dt, sol_stream_t stream);
+                                   size_t workspace_bytes, int32_t strategy, int64_t n_tokens,
+                                   int64_t inner, int64_t d, float eps, sol_dtype dt,
+                                   sol_stream_t stream);
 
 /* The attention input of a block in one pass: AdaLN into the QKV projection, QK RMSNorm
  * + 3D RoPE in its epilogue:
@@ -427,16 +431,15 @@ sol_status sol_adaln_linear_swiglu(void* out, int64_t ld_out, const void* x, int
  * head_dim must be 128 and n_heads even.  Positions: pos [n_tokens, 3] int32, or NULL
  * for the row-major grid (grid_T, grid_H, grid_W) of each sample, samples of
  * sel.tokens_per_sample tokens (0 = one sample), as in sol_qk_rmsnorm_rope3d.
- * workspace and strategies as in sol_adaln_linear (with n_out = 3 * n_heads * head_dim).
+ * workspace and strategy as in sol_adaln_linear (with n_out = 3 * n_heads * head_dim).
  * The projection is not rounded before the norm. */
 sol_status sol_adaln_qkv_rope(void* qkv, int64_t ld_qkv, const void* x, int64_t ld_x,
                               const void* shift, const void* scale, int64_t ld_mod, sol_modsel sel,
                               const void* w, int64_t ld_w, void* workspace, size_t workspace_bytes,
-                              const void* wq,
-                              const void* wk, const int32_t* pos, int32_t grid_T, int32_t grid_H,
-                              int32_t grid_W, const sol_rope3d* rope, int64_t n_tokens,
-                              int32_t n_heads, int32_t head_dim, int64_t d, float eps, sol_dtype dt,
-                              sol_stream_t stream);
+                              int32_t strategy, const void* wq, const void* wk, const int32_t* pos,
+                              int32_t grid_T, int32_t grid_H, int32_t grid_W, const sol_rope3d* rope,
+                              int64_t n_tokens, int32_t n_heads, int32_t head_dim, int64_t d, float eps,
+                              sol_dtype dt, sol_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert L.sol_abi_version() == 1
+    assert L.sol_abi_version() == 2
     assert L.sol_status_string(0) == b"ok"
     for s in range(1, 5):
         assert L.sol_status_string(s) and L.sol_status_string(s) != b"ok"
@@ -179,31 +179,36 @@ def test_linear_epilogue_variants_validation(L):
     assert L.sol_adaln_workspace_bytes(tall, d, k, SEL) >= tall * 8 + tall * k * 2
     assert L.sol_adaln_workspace_bytes(tall, d, k, SEL) < tall * 8 + tall * k * 2 + d * k * 2
     ws = FAKE << 6
-    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, None, need, n, d, k, 1e-6, sol.BF16,
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, None, need, 0, n, d, k, 1e-6, sol.BF16,
                               None) == sol.ERR_INVALID_ARGUMENT
     assert "workspace" in last(L)
-    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws, need - 1, n, d, k, 1e-6, sol.BF16,
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws, need - 1, 0, n, d, k, 1e-6, sol.BF16,
                               None) == sol.ERR_INVALID_ARGUMENT
-    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws + 16, need, n, d, k, 1e-6, sol.BF16,
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws + 16, need, 0, n, d, k, 1e-6, sol.BF16,
                               None) == sol.ERR_MISALIGNED
-    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws, need, n, d, k, float("inf"),
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws, need, 0, n, d, k, float("inf"),
                               sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
     # workspace overlapping x
-    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, x + 1024, need, n, d, k, 1e-6,
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, x + 1024, need, 0, n, d, k, 1e-6,
                               sol.BF16, None) in (sol.ERR_INVALID_ARGUMENT, sol.ERR_MISALIGNED)
     # at most 32 modulation rows: 33 samples of 10 tokens
     many = sol.ModSel(None, 1, 10)
     assert L.sol_adaln_workspace_bytes(330, d, k, many) == 0
-    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, many, w, k, ws, need, 330, d, k, 1e-6, sol.BF16,
+    assert L.sol_adaln_linear(out, d, x, k, None, None, 0, many, w, k, ws, need, 0, 330, d, k, 1e-6, sol.BF16,
                               None) == sol.ERR_UNSUPPORTED
     # the QKV call is built for head_dim 128 and an even head count
-    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, ws, need, None, None, None,
+    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, ws, need, 0, None, None, None,
                                 2, 4, 4, None, n, 4, 64, k, 1e-6, sol.BF16, None) == sol.ERR_UNSUPPORTED
-    assert L.sol_adaln_qkv_rope(out, 1152, x, k, None, None, 0, SEL, w, k, ws, need, None, None, None,
+    assert L.sol_adaln_qkv_rope(out, 1152, x, k, None, None, 0, SEL, w, k, ws, need, 0, None, None, None,
                                 2, 4, 4, None, n, 3, 128, k, 1e-6, sol.BF16, None) == sol.ERR_UNSUPPORTED
-    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, ws, need, None, None, None,
+    assert L.sol_adaln_qkv_rope(out, 768, x, k, None, None, 0, SEL, w, k, ws, need, 0, None, None, None,
                                 2, 4, 4, None, n, 2, 128, k, 1e-6, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
     assert "rope is NULL" in last(L)
+    # the AdaLN strategy is an argument: only the three sol_adaln_strategy values pass
+    for bad in (-1, 3):
+        assert L.sol_adaln_linear(out, d, x, k, None, None, 0, SEL, w, k, ws, need, bad, n, d, k, 1e-6,
+                                  sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
+        assert "strategy" in last(L)
 
 
 def test_adaln_linear_swiglu_validation(L):
@@ -211,13 +216,13 @@ def test_adaln_linear_swiglu_validation(L):
     x, w, out = FAKE, FAKE << 3, FAKE << 4
     need = L.sol_adaln_workspace_bytes(n, 2 * inner, k, SEL)
     ws = FAKE << 6
-    assert L.sol_adaln_linear_swiglu(out, inner, x, k, None, None, 0, SEL, w, k, ws, need, n, inner, k, 1e-6,
+    assert L.sol_adaln_linear_swiglu(out, inner, x, k, None, None, 0, SEL, w, k, ws, need, 0, n, inner, k, 1e-6,
                                      sol.F32, None) == sol.ERR_UNSUPPORTED
-    assert L.sol_adaln_linear_swiglu(out, 192, x, k, None, None, 0, SEL, w, k, ws, need, n, 192, k, 1e-6,
+    assert L.sol_adaln_linear_swiglu(out, 192, x, k, None, None, 0, SEL, w, k, ws, need, 0, n, 192, k, 1e-6,
                                      sol.BF16, None) == sol.ERR_UNSUPPORTED  # inner not a multiple of 128
-    assert L.sol_adaln_linear_swiglu(out, inner, x, k, None, None, 0, SEL, w, k, None, need, n, inner, k, 1e-6,
+    assert L.sol_adaln_linear_swiglu(out, inner, x, k, None, None, 0, SEL, w, k, None, need, 0, n, inner, k, 1e-6,
                                      sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
-    assert L.sol_adaln_linear_swiglu(out, inner, x, k, None, None, 0, SEL, w, k, ws, need - 256, n, inner, k,
+    assert L.sol_adaln_linear_swiglu(out, inner, x, k, None, None, 0, SEL, w, k, ws, need - 256, 0, n, inner, k,
                                      1e-6, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
-    assert L.sol_adaln_linear_swiglu(None, inner, None, k, None, None, 0, SEL, w, k, None, 0, 0, inner, k, 1e-6,
+    assert L.sol_adaln_linear_swiglu(None, inner, None, k, None, None, 0, SEL, w, k, None, 0, 0, 0, inner, k, 1e-6,
                                      sol.BF16, None) == sol.OK

@@ -198,7 +198,7 @@ def adaln_inputs(w, m):
 
 
 @pytest.mark.parametrize("w", [SMALL, PACKED], ids=lambda w: w.name)
-def test_adaln_linear(oracle_mod, monkeypatch, w):
+def test_adaln_linear(oracle_mod, w):
     m = w.n_tokens
     x, shift, scale, sid, _, kw = adaln_inputs(w, m)
     W = wl.linear_weight(w, "w_qkv", 768, w.d, "cuda")
@@ -213,8 +213,7 @@ def test_adaln_linear(oracle_mod, monkeypatch, w):
                                    rr, w.eps)
     check(out, y, bound, f"adaln_linear {w.name}")
     # with the weights folded, the workspace starts with each row's mean and 1/sqrt(var + eps)
-    monkeypatch.setenv("SOL_ADALN_STRATEGY", "fold")
-    sol.adaln_linear(out, x, W, shift, scale, workspace=ws, eps=w.eps, stream_id=sid, **kw)
+    sol.adaln_linear(out, x, W, shift, scale, workspace=ws, strategy="fold", eps=w.eps, stream_id=sid, **kw)
     torch.cuda.synchronize()
     check(out, y, bound, f"adaln_linear {w.name}, weights folded")
     xf = f64(x)
@@ -334,7 +333,7 @@ def test_full_shape_adaln_qkv_rope(oracle_mod):
     ws = sol.adaln_workspace(m, 3 * w.hd, w.d)
     with sol.Rope3D(w.rope_dims, w.theta, w.max_pos) as rope:
         sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, workspace=ws, n_heads=w.n_heads, wq=wq, wk=wk,
-                           grid=w.grid, eps=w.eps)
+                           grid=w.grid, strategy=strategy, eps=w.eps)
         torch.cuda.synchronize()
     Wh = to_oracle(W)
     want, pre, h = oracle_mod.adaln_qkv_rope(
@@ -350,20 +349,15 @@ def test_full_shape_adaln_qkv_rope(oracle_mod):
 
 # ------------------------------------------- the other shapes and strategies of the kernel
 
-@pytest.mark.parametrize("env", [{"SOL_LINEAR_SHAPE": "single"}, {"SOL_ADALN_STRATEGY": "transform"},
-                                 {"SOL_LINEAR_SHAPE": "single", "SOL_ADALN_STRATEGY": "transform"},
-                                 {"SOL_LINEAR_SHAPE": "pair", "SOL_ADALN_STRATEGY": "transform"},
-                                 {"SOL_ADALN_STRATEGY": "fold"}, {"SOL_ADALN_STRATEGY": "stage"},
-                                 {"SOL_LINEAR_SHAPE": "single", "SOL_ADALN_STRATEGY": "stage"}],
-                         ids=lambda e: ",".join(f"{k}={v}" for k, v in e.items()))
-def test_alternative_shapes_and_strategies(oracle_mod, monkeypatch, env):
-    """Single-CTA tiles and each AdaLN strategy -- weights folded, operand transformed, h
-    staged through the workspace (selected per call by the library's environment switches)
-    -- compute the same results under the same bounds."""
-    for k, v in env.items():
-        monkeypatch.setenv(k, v)
+@pytest.mark.parametrize("rows", [None, 128, 77], ids=lambda r: "pair" if r is None else f"single{r}")
+@pytest.mark.parametrize("strategy", ["stage", "fold", "transform"])
+def test_alternative_shapes_and_strategies(oracle_mod, strategy, rows):
+    """Each AdaLN strategy (h staged through the workspace, weights folded, operand
+    transformed; the caller's choice) and both tile shapes (CTA pairs above 128 rows, one
+    CTA per tile at 128 rows or fewer) compute the same results under the same bounds."""
     w = PACKED
-    m = w.n_tokens
+    m = w.n_tokens if rows is None else rows
+    env = f"{strategy}, {m} rows"
     x, shift, scale, sid, pos, kw = adaln_inputs(w, m)
     hd = w.hd
     W = wl.linear_weight(w, "w_qkv", 3 * hd, w.d, "cuda")
@@ -372,7 +366,7 @@ def test_alternative_shapes_and_strategies(oracle_mod, monkeypatch, env):
     ws = sol.adaln_workspace(m, 3 * hd, w.d, **kw)
     with sol.Rope3D(w.rope_dims, w.theta, w.max_pos) as rope:
         sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, workspace=ws, n_heads=w.n_heads, wq=wq, wk=wk,
-                           pos=pos, grid=w.grid, eps=w.eps, stream_id=sid, **kw)
+                           pos=pos, grid=w.grid, strategy=strategy, eps=w.eps, stream_id=sid, **kw)
         torch.cuda.synchronize()
     Wh = to_oracle(W)
     want, pre, h = oracle_mod.adaln_qkv_rope(
@@ -384,7 +378,7 @@ def test_alternative_shapes_and_strategies(oracle_mod, monkeypatch, env):
     bq = qk_bound(pre[:, :2 * hd], E[:, :2 * hd], f64(wq), f64(wk), w.n_heads, w.eps)
     check(qkv[:, :2 * hd], want[:, :2 * hd], bq, f"adaln_qkv_rope q|k {env}")
     check(qkv[:, 2 * hd:], want[:, 2 * hd:], E[:, 2 * hd:], f"adaln_qkv_rope v {env}")
-    # the plain epilogues in the forced shape too
+    # the epilogues without AdaLN in the same shape
     a = wl.activation(w, "attn", m, w.d, "cuda")
     Wup = wl.linear_weight(w, "w_up", 2 * w.inner, w.d, "cuda")
     out = torch.empty((m, w.inner), dtype=torch.bfloat16, device="cuda")
@@ -397,9 +391,19 @@ def test_alternative_shapes_and_strategies(oracle_mod, monkeypatch, env):
     ea, eb = ACC * S[:, :w.inner], ACC * S[:, w.inner:]
     bound = 1.1 * ea * (np.abs(up) + eb) + np.abs(ga / (1 + np.exp(-ga))) * eb
     check(out, oracle_mod.swiglu(np.ascontiguousarray(u), w.inner), bound, f"linear_swiglu {env}")
-    # AdaLN into the up projection with SwiGLU, in the forced shape / strategy
+    gate = wl.modulation(w, "gate_msa", "cuda")
+    Wo = wl.linear_weight(w, "w_o", w.d, w.d, "cuda")
+    xo = torch.empty_like(x)
+    sol.linear_gated_residual(xo, x, a, Wo, gate, stream_id=sid, **kw)
+    torch.cuda.synchronize()
+    Wo_h, G = to_oracle(Wo), to_oracle(gate)
+    want_g = oracle_mod.linear_gated_residual(to_oracle(x), A, Wo_h, G, stream_id=to_oracle(sid), **kw)
+    gmax = np.abs(oracle_mod.to_f64(G)).max(axis=0)
+    check(xo, want_g, ACC * gmax[None, :] * oracle_mod.linear_magnitude(A, Wo_h), f"linear_gated_residual {env}")
+    # AdaLN into the up projection with SwiGLU, same shape and strategy
     ws2 = sol.adaln_workspace(m, 2 * w.inner, w.d, **kw)
-    sol.adaln_linear_swiglu(out, x, Wup, shift, scale, workspace=ws2, eps=w.eps, stream_id=sid, **kw)
+    sol.adaln_linear_swiglu(out, x, Wup, shift, scale, workspace=ws2, strategy=strategy, eps=w.eps, stream_id=sid,
+                            **kw)
     torch.cuda.synchronize()
     want, u2, h2 = oracle_mod.adaln_linear_swiglu(to_oracle(x), Wu, to_oracle(shift), to_oracle(scale), w.inner,
                                                   eps=w.eps, stream_id=to_oracle(sid), **kw)
@@ -422,8 +426,7 @@ def sample_rows(m, n=48, seed=7):
 
 
 @pytest.mark.parametrize("strategy", ["stage", "fold"])
-def test_bench_size_adaln_qkv_rope_sampled(oracle_mod, monkeypatch, strategy):
-    monkeypatch.setenv("SOL_ADALN_STRATEGY", strategy)
+def test_bench_size_adaln_qkv_rope_sampled(oracle_mod, strategy):
     w = FULL
     m = BENCH_M
     x = wl.activation(w, "x", m, w.d, "cuda")
@@ -434,7 +437,7 @@ def test_bench_size_adaln_qkv_rope_sampled(oracle_mod, monkeypatch, strategy):
     ws = sol.adaln_workspace(m, 3 * w.hd, w.d)
     with sol.Rope3D(w.rope_dims, w.theta, w.max_pos) as rope:
         sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, workspace=ws, n_heads=w.n_heads, wq=wq, wk=wk,
-                           grid=w.grid, eps=w.eps)
+                           grid=w.grid, strategy=strategy, eps=w.eps)
         torch.cuda.synchronize()
     rows = sample_rows(m)
     xs = to_oracle(x[torch.from_numpy(rows).cuda()])
@@ -500,10 +503,9 @@ def test_adaln_linear_swiglu(oracle_mod, w):
 
 
 @pytest.mark.parametrize("strategy", ["stage", "fold"])
-def test_bench_size_adaln_linear_swiglu_sampled(oracle_mod, monkeypatch, strategy):
+def test_bench_size_adaln_linear_swiglu_sampled(oracle_mod, strategy):
     """AdaLN -> up projection + SwiGLU at the size bench.py times, both AdaLN strategies,
     checked on sampled rows (the first and last tiles included)."""
-    monkeypatch.setenv("SOL_ADALN_STRATEGY", strategy)
     w = FULL
     m = BENCH_M
     x = wl.activation(w, "x", m, w.d, "cuda")
@@ -511,7 +513,7 @@ def test_bench_size_adaln_linear_swiglu_sampled(oracle_mod, monkeypatch, strateg
     W = wl.linear_weight(w, "w_up", 2 * w.inner, w.d, "cuda")
     out = torch.empty((m, w.inner), dtype=torch.bfloat16, device="cuda")
     ws = sol.adaln_workspace(m, 2 * w.inner, w.d)
-    sol.adaln_linear_swiglu(out, x, W, shift, scale, workspace=ws, eps=w.eps)
+    sol.adaln_linear_swiglu(out, x, W, shift, scale, workspace=ws, strategy=strategy, eps=w.eps)
     torch.cuda.synchronize()
     rows = sample_rows(m, seed=13)
     ri = torch.from_numpy(rows).cuda()

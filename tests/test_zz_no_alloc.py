@@ -4,7 +4,8 @@ sol_qk_rmsnorm_rope3d_noalloc serves callers that cannot allocate device memory 
 they run (engines whose pool already holds the GPU's memory, plugin execute callbacks):
 it keeps its cos/sin table in a fixed array inside the library instead of a handle made
 by cudaMalloc.  Its output must match the regular entry point's within the parity
-tolerance, on consecutive calls that rebuild the shared table for different shapes.
+tolerance, on consecutive calls that rebuild the shared table for different shapes, and
+the fp64 oracle's (bf16 and fp32, positions outside the table clamped).
 
 This file is named so that pytest collects it last.
 """
@@ -14,7 +15,7 @@ import pytest
 import torch
 
 from dit_block_b200 import sol, workloads
-from parity_util import tolerance, to_f64
+from parity_util import assert_close, to_oracle, tolerance, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -116,3 +117,66 @@ def test_noalloc_rejects_tables_beyond_its_array():
     assert e.value.status == sol.ERR_UNSUPPORTED
     assert "65536" in str(e.value)
     torch.cuda.synchronize()
+
+
+def _oracle_qk(oracle_mod, c, q, k, wq, wk, pos):
+    return oracle_mod.qk_rmsnorm_rope3d(
+        to_oracle(q), to_oracle(k), to_oracle(wq), to_oracle(wk), n_heads=c["Hh"], head_dim=c["head_dim"],
+        pos=pos, grid=c["grid"], tokens_per_sample=c["tps"], dims=c["dims"], theta=c["theta"])
+
+
+def test_noalloc_matches_oracle_with_clamped_positions(oracle_mod):
+    """The (16, 56, 56) split at theta 500 straight against the fp64 oracle, with explicit
+    positions, some of them outside the table (the library clamps them into it; the oracle
+    gets the clamped positions)."""
+    c = _case_packed()
+    hd = c["Hh"] * c["head_dim"]
+    q, k = c["qkv"][:, :hd], c["qkv"][:, hd:2 * hd]
+    pos = c["pos"].clone()
+    n = pos.shape[0]
+    mx = torch.tensor(c["max_pos"], dtype=torch.int32, device=DEV)
+    pos[0] = mx + 5          # beyond the table on every axis
+    pos[n // 2] = -3         # below it
+    pos[n - 1, 0] = mx[0]    # exactly one past the last row
+    wq = _randn((128,), BF, 3, std=0.02, mean=1.0)
+    wk = _randn((128,), BF, 4, std=0.02, mean=1.0)
+    gq, gk = torch.empty_like(q), torch.empty_like(k)
+    sol.qk_rmsnorm_rope3d_noalloc(gq, gk, q, k, n_heads=c["Hh"], head_dim=128, wq=wq, wk=wk, pos=pos,
+                                  dims=c["dims"], theta=c["theta"], max_pos=c["max_pos"])
+    torch.cuda.synchronize()
+    clamped = torch.minimum(torch.clamp(pos, min=0), mx - 1)
+    oq, ok = _oracle_qk(oracle_mod, c, q, k, wq, wk, to_oracle(clamped))
+    assert_close(to_f64(gq), oq, BF, "noalloc q vs oracle")
+    assert_close(to_f64(gk), ok, BF, "noalloc k vs oracle")
+    # the regular entry point clamps the same way
+    rq, rk = torch.empty_like(q), torch.empty_like(k)
+    with sol.Rope3D(c["dims"], c["theta"], c["max_pos"]) as rope:
+        sol.qk_rmsnorm_rope3d(rq, rk, q, k, rope, n_heads=c["Hh"], head_dim=128, wq=wq, wk=wk, pos=pos)
+        torch.cuda.synchronize()
+    _close(gq, rq, BF, "clamped q vs regular")
+    _close(gk, rk, BF, "clamped k vs regular")
+
+
+def test_noalloc_f32_matches_oracle_and_regular(oracle_mod):
+    """fp32 path (tight 1e-5 bound): 2 heads of 128 on the 2 x 4 x 4 grid."""
+    grid = (2, 4, 4)
+    n = 32
+    qkv = _randn((n, 3 * 256), torch.float32, 5)
+    c = dict(Hh=2, head_dim=128, dims=(32, 48, 48), theta=10000.0, grid=grid, tps=0)
+    q, k = qkv[:, :256], qkv[:, 256:512]
+    wq = _randn((128,), torch.float32, 6, std=0.02, mean=1.0)
+    wk = _randn((128,), torch.float32, 7, std=0.02, mean=1.0)
+    for call in range(2):  # two calls in a row, the second over the table the first built
+        gq, gk = torch.full_like(q, 7.0), torch.full_like(k, 7.0)
+        sol.qk_rmsnorm_rope3d_noalloc(gq, gk, q, k, n_heads=2, head_dim=128, wq=wq, wk=wk, grid=grid,
+                                      max_pos=grid, dims=c["dims"], theta=c["theta"])
+        torch.cuda.synchronize()
+        oq, ok = _oracle_qk(oracle_mod, c, q, k, wq, wk, None)
+        assert_close(to_f64(gq), oq, torch.float32, f"f32 noalloc q vs oracle, call {call}")
+        assert_close(to_f64(gk), ok, torch.float32, f"f32 noalloc k vs oracle, call {call}")
+        rq, rk = torch.empty_like(q), torch.empty_like(k)
+        with sol.Rope3D(c["dims"], c["theta"], grid) as rope:
+            sol.qk_rmsnorm_rope3d(rq, rk, q, k, rope, n_heads=2, head_dim=128, wq=wq, wk=wk, grid=grid)
+            torch.cuda.synchronize()
+        _close(gq, rq, torch.float32, f"f32 q vs regular, call {call}")
+        _close(gk, rk, torch.float32, f"f32 k vs regular, call {call}")
