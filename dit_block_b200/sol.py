@@ -47,6 +47,17 @@ class QkDesc(ctypes.Structure):
                 ("dt", ctypes.c_int)]
 
 
+class BlockHostDesc(ctypes.Structure):
+    """sol_block_host_desc (include/sol.h)."""
+    _fields_ = [("x", _P), ("qkv", _P), ("y_attn", _P), ("u", _P), ("y_mlp", _P), ("pos", _P),
+                ("stream_id", _P), ("h1", _P), ("qk", _P), ("x1", _P), ("h2", _P), ("act", _P), ("x2", _P),
+                ("shift_msa", _P), ("scale_msa", _P), ("gate_msa", _P), ("shift_mlp", _P), ("scale_mlp", _P),
+                ("gate_mlp", _P), ("wq", _P), ("wk", _P), ("rope", _P), ("grid_T", _I32), ("grid_H", _I32),
+                ("grid_W", _I32), ("n_tokens", _I64), ("tokens_per_sample", _I64), ("n_streams", _I32),
+                ("d", _I64), ("n_heads", _I32), ("head_dim", _I32), ("inner", _I64), ("eps", _F),
+                ("dt", ctypes.c_int)]
+
+
 NORM_PER_HEAD, NORM_ACROSS_HEADS = 0, 1
 ADALN_STAGE, ADALN_FOLD, ADALN_TRANSFORM = 0, 1, 2
 _STRATEGIES = {"stage": ADALN_STAGE, "fold": ADALN_FOLD, "transform": ADALN_TRANSFORM}
@@ -78,6 +89,8 @@ SIGNATURES = {
     "sol_qk_rmsnorm_rope3d_noalloc": ([_P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _P, _P, _I32, _I32,
                                        _I32, _I64, _I32, _I32, _I32, _D, _I32, _I32, _I32, _I64,
                                        _I32, _I32, _F, _E, _P], _E),
+    "sol_dit_block_host_workspace_bytes": ([ctypes.POINTER(BlockHostDesc), _I64, _I32], ctypes.c_size_t),
+    "sol_dit_block_host": ([ctypes.POINTER(BlockHostDesc), _P, ctypes.c_size_t, _I64, _I32, _P, _P, _P], _E),
     "sol_linear": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _E, _P], _E),
     "sol_linear_gated_residual": ([_P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _I64, ModSel, _I64, _I64,
                                    _I64, _E, _P], _E),
@@ -323,6 +336,46 @@ def qk_rmsnorm_rope3d_noalloc(q_out, k_out, q, k, *, n_heads, head_dim, dims=(32
         int(tokens_per_sample), int(dims[0]), int(dims[1]), int(dims[2]), float(theta),
         int(max_pos[0]), int(max_pos[1]), int(max_pos[2]), q.shape[0], int(n_heads),
         int(head_dim), eps, _dtype(q), _stream(stream)), "sol_qk_rmsnorm_rope3d_noalloc")
+
+
+BLOCK_HOST_IN = ("x", "qkv", "y_attn", "u", "y_mlp")
+BLOCK_HOST_OUT = ("h1", "qk", "x1", "h2", "act", "x2")
+BLOCK_HOST_MOD = ("shift_msa", "scale_msa", "gate_msa", "shift_mlp", "scale_mlp", "gate_mlp")
+
+
+def block_host_desc(inputs: dict, outputs: dict, mods: dict, rope: Rope3D, *, n_heads: int, head_dim: int,
+                    inner: int, wq=None, wk=None, pos=None, stream_id=None, grid=(0, 0, 0), tokens_per_sample=0,
+                    n_streams=1, eps=1e-6) -> BlockHostDesc:
+    """sol_block_host_desc over HOST tensors (pinned for overlapped copies): inputs
+    BLOCK_HOST_IN, outputs BLOCK_HOST_OUT (missing or None: not copied back), modulation rows
+    BLOCK_HOST_MOD (missing or None: zero), wq / wk, pos [N, 3] int32, stream_id [N] uint8."""
+    x = inputs["x"]
+    for t in list(inputs.values()) + [v for v in outputs.values() if v is not None]:
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("sol_dit_block_host takes contiguous host tensors")
+    if pos is not None and (pos.dtype != torch.int32 or pos.is_cuda):
+        raise TypeError("pos must be a host int32 [N, 3] tensor")
+    if stream_id is not None and (stream_id.dtype != torch.uint8 or stream_id.is_cuda):
+        raise TypeError("stream_id must be a host uint8 tensor")
+    g = lambda k, dct: _ptr(dct.get(k))
+    return BlockHostDesc(
+        *(g(k, inputs) for k in BLOCK_HOST_IN), _ptr(pos), _ptr(stream_id), *(g(k, outputs) for k in BLOCK_HOST_OUT),
+        *(g(k, mods) for k in BLOCK_HOST_MOD), _ptr(wq), _ptr(wk), rope.handle, int(grid[0]), int(grid[1]),
+        int(grid[2]), x.shape[0], int(tokens_per_sample), int(n_streams), x.shape[1], int(n_heads), int(head_dim),
+        int(inner), float(eps), _dtype(x))
+
+
+def dit_block_host_workspace_bytes(desc: BlockHostDesc, chunk_tokens: int, n_slots: int) -> int:
+    return int(lib().sol_dit_block_host_workspace_bytes(ctypes.byref(desc), int(chunk_tokens), int(n_slots)))
+
+
+def dit_block_host(desc: BlockHostDesc, workspace: torch.Tensor, *, chunk_tokens: int, n_slots: int, s_in, s_comp,
+                   s_out):
+    """One block pass over host tensors (sol_dit_block_host): enqueued on s_comp with the
+    copies on s_in / s_out; the host outputs are filled once s_comp reaches the end."""
+    _check(lib().sol_dit_block_host(ctypes.byref(desc), _ptr(workspace), workspace.numel(), int(chunk_tokens),
+                                    int(n_slots), _stream(s_in), _stream(s_comp), _stream(s_out)),
+           "sol_dit_block_host")
 
 
 def subblock_count(n_tokens: int, tokens_per_sample: int = 0, block_tokens: int = 64) -> int:

@@ -91,7 +91,8 @@ const char* sol_last_error(void);
 int32_t sol_abi_version(void);
 
 /* Error flags raised on the current device by libsol kernels since the last clear:
- * bit 0 = a per-token kernel's bounded wait on its own asynchronous copy gave up;
+ * bit 0 = an AdaLN / prologue kernel's bounded wait on its own asynchronous copy gave up;
+ * bit 1 = a QK RMSNorm + RoPE kernel's bounded wait on its own asynchronous copy gave up;
  * bits 8..15 = a linear-layer kernel (sol_linear*, sol_adaln_*) gave up a bounded wait
  * in its copy / MMA / epilogue / transform pipeline.  The kernel recorded it, drained
  * its own copies and MMAs, stopped early and left its outputs incomplete.  Synchronises
@@ -287,6 +288,95 @@ sol_status sol_dit_epilogue_pool(void* qkv, int64_t ld_qkv, const void* wq, cons
                                  int32_t n_heads, int32_t head_dim, float eps, void* pooled_q,
                                  void* pooled_k, int64_t ld_pool, int32_t block_tokens, sol_dtype dt,
                                  sol_stream_t stream);
+
+/* One pass of the block's per-token hot path over HOST-resident tensors [STM-RES: the
+ * fused operators cut memory traffic and per-step launches; video and audio tokens run
+ * through one packed DiT stack].  Computes exactly what these five device calls compute
+ * over the whole sequence, in this order:
+ *     h1      = sol_adaln_modulate(x; shift_msa, scale_msa)
+ *     q|k     = sol_dit_epilogue(qkv)                    (in place on the qkv rows)
+ *     x1, h2  = sol_dit_prologue(x, y_attn; gate_msa, shift_mlp, scale_mlp)
+ *     act     = sol_swiglu(u)                            (u = [a | b], inner wide)
+ *     x2      = sol_gated_residual(x1, y_mlp; gate_mlp)
+ * but with every token-row tensor in host memory: the sequence is cut into chunks of at
+ * most `chunk_tokens` tokens that never cross a sample, and each chunk is copied in
+ * (cudaMemcpyAsync on s_in), computed (the five launches on s_comp) and copied out
+ * (on s_out) through `n_slots` rotating device buffers in the caller's workspace, so that
+ * the copies of neighbouring chunks overlap the compute.  Inputs and outputs should be
+ * page-locked (cudaHostAlloc / cudaHostRegister) for the copies to run asynchronously.
+ *
+ * Ordering: s_in and s_out first wait for the work already enqueued on s_comp; when the
+ * call returns, s_comp has been made to wait for the last copy-out, so anything enqueued
+ * on s_comp afterwards (a cudaStreamSynchronize, an event) sees the complete pass and
+ * the host outputs filled.  The three streams must be distinct.  The call itself does not
+ * block the host (except where the copies are from pageable memory).
+ *
+ * Host tensors (token-major, rows contiguous: ld = row width):
+ *   x, y_attn, y_mlp   [n_tokens, d]          required
+ *   qkv                [n_tokens, 3 * hd]     required; hd = n_heads * head_dim; q | k | v
+ *   u                  [n_tokens, 2 * inner]  required
+ *   pos                int32 [n_tokens, 3] or NULL: then each sample's tokens sit on the
+ *                      row-major grid_T x grid_H x grid_W grid (as sol_qk_rmsnorm_rope3d)
+ *   stream_id          uint8 [n_tokens] or NULL (every token in stream 0)
+ *   h1, x1, h2, x2     [n_tokens, d]          outputs; NULL = not copied back
+ *   qk                 [n_tokens, 2 * hd]     output: the normalised, rotated q | k; or NULL
+ *   act                [n_tokens, inner]      output, or NULL
+ *   shift_msa, scale_msa, gate_msa, shift_mlp, scale_mlp, gate_mlp
+ *                      [n_samples * n_streams, d] modulation rows (row r = sample *
+ *                      n_streams + stream, as sol_modsel), or NULL (zero); n_samples =
+ *                      ceil(n_tokens / tokens_per_sample), 1 when tokens_per_sample is 0
+ *   wq, wk             [head_dim] RMSNorm weights, or NULL (ones)
+ * The modulation rows and weights are copied once per call (on s_in, ahead of the first
+ * chunk) into the workspace; rope is the device-side table handle of sol_rope3d_create.
+ * Sizes: n_tokens >= 0; tokens_per_sample > 0, or 0 = one sample; n_streams >= 1; d,
+ * n_heads, head_dim, inner as the five device calls accept them; eps >= 0.
+ * workspace: caller-owned device memory of at least
+ * sol_dit_block_host_workspace_bytes(desc, chunk_tokens, n_slots) bytes, 256-byte aligned;
+ * chunk_tokens >= 1, n_slots >= 1 (2 or more overlap copies with compute).  The pass uses
+ * the workspace until s_comp reaches the end of the pass.
+ * Errors: every argument is validated before anything is enqueued; a copy or launch that
+ * the CUDA runtime refuses part-way returns SOL_ERR_CUDA and leaves the pass incomplete
+ * (what was enqueued stays enqueued). */
+typedef struct {
+    const void* x;
+    const void* qkv;
+    const void* y_attn;
+    const void* u;
+    const void* y_mlp;
+    const int32_t* pos;
+    const uint8_t* stream_id;
+    void* h1;
+    void* qk;
+    void* x1;
+    void* h2;
+    void* act;
+    void* x2;
+    const void* shift_msa;
+    const void* scale_msa;
+    const void* gate_msa;
+    const void* shift_mlp;
+    const void* scale_mlp;
+    const void* gate_mlp;
+    const void* wq;
+    const void* wk;
+    const sol_rope3d* rope;
+    int32_t grid_T, grid_H, grid_W;
+    int64_t n_tokens;
+    int64_t tokens_per_sample;
+    int32_t n_streams;
+    int64_t d;
+    int32_t n_heads, head_dim;
+    int64_t inner;
+    float eps;
+    sol_dtype dt;
+} sol_block_host_desc;
+
+/* Device workspace, in bytes, that sol_dit_block_host needs (0 for invalid sizes). */
+size_t sol_dit_block_host_workspace_bytes(const sol_block_host_desc* desc, int64_t chunk_tokens, int32_t n_slots);
+
+sol_status sol_dit_block_host(const sol_block_host_desc* desc, void* workspace, size_t workspace_bytes,
+                              int64_t chunk_tokens, int32_t n_slots, sol_stream_t s_in, sol_stream_t s_comp,
+                              sol_stream_t s_out);
 
 /* QK RMSNorm + 3D RoPE for callers that cannot allocate device memory.  The pages have
  * no counterpart: this entry point exists for hosts that reserve device memory up front

@@ -28,7 +28,7 @@ def last(L):
 
 def test_exports_every_declared_symbol(L):
     names = sol.header_functions()
-    assert len(names) == 24
+    assert len(names) == 26
     for n in names:
         assert hasattr(L, n), f"libsol.so does not export {n}"
         assert n in sol.SIGNATURES, f"binding has no signature for {n}"
@@ -226,3 +226,47 @@ def test_adaln_linear_swiglu_validation(L):
                                      1e-6, sol.BF16, None) == sol.ERR_INVALID_ARGUMENT
     assert L.sol_adaln_linear_swiglu(None, inner, None, k, None, None, 0, SEL, w, k, None, 0, 0, 0, inner, k, 1e-6,
                                      sol.BF16, None) == sol.OK
+
+
+def test_block_host_validation(L):
+    """sol_dit_block_host checks its description, streams and workspace before it enqueues
+    anything (no GPU needed for these refusals)."""
+    import ctypes
+    d = sol.BlockHostDesc()
+    d.x = d.qkv = d.y_attn = d.u = d.y_mlp = FAKE
+    d.rope = FAKE << 2
+    d.grid_T, d.grid_H, d.grid_W = 2, 4, 4
+    d.n_tokens, d.tokens_per_sample, d.n_streams = 32, 0, 1
+    d.d, d.n_heads, d.head_dim, d.inner, d.eps, d.dt = 256, 2, 128, 512, 1e-6, sol.F32
+    ref = ctypes.byref(d)
+    need = L.sol_dit_block_host_workspace_bytes(ref, 16, 2)
+    # constants (6 modulation rows, wq, wk) + 2 slots of 16 rows: x, qkv, y_attn, u, y_mlp,
+    # h1, x1, h2, act, x2 (fp32), positions and stream ids, each region 256-byte aligned
+    slot = 16 * 4 * (256 * 7 + 768 + 1024 + 512) + 256 + 256
+    assert need >= 6 * 256 * 4 + 2 * 128 * 4 + 2 * slot
+    assert L.sol_dit_block_host_workspace_bytes(ref, 0, 2) == 0
+    assert L.sol_dit_block_host_workspace_bytes(None, 16, 2) == 0
+    ws, s1, s2, s3 = FAKE << 8, 1, 2, 3
+    assert L.sol_dit_block_host(None, ws, need, 16, 2, s1, s2, s3) == sol.ERR_INVALID_ARGUMENT
+    assert L.sol_dit_block_host(ref, ws, need, 16, 2, s1, s1, s3) == sol.ERR_INVALID_ARGUMENT
+    assert "distinct" in last(L)
+    assert L.sol_dit_block_host(ref, ws, need - 1, 16, 2, s1, s2, s3) == sol.ERR_INVALID_ARGUMENT
+    assert "workspace" in last(L)
+    assert L.sol_dit_block_host(ref, ws + 16, need, 16, 2, s1, s2, s3) == sol.ERR_MISALIGNED
+    assert L.sol_dit_block_host(ref, ws, need, 16, 0, s1, s2, s3) == sol.ERR_INVALID_ARGUMENT
+    d.y_mlp = None
+    assert L.sol_dit_block_host(ref, ws, need, 16, 2, s1, s2, s3) == sol.ERR_INVALID_ARGUMENT
+    assert "required" in last(L)
+    d.y_mlp = FAKE
+    d.grid_W = 3  # 2 x 4 x 3 = 24 cells for 32 tokens of implicit positions
+    assert L.sol_dit_block_host(ref, ws, need, 16, 2, s1, s2, s3) == sol.ERR_INVALID_ARGUMENT
+    d.grid_W = 4
+    d.d = 250  # not a multiple of 4 fp32 elements
+    assert L.sol_dit_block_host(ref, ws, need, 16, 2, s1, s2, s3) == sol.ERR_MISALIGNED
+    d.d, d.dt = 256, 7
+    assert L.sol_dit_block_host(ref, ws, need, 16, 2, s1, s2, s3) == sol.ERR_UNSUPPORTED
+    d.dt, d.rope = sol.F32, None
+    assert L.sol_dit_block_host(ref, ws, need, 16, 2, s1, s2, s3) == sol.ERR_INVALID_ARGUMENT
+    assert "rope" in last(L)
+    d.rope, d.n_tokens = FAKE << 2, 0
+    assert L.sol_dit_block_host(ref, None, 0, 16, 2, s1, s2, s3) == sol.OK

@@ -1,12 +1,14 @@
-"""The host-buffer pipeline (chunked, three streams) gives bit-identical results to one
-pass of the five launches over the whole sequence, on a video-only grid and on a packed
-video+audio batch whose chunks stop at sample boundaries."""
+"""The host-buffer pass (sol_dit_block_host through pipeline.HostBlockPipeline: chunked,
+three streams, every copy issued by the library) gives bit-identical results to one pass
+of the five launches over the whole sequence, on a video-only grid (positions generated
+per chunk from the implicit grid) and on a packed video+audio batch (explicit positions and
+stream ids) whose chunks stop at sample boundaries; outputs left out stay on the device."""
 from __future__ import annotations
 
 import pytest
 import torch
 
-from dit_block_b200 import block, pipeline, workloads
+from dit_block_b200 import block, pipeline, sol, workloads
 
 pytestmark = pytest.mark.gpu
 
@@ -51,11 +53,46 @@ def test_pipeline_matches_single_pass(w, chunk):
     assert torch.equal(host_out["act"], bufs.act.cpu())
     assert torch.equal(host_out["x2"], bufs.x2.cpu())
     h2d, d2h = pipe.bytes_per_pass(n)
+    layout = 0 if pipe.pos is None else pipe.pos.numel() * 4 + pipe.sid.numel()
     assert h2d == sum(t.numel() * t.element_size() for t in host_in.values()) + \
-        sum(t.numel() * t.element_size() for t in host_mod.values())
+        sum(t.numel() * t.element_size() for t in host_mod.values()) + \
+        pipe.wq.numel() * pipe.wq.element_size() * 2 + layout
     assert d2h == sum(t.numel() * t.element_size() for t in host_out.values())
+    # only x2 back: the other outputs are not copied (their host buffers keep a sentinel)
+    only = {"x2": torch.full_like(host_out["x2"], 7.0)}
+    sentinel = {k: torch.full_like(v, 7.0) for k, v in host_out.items() if k != "x2"}
+    pipe.run(host_in, {**only, **{k: None for k in sentinel}}, host_mod)
+    torch.cuda.synchronize()
+    assert torch.equal(only["x2"], bufs.x2.cpu())
+    assert pipe.bytes_per_pass(n, outputs=("x2",))[1] == only["x2"].numel() * only["x2"].element_size()
+    assert all(torch.all(v == 7.0) for v in sentinel.values())
     pipe.close()
     bufs.close()
+
+
+def test_host_pass_validation():
+    w = CASES[0]
+    n = 40
+    host_in, host_out, host_mod = pipeline.host_buffers(w, n)
+    pipe = pipeline.HostBlockPipeline(w, "cuda", chunk_tokens=16, n_slots=2)
+    d = pipe.desc(host_in, host_out, host_mod)
+    need = sol.dit_block_host_workspace_bytes(d, 16, 2)
+    assert need > 0
+    ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    with pytest.raises(sol.SolError) as e:
+        sol.dit_block_host(d, ws, chunk_tokens=16, n_slots=2, s_in=s1, s_comp=s1, s_out=s2)
+    assert "distinct" in str(e.value)
+    with pytest.raises(sol.SolError) as e:
+        sol.dit_block_host(d, ws[:need - 256], chunk_tokens=16, n_slots=2, s_in=s1, s_comp=s2,
+                           s_out=torch.cuda.Stream())
+    assert "workspace" in str(e.value)
+    bad = pipe.desc(host_in, host_out, host_mod)
+    bad.head_dim = 96  # the epilogue's own check rejects it before anything is enqueued
+    with pytest.raises(sol.SolError):
+        sol.dit_block_host(bad, ws, chunk_tokens=16, n_slots=2, s_in=s1, s_comp=s2, s_out=torch.cuda.Stream())
+    torch.cuda.synchronize()
+    pipe.close()
 
 
 def test_chunks_never_cross_samples():
