@@ -162,6 +162,9 @@ cudaError_t launch_qk_rmsnorm_rope3d(sol_dtype dt, void* q_out, void* k_out, int
                                      float eps, cudaStream_t s)
 {
     (void)grid_T;
+    if (qk_cta_fits(dt, n_heads, head_dim, q, k, n_tokens))
+        return launch_qk_cta(q_out, k_out, ld_qo, ld_ko, q, k, ld_q, ld_k, wq, wk, pos, grid_H, grid_W, tps, rope,
+                             n_tokens, n_heads, eps, s);
     if (qk_regs_fits(dt, n_heads, head_dim))
         return launch_qk_regs(q_out, k_out, ld_qo, ld_ko, q, k, ld_q, ld_k, wq, wk, pos, grid_H, grid_W, tps, rope,
                               n_tokens, n_heads, eps, s);

@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "qk_math.cuh"
 
 namespace sol {
 
@@ -229,15 +230,15 @@ template <int SPW>
 __device__ __forceinline__ void pool_row(const uint4 (&xv)[SPW], bf16* row, float (&acc)[SPW][8], const float (&w)[8],
                                          const float (&cs)[4], const float (&sn)[4], float eps)
 {
+    // the plain epilogue's arithmetic (qk_math.cuh), so the in-place rows are the same bits
+    float kc[16];
+    qk_coefs(w, cs, sn, kc);
     float ss[SPW];
 #pragma unroll
     for (int i = 0; i < SPW; ++i) {
-        float f[8];
-        unpack<bf16>(xv[i], f);
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaf(f[e], f[e], a);
-        ss[i] = a;
+        float2 f[4];
+        unpack2<bf16>(xv[i], f);
+        ss[i] = qk_sumsq(f);
     }
 #pragma unroll
     for (int off = 8; off > 0; off >>= 1) {
@@ -246,16 +247,10 @@ __device__ __forceinline__ void pool_row(const uint4 (&xv)[SPW], bf16* row, floa
     }
 #pragma unroll
     for (int i = 0; i < SPW; ++i) {
-        float f[8], o[8];
-        unpack<bf16>(xv[i], f);
-        const float r = rsqrtf(ss[i] * (1.f / 128.f) + eps);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float a = f[2 * m] * r * w[2 * m];
-            const float b = f[2 * m + 1] * r * w[2 * m + 1];
-            o[2 * m] = a * cs[m] - b * sn[m];
-            o[2 * m + 1] = a * sn[m] + b * cs[m];
-        }
+        float2 f[4];
+        unpack2<bf16>(xv[i], f);
+        float o[8];
+        qk_rotate(f, rsqrtf(ss[i] * (1.f / 128.f) + eps), kc, o);
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[i][e] += o[e];
         st_stream(row + 256 * i, pack<bf16>(o));

@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "qk_math.cuh"
 
 // Launch shape: blocks of 64 threads, >= 4 per SM (the row needs ~200 registers per lane
 // unspilled; the same shape as the AdaLN row kernel).
@@ -30,6 +31,7 @@
 #ifndef SOL_QK_REGS_MINB
 #define SOL_QK_REGS_MINB 4
 #endif
+
 
 namespace sol {
 
@@ -142,31 +144,6 @@ __global__ void __launch_bounds__(SOL_QK_REGS_BLOCK, SOL_QK_REGS_MINB)
             }
         }
 
-        float ss[VPL];
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            float f[8];
-            unpack<bf16>(xv[i], f);
-            float a = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) a = fmaf(f[e], f[e], a);
-            ss[i] = a;
-        }
-        float r_row = 0.f;
-        if constexpr (ACROSS) {
-            float tot = 0.f;
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) tot += ss[i];
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
-            r_row = rsqrtf(tot * (1.f / (256.f * VPL)) + eps);
-        } else {
-#pragma unroll
-            for (int off = 8; off > 0; off >>= 1) {
-#pragma unroll
-                for (int i = 0; i < VPL; ++i) ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], off);
-            }
-        }
         float w[8];  // selects, not an indexed array (which would live in local memory)
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = isk ? fwk[e] : fwq[e];
@@ -182,18 +159,11 @@ __global__ void __launch_bounds__(SOL_QK_REGS_BLOCK, SOL_QK_REGS_MINB)
             dst = (isk ? k_out + n * ld_ko : q_out + n * ld_qo) + 8 * lane;
             slot_step = 256;
         }
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            float f[8], o[8];
-            unpack<bf16>(xv[i], f);
-            float r;
+        // slot i's 8 elements f, scaled by 1 / rms r and the weights, rotated and stored
+        auto emit = [&](int i, const float* f, float r) {
+            float o[8];
             if constexpr (ACROSS) {
-                r = r_row;
-                if (wrow) {
-                    unpack<bf16>(ld_cached(wrow + 256 * i + 8 * lane), w);
-                }
-            } else {
-                r = rsqrtf(ss[i] * (1.f / 128.f) + eps);
+                if (wrow) unpack<bf16>(ld_cached(wrow + 256 * i + 8 * lane), w);
             }
             if constexpr (HALF) {
                 float a[8];
@@ -218,6 +188,71 @@ __global__ void __launch_bounds__(SOL_QK_REGS_BLOCK, SOL_QK_REGS_MINB)
                 dst += slot_step;
             } else {
                 st_stream(dst + 256 * i, pack<bf16>(o));
+            }
+        };
+
+        if constexpr (ACROSS) {
+            // one norm over the whole row: every slot's sum first, then the output pass
+            float tot = 0.f;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                float f[8];
+                unpack<bf16>(xv[i], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) tot = fmaf(f[e], f[e], tot);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
+            const float r_row = rsqrtf(tot * (1.f / (256.f * VPL)) + eps);
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                float f[8];
+                unpack<bf16>(xv[i], f);
+                emit(i, f, r_row);
+            }
+        } else {
+            // per head vector: GS slots at a time -- widen once, sums of squares, GS
+            // independent half-warp trees, then normalise, rotate and store them
+            constexpr int GS = 4;
+            float kc[16];  // interleaved pairs: weights folded into the rotation once per row
+            if constexpr (!HALF) qk_coefs(w, cs, sn, kc);
+#pragma unroll
+            for (int i0 = 0; i0 < VPL; i0 += GS) {
+                float2 f[GS][4];
+                float ss[GS];
+#pragma unroll
+                for (int u = 0; u < GS; ++u) {
+                    ss[u] = 0.f;
+                    if (i0 + u < VPL) {
+                        unpack2<bf16>(xv[i0 + u], f[u]);
+                        ss[u] = qk_sumsq(f[u]);
+                    }
+                }
+#pragma unroll
+                for (int off = 8; off > 0; off >>= 1) {
+#pragma unroll
+                    for (int u = 0; u < GS; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
+                }
+#pragma unroll
+                for (int u = 0; u < GS; ++u) {
+                    if (i0 + u < VPL) {
+                        const float r = rsqrtf(ss[u] * (1.f / 128.f) + eps);
+                        if constexpr (HALF) {
+                            float ff[8];
+                            unpack<bf16>(xv[i0 + u], ff);
+                            emit(i0 + u, ff, r);
+                        } else {
+                            float o[8];
+                            qk_rotate(f[u], r, kc, o);
+                            if constexpr (STRIDED) {
+                                st_stream(dst, pack<bf16>(o));
+                                dst += slot_step;
+                            } else {
+                                st_stream(dst + 256 * (i0 + u), pack<bf16>(o));
+                            }
+                        }
+                    }
+                }
             }
         }
     }

@@ -66,6 +66,16 @@ cudaError_t launch_qk_regs(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_k
                            int64_t ld_q, int64_t ld_k, const void* wq, const void* wk, const int32_t* pos,
                            int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope, int64_t n_tokens,
                            int32_t n_heads, float eps, cudaStream_t s);
+// QK RMSNorm + 3D RoPE with one CTA per token, its q and k rows staged in shared memory by
+// bulk copies (k_qk_cta.cu): bf16, head_dim 128, an even number of heads up to 48, q and k
+// both given.
+bool qk_cta_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim, const void* q, const void* k, int64_t n_tokens);
+cudaError_t launch_qk_cta(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, const void* q, const void* k,
+                          int64_t ld_q, int64_t ld_k, const void* wq, const void* wk, const int32_t* pos,
+                          int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope, int64_t n_tokens,
+                          int32_t n_heads, float eps, cudaStream_t s);
+// Error flags of that kernel's bounded wait (bit 1); optionally cleared.  Synchronous.
+uint32_t qk_device_error(bool clear);
 // The same kernel for the convention variants (norm across heads, rotate-half pairs, strided
 // outputs): bf16, head_dim 128, a multiple of 8 heads up to 48.
 bool qk_regs_ex_fits(sol_dtype dt, bool half, int32_t n_heads, int32_t head_dim, const RopeDev& rope);
