@@ -9,14 +9,16 @@ dit_block_b200/block.py).  Default workload: the full-resolution 10 s grid, 61x4
 
 N > 1 is launched by torchrun, one rank per GPU; every rank processes its own copy of
 the workload (weak scaling, no collective on the data path) and the time is the max
-over ranks.  Rank 0 prints one JSON line.
+over ranks.  With --shard the ranks split one workload's tokens into contiguous ranges
+instead (strong scaling, still no collective on the data path).  Rank 0 prints one JSON
+line.
 
 value       algorithmic HBM bytes of all ranks' steps / device time (GB/s); every tensor
             element an op must read or write counts once (216,064 B per token per step).
-e2e         the same metric through the public host-buffer API (HostBlockPipeline): per
+e2e         the same metric through the C ABI's host-buffer call (sol_dit_block_host): per
             step, pinned host -> device copies of every input, the five launches,
             device -> host copies of every output, all inside the timed region, chunked
-            and overlapped across three streams.
+            and overlapped across three streams by the library.
 roofline    the SwiGLU launch (the largest byte mover): achieved GB/s from CUDA events
             around each launch in the timed steps, against the measured HBM copy peak.
 cpu_baseline / --impl reference
@@ -46,7 +48,8 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 SPEC_HBM_GBS = 8000.0
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_swiglu_fullres_10s.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_swiglu.json")
+PER_CONFIG = ("lowres", "fullres_5s", "fullres_10s", "packed_av")
 OPS = ("adaln_modulate", "dit_epilogue", "dit_prologue", "swiglu", "gated_residual")
 DOMINANT = "swiglu"
 
@@ -155,25 +158,20 @@ def source_digest() -> str:
 
 
 def ncu_traffic(n_tokens: int):
-    """DRAM bytes of one SwiGLU launch from the committed ncu summary, scaled to n_tokens;
-    None if absent or taken on different kernel source."""
+    """DRAM bytes of one SwiGLU launch over n_tokens tokens: the ncu capture committed in
+    profiles/traffic_swiglu.json (dram__bytes_read.sum + dram__bytes_write.sum of one launch
+    on a small case), scaled by tokens -- SwiGLU's traffic grows in proportion to the rows
+    it streams.  None if the file is absent or was taken on different kernel source."""
     try:
         with open(TRAFFIC_FILE) as f:
-            text = f.read()
-    except OSError:
+            t = json.load(f)
+    except (OSError, ValueError):
         return None
-    kv = {}
-    for line in text.splitlines():
-        line = line.strip().strip("`")
-        if line.startswith("- ") and ":" in line:
-            k, v = line[2:].split(":", 1)
-            kv[k.strip()] = v.strip()
     try:
-        if kv.get("kernel_source_sha256_16") != source_digest():
+        if t["kernel_source_sha256_16"] != source_digest():
             return None
-        per_token = float(kv["dram_bytes_per_token"])
-        return per_token * n_tokens
-    except (KeyError, ValueError):
+        return (float(t["dram_bytes_read"]) + float(t["dram_bytes_write"])) / float(t["tokens"]) * n_tokens
+    except (KeyError, ValueError, ZeroDivisionError):
         return None
 
 
@@ -305,7 +303,15 @@ def run_ours(args, w):
     build.build()
     sol.lib()
 
-    bufs = block.BlockBuffers.allocate(w, dev, n_tokens=args.tokens)
+    if args.shard:
+        # strong scaling: rank r takes its contiguous range of the workload's tokens
+        from dit_block_b200 import shard
+        n_total = w.n_tokens if args.tokens is None else min(args.tokens, w.n_tokens)
+        t0, t1 = shard.token_ranges(n_total, world)[rank]
+        bufs = shard.ShardBuffers(w, t0, t1, dev)
+    else:
+        bufs = block.BlockBuffers.allocate(w, dev, n_tokens=args.tokens)
+        n_total = bufs.n_tokens * world
     n = bufs.n_tokens
     bpt = bytes_per_token(w)
     step_bytes = sum(bpt.values()) * n
@@ -323,39 +329,35 @@ def run_ours(args, w):
     barrier()
     torch.cuda.synchronize(dev)
     clocks = ClockSampler(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(OPS) + 1)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.start()
-    start.record(stream)
-    for s in range(args.steps):
-        ev[s][0].record(stream)
-        for j, op in enumerate(OPS):
-            bufs.launch(op)
-            ev[s][j + 1].record(stream)
-    end.record(stream)
-    torch.cuda.synchronize(dev)
+    total_ms, op_times = time_passes(bufs, args.steps, stream)
     barrier()
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
-    total_ms = start.elapsed_time(end)
-    op_times = {op: [ev[s][j].elapsed_time(ev[s][j + 1]) for s in range(args.steps)] for j, op in enumerate(OPS)}
     per_op_ms = {op: sum(t) / len(t) for op, t in op_times.items()}
     total_ms, = max_over_ranks([total_ms], world, dev)
     ms_step = total_ms / args.steps
-    value = step_bytes * world * args.steps / (total_ms * 1e-3) / 1e9
+    all_bytes = sum(bpt.values()) * n_total  # every rank's tokens of one step
+    value = all_bytes * args.steps / (total_ms * 1e-3) / 1e9
+
+    peak, peak_kind = measured_peak()
+    headline = config_entry(w, n, total_ms, args.steps, op_times, peak)
 
     # ---- ops beyond the block pass, each timed alone on the same workload
-    next_ops = {} if args.no_next else time_next_ops(bufs, dev, args)
-    linear_ops = {} if (args.no_next or args.linear_tokens <= 0) else time_linear_ops(w, dev, args.linear_tokens)
+    extras = not args.shard
+    next_ops = {} if (args.no_next or not extras) else time_next_ops(bufs, dev, args)
+    linear_ops = {} if (args.no_next or args.linear_tokens <= 0 or not extras) else \
+        time_linear_ops(w, dev, args.linear_tokens)
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and extras:
         e2e = run_e2e(args, bufs, dev, world, step_bytes)
+    elif args.shard:
+        e2e = {"value": None, "unit": "GB/s", "error": "not measured for token shards (run without --shard)"}
 
     mix_ref = stream_mix_reference(n, w.d, dev)
 
-    peak, peak_kind = measured_peak()
     dom_ms = per_op_ms[DOMINANT]
     dom_bytes = bpt[DOMINANT] * n
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
@@ -364,18 +366,21 @@ def run_ours(args, w):
                    "ms_median": round(statistics.median(op_times[op]), 4), "ms_min": round(min(op_times[op]), 4),
                    "GB_s": round(bpt[op] * n / (per_op_ms[op] * 1e-3) / 1e9, 1),
                    "frac_of_measured_peak": round(bpt[op] * n / (per_op_ms[op] * 1e-3) / 1e9 / peak, 4),
+                   "frac_of_spec_peak": round(bpt[op] * n / (per_op_ms[op] * 1e-3) / 1e9 / SPEC_HBM_GBS, 4),
                    "bytes_per_token": bpt[op]} for op in OPS}
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(w),
-        "data": "synthetic",
-        "config": {"workload": w.name, "tokens": n, "grid": list(w.grid), "batch": w.batch,
+        "higher_is_better": True, "scaling": "strong" if args.shard else "weak", "vs_baseline": None,
+        "dtype": dtype_name(w), "data": "synthetic",
+        "config": {"workload": w.name, "tokens": n_total, "tokens_per_rank": n, "grid": list(w.grid),
+                   "batch": w.batch,
                    "d": w.d, "heads": f"{w.n_heads}x{w.head_dim}", "swiglu_inner": w.inner,
                    "bytes_per_token": sum(bpt.values()),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "parallelism": (f"token shards x{world}" if args.shard else f"replicas x{world}")
+                   if world > 1 else "single GPU",
                    "l2": "no flush: every op streams >= 2.5 GB, far above the 126 MB L2"},
-        "tokens_per_s": round(n * world * args.steps / (total_ms * 1e-3), 1),
+        "tokens_per_s": round(n_total * args.steps / (total_ms * 1e-3), 1),
         "frac_of_measured_hbm_peak": round(value / world / peak, 4),
         "frac_of_spec_hbm_peak": round(value / world / SPEC_HBM_GBS, 4),
         "per_op": per_op,
@@ -387,20 +392,90 @@ def run_ours(args, w):
                      "mix_reference": mix_ref,
                      "frac_of_torch_add_2r1w": round(achieved / mix_ref["torch_add_2r1w_GB_s"], 4)},
         "clocks": clk,
+        "per_config": None,
         "next_ops": next_ops,
         "linear_ops": linear_ops,
         "gpu_launches": len(OPS) * args.steps,
         "e2e": e2e,
     }
+    full_size = args.tokens is None or args.tokens >= w.n_tokens
+    bufs.close()
+    del bufs
+    torch.cuda.empty_cache()
+    if not args.no_per_config and full_size and w.dtype == torch.bfloat16 and not args.shard:
+        # every bf16 workload, one at a time; each rank times its own copy (the max over
+        # ranks is taken for the chain time)
+        pc = time_per_config(args, dev, peak, {w.name: headline})
+        for name, e in pc.items():
+            e["chain_ms"], = max_over_ranks([e["chain_ms"]], world, dev)
+        line["per_config"] = pc
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    bufs.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def time_passes(bufs, steps: int, stream):
+    """Device time of `steps` back-to-back passes (CUDA events on `stream`) and each
+    launch's own duration per pass (events between the launches)."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(OPS) + 1)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(steps):
+        ev[s][0].record(stream)
+        for j, op in enumerate(OPS):
+            bufs.launch(op)
+            ev[s][j + 1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    op_times = {op: [ev[s][j].elapsed_time(ev[s][j + 1]) for s in range(steps)] for j, op in enumerate(OPS)}
+    return start.elapsed_time(end), op_times
+
+
+def config_entry(w, n: int, total_ms: float, steps: int, op_times: dict, peak: float) -> dict:
+    """Chain and per-op throughput of one workload, as fractions of the measured copy peak
+    and of the 8 TB/s spec."""
+    bpt = bytes_per_token(w)
+    step_bytes = sum(bpt.values()) * n
+    ms = total_ms / steps
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    ops = {}
+    for op in OPS:
+        t = sum(op_times[op]) / len(op_times[op])
+        g = bpt[op] * n / (t * 1e-3) / 1e9
+        ops[op] = {"ms": round(t, 4), "ms_median": round(statistics.median(op_times[op]), 4),
+                   "GB_s": round(g, 1), "frac_of_measured_peak": round(g / peak, 4),
+                   "frac_of_spec_peak": round(g / SPEC_HBM_GBS, 4)}
+    return {"tokens": n, "steps": steps, "chain_ms": round(ms, 4), "GB_s": round(gbs, 1),
+            "tokens_per_s": round(n / (ms * 1e-3), 1), "frac_of_measured_peak": round(gbs / peak, 4),
+            "frac_of_spec_peak": round(gbs / SPEC_HBM_GBS, 4), "per_op": ops}
+
+
+def time_per_config(args, dev, peak: float, done: dict) -> dict:
+    """Every bf16 workload timed like the headline (one at a time: its buffers are
+    allocated, timed over args.config_steps passes and freed before the next)."""
+    from dit_block_b200 import block
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for name in PER_CONFIG:
+        if name in done:
+            out[name] = done[name]
+            continue
+        w = workloads.WORKLOADS[name]
+        bufs = block.BlockBuffers.allocate(w, dev)
+        for _ in range(args.warmup):
+            bufs.step()
+        torch.cuda.synchronize(dev)
+        total, op_times = time_passes(bufs, args.config_steps, stream)
+        out[name] = config_entry(w, bufs.n_tokens, total, args.config_steps, op_times, peak)
+        bufs.close()
+        del bufs
+        torch.cuda.empty_cache()
+    return out
 
 
 def stream_mix_reference(n: int, d: int, dev) -> dict:
@@ -622,9 +697,10 @@ def run_linear_only(args, w):
 
 
 def run_e2e(args, bufs, dev, world, step_bytes):
-    """The pass through the public host-buffer API (dit_block_b200.pipeline): pinned host
-    inputs in, five launches per chunk, pinned host outputs back; every copy is inside
-    the timed region and overlapped with compute across three streams."""
+    """The pass through the C ABI's host-buffer call (sol_dit_block_host, driven by
+    dit_block_b200.pipeline): pinned host inputs in, five launches per chunk, pinned host
+    outputs back; every copy is inside the timed region and overlapped with compute across
+    three streams by the library."""
     from dit_block_b200 import pipeline
     w, i = bufs.w, bufs.inp
     n = bufs.n_tokens
@@ -669,7 +745,7 @@ def run_e2e(args, bufs, dev, world, step_bytes):
     del host_in, host_out, host_mod
     return {"value": round(val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": args.e2e_steps, "ms_per_step": round(ms / args.e2e_steps, 2),
-            "api": "dit_block_b200.pipeline.HostBlockPipeline.run (pinned host buffers)",
+            "api": "sol_dit_block_host (C ABI; pinned host buffers, via dit_block_b200.pipeline.HostBlockPipeline)",
             "chunk_tokens": args.e2e_chunk}
 
 
@@ -692,6 +768,12 @@ def main(argv=None):
     p.add_argument("--linear-only", action="store_true",
                    help="time only the fused linear layers (prints their own JSON line)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--shard", action="store_true",
+                   help="strong scaling: split the workload's tokens into one contiguous range per rank "
+                        "(no collective on the data path) instead of a full replica per rank")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="skip timing the other bf16 workloads (per_config)")
+    p.add_argument("--config-steps", type=int, default=20, help="passes timed per workload in per_config")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-tokens", type=int, default=256, help="oracle token sample per reference step")
     args = p.parse_args(argv)
