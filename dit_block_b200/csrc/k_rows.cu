@@ -584,6 +584,8 @@ cudaError_t launch_adaln_rows(sol_dtype dt, void* x_out, int64_t ld_xo, void* h,
                               int64_t ld_mod, const ModSel& sel, int64_t n_tokens, int64_t d,
                               float eps, cudaStream_t s)
 {
+    if (!y && ld_x == ld_h && adaln_stage_fits(dt, d, n_tokens))
+        return launch_adaln_stage(h, x, ld_h, shift, scale, ld_mod, sel, n_tokens, d, eps, s);
     if (!y && SOL_ADALN_FOUR_WARPS && ld_x == ld_h && prologue_regs_fits(dt, d))
         return launch_prologue_regs(nullptr, h, x, nullptr, nullptr, shift, scale, ld_h, ld_mod, sel, n_tokens, d,
                                     eps, s);

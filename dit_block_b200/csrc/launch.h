@@ -164,6 +164,14 @@ cudaError_t launch_prologue_regs(void* x_out, void* h, const void* x, const void
                                  const void* shift, const void* scale, int64_t ld, int64_t ld_mod, const ModSel& sel,
                                  int64_t n_tokens, int64_t d, float eps, cudaStream_t s);
 
+// AdaLN with one CTA per row staged in shared memory by a bulk copy (k_rows_stage.cu): bf16,
+// d a multiple of 1024 up to 6144, h and x with one row stride.
+bool adaln_stage_fits(sol_dtype dt, int64_t d, int64_t n_tokens);
+cudaError_t launch_adaln_stage(void* h, const void* x, int64_t ld, const void* shift, const void* scale, int64_t ld_mod,
+                               const ModSel& sel, int64_t n_tokens, int64_t d, float eps, cudaStream_t s);
+// Error flags of that kernel's bounded wait (bit 0); optionally cleared.  Synchronous.
+uint32_t rows_stage_device_error(bool clear);
+
 // Whether a row of `vpr` 16-byte vectors fits the register-resident AdaLN kernel.
 bool adaln_row_fits(int64_t vpr);
 
