@@ -10,10 +10,10 @@
 // CTAs retire new ones start their copies while the others compute and store: 6.80 TB/s
 // (128-thread CTAs: 6.73).
 //
-// Per CTA (T threads): thread 0 starts the two copies on one mbarrier; threads 0..63
-// compute the token's position and the (cos, sin) of the 64 rotary pairs of a head vector
-// into shared memory; then every thread takes vectors c = t + T u of the token's q | k
-// vectors.  T is a multiple of the 16 vectors of a head vector, so thread t owns the same
+// Per CTA (T threads): thread 0 starts the two copies on one mbarrier; thread p < 64
+// computes the token's position, pair p's (cos, sin) and its rotation coefficients with the
+// q and k weights folded in (qk_coefs), into shared memory; then every thread takes vectors
+// c = t + T u of the token's q | k vectors.  T is a multiple of the 16 vectors of a head vector, so thread t owns the same
 // 8-element slice (8 * (t % 16) ..) of every head vector it touches and each head vector's
 // sum of squares is one half-warp shuffle tree.  The per-slot arithmetic is qk_math.cuh's
 // (bit-identical to k_qk_regs.cu's and k_qk_pool.cu's).  The wait on the copies is bounded;
@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(kQkCtaThreads)
              int32_t grid_H, int32_t grid_W, uint32_t tokens_per_sample, RopeDev rope, int32_t n_heads, float eps)
 {
     extern __shared__ __align__(128) uint4 rows[];  // [q row | k row], 2 * qv vectors
-    __shared__ float2 csn[64];                     // (cos, sin) of pair j of a head vector
+    __shared__ float4 kcs[2][4][16];  // rotation coefficients of pair 4 j + m at [q or k][m][j]
     __shared__ __align__(8) uint64_t bar;
     const uint32_t n = blockIdx.x;  // < 2^31 (checked on the host)
     const int t = threadIdx.x;
@@ -63,7 +63,8 @@ __global__ void __launch_bounds__(kQkCtaThreads)
         bulk_g2s(smem_u32(rows + qv), k + (int64_t)n * ld_k, row_bytes, smem_u32(&bar));
     }
     if (t < 64) {
-        // the token's (t, h, w) position, then pair t's axis and angle
+        // the token's (t, h, w) position, then pair t's angle and its rotation coefficients
+        // with the q and k weights folded in (qk_coefs of qk_math.cuh, per pair)
         uint32_t p0, p1, p2;
         if (pos) {
             p0 = (uint32_t)min(max(__ldg(pos + 3 * (int64_t)n + 0), 0), rope.max[0] - 1);
@@ -81,9 +82,20 @@ __global__ void __launch_bounds__(kQkCtaThreads)
         const float2* tp = t < h0    ? rope.tab[0] + (int64_t)p0 * rope.half[0] + t
                            : t < h01 ? rope.tab[1] + (int64_t)p1 * rope.half[1] + (t - h0)
                                      : rope.tab[2] + (int64_t)p2 * rope.half[2] + (t - h01);
-        csn[t] = __ldg(tp);
+        const float2 a = __ldg(tp);
+#pragma unroll
+        for (int isk = 0; isk < 2; ++isk) {
+            const bf16* wrow = isk ? wk : wq;
+            float w0 = 1.f, w1 = 1.f;
+            if (wrow) {
+                const __nv_bfloat162 wp = __ldg(reinterpret_cast<const __nv_bfloat162*>(wrow) + t);
+                w0 = __low2float(wp);
+                w1 = __high2float(wp);
+            }
+            kcs[isk][t & 3][t >> 2] = make_float4(w0 * a.x, w1 * a.y, w0 * a.y, w1 * a.x);
+        }
     }
-    __syncthreads();  // the barrier is initialised and the angles are in place
+    __syncthreads();  // the barrier is initialised and the coefficients are in place
 
     // every thread waits (bounded) for the copies; the give-up decision is the CTA's
     const bool landed = mbar_wait_bounded(smem_u32(&bar), 0, kQkWaitLimit);
@@ -95,14 +107,7 @@ __global__ void __launch_bounds__(kQkCtaThreads)
         return;
     }
 
-    const int sub = t & 15;  // element slice 8 * sub .. + 7 of every head vector
-    float cs[4], sn[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const float2 v = csn[4 * sub + m];
-        cs[m] = v.x;
-        sn[m] = v.y;
-    }
+    const int sub = t & 15;  // element slice 8 * sub .. + 7 of every head vector: pairs 4 sub ..
     // sums of squares and the half-warp trees of every slot (slots past the row are zero,
     // and uniform over each warp: T u + t and 2 * qv are multiples of 32)
     float ss[U];
@@ -126,16 +131,15 @@ __global__ void __launch_bounds__(kQkCtaThreads)
         const int c = t + kQkCtaThreads * u;
         if (c >= 2 * qv) continue;
         const bool isk = c >= qv;
-        const bf16* wrow = isk ? wk : wq;  // this thread's slice of the weights (an L1 hit)
-        float w[8];
-        if (wrow) {
-            unpack<bf16>(ld_cached(wrow + 8 * sub), w);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = 1.f;
-        }
         float kc[16];
-        qk_coefs(w, cs, sn, kc);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float4 v = kcs[isk ? 1 : 0][m][sub];  // lanes read consecutive 16-byte words
+            kc[4 * m + 0] = v.x;
+            kc[4 * m + 1] = v.y;
+            kc[4 * m + 2] = v.z;
+            kc[4 * m + 3] = v.w;
+        }
         float2 f[4];
         unpack2<bf16>(rows[c], f);
         float o[8];
@@ -159,8 +163,13 @@ cudaError_t launch_u(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, con
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (smem > 48 * 1024 && attr_set[dev].load(std::memory_order_acquire) < smem) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr_set[dev].load(std::memory_order_acquire) < smem) {
+        // the whole of the SM's unified L1 / shared memory as shared memory, so that the
+        // thread limit (8 CTAs of 256), not the carveout, bounds the resident CTAs
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e == cudaSuccess && smem > 48 * 1024)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr_set[dev].store(smem, std::memory_order_release);
     }

@@ -333,7 +333,7 @@ def test_full_shape_adaln_qkv_rope(oracle_mod):
     ws = sol.adaln_workspace(m, 3 * w.hd, w.d)
     with sol.Rope3D(w.rope_dims, w.theta, w.max_pos) as rope:
         sol.adaln_qkv_rope(qkv, x, W, rope, shift, scale, workspace=ws, n_heads=w.n_heads, wq=wq, wk=wk,
-                           grid=w.grid, strategy=strategy, eps=w.eps)
+                           grid=w.grid, eps=w.eps)
         torch.cuda.synchronize()
     Wh = to_oracle(W)
     want, pre, h = oracle_mod.adaln_qkv_rope(
