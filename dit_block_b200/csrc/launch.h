@@ -172,6 +172,9 @@ cudaError_t launch_adaln_stage(void* h, const void* x, int64_t ld, const void* s
 // Error flags of that kernel's bounded wait (bit 0); optionally cleared.  Synchronous.
 uint32_t rows_stage_device_error(bool clear);
 
+// Error flags of sol_selftest_wait_timeout (bit 2); optionally cleared.  Synchronous.
+uint32_t selftest_device_error(bool clear);
+
 // Whether a row of `vpr` 16-byte vectors fits the register-resident AdaLN kernel.
 bool adaln_row_fits(int64_t vpr);
 

@@ -205,9 +205,10 @@ sol_status sol_device_errors(uint32_t* flags, int32_t clear)
     const uint32_t rows = sol::rows_device_error(clear != 0);
     const uint32_t staged = sol::rows_stage_device_error(clear != 0);
     const uint32_t qk = sol::qk_device_error(clear != 0);
-    CHECK(rows != 0xffffffffu && staged != 0xffffffffu && qk != 0xffffffffu, SOL_ERR_CUDA,
+    const uint32_t self = sol::selftest_device_error(clear != 0);
+    CHECK(rows != 0xffffffffu && staged != 0xffffffffu && qk != 0xffffffffu && self != 0xffffffffu, SOL_ERR_CUDA,
           "reading the device error flags failed");
-    *flags = rows | staged | qk | ((sol::gemm_device_error(clear != 0) & 0xffu) << 8);
+    *flags = rows | staged | qk | self | ((sol::gemm_device_error(clear != 0) & 0xffu) << 8);
     return SOL_OK;
 }
 

@@ -70,6 +70,7 @@ SIGNATURES = {
     "sol_last_error": ([], ctypes.c_char_p),
     "sol_abi_version": ([], _I32),
     "sol_device_errors": ([ctypes.POINTER(ctypes.c_uint32), _I32], _E),
+    "sol_selftest_wait_timeout": ([_I32, _P], _E),
     "sol_adaln_modulate": ([_P, _I64, _P, _I64, _P, _P, _I64, ModSel, _I64, _I64, _F, _E, _P], _E),
     "sol_gated_residual": ([_P, _I64, _P, _I64, _P, _I64, _P, _I64, ModSel, _I64, _I64, _E, _P], _E),
     "sol_gated_residual_cache_diff": ([_P, _I64, _P, _I64, _P, _I64, _P, _I64, ModSel, _P, _I64, _I32,
@@ -149,6 +150,12 @@ def device_errors(clear: bool = False) -> int:
     f = ctypes.c_uint32(0)
     _check(lib().sol_device_errors(ctypes.byref(f), int(clear)), "sol_device_errors")
     return int(f.value)
+
+
+def selftest_wait_timeout(polls: int = 8, stream=None):
+    """Run the bounded-wait failure path on purpose (sol_selftest_wait_timeout): afterwards
+    device_errors() reports bit 2 until cleared."""
+    _check(lib().sol_selftest_wait_timeout(int(polls), _stream(stream)), "sol_selftest_wait_timeout")
 
 
 # ------------------------------------------------------------------------- marshalling

@@ -93,12 +93,21 @@ int32_t sol_abi_version(void);
 /* Error flags raised on the current device by libsol kernels since the last clear:
  * bit 0 = an AdaLN / prologue kernel's bounded wait on its own asynchronous copy gave up;
  * bit 1 = a QK RMSNorm + RoPE kernel's bounded wait on its own asynchronous copy gave up;
+ * bit 2 = sol_selftest_wait_timeout's wait gave up (as it is meant to);
  * bits 8..15 = a linear-layer kernel (sol_linear*, sol_adaln_*) gave up a bounded wait
  * in its copy / MMA / epilogue / transform pipeline.  The kernel recorded it, drained
  * its own copies and MMAs, stopped early and left its outputs incomplete.  Synchronises
  * the current device first; clear != 0 resets the flags.  Never set in normal
  * operation. */
 sol_status sol_device_errors(uint32_t* flags, int32_t clear);
+
+/* Diagnostic of the failure path above, safe to run at any time: launches one CTA on
+ * `stream` that waits, with the same bounded wait the kernels use, on an mbarrier phase
+ * that can never complete (it expects two arrivals and gets one); after `polls` polls
+ * (1..1000, each suspending for at most about a millisecond) the wait gives up, the CTA
+ * records bit 2 of the device error flags and returns.  Nothing faults and the context stays
+ * usable: a caller can check that sol_device_errors reports the bit, clear it and go on. */
+sol_status sol_selftest_wait_timeout(int32_t polls, sol_stream_t stream);
 
 /* AdaLN modulation [XHH-QA, STM-GAN]:
  *     mu = mean_i x_i,  var = mean_i (x_i - mu)^2  (biased, two passes),

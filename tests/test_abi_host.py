@@ -28,7 +28,7 @@ def last(L):
 
 def test_exports_every_declared_symbol(L):
     names = sol.header_functions()
-    assert len(names) == 26
+    assert len(names) == 27
     for n in names:
         assert hasattr(L, n), f"libsol.so does not export {n}"
         assert n in sol.SIGNATURES, f"binding has no signature for {n}"
@@ -270,3 +270,9 @@ def test_block_host_validation(L):
     assert "rope" in last(L)
     d.rope, d.n_tokens = FAKE << 2, 0
     assert L.sol_dit_block_host(ref, None, 0, 16, 2, s1, s2, s3) == sol.OK
+
+
+def test_selftest_validation(L):
+    for bad in (0, -3, 1001):
+        assert L.sol_selftest_wait_timeout(bad, None) == sol.ERR_INVALID_ARGUMENT
+        assert "polls" in last(L)
