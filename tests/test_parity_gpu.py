@@ -119,8 +119,10 @@ QK_CASES = [  # dtype, head_dim, dims, n_heads, grid (T,H,W), samples
     (torch.float32, 128, (32, 48, 48), 2, (2, 4, 4), 1),
     (torch.float32, 64, (16, 24, 24), 3, (5, 2, 3), 2),
     (torch.float32, 32, (8, 12, 12), 7, (3, 3, 3), 1),
-    (BF, 128, (32, 48, 48), 48, (2, 3, 4), 2),   # register kernel, 24 slots per lane (the most)
-    (BF, 128, (32, 48, 48), 2, (3, 3, 3), 1),    # register kernel, 1 slot per lane
+    (BF, 128, (32, 48, 48), 48, (2, 3, 4), 2),   # CTA-per-token kernel at its widest (6 vectors a thread)
+    (BF, 128, (32, 48, 48), 2, (3, 3, 3), 1),    # CTA-per-token kernel, 2 of its 8 warps busy
+    (BF, 128, (32, 48, 48), 6, (2, 3, 5), 2),    # 6 of 8 warps busy
+    (BF, 128, (16, 56, 56), 24, (3, 2, 2), 1),   # 3 vectors a thread, another split
 ]
 
 
@@ -153,6 +155,33 @@ def test_qk_rmsnorm_rope3d_and_epilogue(orc, dtype, head_dim, dims, Hh, grid, B)
     # the separate-output call and the in-place epilogue agree bit for bit
     assert torch.equal(epi[:, :hd], qo) and torch.equal(epi[:, hd:2 * hd], ko)
     rope.close()
+
+
+def test_qk_separate_strided_tensors_and_guard_bands(orc):
+    """q and k in separate tensors with different row strides, written out of place into
+    outputs with other strides: every row matches the oracle and nothing between or around
+    the output rows is written."""
+    n, Hh = 101, 40
+    hd = Hh * 128
+    qb, q = _guarded(n, hd, hd + 64, BF)
+    kb, k = _guarded(n, hd, hd + 128, BF)
+    q.copy_(randn((n, hd), BF, 31, std=1.5))
+    k.copy_(randn((n, hd), BF, 32, std=1.5))
+    qob, qo = _guarded(n, hd, hd + 256, BF)
+    kob, ko = _guarded(n, hd, hd + 8, BF)
+    wq = randn((128,), BF, 33, std=0.02, mean=1.0)
+    wk = randn((128,), BF, 34, std=0.02, mean=1.0)
+    grid = (3, 5, 7)
+    with sol.Rope3D((32, 48, 48), 10000.0, (4, 5, 7)) as rope:
+        sol.qk_rmsnorm_rope3d(qo, ko, q, k, rope, n_heads=Hh, head_dim=128, wq=wq, wk=wk, grid=grid,
+                              tokens_per_sample=0)
+        torch.cuda.synchronize()
+    want_q, want_k = orc.qk_rmsnorm_rope3d(to_oracle(q.contiguous()), to_oracle(k.contiguous()), to_oracle(wq),
+                                          to_oracle(wk), n_heads=Hh, head_dim=128, grid=grid)
+    assert_close(to_f64(qo.contiguous()), want_q, BF, "strided q")
+    assert_close(to_f64(ko.contiguous()), want_k, BF, "strided k")
+    assert _guards_intact(qob, n, hd, hd + 256) and _guards_intact(kob, n, hd, hd + 8)
+    assert _guards_intact(qb, n, hd, hd + 64) and _guards_intact(kb, n, hd, hd + 128)
 
 
 def test_qk_explicit_positions_packed_and_clamped(orc):
