@@ -6,19 +6,20 @@
 // bound by the bytes each SM keeps in flight.  Rows held in registers cap that at what the
 // register file spares (a persistent warp per row, k_qk_regs.cu: 8 warps x 10 KB per SM,
 // 6.22 TB/s at 245,952 tokens x 40 heads); here a token's 20 KB waits in shared memory, so
-// 8 resident CTAs of 256 threads (40 registers each) keep 160 KB in flight per SM, and as
-// CTAs retire new ones start their copies while the others compute and store: 6.80 TB/s
-// (128-thread CTAs: 6.73).
+// 8 resident CTAs of 256 threads (32 registers each) keep 160 KB in flight per SM, and as
+// CTAs retire new ones start their copies while the others compute and store: 6.80-6.91
+// TB/s (128-thread CTAs: 6.73).
 //
 // Per CTA (T threads): thread 0 starts the two copies on one mbarrier; thread p < 64
 // computes the token's position, pair p's (cos, sin) and its rotation coefficients with the
 // q and k weights folded in (qk_coefs), into shared memory; then every thread takes vectors
-// c = t + T u of the token's q | k vectors.  T is a multiple of the 16 vectors of a head vector, so thread t owns the same
-// 8-element slice (8 * (t % 16) ..) of every head vector it touches and each head vector's
-// sum of squares is one half-warp shuffle tree.  The per-slot arithmetic is qk_math.cuh's
-// (bit-identical to k_qk_regs.cu's and k_qk_pool.cu's).  The wait on the copies is bounded;
-// on give-up the CTA records bit 1 of the device error flags, waits once more (bounded) for
-// its copies and returns.
+// c = t + T u of the token's q | k vectors.  T is a multiple of the 16 vectors of a head
+// vector, so thread t owns the same 8-element slice (8 * (t % 16) ..) of every head vector
+// it touches and each head vector's sum of squares is one half-warp shuffle tree.  The
+// per-slot arithmetic of the default convention is qk_math.cuh's (bit-identical to
+// k_qk_regs.cu's and k_qk_pool.cu's).  The wait on the copies is bounded; on give-up the
+// CTA records bit 1 of the device error flags, waits once more (bounded) for its copies and
+// returns.
 #include <algorithm>
 #include <atomic>
 

@@ -242,7 +242,10 @@ EX_CASES = [  # dtype, head_dim, dims, n_heads, grid, samples
     (BF, 64, (16, 16, 32), 5, (4, 3, 3), 3),
     (torch.float32, 128, (32, 48, 48), 3, (2, 4, 4), 1),
     (torch.float32, 32, (8, 8, 16), 7, (3, 3, 3), 2),
-    (BF, 128, (32, 48, 48), 8, (2, 3, 5), 3),   # register kernel, 4 slots per lane
+    (BF, 128, (32, 48, 48), 8, (2, 3, 5), 3),   # 8 heads: rotate-half across heads on the register kernel
+    (BF, 128, (32, 48, 48), 48, (2, 3, 4), 2),  # CTA-per-token kernel at its widest (6 slots a thread)
+    (BF, 128, (32, 48, 48), 2, (3, 3, 3), 1),   # CTA-per-token kernel, one slot, 2 of 8 warps busy
+    (BF, 128, (16, 48, 64), 6, (2, 3, 5), 2),   # another split: rotate-half chunk edges move
 ]
 
 
