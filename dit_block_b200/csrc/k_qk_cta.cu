@@ -5,21 +5,32 @@
 // Why: the op is an in-place stream of 4 bytes per element with little arithmetic, so it is
 // bound by the bytes each SM keeps in flight.  Rows held in registers cap that at what the
 // register file spares (a persistent warp per row, k_qk_regs.cu: 8 warps x 10 KB per SM,
-// 6.22 TB/s at 245,952 tokens x 40 heads); here a token's 20 KB waits in shared memory, so
-// 8 resident CTAs of 256 threads (32 registers each) keep 160 KB in flight per SM, and as
-// CTAs retire new ones start their copies while the others compute and store: 6.80-6.91
-// TB/s (128-thread CTAs: 6.73).
+// 6.22 TB/s at 245,952 tokens x 40 heads); here a token's 20 KB waits in shared memory, and
+// as CTAs retire new ones start their copies while the others compute and store.
 //
-// Per CTA (T threads): thread 0 starts the two copies on one mbarrier; thread p < 64
-// computes the token's position, pair p's (cos, sin) and its rotation coefficients with the
-// q and k weights folded in (qk_coefs), into shared memory; then every thread takes vectors
-// c = t + T u of the token's q | k vectors.  T is a multiple of the 16 vectors of a head
-// vector, so thread t owns the same 8-element slice (8 * (t % 16) ..) of every head vector
-// it touches and each head vector's sum of squares is one half-warp shuffle tree.  The
-// per-slot arithmetic of the default convention is qk_math.cuh's (bit-identical to
-// k_qk_regs.cu's and k_qk_pool.cu's).  The wait on the copies is bounded; on give-up the
-// CTA records bit 1 of the device error flags, waits once more (bounded) for its copies and
-// returns.
+// Two kernels:
+//   k_qk_head    RMS per head vector (the plain op and every per-head convention): 128
+//                threads, 9 resident CTAs per SM (shared memory bounds them: 9 x 22.6 KB =
+//                180 KB in flight), 46-56 registers.  The q row is done, then the k row; a
+//                thread takes vectors t + 128 u of the row and keeps the row's 16 rotation
+//                coefficients of its slice in registers for all of them.  6.8 TB/s alone and
+//                inside the block pass, also at the 1.5 GHz the power cap holds in long runs
+//                (an earlier 256-thread form that read its coefficients from shared memory
+//                per vector streamed 6.9 alone but 6.0 there: its shared-memory pipe ran
+//                near full, and its compute phase, which holds the CTA's rows, followed the
+//                clock).
+//   k_qk_across  one RMS over the whole q (k) row: 256 threads, vectors t + 256 u of the
+//                [q | k] row, one CTA reduction for the two row sums.
+//
+// Per CTA: thread 0 starts the two copies on one mbarrier; thread p < 64 computes the
+// token's position, pair p's (cos, sin) and, per head, its rotation coefficients with the q
+// and k weights folded in (qk_coefs), into shared memory.  The thread counts are multiples
+// of the 16 vectors of a head vector, so thread t owns the same 8-element slice
+// (8 * (t % 16) ..) of every head vector it touches and each head vector's sum of squares
+// is one half-warp shuffle tree.  The per-slot arithmetic of the default convention is
+// qk_math.cuh's (bit-identical to k_qk_regs.cu's and k_qk_pool.cu's).  The wait on the
+// copies is bounded; on give-up the CTA records bit 1 of the device error flags, waits once
+// more (bounded) for its copies and returns.
 #include <algorithm>
 #include <atomic>
 
@@ -29,16 +40,14 @@
 #include "launch.h"
 #include "qk_math.cuh"
 
-#ifndef SOL_QK_CTA_THREADS
-#define SOL_QK_CTA_THREADS 256
-#endif
-
 namespace sol {
 
 static __device__ unsigned int g_qk_error;
 
 namespace {
-constexpr int kQkCtaThreads = SOL_QK_CTA_THREADS;
+constexpr int kHeadThreads = 128;        // k_qk_head
+constexpr int kHeadCtas = 9;             // resident k_qk_head CTAs per SM (launch bounds)
+constexpr int kAcrossThreads = 256;      // k_qk_across
 constexpr uint32_t kQkWaitLimit = 4096;  // polls of <= ~1 ms each
 
 __device__ __forceinline__ void st_stream8(void* p, uint32_t x, uint32_t y)
@@ -47,149 +56,108 @@ __device__ __forceinline__ void st_stream8(void* p, uint32_t x, uint32_t y)
 }
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Thread 0: start the bulk copies of the token's q and k rows (16 * qv bytes each).
+__device__ __forceinline__ void start_row_copies(uint4* rows, uint64_t* bar, const bf16* q, const bf16* k,
+                                                 int64_t ld_q, int64_t ld_k, uint32_t n, int qv)
+{
+    const uint32_t row_bytes = 16u * (uint32_t)qv;
+    mbar_init(smem_u32(bar), 1);
+    mbar_fence_init();
+    mbar_arrive_expect_tx(smem_u32(bar), 2 * row_bytes);
+    bulk_g2s(smem_u32(rows), q + (int64_t)n * ld_q, row_bytes, smem_u32(bar));
+    bulk_g2s(smem_u32(rows + qv), k + (int64_t)n * ld_k, row_bytes, smem_u32(bar));
+}
+
+// Pair p's (cos, sin) for token n: its axis chunk, the token's position on that axis (from
+// pos, clamped to the table, or from the token's place in its sample's T x H x W grid) and
+// the pair's index j within the chunk.
+__device__ __forceinline__ float2 pair_angle(int p, uint32_t n, const int32_t* __restrict__ pos, int32_t grid_H,
+                                             int32_t grid_W, uint32_t tokens_per_sample, RopeDev rope)
+{
+    uint32_t p0, p1, p2;
+    if (pos) {
+        p0 = (uint32_t)min(max(__ldg(pos + 3 * (int64_t)n + 0), 0), rope.max[0] - 1);
+        p1 = (uint32_t)min(max(__ldg(pos + 3 * (int64_t)n + 1), 0), rope.max[1] - 1);
+        p2 = (uint32_t)min(max(__ldg(pos + 3 * (int64_t)n + 2), 0), rope.max[2] - 1);
+    } else {
+        const uint32_t nl = tokens_per_sample ? n % tokens_per_sample : n;
+        const uint32_t hw = (uint32_t)grid_H * (uint32_t)grid_W;
+        p0 = nl / hw;
+        const uint32_t r = nl - p0 * hw;
+        p1 = r / (uint32_t)grid_W;
+        p2 = r - p1 * (uint32_t)grid_W;
+    }
+    const int h0 = rope.half[0], h01 = rope.half[0] + rope.half[1];
+    const float2* tp = p < h0    ? rope.tab[0] + (int64_t)p0 * rope.half[0] + p
+                       : p < h01 ? rope.tab[1] + (int64_t)p1 * rope.half[1] + (p - h0)
+                                 : rope.tab[2] + (int64_t)p2 * rope.half[2] + (p - h01);
+    return __ldg(tp);
+}
+
+// Every thread waits (bounded) for the copies; the give-up decision is the CTA's.  Returns
+// false (after recording the error and draining the copies) when the CTA must exit.
+__device__ __forceinline__ bool rows_landed(uint64_t* bar)
+{
+    const bool landed = mbar_wait_bounded(smem_u32(bar), 0, kQkWaitLimit);
+    if (__syncthreads_or(!landed)) {
+        if (threadIdx.x == 0) {
+            atomicOr(&g_qk_error, 2u);
+            mbar_wait_bounded(smem_u32(bar), 0, kQkWaitLimit);  // the copies must land before exit
+        }
+        return false;
+    }
+    return true;
+}
 }  // namespace
 
-// Convention variants (sol_qk_rmsnorm_rope3d_ex) in the same kernel:
-//   HALF     rotate-half pairs (element j of an axis chunk with element j + D_c / 2) in place
-//            of interleaved ones, per head.  Pair p of a head vector has the angle of
-//            interleaved pair p (index j within its axis chunk) and its two elements D_c / 2
-//            apart; with chunk halves that are multiples of 4, thread `sub` takes pairs
-//            4 sub .. 4 sub + 3: 4 consecutive first elements and their 4 partners, two
-//            8-byte pieces of the staged row, written back as two 8-byte pieces.  The pair
-//            coefficients (weights folded in) and the arithmetic are the interleaved ones.
-//   ACROSS   one RMS over the whole q (k) row (interleaved pairs), weights [n_heads * 128]
-//            laid out like the row: the slot sums meet in a CTA reduction (one barrier); the
-//            weights differ per head, so they are read per slot (through L1), and the staged
-//            table holds the bare (cos, sin).
-//   STRIDED  outputs at (sample, token, head) element strides, e.g. [sample, head, token, dim].
-// The default (per head, interleaved, token-major) is the plain op's path exactly.
-template <int U, bool ACROSS, bool HALF, bool STRIDED>
-__global__ void __launch_bounds__(kQkCtaThreads, 2048 / kQkCtaThreads)
-    k_qk_cta(bf16* q_out, bf16* k_out, int64_t ld_qo, int64_t ld_ko, QkOutStrides os, const bf16* q, const bf16* k,
-             int64_t ld_q, int64_t ld_k, const bf16* __restrict__ wq, const bf16* __restrict__ wk,
-             const int32_t* __restrict__ pos, int32_t grid_H, int32_t grid_W, uint32_t tokens_per_sample, RopeDev rope,
-             int32_t n_heads, float eps)
+// RMS per head vector.  HALF: rotate-half pairs (element j of an axis chunk with element
+// j + D_c / 2) in place of interleaved ones.  Pair p of a head vector has the angle of
+// interleaved pair p (index j within its axis chunk) and its two elements D_c / 2 apart, so
+// the pair coefficients (weights folded in) and the arithmetic are the interleaved ones;
+// with chunk halves that are multiples of 4, thread `sub` takes pairs 4 sub .. 4 sub + 3: 4
+// consecutive first elements and their 4 partners, two 8-byte pieces of the staged row,
+// written back as two 8-byte pieces.  STRIDED: outputs at (sample, token, head) element
+// strides, e.g. [sample, head, token, dim].  UQ = vectors per thread and row.
+template <int UQ, bool HALF, bool STRIDED>
+__global__ void __launch_bounds__(kHeadThreads, kHeadCtas)
+    k_qk_head(bf16* q_out, bf16* k_out, int64_t ld_qo, int64_t ld_ko, QkOutStrides os, const bf16* q, const bf16* k,
+              int64_t ld_q, int64_t ld_k, const bf16* __restrict__ wq, const bf16* __restrict__ wk,
+              const int32_t* __restrict__ pos, int32_t grid_H, int32_t grid_W, uint32_t tokens_per_sample,
+              RopeDev rope, int32_t n_heads, float eps)
 {
-    static_assert(!(ACROSS && HALF), "rotate-half across heads runs on the row-in-registers kernel");
     extern __shared__ __align__(128) uint4 rows[];  // [q row | k row], 2 * qv vectors
-    // per head: rotation coefficients of pair 4 j + m at [q or k][m][j], with the q, k
-    // weights folded in; across heads: (cos, sin) of pair 4 j + m at [0][m][j].xy
+    // rotation coefficients of pair 4 j + m at [q or k][m][j], weights folded in
     __shared__ float4 kcs[2][4][16];
-    __shared__ float red[2][kQkCtaThreads / 32];
     __shared__ __align__(8) uint64_t bar;
     const uint32_t n = blockIdx.x;  // < 2^31 (checked on the host)
     const int t = threadIdx.x;
     const int qv = 16 * n_heads;    // 16-byte vectors of the q row (and of the k row)
-    const uint32_t row_bytes = 16u * (uint32_t)qv;
 
-    if (t == 0) {
-        mbar_init(smem_u32(&bar), 1);
-        mbar_fence_init();
-        mbar_arrive_expect_tx(smem_u32(&bar), 2 * row_bytes);
-        bulk_g2s(smem_u32(rows), q + (int64_t)n * ld_q, row_bytes, smem_u32(&bar));
-        bulk_g2s(smem_u32(rows + qv), k + (int64_t)n * ld_k, row_bytes, smem_u32(&bar));
-    }
+    if (t == 0) start_row_copies(rows, &bar, q, k, ld_q, ld_k, n, qv);
     const int h0 = rope.half[0], h01 = rope.half[0] + rope.half[1];
     if (t < 64) {
-        // the token's (t, h, w) position, then pair t's angle: index j within its axis chunk
-        uint32_t p0, p1, p2;
-        if (pos) {
-            p0 = (uint32_t)min(max(__ldg(pos + 3 * (int64_t)n + 0), 0), rope.max[0] - 1);
-            p1 = (uint32_t)min(max(__ldg(pos + 3 * (int64_t)n + 1), 0), rope.max[1] - 1);
-            p2 = (uint32_t)min(max(__ldg(pos + 3 * (int64_t)n + 2), 0), rope.max[2] - 1);
-        } else {
-            const uint32_t nl = tokens_per_sample ? n % tokens_per_sample : n;
-            const uint32_t hw = (uint32_t)grid_H * (uint32_t)grid_W;
-            p0 = nl / hw;
-            const uint32_t r = nl - p0 * hw;
-            p1 = r / (uint32_t)grid_W;
-            p2 = r - p1 * (uint32_t)grid_W;
+        const float2 a = pair_angle(t, n, pos, grid_H, grid_W, tokens_per_sample, rope);
+        // the pair's two elements: (2 t, 2 t + 1), or rotate-half (e, e + D_c / 2)
+        int ea = 2 * t, eb = 2 * t + 1;
+        if constexpr (HALF) {
+            const int hc = t < h0 ? rope.half[0] : (t < h01 ? rope.half[1] : rope.half[2]);
+            ea = t < h0 ? t : (t < h01 ? t + h0 : t + h01);  // chunk start 2 (pairs before) + j
+            eb = ea + hc;
         }
-        const float2* tp = t < h0    ? rope.tab[0] + (int64_t)p0 * rope.half[0] + t
-                           : t < h01 ? rope.tab[1] + (int64_t)p1 * rope.half[1] + (t - h0)
-                                     : rope.tab[2] + (int64_t)p2 * rope.half[2] + (t - h01);
-        const float2 a = __ldg(tp);
-        if constexpr (ACROSS) {
-            kcs[0][t & 3][t >> 2] = make_float4(a.x, a.y, 0.f, 0.f);
-        } else {
-            // the pair's two elements: (2 t, 2 t + 1), or rotate-half (e, e + D_c / 2)
-            int ea = 2 * t, eb = 2 * t + 1;
-            if constexpr (HALF) {
-                const int hc = t < h0 ? rope.half[0] : (t < h01 ? rope.half[1] : rope.half[2]);
-                ea = t < h0 ? t : (t < h01 ? t + h0 : t + h01);  // chunk start 2 (pairs before) + j
-                eb = ea + hc;
-            }
-            // the q and k weights folded in (qk_coefs of qk_math.cuh, per pair)
+        // the q and k weights folded in (qk_coefs of qk_math.cuh, per pair)
 #pragma unroll
-            for (int isk = 0; isk < 2; ++isk) {
-                const bf16* wrow = isk ? wk : wq;
-                const float wa = wrow ? __bfloat162float(wrow[ea]) : 1.f;
-                const float wb = wrow ? __bfloat162float(wrow[eb]) : 1.f;
-                kcs[isk][t & 3][t >> 2] = make_float4(wa * a.x, wb * a.y, wa * a.y, wb * a.x);
-            }
+        for (int isk = 0; isk < 2; ++isk) {
+            const bf16* wrow = isk ? wk : wq;
+            const float wa = wrow ? __bfloat162float(wrow[ea]) : 1.f;
+            const float wb = wrow ? __bfloat162float(wrow[eb]) : 1.f;
+            kcs[isk][t & 3][t >> 2] = make_float4(wa * a.x, wb * a.y, wa * a.y, wb * a.x);
         }
     }
     __syncthreads();  // the barrier is initialised and the coefficients are in place
-
-    // every thread waits (bounded) for the copies; the give-up decision is the CTA's
-    const bool landed = mbar_wait_bounded(smem_u32(&bar), 0, kQkWaitLimit);
-    if (__syncthreads_or(!landed)) {
-        if (t == 0) {
-            atomicOr(&g_qk_error, 2u);
-            mbar_wait_bounded(smem_u32(&bar), 0, kQkWaitLimit);  // the copies must land before exit
-        }
-        return;
-    }
+    if (!rows_landed(&bar)) return;
 
     const int sub = t & 15;  // pairs 4 sub .. 4 sub + 3 of every head vector the thread touches
-    // sums of squares; per head: the half-warp trees of every slot (slots past the row are
-    // zero, and uniform over each warp: T u + t and 2 * qv are multiples of 32); across
-    // heads: one CTA reduction per row
-    float ss[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        ss[u] = 0.f;
-        const int c = t + kQkCtaThreads * u;
-        if (c < 2 * qv) {
-            float2 f[4];
-            unpack2<bf16>(rows[c], f);
-            ss[u] = qk_sumsq(f);
-        }
-    }
-    float r_row[2] = {0.f, 0.f};
-    if constexpr (ACROSS) {
-        float sq = 0.f, sk = 0.f;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int c = t + kQkCtaThreads * u;
-            if (c < qv)
-                sq += ss[u];
-            else
-                sk += ss[u];
-        }
-        sq = warp_sum(sq);
-        sk = warp_sum(sk);
-        if ((t & 31) == 0) {
-            red[0][t >> 5] = sq;
-            red[1][t >> 5] = sk;
-        }
-        __syncthreads();
-        float tq = 0.f, tk = 0.f;
-#pragma unroll
-        for (int w = 0; w < kQkCtaThreads / 32; ++w) {
-            tq += red[0][w];
-            tk += red[1][w];
-        }
-        const float inv = 1.f / (128.f * (float)n_heads);
-        r_row[0] = rsqrtf(tq * inv + eps);
-        r_row[1] = rsqrtf(tk * inv + eps);
-    } else {
-#pragma unroll
-        for (int off = 8; off > 0; off >>= 1) {
-#pragma unroll
-            for (int u = 0; u < U; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
-        }
-    }
     // rotate-half: this thread's first elements e0 .. e0 + 3 and their partners at + hp
     int e0 = 8 * sub, hp = 0;
     if constexpr (HALF) {
@@ -203,41 +171,45 @@ __global__ void __launch_bounds__(kQkCtaThreads, 2048 / kQkCtaThreads)
         const uint32_t sample = tokens_per_sample ? n / tokens_per_sample : 0;
         obase = (int64_t)sample * os.sample + (int64_t)(n - sample * tokens_per_sample) * os.token;
     }
-    // (across heads no slot sum is needed any more: one slot at a time keeps registers low)
-#pragma unroll(ACROSS ? 1 : U)
-    for (int u = 0; u < U; ++u) {
-        const int c = t + kQkCtaThreads * u;
-        if (c >= 2 * qv) continue;
-        const int isk = c >= qv ? 1 : 0;
-        const int v = c - isk * qv;  // vector within the row: head v / 16, slice v % 16
-        const int hh = v >> 4;
-        float o[8];
-        if constexpr (ACROSS) {
-            // weights per slot, then the bare rotation
-            const float r = isk ? r_row[1] : r_row[0];
-            const bf16* wrow = isk ? wk : wq;
-            float w[8];
-            if (wrow) {
-                unpack<bf16>(ld_cached(wrow + 8 * v), w);
-            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) w[e] = 1.f;
+    for (int isk = 0; isk < 2; ++isk) {
+        const uint4* row = rows + isk * qv;
+        // sums of squares of the head vectors: the half-warp tree of every slot (slots past
+        // the row are zero, and uniform over each warp: qv is a multiple of 32)
+        float ss[UQ];
+#pragma unroll
+        for (int u = 0; u < UQ; ++u) {
+            ss[u] = 0.f;
+            const int c = t + kHeadThreads * u;
+            if (c < qv) {
+                float2 f[4];
+                unpack2<bf16>(row[c], f);
+                ss[u] = qk_sumsq(f);
             }
-            float f[8], a[8];
-            unpack<bf16>(rows[c], f);
+        }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a[e] = f[e] * r * w[e];
+        for (int off = 8; off > 0; off >>= 1) {
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 cssn = kcs[0][m][sub];
-                o[2 * m] = a[2 * m] * cssn.x - a[2 * m + 1] * cssn.y;
-                o[2 * m + 1] = a[2 * m] * cssn.y + a[2 * m + 1] * cssn.x;
-            }
-        } else {
-            // the 4 pairs as (first, second) element, rotated with the folded coefficients
+            for (int u = 0; u < UQ; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
+        }
+        float kc[16];  // this slice's coefficients, for every head vector of the row
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float4 x = kcs[isk][m][sub];  // lanes read consecutive 16-byte words
+            kc[4 * m + 0] = x.x;
+            kc[4 * m + 1] = x.y;
+            kc[4 * m + 2] = x.z;
+            kc[4 * m + 3] = x.w;
+        }
+        bf16* const out = isk ? k_out : q_out;
+#pragma unroll
+        for (int u = 0; u < UQ; ++u) {
+            const int c = t + kHeadThreads * u;
+            if (c >= qv) continue;
+            // the 4 pairs as (first, second) element
             float2 f[4];
             if constexpr (HALF) {
-                const bf16* hrow = reinterpret_cast<const bf16*>(rows + (c - sub));  // the head vector
+                const bf16* hrow = reinterpret_cast<const bf16*>(row + (c - sub));  // the head vector
                 const uint2 a = *reinterpret_cast<const uint2*>(hrow + e0);
                 const uint2 b = *reinterpret_cast<const uint2*>(hrow + e0 + hp);
                 f[0] = make_float2(bf_lo(a.x), bf_lo(b.x));
@@ -245,109 +217,228 @@ __global__ void __launch_bounds__(kQkCtaThreads, 2048 / kQkCtaThreads)
                 f[2] = make_float2(bf_lo(a.y), bf_lo(b.y));
                 f[3] = make_float2(bf_hi(a.y), bf_hi(b.y));
             } else {
-                unpack2<bf16>(rows[c], f);
+                unpack2<bf16>(row[c], f);
             }
-            float kc[16];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 x = kcs[isk][m][sub];  // lanes read consecutive 16-byte words
-                kc[4 * m + 0] = x.x;
-                kc[4 * m + 1] = x.y;
-                kc[4 * m + 2] = x.z;
-                kc[4 * m + 3] = x.w;
-            }
+            float o[8];
             qk_rotate(f, rsqrtf(ss[u] * (1.f / 128.f) + eps), kc, o);
-        }
-        bf16* dst;  // the head vector's output
-        if constexpr (STRIDED) {
-            dst = (isk ? k_out : q_out) + obase + (int64_t)hh * os.head;
-        } else {
-            dst = isk ? k_out + (int64_t)n * ld_ko + 128 * hh : q_out + (int64_t)n * ld_qo + 128 * hh;
-        }
-        if constexpr (HALF) {
-            st_stream8(dst + e0, pack2_bf16(o[0], o[2]), pack2_bf16(o[4], o[6]));
-            st_stream8(dst + e0 + hp, pack2_bf16(o[1], o[3]), pack2_bf16(o[5], o[7]));
-        } else {
-            st_stream(dst + 8 * sub, pack<bf16>(o));
+            bf16* dst;  // the head vector's output
+            if constexpr (STRIDED)
+                dst = out + obase + (int64_t)(c >> 4) * os.head;
+            else
+                dst = out + (int64_t)n * (isk ? ld_ko : ld_qo) + 8 * (c - sub);
+            if constexpr (HALF) {
+                st_stream8(dst + e0, pack2_bf16(o[0], o[2]), pack2_bf16(o[4], o[6]));
+                st_stream8(dst + e0 + hp, pack2_bf16(o[1], o[3]), pack2_bf16(o[5], o[7]));
+            } else {
+                st_stream(dst + 8 * sub, pack<bf16>(o));
+            }
         }
     }
-    (void)r_row;
     (void)hp;
+}
+
+// One RMS over the whole q (k) row (interleaved pairs), weights [n_heads * 128] laid out
+// like the row: the slot sums meet in a CTA reduction (one barrier); the weights differ per
+// head, so they are read per slot (through L1) and multiply the elements before a rotation
+// with the bare (cos, sin).  U = vectors per thread of the [q | k] row.
+template <int U, bool STRIDED>
+__global__ void __launch_bounds__(kAcrossThreads, 2048 / kAcrossThreads)
+    k_qk_across(bf16* q_out, bf16* k_out, int64_t ld_qo, int64_t ld_ko, QkOutStrides os, const bf16* q,
+                const bf16* k, int64_t ld_q, int64_t ld_k, const bf16* __restrict__ wq, const bf16* __restrict__ wk,
+                const int32_t* __restrict__ pos, int32_t grid_H, int32_t grid_W, uint32_t tokens_per_sample,
+                RopeDev rope, int32_t n_heads, float eps)
+{
+    extern __shared__ __align__(128) uint4 rows[];  // [q row | k row], 2 * qv vectors
+    __shared__ float2 cs[4][16];                     // (cos, sin) of pair 4 j + m at [m][j]
+    __shared__ float red[2][kAcrossThreads / 32];
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t n = blockIdx.x;
+    const int t = threadIdx.x;
+    const int qv = 16 * n_heads;
+
+    if (t == 0) start_row_copies(rows, &bar, q, k, ld_q, ld_k, n, qv);
+    if (t < 64) cs[t & 3][t >> 2] = pair_angle(t, n, pos, grid_H, grid_W, tokens_per_sample, rope);
+    __syncthreads();  // the barrier is initialised and the angles are in place
+    if (!rows_landed(&bar)) return;
+
+    const int sub = t & 15;
+    float sq = 0.f, sk = 0.f;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int c = t + kAcrossThreads * u;
+        if (c < 2 * qv) {  // uniform over each warp
+            float2 f[4];
+            unpack2<bf16>(rows[c], f);
+            const float s = qk_sumsq(f);
+            if (c < qv)
+                sq += s;
+            else
+                sk += s;
+        }
+    }
+    sq = warp_sum(sq);
+    sk = warp_sum(sk);
+    if ((t & 31) == 0) {
+        red[0][t >> 5] = sq;
+        red[1][t >> 5] = sk;
+    }
+    __syncthreads();
+    float tq = 0.f, tk = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAcrossThreads / 32; ++w) {
+        tq += red[0][w];
+        tk += red[1][w];
+    }
+    const float inv = 1.f / (128.f * (float)n_heads);
+    const float rq = rsqrtf(tq * inv + eps), rk = rsqrtf(tk * inv + eps);
+    int64_t obase = 0;
+    if constexpr (STRIDED) {
+        const uint32_t sample = tokens_per_sample ? n / tokens_per_sample : 0;
+        obase = (int64_t)sample * os.sample + (int64_t)(n - sample * tokens_per_sample) * os.token;
+    }
+    // one slot at a time (a rolled loop) keeps the registers low
+#pragma unroll 1
+    for (int u = 0; u < U; ++u) {
+        const int c = t + kAcrossThreads * u;
+        if (c >= 2 * qv) continue;
+        const int isk = c >= qv ? 1 : 0;
+        const int v = c - isk * qv;  // vector within the row: head v / 16, slice v % 16
+        const float r = isk ? rk : rq;
+        const bf16* wrow = isk ? wk : wq;
+        float w[8];
+        if (wrow) {
+            unpack<bf16>(ld_cached(wrow + 8 * v), w);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = 1.f;
+        }
+        float f[8], a[8], o[8];
+        unpack<bf16>(rows[c], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a[e] = f[e] * r * w[e];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float2 x = cs[m][sub];
+            o[2 * m] = a[2 * m] * x.x - a[2 * m + 1] * x.y;
+            o[2 * m + 1] = a[2 * m] * x.y + a[2 * m + 1] * x.x;
+        }
+        bf16* dst;
+        if constexpr (STRIDED)
+            dst = (isk ? k_out : q_out) + obase + (int64_t)(v >> 4) * os.head + 8 * sub;
+        else
+            dst = isk ? k_out + (int64_t)n * ld_ko + 8 * v : q_out + (int64_t)n * ld_qo + 8 * v;
+        st_stream(dst, pack<bf16>(o));
+    }
 }
 
 namespace {
 
-template <int U, bool ACROSS, bool HALF, bool STRIDED>
-cudaError_t launch_u(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, const QkOutStrides& os, const void* q,
-                     const void* k, int64_t ld_q, int64_t ld_k, const void* wq, const void* wk, const int32_t* pos,
-                     int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope, int64_t n_tokens,
-                     int32_t n_heads, float eps, cudaStream_t s)
+// Launch arguments shared by both kernels.
+struct QkLaunch {
+    void* q_out;
+    void* k_out;
+    int64_t ld_qo, ld_ko;
+    QkOutStrides os;
+    const void* q;
+    const void* k;
+    int64_t ld_q, ld_k;
+    const void* wq;
+    const void* wk;
+    const int32_t* pos;
+    int32_t grid_H, grid_W;
+    int64_t tps;
+    RopeDev rope;
+    int64_t n_tokens;
+    int32_t n_heads;
+    float eps;
+};
+
+// Set the kernel's shared-memory attributes once per device (for the largest row seen),
+// then launch one CTA per token.  carveout_pct < 0: all of the unified L1 / shared memory as
+// shared memory.
+template <typename Kern>
+cudaError_t launch_rows(Kern kern, int threads, int carveout_pct, const QkLaunch& a, std::atomic<size_t>* attr_set,
+                        cudaStream_t s)
 {
-    auto kern = k_qk_cta<U, ACROSS, HALF, STRIDED>;
-    const size_t smem = (size_t)2 * 16 * 16 * n_heads;
-    static std::atomic<size_t> attr_set[64];  // per device: the larger dynamic shared memory it allows
+    const size_t smem = (size_t)2 * 16 * 16 * a.n_heads;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (attr_set[dev].load(std::memory_order_acquire) < smem) {
-        // enough of the SM's unified L1 / shared memory as shared memory that the thread
-        // limit (8 CTAs of 256), not the carveout, bounds the resident CTAs: all of it, or
-        // for the across-heads variants, which read their weights per slot through L1, just
-        // enough (per CTA: the row, ~2 KB of static arrays and the 1 KB the system keeps)
-        int carveout = (int)cudaSharedmemCarveoutMaxShared;
-        if (ACROSS) {
-            const size_t need = (smem + 3 * 1024) * (2048 / kQkCtaThreads);
-            carveout = (int)std::min<size_t>(100, (need * 100 + 228 * 1024 - 1) / (228 * 1024));
-        }
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, carveout);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 carveout_pct < 0 ? (int)cudaSharedmemCarveoutMaxShared : carveout_pct);
         if (e == cudaSuccess && smem > 48 * 1024)
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr_set[dev].store(smem, std::memory_order_release);
     }
-    kern<<<(unsigned)n_tokens, kQkCtaThreads, smem, s>>>(
-        static_cast<bf16*>(q_out), static_cast<bf16*>(k_out), ld_qo, ld_ko, os, static_cast<const bf16*>(q),
-        static_cast<const bf16*>(k), ld_q, ld_k, static_cast<const bf16*>(wq), static_cast<const bf16*>(wk), pos,
-        grid_H, grid_W, (uint32_t)tps, rope, n_heads, eps);
+    kern<<<(unsigned)a.n_tokens, threads, smem, s>>>(
+        static_cast<bf16*>(a.q_out), static_cast<bf16*>(a.k_out), a.ld_qo, a.ld_ko, a.os,
+        static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), a.ld_q, a.ld_k, static_cast<const bf16*>(a.wq),
+        static_cast<const bf16*>(a.wk), a.pos, a.grid_H, a.grid_W, (uint32_t)a.tps, a.rope, a.n_heads, a.eps);
     return cudaGetLastError();
 }
 
-template <bool ACROSS, bool HALF, bool STRIDED>
-cudaError_t dispatch_u(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, const QkOutStrides& os, const void* q,
-                       const void* k, int64_t ld_q, int64_t ld_k, const void* wq, const void* wk, const int32_t* pos,
-                       int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope, int64_t n_tokens,
-                       int32_t n_heads, float eps, cudaStream_t s)
+template <int UQ, bool HALF, bool STRIDED> cudaError_t launch_head(const QkLaunch& a, cudaStream_t s)
 {
-    switch ((32 * n_heads + kQkCtaThreads - 1) / kQkCtaThreads) {
-#define SOL_QK_CTA_U(u)                                                                                        \
-    case u:                                                                                                    \
-        return launch_u<u, ACROSS, HALF, STRIDED>(q_out, k_out, ld_qo, ld_ko, os, q, k, ld_q, ld_k, wq, wk, pos, \
-                                                  grid_H, grid_W, tps, rope, n_tokens, n_heads, eps, s);
-        SOL_QK_CTA_U(1) SOL_QK_CTA_U(2) SOL_QK_CTA_U(3) SOL_QK_CTA_U(4) SOL_QK_CTA_U(5) SOL_QK_CTA_U(6)
-#undef SOL_QK_CTA_U
+    // 9 CTAs of 22.6 KB need all of the shared part
+    static std::atomic<size_t> attr_set[64];  // per device: the larger dynamic shared memory it allows
+    return launch_rows(k_qk_head<UQ, HALF, STRIDED>, kHeadThreads, -1, a, attr_set, s);
+}
+
+template <int U, bool STRIDED> cudaError_t launch_across(const QkLaunch& a, cudaStream_t s)
+{
+    // just enough shared memory for 8 CTAs (per CTA: the rows, ~0.6 KB of static arrays and
+    // the 1 KB the system keeps): the rest stays L1 for the weights read per slot
+    static std::atomic<size_t> attr_set[64];
+    const size_t need = ((size_t)2 * 16 * 16 * a.n_heads + 2 * 1024) * (2048 / kAcrossThreads);
+    const int pct = (int)std::min<size_t>(100, (need * 100 + 228 * 1024 - 1) / (228 * 1024));
+    return launch_rows(k_qk_across<U, STRIDED>, kAcrossThreads, pct, a, attr_set, s);
+}
+
+template <bool HALF, bool STRIDED> cudaError_t dispatch_head(const QkLaunch& a, cudaStream_t s)
+{
+    switch ((16 * a.n_heads + kHeadThreads - 1) / kHeadThreads) {
+    case 1: return launch_head<1, HALF, STRIDED>(a, s);
+    case 2: return launch_head<2, HALF, STRIDED>(a, s);
+    case 3: return launch_head<3, HALF, STRIDED>(a, s);
+    case 4: return launch_head<4, HALF, STRIDED>(a, s);
+    case 5: return launch_head<5, HALF, STRIDED>(a, s);
+    case 6: return launch_head<6, HALF, STRIDED>(a, s);
     }
     return cudaErrorInvalidValue;
 }
 
-}  // namespace
-
-bool qk_cta_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim, const void* q, const void* k, int64_t n_tokens)
+template <bool STRIDED> cudaError_t dispatch_across(const QkLaunch& a, cudaStream_t s)
 {
-    // the copies need 16-byte aligned rows (the API's rule); 256 threads cover up to 48 heads
-    // with 6 vectors each
-    return dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads >= 2 && n_heads % 2 == 0 && n_heads <= 48 && q && k &&
-           n_tokens < ((int64_t)1 << 31);
+    switch ((32 * a.n_heads + kAcrossThreads - 1) / kAcrossThreads) {
+    case 1: return launch_across<1, STRIDED>(a, s);
+    case 2: return launch_across<2, STRIDED>(a, s);
+    case 3: return launch_across<3, STRIDED>(a, s);
+    case 4: return launch_across<4, STRIDED>(a, s);
+    case 5: return launch_across<5, STRIDED>(a, s);
+    case 6: return launch_across<6, STRIDED>(a, s);
+    }
+    return cudaErrorInvalidValue;
 }
 
-namespace {
 // token-major outputs (head stride 128, samples back to back) take the unstrided stores
 bool out_token_major(const QkOutStrides& os, int64_t tps, int64_t n_tokens)
 {
     const int64_t tps_eff = tps > 0 ? tps : n_tokens;
     return os.head == 128 && (os.sample == tps_eff * os.token || n_tokens <= tps_eff);
 }
+
 }  // namespace
+
+bool qk_cta_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim, const void* q, const void* k, int64_t n_tokens)
+{
+    // the copies need 16-byte aligned rows (the API's rule); the thread counts cover up to 48
+    // heads with 6 vectors a thread and row (k_qk_head) or [q | k] row (k_qk_across)
+    return dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads >= 2 && n_heads % 2 == 0 && n_heads <= 48 && q && k &&
+           n_tokens < ((int64_t)1 << 31);
+}
 
 bool qk_cta_ex_fits(sol_dtype dt, bool across, bool half, int32_t n_heads, int32_t head_dim,
                     const void* q, const void* k, int64_t n_tokens, int64_t tps, const RopeDev& rope)
@@ -370,9 +461,9 @@ cudaError_t launch_qk_cta(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko
 {
     if (n_tokens == 0) return cudaSuccess;
     if (tps >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
-    const QkOutStrides os{0, 0, 0};  // unused: token-major outputs
-    return dispatch_u<false, false, false>(q_out, k_out, ld_qo, ld_ko, os, q, k, ld_q, ld_k, wq, wk, pos, grid_H,
-                                           grid_W, tps, rope, n_tokens, n_heads, eps, s);
+    const QkLaunch a{q_out, k_out, ld_qo, ld_ko, QkOutStrides{0, 0, 0}, q, k, ld_q, ld_k, wq, wk, pos,
+                     grid_H, grid_W, tps, rope, n_tokens, n_heads, eps};
+    return dispatch_head<false, false>(a, s);
 }
 
 cudaError_t launch_qk_cta_ex(bool across, bool half, void* q_out, void* k_out, const QkOutStrides& os, const void* q,
@@ -382,18 +473,13 @@ cudaError_t launch_qk_cta_ex(bool across, bool half, void* q_out, void* k_out, c
 {
     if (n_tokens == 0) return cudaSuccess;
     if (half && across) return cudaErrorInvalidValue;  // outside qk_cta_ex_fits
+    if (tps >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const bool token_major = out_token_major(os, tps, n_tokens);
-    const int64_t ld_o = os.token;
-#define SOL_QK_CTA_EX_ARGS q_out, k_out, ld_o, ld_o, os, q, k, ld_q, ld_k, wq, wk, pos, grid_H, grid_W, tps, rope, n_tokens, n_heads, eps, s
-    if (token_major) {
-        if (half) return dispatch_u<false, true, false>(SOL_QK_CTA_EX_ARGS);
-        return across ? dispatch_u<true, false, false>(SOL_QK_CTA_EX_ARGS)
-                      : dispatch_u<false, false, false>(SOL_QK_CTA_EX_ARGS);
-    }
-    if (half) return dispatch_u<false, true, true>(SOL_QK_CTA_EX_ARGS);
-    return across ? dispatch_u<true, false, true>(SOL_QK_CTA_EX_ARGS)
-                  : dispatch_u<false, false, true>(SOL_QK_CTA_EX_ARGS);
-#undef SOL_QK_CTA_EX_ARGS
+    const QkLaunch a{q_out, k_out, os.token, os.token, os, q, k, ld_q, ld_k, wq, wk, pos,
+                     grid_H, grid_W, tps, rope, n_tokens, n_heads, eps};
+    if (across) return token_major ? dispatch_across<false>(a, s) : dispatch_across<true>(a, s);
+    if (half) return token_major ? dispatch_head<true, false>(a, s) : dispatch_head<true, true>(a, s);
+    return token_major ? dispatch_head<false, false>(a, s) : dispatch_head<false, true>(a, s);
 }
 
 uint32_t qk_device_error(bool clear)
