@@ -8,24 +8,20 @@
 // 6.22 TB/s at 245,952 tokens x 40 heads); here a token's 20 KB waits in shared memory, and
 // as CTAs retire new ones start their copies while the others compute and store.
 //
-// Two kernels:
-//   k_qk_head    RMS per head vector (the plain op and every per-head convention): 128
-//                threads, 9 resident CTAs per SM (shared memory bounds them: 9 x 22.6 KB =
-//                180 KB in flight), 46-56 registers.  The q row is done, then the k row; a
-//                thread takes vectors t + 128 u of the row and keeps the row's 16 rotation
-//                coefficients of its slice in registers for all of them.  6.8 TB/s alone and
-//                inside the block pass, also at the 1.5 GHz the power cap holds in long runs
-//                (an earlier 256-thread form that read its coefficients from shared memory
-//                per vector streamed 6.9 alone but 6.0 there: its shared-memory pipe ran
-//                near full, and its compute phase, which holds the CTA's rows, followed the
-//                clock).
-//   k_qk_across  one RMS over the whole q (k) row: 256 threads, vectors t + 256 u of the
-//                [q | k] row, one CTA reduction for the two row sums.
+// k_qk_head (the plain op and every convention of sol_qk_rmsnorm_rope3d_ex): 128 threads, 9
+// resident CTAs per SM (shared memory bounds them: 9 x 22.6 KB = 180 KB in flight), 48-56
+// registers.  The q row is done, then the k row; a thread takes vectors t + 128 u of the row
+// and keeps the row's 16 rotation coefficients of its slice in registers for all of them.
+// 6.8-6.9 TB/s alone and inside the block pass, also at
+// the 1.5 GHz the power cap holds in long runs (an earlier 256-thread form that read its
+// coefficients from shared memory per vector streamed 6.9 alone but 6.0 there: its
+// shared-memory pipe ran near full, and its compute phase, which holds the CTA's rows,
+// followed the clock).
 //
 // Per CTA: thread 0 starts the two copies on one mbarrier; thread p < 64 computes the
 // token's position, pair p's (cos, sin) and, per head, its rotation coefficients with the q
-// and k weights folded in (qk_coefs), into shared memory.  The thread counts are multiples
-// of the 16 vectors of a head vector, so thread t owns the same 8-element slice
+// and k weights folded in (qk_coefs), into shared memory.  128 is a multiple of the 16
+// vectors of a head vector, so thread t owns the same 8-element slice
 // (8 * (t % 16) ..) of every head vector it touches and each head vector's sum of squares
 // is one half-warp shuffle tree.  The per-slot arithmetic of the default convention is
 // qk_math.cuh's (bit-identical to k_qk_regs.cu's and k_qk_pool.cu's).  The wait on the
@@ -47,7 +43,6 @@ static __device__ unsigned int g_qk_error;
 namespace {
 constexpr int kHeadThreads = 128;        // k_qk_head
 constexpr int kHeadCtas = 9;             // resident k_qk_head CTAs per SM (launch bounds)
-constexpr int kAcrossThreads = 256;      // k_qk_across
 constexpr uint32_t kQkWaitLimit = 4096;  // polls of <= ~1 ms each
 
 __device__ __forceinline__ void st_stream8(void* p, uint32_t x, uint32_t y)
@@ -111,15 +106,21 @@ __device__ __forceinline__ bool rows_landed(uint64_t* bar)
 }
 }  // namespace
 
-// RMS per head vector.  HALF: rotate-half pairs (element j of an axis chunk with element
-// j + D_c / 2) in place of interleaved ones.  Pair p of a head vector has the angle of
-// interleaved pair p (index j within its axis chunk) and its two elements D_c / 2 apart, so
-// the pair coefficients (weights folded in) and the arithmetic are the interleaved ones;
-// with chunk halves that are multiples of 4, thread `sub` takes pairs 4 sub .. 4 sub + 3: 4
-// consecutive first elements and their 4 partners, two 8-byte pieces of the staged row,
-// written back as two 8-byte pieces.  STRIDED: outputs at (sample, token, head) element
-// strides, e.g. [sample, head, token, dim].  UQ = vectors per thread and row.
-template <int UQ, bool HALF, bool STRIDED>
+// UQ = vectors per thread and row.  The default (per head, interleaved pairs, token-major
+// rows) is the plain op.
+//   ACROSS   one RMS over the whole q (k) row, weights [n_heads * 128] laid out like the
+//            row: the thread sums of the two rows meet in one CTA reduction (one barrier);
+//            the weights differ per head, so each vector's are read (through L1) and
+//            multiply its elements before a rotation with the bare (cos, sin).
+//   HALF     rotate-half pairs (element j of an axis chunk with element j + D_c / 2) in
+//            place of interleaved ones.  Pair p of a head vector has the angle of interleaved
+//            pair p (index j within its axis chunk) and its two elements D_c / 2 apart, so
+//            the pair coefficients and the arithmetic are the interleaved ones; with chunk
+//            halves that are multiples of 4, thread `sub` takes pairs 4 sub .. 4 sub + 3: 4
+//            consecutive first elements and their 4 partners, two 8-byte pieces of the
+//            staged row, written back as two 8-byte pieces.
+//   STRIDED  outputs at (sample, token, head) element strides, e.g. [sample, head, token, dim].
+template <int UQ, bool ACROSS, bool HALF, bool STRIDED>
 __global__ void __launch_bounds__(kHeadThreads, kHeadCtas)
     k_qk_head(bf16* q_out, bf16* k_out, int64_t ld_qo, int64_t ld_ko, QkOutStrides os, const bf16* q, const bf16* k,
               int64_t ld_q, int64_t ld_k, const bf16* __restrict__ wq, const bf16* __restrict__ wk,
@@ -127,8 +128,10 @@ __global__ void __launch_bounds__(kHeadThreads, kHeadCtas)
               RopeDev rope, int32_t n_heads, float eps)
 {
     extern __shared__ __align__(128) uint4 rows[];  // [q row | k row], 2 * qv vectors
-    // rotation coefficients of pair 4 j + m at [q or k][m][j], weights folded in
+    // rotation coefficients of pair 4 j + m at [q or k][m][j], weights folded in; across
+    // heads [0][m][j], without weights
     __shared__ float4 kcs[2][4][16];
+    __shared__ float red[2][kHeadThreads / 32];
     __shared__ __align__(8) uint64_t bar;
     const uint32_t n = blockIdx.x;  // < 2^31 (checked on the host)
     const int t = threadIdx.x;
@@ -136,7 +139,10 @@ __global__ void __launch_bounds__(kHeadThreads, kHeadCtas)
 
     if (t == 0) start_row_copies(rows, &bar, q, k, ld_q, ld_k, n, qv);
     const int h0 = rope.half[0], h01 = rope.half[0] + rope.half[1];
-    if (t < 64) {
+    if (ACROSS && t < 64) {
+        const float2 a = pair_angle(t, n, pos, grid_H, grid_W, tokens_per_sample, rope);
+        kcs[0][t & 3][t >> 2] = make_float4(a.x, a.y, a.y, a.x);
+    } else if (t < 64) {
         const float2 a = pair_angle(t, n, pos, grid_H, grid_W, tokens_per_sample, rope);
         // the pair's two elements: (2 t, 2 t + 1), or rotate-half (e, e + D_c / 2)
         int ea = 2 * t, eb = 2 * t + 1;
@@ -171,6 +177,36 @@ __global__ void __launch_bounds__(kHeadThreads, kHeadCtas)
         const uint32_t sample = tokens_per_sample ? n / tokens_per_sample : 0;
         obase = (int64_t)sample * os.sample + (int64_t)(n - sample * tokens_per_sample) * os.token;
     }
+    float r_row[2] = {0.f, 0.f};
+    if constexpr (ACROSS) {
+        float sr[2] = {0.f, 0.f};
+#pragma unroll
+        for (int isk = 0; isk < 2; ++isk) {
+#pragma unroll
+            for (int u = 0; u < UQ; ++u) {
+                const int c = t + kHeadThreads * u;
+                if (c < qv) {
+                    float2 f[4];
+                    unpack2<bf16>(rows[isk * qv + c], f);
+                    sr[isk] += qk_sumsq(f);
+                }
+            }
+            sr[isk] = warp_sum(sr[isk]);
+        }
+        if ((t & 31) == 0) {
+            red[0][t >> 5] = sr[0];
+            red[1][t >> 5] = sr[1];
+        }
+        __syncthreads();
+        const float inv = 1.f / (128.f * (float)n_heads);
+#pragma unroll
+        for (int isk = 0; isk < 2; ++isk) {
+            float tot = 0.f;
+#pragma unroll
+            for (int w = 0; w < kHeadThreads / 32; ++w) tot += red[isk][w];
+            r_row[isk] = rsqrtf(tot * inv + eps);
+        }
+    }
 #pragma unroll
     for (int isk = 0; isk < 2; ++isk) {
         const uint4* row = rows + isk * qv;
@@ -181,21 +217,23 @@ __global__ void __launch_bounds__(kHeadThreads, kHeadCtas)
         for (int u = 0; u < UQ; ++u) {
             ss[u] = 0.f;
             const int c = t + kHeadThreads * u;
-            if (c < qv) {
+            if (!ACROSS && c < qv) {
                 float2 f[4];
                 unpack2<bf16>(row[c], f);
                 ss[u] = qk_sumsq(f);
             }
         }
+        if constexpr (!ACROSS) {
 #pragma unroll
-        for (int off = 8; off > 0; off >>= 1) {
+            for (int off = 8; off > 0; off >>= 1) {
 #pragma unroll
-            for (int u = 0; u < UQ; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
+                for (int u = 0; u < UQ; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
+            }
         }
         float kc[16];  // this slice's coefficients, for every head vector of the row
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            const float4 x = kcs[isk][m][sub];  // lanes read consecutive 16-byte words
+            const float4 x = kcs[ACROSS ? 0 : isk][m][sub];  // lanes read consecutive 16-byte words
             kc[4 * m + 0] = x.x;
             kc[4 * m + 1] = x.y;
             kc[4 * m + 2] = x.z;
@@ -219,8 +257,28 @@ __global__ void __launch_bounds__(kHeadThreads, kHeadCtas)
             } else {
                 unpack2<bf16>(row[c], f);
             }
+            if constexpr (ACROSS) {
+                // the weights of these elements (per head, so per slot), before the rotation
+                const bf16* wrow = isk ? wk : wq;
+                if (wrow) {
+                    float2 w[4];
+                    if constexpr (HALF) {
+                        const bf16* wh = wrow + 8 * (c - sub);
+                        const uint2 a = __ldg(reinterpret_cast<const uint2*>(wh + e0));
+                        const uint2 b = __ldg(reinterpret_cast<const uint2*>(wh + e0 + hp));
+                        w[0] = make_float2(bf_lo(a.x), bf_lo(b.x));
+                        w[1] = make_float2(bf_hi(a.x), bf_hi(b.x));
+                        w[2] = make_float2(bf_lo(a.y), bf_lo(b.y));
+                        w[3] = make_float2(bf_hi(a.y), bf_hi(b.y));
+                    } else {
+                        unpack2<bf16>(ld_cached(wrow + 8 * c), w);
+                    }
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) f[m] = __fmul2_rn(f[m], w[m]);
+                }
+            }
             float o[8];
-            qk_rotate(f, rsqrtf(ss[u] * (1.f / 128.f) + eps), kc, o);
+            qk_rotate(f, ACROSS ? r_row[isk] : rsqrtf(ss[u] * (1.f / 128.f) + eps), kc, o);
             bf16* dst;  // the head vector's output
             if constexpr (STRIDED)
                 dst = out + obase + (int64_t)(c >> 4) * os.head;
@@ -235,105 +293,12 @@ __global__ void __launch_bounds__(kHeadThreads, kHeadCtas)
         }
     }
     (void)hp;
-}
-
-// One RMS over the whole q (k) row (interleaved pairs), weights [n_heads * 128] laid out
-// like the row: the slot sums meet in a CTA reduction (one barrier); the weights differ per
-// head, so they are read per slot (through L1) and multiply the elements before a rotation
-// with the bare (cos, sin).  U = vectors per thread of the [q | k] row.
-template <int U, bool STRIDED>
-__global__ void __launch_bounds__(kAcrossThreads, 2048 / kAcrossThreads)
-    k_qk_across(bf16* q_out, bf16* k_out, int64_t ld_qo, int64_t ld_ko, QkOutStrides os, const bf16* q,
-                const bf16* k, int64_t ld_q, int64_t ld_k, const bf16* __restrict__ wq, const bf16* __restrict__ wk,
-                const int32_t* __restrict__ pos, int32_t grid_H, int32_t grid_W, uint32_t tokens_per_sample,
-                RopeDev rope, int32_t n_heads, float eps)
-{
-    extern __shared__ __align__(128) uint4 rows[];  // [q row | k row], 2 * qv vectors
-    __shared__ float2 cs[4][16];                     // (cos, sin) of pair 4 j + m at [m][j]
-    __shared__ float red[2][kAcrossThreads / 32];
-    __shared__ __align__(8) uint64_t bar;
-    const uint32_t n = blockIdx.x;
-    const int t = threadIdx.x;
-    const int qv = 16 * n_heads;
-
-    if (t == 0) start_row_copies(rows, &bar, q, k, ld_q, ld_k, n, qv);
-    if (t < 64) cs[t & 3][t >> 2] = pair_angle(t, n, pos, grid_H, grid_W, tokens_per_sample, rope);
-    __syncthreads();  // the barrier is initialised and the angles are in place
-    if (!rows_landed(&bar)) return;
-
-    const int sub = t & 15;
-    float sq = 0.f, sk = 0.f;
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const int c = t + kAcrossThreads * u;
-        if (c < 2 * qv) {  // uniform over each warp
-            float2 f[4];
-            unpack2<bf16>(rows[c], f);
-            const float s = qk_sumsq(f);
-            if (c < qv)
-                sq += s;
-            else
-                sk += s;
-        }
-    }
-    sq = warp_sum(sq);
-    sk = warp_sum(sk);
-    if ((t & 31) == 0) {
-        red[0][t >> 5] = sq;
-        red[1][t >> 5] = sk;
-    }
-    __syncthreads();
-    float tq = 0.f, tk = 0.f;
-#pragma unroll
-    for (int w = 0; w < kAcrossThreads / 32; ++w) {
-        tq += red[0][w];
-        tk += red[1][w];
-    }
-    const float inv = 1.f / (128.f * (float)n_heads);
-    const float rq = rsqrtf(tq * inv + eps), rk = rsqrtf(tk * inv + eps);
-    int64_t obase = 0;
-    if constexpr (STRIDED) {
-        const uint32_t sample = tokens_per_sample ? n / tokens_per_sample : 0;
-        obase = (int64_t)sample * os.sample + (int64_t)(n - sample * tokens_per_sample) * os.token;
-    }
-    // one slot at a time (a rolled loop) keeps the registers low
-#pragma unroll 1
-    for (int u = 0; u < U; ++u) {
-        const int c = t + kAcrossThreads * u;
-        if (c >= 2 * qv) continue;
-        const int isk = c >= qv ? 1 : 0;
-        const int v = c - isk * qv;  // vector within the row: head v / 16, slice v % 16
-        const float r = isk ? rk : rq;
-        const bf16* wrow = isk ? wk : wq;
-        float w[8];
-        if (wrow) {
-            unpack<bf16>(ld_cached(wrow + 8 * v), w);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = 1.f;
-        }
-        float f[8], a[8], o[8];
-        unpack<bf16>(rows[c], f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) a[e] = f[e] * r * w[e];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float2 x = cs[m][sub];
-            o[2 * m] = a[2 * m] * x.x - a[2 * m + 1] * x.y;
-            o[2 * m + 1] = a[2 * m] * x.y + a[2 * m + 1] * x.x;
-        }
-        bf16* dst;
-        if constexpr (STRIDED)
-            dst = (isk ? k_out : q_out) + obase + (int64_t)(v >> 4) * os.head + 8 * sub;
-        else
-            dst = isk ? k_out + (int64_t)n * ld_ko + 8 * v : q_out + (int64_t)n * ld_qo + 8 * v;
-        st_stream(dst, pack<bf16>(o));
-    }
+    (void)r_row;
 }
 
 namespace {
 
-// Launch arguments shared by both kernels.
+// Launch arguments.
 struct QkLaunch {
     void* q_out;
     void* k_out;
@@ -353,12 +318,11 @@ struct QkLaunch {
     float eps;
 };
 
-// Set the kernel's shared-memory attributes once per device (for the largest row seen),
-// then launch one CTA per token.  carveout_pct < 0: all of the unified L1 / shared memory as
-// shared memory.
+// Set the kernel's shared-memory attributes once per device (for the largest row seen:
+// all of the unified L1 / shared memory as shared memory, since 9 CTAs of 22.6 KB need it),
+// then launch one CTA per token.
 template <typename Kern>
-cudaError_t launch_rows(Kern kern, int threads, int carveout_pct, const QkLaunch& a, std::atomic<size_t>* attr_set,
-                        cudaStream_t s)
+cudaError_t launch_rows(Kern kern, const QkLaunch& a, std::atomic<size_t>* attr_set, cudaStream_t s)
 {
     const size_t smem = (size_t)2 * 16 * 16 * a.n_heads;
     int dev = 0;
@@ -367,58 +331,34 @@ cudaError_t launch_rows(Kern kern, int threads, int carveout_pct, const QkLaunch
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (attr_set[dev].load(std::memory_order_acquire) < smem) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 carveout_pct < 0 ? (int)cudaSharedmemCarveoutMaxShared : carveout_pct);
+                                 (int)cudaSharedmemCarveoutMaxShared);
         if (e == cudaSuccess && smem > 48 * 1024)
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr_set[dev].store(smem, std::memory_order_release);
     }
-    kern<<<(unsigned)a.n_tokens, threads, smem, s>>>(
+    kern<<<(unsigned)a.n_tokens, kHeadThreads, smem, s>>>(
         static_cast<bf16*>(a.q_out), static_cast<bf16*>(a.k_out), a.ld_qo, a.ld_ko, a.os,
         static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k), a.ld_q, a.ld_k, static_cast<const bf16*>(a.wq),
         static_cast<const bf16*>(a.wk), a.pos, a.grid_H, a.grid_W, (uint32_t)a.tps, a.rope, a.n_heads, a.eps);
     return cudaGetLastError();
 }
 
-template <int UQ, bool HALF, bool STRIDED> cudaError_t launch_head(const QkLaunch& a, cudaStream_t s)
+template <int UQ, bool ACROSS, bool HALF, bool STRIDED> cudaError_t launch_head(const QkLaunch& a, cudaStream_t s)
 {
-    // 9 CTAs of 22.6 KB need all of the shared part
     static std::atomic<size_t> attr_set[64];  // per device: the larger dynamic shared memory it allows
-    return launch_rows(k_qk_head<UQ, HALF, STRIDED>, kHeadThreads, -1, a, attr_set, s);
+    return launch_rows(k_qk_head<UQ, ACROSS, HALF, STRIDED>, a, attr_set, s);
 }
 
-template <int U, bool STRIDED> cudaError_t launch_across(const QkLaunch& a, cudaStream_t s)
-{
-    // just enough shared memory for 8 CTAs (per CTA: the rows, ~0.6 KB of static arrays and
-    // the 1 KB the system keeps): the rest stays L1 for the weights read per slot
-    static std::atomic<size_t> attr_set[64];
-    const size_t need = ((size_t)2 * 16 * 16 * a.n_heads + 2 * 1024) * (2048 / kAcrossThreads);
-    const int pct = (int)std::min<size_t>(100, (need * 100 + 228 * 1024 - 1) / (228 * 1024));
-    return launch_rows(k_qk_across<U, STRIDED>, kAcrossThreads, pct, a, attr_set, s);
-}
-
-template <bool HALF, bool STRIDED> cudaError_t dispatch_head(const QkLaunch& a, cudaStream_t s)
+template <bool ACROSS, bool HALF, bool STRIDED> cudaError_t dispatch_head(const QkLaunch& a, cudaStream_t s)
 {
     switch ((16 * a.n_heads + kHeadThreads - 1) / kHeadThreads) {
-    case 1: return launch_head<1, HALF, STRIDED>(a, s);
-    case 2: return launch_head<2, HALF, STRIDED>(a, s);
-    case 3: return launch_head<3, HALF, STRIDED>(a, s);
-    case 4: return launch_head<4, HALF, STRIDED>(a, s);
-    case 5: return launch_head<5, HALF, STRIDED>(a, s);
-    case 6: return launch_head<6, HALF, STRIDED>(a, s);
-    }
-    return cudaErrorInvalidValue;
-}
-
-template <bool STRIDED> cudaError_t dispatch_across(const QkLaunch& a, cudaStream_t s)
-{
-    switch ((32 * a.n_heads + kAcrossThreads - 1) / kAcrossThreads) {
-    case 1: return launch_across<1, STRIDED>(a, s);
-    case 2: return launch_across<2, STRIDED>(a, s);
-    case 3: return launch_across<3, STRIDED>(a, s);
-    case 4: return launch_across<4, STRIDED>(a, s);
-    case 5: return launch_across<5, STRIDED>(a, s);
-    case 6: return launch_across<6, STRIDED>(a, s);
+    case 1: return launch_head<1, ACROSS, HALF, STRIDED>(a, s);
+    case 2: return launch_head<2, ACROSS, HALF, STRIDED>(a, s);
+    case 3: return launch_head<3, ACROSS, HALF, STRIDED>(a, s);
+    case 4: return launch_head<4, ACROSS, HALF, STRIDED>(a, s);
+    case 5: return launch_head<5, ACROSS, HALF, STRIDED>(a, s);
+    case 6: return launch_head<6, ACROSS, HALF, STRIDED>(a, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -434,8 +374,8 @@ bool out_token_major(const QkOutStrides& os, int64_t tps, int64_t n_tokens)
 
 bool qk_cta_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim, const void* q, const void* k, int64_t n_tokens)
 {
-    // the copies need 16-byte aligned rows (the API's rule); the thread counts cover up to 48
-    // heads with 6 vectors a thread and row (k_qk_head) or [q | k] row (k_qk_across)
+    // the copies need 16-byte aligned rows (the API's rule); 128 threads cover up to 48 heads
+    // with 6 vectors a thread and row
     return dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads >= 2 && n_heads % 2 == 0 && n_heads <= 48 && q && k &&
            n_tokens < ((int64_t)1 << 31);
 }
@@ -444,13 +384,9 @@ bool qk_cta_ex_fits(sol_dtype dt, bool across, bool half, int32_t n_heads, int32
                     const void* q, const void* k, int64_t n_tokens, int64_t tps, const RopeDev& rope)
 {
     if (!qk_cta_fits(dt, n_heads, head_dim, q, k, n_tokens) || tps >= ((int64_t)1 << 31)) return false;
-    if (half) {
-        // rotate-half per head only: across heads the row-in-registers kernel measured faster
-        // (and one kernel serves every output layout, so results do not depend on the layout)
-        if (across) return false;
+    if (half)  // a thread's 4 pairs in one chunk half, its pieces 8-byte aligned
         for (int c = 0; c < 3; ++c)
             if (rope.half[c] % 4 != 0) return false;
-    }
     return true;
 }
 
@@ -463,7 +399,7 @@ cudaError_t launch_qk_cta(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko
     if (tps >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const QkLaunch a{q_out, k_out, ld_qo, ld_ko, QkOutStrides{0, 0, 0}, q, k, ld_q, ld_k, wq, wk, pos,
                      grid_H, grid_W, tps, rope, n_tokens, n_heads, eps};
-    return dispatch_head<false, false>(a, s);
+    return dispatch_head<false, false, false>(a, s);
 }
 
 cudaError_t launch_qk_cta_ex(bool across, bool half, void* q_out, void* k_out, const QkOutStrides& os, const void* q,
@@ -472,14 +408,14 @@ cudaError_t launch_qk_cta_ex(bool across, bool half, void* q_out, void* k_out, c
                              int64_t n_tokens, int32_t n_heads, float eps, cudaStream_t s)
 {
     if (n_tokens == 0) return cudaSuccess;
-    if (half && across) return cudaErrorInvalidValue;  // outside qk_cta_ex_fits
     if (tps >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const bool token_major = out_token_major(os, tps, n_tokens);
     const QkLaunch a{q_out, k_out, os.token, os.token, os, q, k, ld_q, ld_k, wq, wk, pos,
                      grid_H, grid_W, tps, rope, n_tokens, n_heads, eps};
-    if (across) return token_major ? dispatch_across<false>(a, s) : dispatch_across<true>(a, s);
-    if (half) return token_major ? dispatch_head<true, false>(a, s) : dispatch_head<true, true>(a, s);
-    return token_major ? dispatch_head<false, false>(a, s) : dispatch_head<false, true>(a, s);
+    if (across && half) return token_major ? dispatch_head<true, true, false>(a, s) : dispatch_head<true, true, true>(a, s);
+    if (across) return token_major ? dispatch_head<true, false, false>(a, s) : dispatch_head<true, false, true>(a, s);
+    if (half) return token_major ? dispatch_head<false, true, false>(a, s) : dispatch_head<false, true, true>(a, s);
+    return token_major ? dispatch_head<false, false, false>(a, s) : dispatch_head<false, false, true>(a, s);
 }
 
 uint32_t qk_device_error(bool clear)

@@ -12,9 +12,9 @@
 //   * all VPL loads are in flight before any is used, and the row is written only after
 //     it was read completely (in place is safe).
 // Arithmetic is fp32: v / sqrt(mean(v^2) + eps) * w, then the interleaved rotation of
-// pairs (2j, 2j + 1), as the per-step kernel (k_qk.cu) computes it.  The same kernel serves
-// the convention variants of k_qk_ex.cu (norm across all heads, rotate-half pairs, strided
-// outputs) for bf16 with a multiple of 8 heads.
+// pairs (2j, 2j + 1), as the per-step kernel (k_qk.cu) computes it.  The staged kernel of
+// k_qk_cta.cu takes the same shapes when q and k are both given; this one serves the calls
+// with q or k alone.
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -35,68 +35,37 @@
 
 namespace sol {
 
-// ACROSS: RMSNorm over the whole q (or k) row, weights [n_heads * 128], instead of per head
-// vector.  The row is in registers, so the norm is one full-warp reduction of the slots'
-// partial sums -- no second pass over HBM.
-// HALF: rotate-half pairs (element j of an axis chunk with element j + D_c/2).  The chunk
-// halves are multiples of 8 elements, so a lane's 8 elements sit in one half of one chunk
-// and their partners in lane +-(D_c/2)/8 of the same half-warp (the same head vector): one
-// shuffle per element, and the lane's 8 (cos, sin) entries are consecutive in the table.
-// STRIDED: outputs at (sample, token, head) element strides, e.g. [sample, head, token, dim].
-template <int VPL, bool ACROSS, bool HALF, bool STRIDED>
+template <int VPL>
 __global__ void __launch_bounds__(SOL_QK_REGS_BLOCK, SOL_QK_REGS_MINB)
-    k_qk_regs(bf16* q_out, bf16* k_out, int64_t ld_qo, int64_t ld_ko, QkOutStrides os, const bf16* q, const bf16* k,
-              int64_t ld_q, int64_t ld_k, const bf16* __restrict__ wq, const bf16* __restrict__ wk,
-              const int32_t* __restrict__ pos, int32_t grid_H, int32_t grid_W, int64_t tokens_per_sample,
-              RopeDev rope, int64_t n_tokens, float eps)
+    k_qk_regs(bf16* q_out, bf16* k_out, int64_t ld_qo, int64_t ld_ko, const bf16* q, const bf16* k, int64_t ld_q,
+              int64_t ld_k, const bf16* __restrict__ wq, const bf16* __restrict__ wk, const int32_t* __restrict__ pos,
+              int32_t grid_H, int32_t grid_W, int64_t tokens_per_sample, RopeDev rope, int64_t n_tokens, float eps)
 {
-    constexpr int NT = HALF ? 8 : 4;  // (cos, sin) entries per lane and row
     const int lane = threadIdx.x & 31;
     const int sub = lane & 15;  // element slice 8 * sub .. + 7 of every head vector
     float fwq[8], fwk[8];
-    if (!ACROSS && wq) {
+    if (wq) {
         unpack<bf16>(ld_cached(wq + 8 * sub), fwq);
     } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) fwq[e] = 1.f;
     }
-    if (!ACROSS && wk) {
+    if (wk) {
         unpack<bf16>(ld_cached(wk + 8 * sub), fwk);
     } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) fwk[e] = 1.f;
     }
-    // interleaved: this lane's four rotary pairs (axis, table column, row stride);
-    // rotate-half: the chunk half holding the lane's 8 elements, its first table column,
-    // the partner lane and the sign of the partner's term
+    // this lane's four rotary pairs: axis, table column, row stride
     const float2* tb[4];
     int stride[4], axis[4];
-    const float4* tbh = nullptr;
-    int strideh = 0, axish = 0, partner = lane;
-    float sgn = 1.f;
-    if constexpr (HALF) {
-        const int i0 = 8 * sub;
-        const int c0 = 2 * rope.half[0], c1 = c0 + 2 * rope.half[1];
-        axish = i0 < c0 ? 0 : (i0 < c1 ? 1 : 2);
-        const int off = axish == 0 ? 0 : (axish == 1 ? c0 : c1);
-        const int hw = axish == 0 ? rope.half[0] : (axish == 1 ? rope.half[1] : rope.half[2]);
-        const bool first = i0 - off < hw;
-        const int j0 = first ? i0 - off : i0 - off - hw;
-        const float2* t = axish == 0 ? rope.tab[0] : (axish == 1 ? rope.tab[1] : rope.tab[2]);
-        tbh = reinterpret_cast<const float4*>(t + j0);  // 16-byte aligned: j0 and hw are multiples of 8
-        strideh = hw / 2;                               // one table row = hw float2 = hw / 2 float4
-        partner = first ? lane + hw / 8 : lane - hw / 8;
-        sgn = first ? -1.f : 1.f;
-    } else {
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int pi = 4 * sub + m;
-            const int h0 = rope.half[0], h01 = rope.half[0] + rope.half[1];
-            axis[m] = pi < h0 ? 0 : (pi < h01 ? 1 : 2);
-            tb[m] = axis[m] == 0 ? rope.tab[0] + pi
-                                 : (axis[m] == 1 ? rope.tab[1] + (pi - h0) : rope.tab[2] + (pi - h01));
-            stride[m] = axis[m] == 0 ? rope.half[0] : (axis[m] == 1 ? rope.half[1] : rope.half[2]);
-        }
+    for (int m = 0; m < 4; ++m) {
+        const int pi = 4 * sub + m;
+        const int h0 = rope.half[0], h01 = rope.half[0] + rope.half[1];
+        axis[m] = pi < h0 ? 0 : (pi < h01 ? 1 : 2);
+        tb[m] = axis[m] == 0 ? rope.tab[0] + pi : (axis[m] == 1 ? rope.tab[1] + (pi - h0) : rope.tab[2] + (pi - h01));
+        stride[m] = axis[m] == 0 ? rope.half[0] : (axis[m] == 1 ? rope.half[1] : rope.half[2]);
     }
 
     const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -122,136 +91,47 @@ __global__ void __launch_bounds__(SOL_QK_REGS_BLOCK, SOL_QK_REGS_MINB)
             p1 = (int)((nl / grid_W) % grid_H);
             p2 = (int)(nl % grid_W);
         }
-        float cs[NT], sn[NT];
-        if constexpr (HALF) {
-            const int pm = axish == 0 ? p0 : (axish == 1 ? p1 : p2);
-            const float4* t = tbh + (int64_t)pm * strideh;
+        float cs[4], sn[4];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 v = __ldg(t + m);
-                cs[2 * m] = v.x;
-                sn[2 * m] = v.y;
-                cs[2 * m + 1] = v.z;
-                sn[2 * m + 1] = v.w;
-            }
-        } else {
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int pm = axis[m] == 0 ? p0 : (axis[m] == 1 ? p1 : p2);
-                const float2 t = __ldg(tb[m] + (int64_t)pm * stride[m]);
-                cs[m] = t.x;
-                sn[m] = t.y;
-            }
+        for (int m = 0; m < 4; ++m) {
+            const int pm = axis[m] == 0 ? p0 : (axis[m] == 1 ? p1 : p2);
+            const float2 t = __ldg(tb[m] + (int64_t)pm * stride[m]);
+            cs[m] = t.x;
+            sn[m] = t.y;
         }
-
         float w[8];  // selects, not an indexed array (which would live in local memory)
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = isk ? fwk[e] : fwq[e];
-        const bf16* wrow = isk ? wk : wq;  // across heads: [n_heads * 128], laid out like the row
-        bf16* dst;
-        int64_t slot_step;  // elements between register slots i and i + 1 in the output
-        if constexpr (STRIDED) {
-            const int64_t sample = tokens_per_sample > 0 ? n / tokens_per_sample : 0;
-            const int64_t nl = n - sample * tokens_per_sample;
-            dst = (isk ? k_out : q_out) + sample * os.sample + nl * os.token + (lane >> 4) * os.head + 8 * sub;
-            slot_step = 2 * os.head;
-        } else {
-            dst = (isk ? k_out + n * ld_ko : q_out + n * ld_qo) + 8 * lane;
-            slot_step = 256;
-        }
-        // slot i's 8 elements f, scaled by 1 / rms r and the weights, rotated and stored
-        auto emit = [&](int i, const float* f, float r) {
-            float o[8];
-            if constexpr (ACROSS) {
-                if (wrow) unpack<bf16>(ld_cached(wrow + 256 * i + 8 * lane), w);
-            }
-            if constexpr (HALF) {
-                float a[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) a[e] = f[e] * r * w[e];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float b = __shfl_sync(0xffffffffu, a[e], partner);
-                    o[e] = a[e] * cs[e] + sgn * b * sn[e];
-                }
-            } else {
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const float a = f[2 * m] * r * w[2 * m];
-                    const float b = f[2 * m + 1] * r * w[2 * m + 1];
-                    o[2 * m] = a * cs[m] - b * sn[m];
-                    o[2 * m + 1] = a * sn[m] + b * cs[m];
-                }
-            }
-            if constexpr (STRIDED) {
-                st_stream(dst, pack<bf16>(o));  // advanced slot by slot: no table of 64-bit addresses
-                dst += slot_step;
-            } else {
-                st_stream(dst + 256 * i, pack<bf16>(o));
-            }
-        };
+        float kc[16];  // weights folded into the rotation once per row
+        qk_coefs(w, cs, sn, kc);
+        bf16* dst = (isk ? k_out + n * ld_ko : q_out + n * ld_qo) + 8 * lane;
 
-        if constexpr (ACROSS) {
-            // one norm over the whole row: every slot's sum first, then the output pass
-            float tot = 0.f;
+        // GS slots at a time: widen once, sums of squares, GS independent half-warp trees,
+        // then normalise, rotate and store them
+        constexpr int GS = 4;
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                float f[8];
-                unpack<bf16>(xv[i], f);
+        for (int i0 = 0; i0 < VPL; i0 += GS) {
+            float2 f[GS][4];
+            float ss[GS];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) tot = fmaf(f[e], f[e], tot);
+            for (int u = 0; u < GS; ++u) {
+                ss[u] = 0.f;
+                if (i0 + u < VPL) {
+                    unpack2<bf16>(xv[i0 + u], f[u]);
+                    ss[u] = qk_sumsq(f[u]);
+                }
             }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
-            const float r_row = rsqrtf(tot * (1.f / (256.f * VPL)) + eps);
+            for (int off = 8; off > 0; off >>= 1) {
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                float f[8];
-                unpack<bf16>(xv[i], f);
-                emit(i, f, r_row);
+                for (int u = 0; u < GS; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
             }
-        } else {
-            // per head vector: GS slots at a time -- widen once, sums of squares, GS
-            // independent half-warp trees, then normalise, rotate and store them
-            constexpr int GS = 4;
-            float kc[16];  // interleaved pairs: weights folded into the rotation once per row
-            if constexpr (!HALF) qk_coefs(w, cs, sn, kc);
 #pragma unroll
-            for (int i0 = 0; i0 < VPL; i0 += GS) {
-                float2 f[GS][4];
-                float ss[GS];
-#pragma unroll
-                for (int u = 0; u < GS; ++u) {
-                    ss[u] = 0.f;
-                    if (i0 + u < VPL) {
-                        unpack2<bf16>(xv[i0 + u], f[u]);
-                        ss[u] = qk_sumsq(f[u]);
-                    }
-                }
-#pragma unroll
-                for (int off = 8; off > 0; off >>= 1) {
-#pragma unroll
-                    for (int u = 0; u < GS; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
-                }
-#pragma unroll
-                for (int u = 0; u < GS; ++u) {
-                    if (i0 + u < VPL) {
-                        const float r = rsqrtf(ss[u] * (1.f / 128.f) + eps);
-                        if constexpr (HALF) {
-                            float ff[8];
-                            unpack<bf16>(xv[i0 + u], ff);
-                            emit(i0 + u, ff, r);
-                        } else {
-                            float o[8];
-                            qk_rotate(f[u], r, kc, o);
-                            if constexpr (STRIDED) {
-                                st_stream(dst, pack<bf16>(o));
-                                dst += slot_step;
-                            } else {
-                                st_stream(dst + 256 * (i0 + u), pack<bf16>(o));
-                            }
-                        }
-                    }
+            for (int u = 0; u < GS; ++u) {
+                if (i0 + u < VPL) {
+                    float o[8];
+                    qk_rotate(f[u], rsqrtf(ss[u] * (1.f / 128.f) + eps), kc, o);
+                    st_stream(dst + 256 * (i0 + u), pack<bf16>(o));
                 }
             }
         }
@@ -260,18 +140,17 @@ __global__ void __launch_bounds__(SOL_QK_REGS_BLOCK, SOL_QK_REGS_MINB)
 
 namespace {
 
-template <int VPL, bool ACROSS, bool HALF, bool STRIDED>
-cudaError_t launch_vpl(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, const QkOutStrides& os,
-                       const void* q, const void* k, int64_t ld_q, int64_t ld_k, const void* wq, const void* wk,
-                       const int32_t* pos, int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope,
-                       int64_t n_tokens, float eps, cudaStream_t s)
+template <int VPL>
+cudaError_t launch_vpl(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, const void* q, const void* k,
+                       int64_t ld_q, int64_t ld_k, const void* wq, const void* wk, const int32_t* pos, int32_t grid_H,
+                       int32_t grid_W, int64_t tps, const RopeDev& rope, int64_t n_tokens, float eps, cudaStream_t s)
 {
-    auto kern = k_qk_regs<VPL, ACROSS, HALF, STRIDED>;
+    auto kern = k_qk_regs<VPL>;
     constexpr int block = SOL_QK_REGS_BLOCK;
     const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), block, 0);
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t grid = std::min<int64_t>((int64_t)per_sm * sm_count(), (2 * n_tokens + block / 32 - 1) / (block / 32));
-    kern<<<(unsigned)grid, block, 0, s>>>(static_cast<bf16*>(q_out), static_cast<bf16*>(k_out), ld_qo, ld_ko, os,
+    kern<<<(unsigned)grid, block, 0, s>>>(static_cast<bf16*>(q_out), static_cast<bf16*>(k_out), ld_qo, ld_ko,
                                         static_cast<const bf16*>(q), static_cast<const bf16*>(k), ld_q, ld_k,
                                         static_cast<const bf16*>(wq), static_cast<const bf16*>(wk), pos, grid_H,
                                         grid_W, tps, rope, n_tokens, eps);
@@ -290,61 +169,17 @@ cudaError_t launch_qk_regs(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_k
                            int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope, int64_t n_tokens,
                            int32_t n_heads, float eps, cudaStream_t s)
 {
-    const QkOutStrides os{0, 0, 0};  // unused: token-major outputs
     switch (n_heads / 2) {
 #define SOL_QK_VPL(v)                                                                                              \
     case v:                                                                                                        \
-        return launch_vpl<v, false, false, false>(q_out, k_out, ld_qo, ld_ko, os, q, k, ld_q, ld_k, wq, wk, pos,  \
-                                                  grid_H, grid_W, tps, rope, n_tokens, eps, s);
+        return launch_vpl<v>(q_out, k_out, ld_qo, ld_ko, q, k, ld_q, ld_k, wq, wk, pos, grid_H, grid_W, tps, rope, \
+                             n_tokens, eps, s);
         SOL_QK_VPL(1) SOL_QK_VPL(2) SOL_QK_VPL(3) SOL_QK_VPL(4) SOL_QK_VPL(5) SOL_QK_VPL(6) SOL_QK_VPL(7)
         SOL_QK_VPL(8) SOL_QK_VPL(9) SOL_QK_VPL(10) SOL_QK_VPL(11) SOL_QK_VPL(12) SOL_QK_VPL(13) SOL_QK_VPL(14)
         SOL_QK_VPL(15) SOL_QK_VPL(16) SOL_QK_VPL(17) SOL_QK_VPL(18) SOL_QK_VPL(19) SOL_QK_VPL(20)
         SOL_QK_VPL(21) SOL_QK_VPL(22) SOL_QK_VPL(23) SOL_QK_VPL(24)
 #undef SOL_QK_VPL
     }
-    return cudaErrorInvalidValue;
-}
-
-// The convention variants run here for bf16, head_dim 128 and a multiple of 8 heads up to
-// 48 (the instantiations are bounded to keep the build short); rotate-half also needs
-// chunk halves that are multiples of 8 and 16-byte aligned tables.
-bool qk_regs_ex_fits(sol_dtype dt, bool half, int32_t n_heads, int32_t head_dim, const RopeDev& rope)
-{
-    if (!(dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads % 8 == 0 && n_heads >= 8 && n_heads <= 48))
-        return false;
-    if (half)
-        for (int c = 0; c < 3; ++c)
-            if (rope.half[c] % 8 != 0 || reinterpret_cast<uintptr_t>(rope.tab[c]) % 16 != 0) return false;
-    return true;
-}
-
-cudaError_t launch_qk_regs_ex(bool across, bool half, void* q_out, void* k_out, const QkOutStrides& os, const void* q,
-                              const void* k, int64_t ld_q, int64_t ld_k, const void* wq, const void* wk,
-                              const int32_t* pos, int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope,
-                              int64_t n_tokens, int32_t n_heads, float eps, cudaStream_t s)
-{
-    // token-major outputs (head stride 128, samples back to back) take the unstrided stores
-    const int64_t tps_eff = tps > 0 ? tps : n_tokens;
-    const bool token_major = os.head == 128 && (os.sample == tps_eff * os.token || n_tokens <= tps_eff);
-    const int64_t ld_o = os.token;
-#define SOL_QK_EX_ARGS q_out, k_out, ld_o, ld_o, os, q, k, ld_q, ld_k, wq, wk, pos, grid_H, grid_W, tps, rope, n_tokens, eps, s
-#define SOL_QK_EX_VPL(v)                                                                                          \
-    case v:                                                                                                       \
-        if (token_major) {                                                                                        \
-            if (across) return half ? launch_vpl<v, true, true, false>(SOL_QK_EX_ARGS)                            \
-                                    : launch_vpl<v, true, false, false>(SOL_QK_EX_ARGS);                          \
-            return half ? launch_vpl<v, false, true, false>(SOL_QK_EX_ARGS)                                       \
-                        : launch_vpl<v, false, false, false>(SOL_QK_EX_ARGS);                                     \
-        }                                                                                                         \
-        if (across) return half ? launch_vpl<v, true, true, true>(SOL_QK_EX_ARGS)                                 \
-                                : launch_vpl<v, true, false, true>(SOL_QK_EX_ARGS);                               \
-        return half ? launch_vpl<v, false, true, true>(SOL_QK_EX_ARGS)                                            \
-                    : launch_vpl<v, false, false, true>(SOL_QK_EX_ARGS);
-    switch (n_heads / 2) {
-        SOL_QK_EX_VPL(4) SOL_QK_EX_VPL(8) SOL_QK_EX_VPL(12) SOL_QK_EX_VPL(16) SOL_QK_EX_VPL(20) SOL_QK_EX_VPL(24)
-    }
-#undef SOL_QK_EX_VPL
-#undef SOL_QK_EX_ARGS
     return cudaErrorInvalidValue;
 }
 

@@ -60,7 +60,7 @@ cudaError_t launch_qk_rmsnorm_rope3d(sol_dtype dt, void* q_out, void* k_out, int
                                      int32_t head_dim, float eps, cudaStream_t s);
 
 // QK RMSNorm + 3D RoPE with one warp per (token, q or k) row in registers (k_qk_regs.cu):
-// bf16, head_dim 128, an even number of heads.
+// bf16, head_dim 128, an even number of heads; q or k may be NULL.
 bool qk_regs_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim);
 cudaError_t launch_qk_regs(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko, const void* q, const void* k,
                            int64_t ld_q, int64_t ld_k, const void* wq, const void* wk, const int32_t* pos,
@@ -74,8 +74,8 @@ cudaError_t launch_qk_cta(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko
                           int64_t ld_q, int64_t ld_k, const void* wq, const void* wk, const int32_t* pos,
                           int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope, int64_t n_tokens,
                           int32_t n_heads, float eps, cudaStream_t s);
-// The same kernel for the convention variants: norm across heads, strided outputs, and
-// rotate-half pairs per head (chunk halves multiples of 4); not rotate-half across heads.
+// The same kernel for the convention variants: norm across heads, rotate-half pairs (chunk
+// halves multiples of 4), strided outputs.
 bool qk_cta_ex_fits(sol_dtype dt, bool across, bool half, int32_t n_heads, int32_t head_dim,
                     const void* q, const void* k, int64_t n_tokens, int64_t tps, const RopeDev& rope);
 cudaError_t launch_qk_cta_ex(bool across, bool half, void* q_out, void* k_out, const QkOutStrides& os, const void* q,
@@ -84,13 +84,6 @@ cudaError_t launch_qk_cta_ex(bool across, bool half, void* q_out, void* k_out, c
                              int64_t n_tokens, int32_t n_heads, float eps, cudaStream_t s);
 // Error flags of that kernel's bounded wait (bit 1); optionally cleared.  Synchronous.
 uint32_t qk_device_error(bool clear);
-// The same kernel for the convention variants (norm across heads, rotate-half pairs, strided
-// outputs): bf16, head_dim 128, a multiple of 8 heads up to 48.
-bool qk_regs_ex_fits(sol_dtype dt, bool half, int32_t n_heads, int32_t head_dim, const RopeDev& rope);
-cudaError_t launch_qk_regs_ex(bool across, bool half, void* q_out, void* k_out, const QkOutStrides& os, const void* q,
-                              const void* k, int64_t ld_q, int64_t ld_k, const void* wq, const void* wk,
-                              const int32_t* pos, int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope,
-                              int64_t n_tokens, int32_t n_heads, float eps, cudaStream_t s);
 
 // QK RMSNorm + 3D RoPE, convention variants (k_qk_ex.cu): `across` = RMS over all heads
 // with weights [n_heads * head_dim]; `half` = rotate-half pairs; any output strides.
