@@ -295,6 +295,47 @@ def test_qk_ex_conventions_and_layouts(orc, dtype, head_dim, dims, Hh, grid, B, 
     rope.close()
 
 
+@pytest.mark.parametrize("span", [sol.NORM_PER_HEAD, sol.NORM_ACROSS_HEADS])
+@pytest.mark.parametrize("pairing", [sol.ROPE_INTERLEAVED, sol.ROPE_HALF])
+def test_qk_ex_explicit_positions_packed_and_clamped(orc, span, pairing):
+    """Explicit packed video+audio positions through the staged kernel (bf16, 128-dim heads,
+    an even head count), token-major and head-major; positions past the table clamp."""
+    w = workloads.Workload("t", 7, BF, 2, (2, 3, 4), 5, 64, 4, 128, 64)
+    pos, sid = workloads.token_layout(w)
+    n, hd = pos.shape[0], w.hd
+    q, k = randn((n, hd), BF, 41, std=1.5), randn((n, hd), BF, 42, std=1.5)
+    wlen = hd if span == sol.NORM_ACROSS_HEADS else 128
+    wq, wk = randn((wlen,), BF, 43, std=0.02, mean=1.0), randn((wlen,), BF, 44, std=0.02, mean=1.0)
+    rope = sol.Rope3D(w.rope_dims, w.theta, w.max_pos)
+    P = pos.to(DEV)
+    common = dict(n_heads=w.n_heads, head_dim=128, wq=wq, wk=wk, norm_span=span, pairing=pairing)
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    sol.qk_rmsnorm_rope3d_ex(qo, ko, q, k, rope, pos=P, **common)
+    # one sample of n tokens, head-major [1, heads, n, 128]
+    qh = torch.empty((1, w.n_heads, n, 128), dtype=BF, device=DEV)
+    kh = torch.empty_like(qh)
+    sol.qk_rmsnorm_rope3d_ex(qh, kh, q, k, rope, pos=P, out_strides=(128, n * 128, w.n_heads * n * 128), **common)
+    torch.cuda.synchronize()
+    want_q, want_k = orc.qk_rmsnorm_rope3d_ex(to_oracle(q), to_oracle(k), to_oracle(wq), to_oracle(wk),
+                                              n_heads=w.n_heads, head_dim=128, pos=pos.numpy(),
+                                              dims=w.rope_dims, theta=w.theta, norm_span=span, pairing=pairing)
+    assert_close(to_f64(qo), want_q, BF, "q")
+    assert_close(to_f64(ko), want_k, BF, "k")
+    assert torch.equal(qh[0].permute(1, 0, 2).reshape(n, hd), qo)
+    assert torch.equal(kh[0].permute(1, 0, 2).reshape(n, hd), ko)
+    big = P.clone()
+    big[:, 0] += 1000
+    big[:3, 1] = -4
+    clamped = torch.minimum(big, torch.tensor(w.max_pos, device=DEV, dtype=torch.int32) - 1).clamp_min(0)
+    a, b = torch.empty_like(q), torch.empty_like(q)
+    sol.qk_rmsnorm_rope3d_ex(a, b, q, k, rope, pos=big.contiguous(), **common)
+    c, d = torch.empty_like(q), torch.empty_like(q)
+    sol.qk_rmsnorm_rope3d_ex(c, d, q, k, rope, pos=clamped.contiguous(), **common)
+    torch.cuda.synchronize()
+    assert torch.equal(a, c) and torch.equal(b, d)
+    rope.close()
+
+
 def test_qk_ex_rejects_bad_layouts():
     rope = sol.Rope3D((32, 48, 48), 10000.0, (4, 4, 4))
     q = randn((8, 128), BF, 1)
