@@ -418,6 +418,237 @@ cudaError_t launch_qk_cta_ex(bool across, bool half, void* q_out, void* k_out, c
     return token_major ? dispatch_head<false, false, false>(a, s) : dispatch_head<false, false, true>(a, s);
 }
 
+// ---------------------------------------------------------------------------------
+// The QKV epilogue fused with the 64-token block means of SubBlock routing
+// (sol_dit_epilogue_pool), staged: one CTA of 128 threads per (block, q or k) walks the
+// block's tokens through a ring of kPoolSlots row buffers that thread 0 refills by bulk
+// copies as rows are consumed, so up to kPoolSlots rows per CTA (4 CTAs per SM) are in
+// flight while the block sums stay in fp32 registers.  Thread t owns vectors t + 128 u of
+// the row (the same 8-element slice of every head vector it touches) and the 4 rotary
+// pairs of that slice: its coefficients are recomputed per token from its weights and the
+// token's angles (qk_coefs), and the per-vector arithmetic is qk_math.cuh's, so the
+// in-place rows equal the plain epilogue's bit for bit and the sums are taken over the
+// same fp32 outputs, token by token.  Every wait on a row is bounded; on give-up the CTA
+// records bit 1 of the device error flags, waits (bounded) for its copies in flight and
+// returns.
+constexpr int kPoolSlots = 4;
+constexpr int kPoolCtas = 4;  // resident CTAs per SM (launch bounds)
+
+template <int UQ>
+__global__ void __launch_bounds__(kHeadThreads, kPoolCtas)
+    k_qk_pool_stage(bf16* q, bf16* k, int64_t ld_q, int64_t ld_k, bf16* pq, bf16* pk, int64_t ld_pq, int64_t ld_pk,
+                    const bf16* __restrict__ wq, const bf16* __restrict__ wk, const int32_t* __restrict__ pos,
+                    int32_t grid_H, int32_t grid_W, int64_t tps, int32_t block, int64_t bps, RopeDev rope,
+                    int64_t n_tokens, int32_t n_heads, float eps)
+{
+    extern __shared__ __align__(128) uint4 ring[];  // kPoolSlots rows of qv vectors
+    __shared__ __align__(8) uint64_t full[kPoolSlots];
+    const int t = threadIdx.x;
+    const int sub = t & 15;
+    const int qv = 16 * n_heads;
+    const uint32_t row_bytes = 16u * (uint32_t)qv;
+    const int64_t blk = (int64_t)(blockIdx.x >> 1);
+    const bool isk = (blockIdx.x & 1) != 0;
+    // the block's tokens [t0, t1): blocks restart at every sample boundary
+    const int64_t sample = blk / bps;
+    const int64_t t0 = sample * tps + (blk - sample * bps) * block;
+    int64_t t1 = t0 + block;
+    if (t1 > (sample + 1) * tps) t1 = (sample + 1) * tps;
+    if (t1 > n_tokens) t1 = n_tokens;
+    const int cnt = (int)(t1 - t0);
+    bf16* const rows_g = isk ? k : q;
+    const int64_t ld = isk ? ld_k : ld_q;
+
+    if (t == 0) {
+#pragma unroll
+        for (int i = 0; i < kPoolSlots; ++i) mbar_init(smem_u32(&full[i]), 1);
+        mbar_fence_init();
+        for (int i = 0; i < kPoolSlots && i < cnt; ++i) {
+            mbar_arrive_expect_tx(smem_u32(&full[i]), row_bytes);
+            bulk_g2s(smem_u32(ring + i * qv), rows_g + (t0 + i) * ld, row_bytes, smem_u32(&full[i]));
+        }
+    }
+    // this slice's weights, and its 4 pairs' axis, table column and table row stride
+    float w[8];
+    const bf16* wsrc = isk ? wk : wq;
+    if (wsrc) {
+        unpack<bf16>(ld_cached(wsrc + 8 * sub), w);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = 1.f;
+    }
+    const int h0 = rope.half[0], h01 = rope.half[0] + rope.half[1];
+    int axis[4];
+    const float2* tb[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int pi = 4 * sub + m;
+        axis[m] = pi < h0 ? 0 : (pi < h01 ? 1 : 2);
+        tb[m] = axis[m] == 0 ? rope.tab[0] + pi : (axis[m] == 1 ? rope.tab[1] + (pi - h0) : rope.tab[2] + (pi - h01));
+    }
+    // the grid position of the next token (implicit positions)
+    uint32_t g0 = 0, g1 = 0, g2 = 0;
+    if (!pos) {
+        const uint32_t nl = (uint32_t)(t0 - sample * tps);
+        const uint32_t hw = (uint32_t)grid_H * (uint32_t)grid_W;
+        g0 = nl / hw;
+        const uint32_t r = nl - g0 * hw;
+        g1 = r / (uint32_t)grid_W;
+        g2 = r - g1 * (uint32_t)grid_W;
+    }
+    float acc[UQ][8];
+#pragma unroll
+    for (int u = 0; u < UQ; ++u)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+    __syncthreads();  // the barriers are initialised
+
+    for (int i = 0; i < cnt; ++i) {
+        const int slot = i % kPoolSlots;
+        const bool landed = mbar_wait_bounded(smem_u32(&full[slot]), (uint32_t)(i / kPoolSlots) & 1u, kQkWaitLimit);
+        if (__syncthreads_or(!landed)) {
+            if (t == 0) {
+                atomicOr(&g_qk_error, 2u);
+                for (int j = i; j < cnt && j < i + kPoolSlots; ++j)  // the copies in flight must land
+                    mbar_wait_bounded(smem_u32(&full[j % kPoolSlots]), (uint32_t)(j / kPoolSlots) & 1u,
+                                      kQkWaitLimit);
+            }
+            return;
+        }
+        const int64_t n = t0 + i;
+        uint32_t p[3];
+        if (pos) {
+            p[0] = (uint32_t)min(max(__ldg(pos + 3 * n + 0), 0), rope.max[0] - 1);
+            p[1] = (uint32_t)min(max(__ldg(pos + 3 * n + 1), 0), rope.max[1] - 1);
+            p[2] = (uint32_t)min(max(__ldg(pos + 3 * n + 2), 0), rope.max[2] - 1);
+        } else {
+            p[0] = g0;
+            p[1] = g1;
+            p[2] = g2;
+            if (++g2 == (uint32_t)grid_W) {
+                g2 = 0;
+                if (++g1 == (uint32_t)grid_H) {
+                    g1 = 0;
+                    ++g0;
+                }
+            }
+        }
+        float cs[4], sn[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t pm = axis[m] == 0 ? p[0] : (axis[m] == 1 ? p[1] : p[2]);
+            const int st = axis[m] == 0 ? rope.half[0] : (axis[m] == 1 ? rope.half[1] : rope.half[2]);
+            const float2 a = __ldg(tb[m] + (int64_t)pm * st);
+            cs[m] = a.x;
+            sn[m] = a.y;
+        }
+        float kc[16];
+        qk_coefs(w, cs, sn, kc);
+        const uint4* row = ring + slot * qv;
+        float ss[UQ];
+#pragma unroll
+        for (int u = 0; u < UQ; ++u) {
+            ss[u] = 0.f;
+            const int c = t + kHeadThreads * u;
+            if (c < qv) {
+                float2 f[4];
+                unpack2<bf16>(row[c], f);
+                ss[u] = qk_sumsq(f);
+            }
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) {
+#pragma unroll
+            for (int u = 0; u < UQ; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
+        }
+        bf16* const dst = rows_g + n * ld;
+#pragma unroll
+        for (int u = 0; u < UQ; ++u) {
+            const int c = t + kHeadThreads * u;
+            if (c >= qv) continue;
+            float2 f[4];
+            unpack2<bf16>(row[c], f);
+            float o[8];
+            qk_rotate(f, rsqrtf(ss[u] * (1.f / 128.f) + eps), kc, o);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[u][e] += o[e];
+            st_stream(dst + 8 * c, pack<bf16>(o));
+        }
+        __syncthreads();  // every thread is done with the slot
+        if (t == 0 && i + kPoolSlots < cnt) {
+            mbar_arrive_expect_tx(smem_u32(&full[slot]), row_bytes);
+            bulk_g2s(smem_u32(ring + slot * qv), rows_g + (n + kPoolSlots) * ld, row_bytes, smem_u32(&full[slot]));
+        }
+    }
+    const float inv = 1.f / (float)cnt;
+    bf16* const out = isk ? pk + blk * ld_pk : pq + blk * ld_pq;
+#pragma unroll
+    for (int u = 0; u < UQ; ++u) {
+        const int c = t + kHeadThreads * u;
+        if (c >= qv) continue;
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = acc[u][e] * inv;
+        st_stream(out + 8 * c, pack<bf16>(o));
+    }
+}
+
+namespace {
+template <int UQ>
+cudaError_t launch_pool_stage(void* q, void* k, int64_t ld_q, int64_t ld_k, void* pq, void* pk, int64_t ld_pq,
+                              int64_t ld_pk, const void* wq, const void* wk, const int32_t* pos, int32_t grid_H,
+                              int32_t grid_W, int64_t tps, int32_t block, int64_t bps, int64_t n_blocks,
+                              const RopeDev& rope, int64_t n_tokens, int32_t n_heads, float eps, cudaStream_t s)
+{
+    auto kern = k_qk_pool_stage<UQ>;
+    const size_t smem = (size_t)kPoolSlots * 16 * 16 * n_heads;  // up to 48 KB (48 heads)
+    static std::atomic<size_t> attr_set[64];  // per device: the larger dynamic shared memory it allows
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (attr_set[dev].load(std::memory_order_acquire) < smem) {
+        // 4 CTAs of up to 48 KB: all of the unified L1 / shared memory as shared memory; the
+        // dynamic part plus the barriers may pass the 48 KB a launch gets without asking
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set[dev].store(smem, std::memory_order_release);
+    }
+    kern<<<(unsigned)(2 * n_blocks), kHeadThreads, smem, s>>>(
+        static_cast<bf16*>(q), static_cast<bf16*>(k), ld_q, ld_k, static_cast<bf16*>(pq), static_cast<bf16*>(pk),
+        ld_pq, ld_pk, static_cast<const bf16*>(wq), static_cast<const bf16*>(wk), pos, grid_H, grid_W, tps, block,
+        bps, rope, n_tokens, n_heads, eps);
+    return cudaGetLastError();
+}
+}  // namespace
+
+bool qk_pool_stage_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim, const void* q, const void* k,
+                        int64_t tps, int64_t n_blocks)
+{
+    return dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads >= 2 && n_heads % 2 == 0 && n_heads <= 48 && q && k &&
+           tps < ((int64_t)1 << 31) && 2 * n_blocks < ((int64_t)1 << 31);
+}
+
+cudaError_t launch_qk_pool_stage(void* q, void* k, int64_t ld_q, int64_t ld_k, void* pq, void* pk, int64_t ld_pq,
+                                 int64_t ld_pk, const void* wq, const void* wk, const int32_t* pos, int32_t grid_H,
+                                 int32_t grid_W, int64_t tps, int32_t block, int64_t bps, int64_t n_blocks,
+                                 const RopeDev& rope, int64_t n_tokens, int32_t n_heads, float eps, cudaStream_t s)
+{
+    if (n_blocks == 0) return cudaSuccess;
+    switch ((16 * n_heads + kHeadThreads - 1) / kHeadThreads) {
+#define SOL_POOL_STAGE_U(u)                                                                                      \
+    case u:                                                                                                      \
+        return launch_pool_stage<u>(q, k, ld_q, ld_k, pq, pk, ld_pq, ld_pk, wq, wk, pos, grid_H, grid_W, tps, block, \
+                                    bps, n_blocks, rope, n_tokens, n_heads, eps, s);
+        SOL_POOL_STAGE_U(1) SOL_POOL_STAGE_U(2) SOL_POOL_STAGE_U(3) SOL_POOL_STAGE_U(4) SOL_POOL_STAGE_U(5)
+        SOL_POOL_STAGE_U(6)
+#undef SOL_POOL_STAGE_U
+    }
+    return cudaErrorInvalidValue;
+}
+
 uint32_t qk_device_error(bool clear)
 {
     unsigned int v = 0;

@@ -4,8 +4,10 @@
 // keeps a fraction of the key blocks; "SGLang acelera video do MiniMax-H3",
 // "De onde vem os ganhos"].
 //
-// Two kernels.  bf16 with head_dim 128 and a multiple of 8 heads takes the row-in-registers
-// kernel k_qk_pool_regs (below).  Every other shape takes k_qk_rope_pool:
+// bf16 with head_dim 128 and an even number of heads up to 48 takes the staged kernel
+// k_qk_pool_stage (k_qk_cta.cu: a ring of bulk-copied rows per block, 6.27-6.41 TB/s at
+// 245,952 tokens x 40 heads, where a row-in-registers kernel that walked each block two
+// tokens at a time reached 6.08).  Every other shape takes k_qk_rope_pool:
 // a CTA of 8 warps owns one block of `block` tokens at a time (blocks restart at every
 // sample boundary; blocks walked with a grid stride).  Each warp takes a contiguous run
 // of the block's tokens and walks it in chunks of up to 8 tokens: it first stages the
@@ -22,7 +24,6 @@
 
 #include "common.cuh"
 #include "launch.h"
-#include "qk_math.cuh"
 
 namespace sol {
 
@@ -202,170 +203,6 @@ k_qk_rope_pool(T* q, T* k, int64_t ld_q, int64_t ld_k, T* pq, T* pk, int64_t ld_
     }
 }
 
-// Row-in-registers variant (bf16, head_dim 128, a multiple of 8 heads up to 48): a CTA of
-// SOL_POOL_PARTS warps owns one (block, q or k) pair; warp p holds a part of the row --
-// register slots p * SPW .. + SPW - 1 in the layout of k_qk_regs.cu (slot i of lanes 0-15 /
-// 16-31 is head vector 2i / 2i + 1, so each lane owns the same 8-element slice of every
-// head vector) -- and walks the block's tokens SOL_POOL_TPI at a time, their loads in
-// flight together.  The block sums stay in fp32 registers (8 per slot per lane), so there
-// is no shared memory and no atomic.  The in-place q / k arithmetic is exactly the plain
-// epilogue's.  One CTA per (block, q or k), no persistent grid.
-// Shape, from a sweep on B200 at 245,952 tokens x 40 heads (the plain epilogue: 1.60 ms;
-// the shared-memory kernel above: 2.04 ms): 4 warps per row, 2 tokens per iteration, >= 3
-// CTAs per SM (165 registers): 1.66 ms; the same with 4 tokens and 2 CTAs: 1.70; 2 warps
-// per row with 1 or 2 tokens: 1.77-1.80; 4 warps with 2 or 3 tokens and 2 CTAs: 1.78-1.91.
-#ifndef SOL_POOL_PARTS
-#define SOL_POOL_PARTS 4  // warps per row (each holds n_heads / (2 * SOL_POOL_PARTS) register slots)
-#endif
-#ifndef SOL_POOL_TPI
-#define SOL_POOL_TPI 2  // tokens whose loads are in flight together
-#endif
-#ifndef SOL_POOL_REGS_MINB
-#define SOL_POOL_REGS_MINB 3
-#endif
-
-namespace {
-
-template <int SPW>
-__device__ __forceinline__ void pool_row(const uint4 (&xv)[SPW], bf16* row, float (&acc)[SPW][8], const float (&w)[8],
-                                         const float (&cs)[4], const float (&sn)[4], float eps)
-{
-    // the plain epilogue's arithmetic (qk_math.cuh), so the in-place rows are the same bits
-    float kc[16];
-    qk_coefs(w, cs, sn, kc);
-    float ss[SPW];
-#pragma unroll
-    for (int i = 0; i < SPW; ++i) {
-        float2 f[4];
-        unpack2<bf16>(xv[i], f);
-        ss[i] = qk_sumsq(f);
-    }
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) {
-#pragma unroll
-        for (int i = 0; i < SPW; ++i) ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], off);
-    }
-#pragma unroll
-    for (int i = 0; i < SPW; ++i) {
-        float2 f[4];
-        unpack2<bf16>(xv[i], f);
-        float o[8];
-        qk_rotate(f, rsqrtf(ss[i] * (1.f / 128.f) + eps), kc, o);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[i][e] += o[e];
-        st_stream(row + 256 * i, pack<bf16>(o));
-    }
-}
-
-}  // namespace
-
-template <int SPW, int TPI, int PARTS>
-__global__ void __launch_bounds__(32 * PARTS, SOL_POOL_REGS_MINB)
-    k_qk_pool_regs(bf16* q, bf16* k, int64_t ld_q, int64_t ld_k, bf16* pq, bf16* pk, int64_t ld_pq, int64_t ld_pk,
-                   const bf16* __restrict__ wq, const bf16* __restrict__ wk, const int32_t* __restrict__ pos,
-                   int32_t grid_H, int32_t grid_W, int64_t tps, int32_t block, int64_t bps, int64_t n_blocks,
-                   RopeDev rope, int64_t n_tokens, float eps)
-{
-    const int lane = threadIdx.x & 31;
-    const int sub = lane & 15;
-    const int part = threadIdx.x >> 5;  // which SPW slots of the row this warp holds
-    const float2* tb[4];
-    int stride[4], axis[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const int pi = 4 * sub + m;
-        const int h0 = rope.half[0], h01 = rope.half[0] + rope.half[1];
-        axis[m] = pi < h0 ? 0 : (pi < h01 ? 1 : 2);
-        tb[m] = axis[m] == 0 ? rope.tab[0] + pi : (axis[m] == 1 ? rope.tab[1] + (pi - h0) : rope.tab[2] + (pi - h01));
-        stride[m] = axis[m] == 0 ? rope.half[0] : (axis[m] == 1 ? rope.half[1] : rope.half[2]);
-    }
-    for (int64_t c = blockIdx.x; c < 2 * n_blocks; c += gridDim.x) {
-        const int64_t blk = c >> 1;
-        const bool isk = (c & 1) != 0;  // uniform over the CTA
-        const bf16* wsrc = isk ? wk : wq;
-        float w[8];
-        if (wsrc) {
-            unpack<bf16>(ld_cached(wsrc + 8 * sub), w);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = 1.f;
-        }
-        const int64_t sample = blk / bps;
-        const int64_t t0 = sample * tps + (blk - sample * bps) * block;
-        int64_t t1 = t0 + block;
-        if (t1 > (sample + 1) * tps) t1 = (sample + 1) * tps;
-        if (t1 > n_tokens) t1 = n_tokens;
-        bf16* rows = (isk ? k : q) + 256 * SPW * part + 8 * lane;
-        const int64_t ld = isk ? ld_k : ld_q;
-        int g0 = 0, g1 = 0, g2 = 0;  // grid position of the next token (implicit positions)
-        if (!pos) {
-            const int64_t nl = t0 - sample * tps;
-            g0 = (int)(nl / ((int64_t)grid_H * grid_W));
-            g1 = (int)((nl / grid_W) % grid_H);
-            g2 = (int)(nl % grid_W);
-        }
-        auto next_angles = [&](int64_t n, float (&cs)[4], float (&sn)[4]) {
-            int p0, p1, p2;
-            if (pos) {
-                p0 = min(max(__ldg(pos + 3 * n + 0), 0), rope.max[0] - 1);
-                p1 = min(max(__ldg(pos + 3 * n + 1), 0), rope.max[1] - 1);
-                p2 = min(max(__ldg(pos + 3 * n + 2), 0), rope.max[2] - 1);
-            } else {
-                p0 = g0;
-                p1 = g1;
-                p2 = g2;
-                if (++g2 == grid_W) {
-                    g2 = 0;
-                    if (++g1 == grid_H) {
-                        g1 = 0;
-                        ++g0;
-                    }
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int pm = axis[m] == 0 ? p0 : (axis[m] == 1 ? p1 : p2);
-                const float2 t = __ldg(tb[m] + (int64_t)pm * stride[m]);
-                cs[m] = t.x;
-                sn[m] = t.y;
-            }
-        };
-        float acc[SPW][8];
-#pragma unroll
-        for (int i = 0; i < SPW; ++i)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
-        for (int64_t n = t0; n < t1; n += TPI) {
-            const int cnt = t1 - n < TPI ? (int)(t1 - n) : TPI;  // uniform over the CTA
-            uint4 xv[TPI][SPW];
-#pragma unroll
-            for (int t = 0; t < TPI; ++t) {
-                if (t < cnt) {
-#pragma unroll
-                    for (int i = 0; i < SPW; ++i) xv[t][i] = ld_stream(rows + (n + t) * ld + 256 * i);
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < TPI; ++t) {
-                if (t < cnt) {
-                    float cs[4], sn[4];
-                    next_angles(n + t, cs, sn);
-                    pool_row<SPW>(xv[t], rows + (n + t) * ld, acc, w, cs, sn, eps);
-                }
-            }
-        }
-        const float inv = 1.f / (float)(t1 - t0);
-        bf16* out = (isk ? pk + blk * ld_pk : pq + blk * ld_pq) + 256 * SPW * part + 8 * lane;
-#pragma unroll
-        for (int i = 0; i < SPW; ++i) {
-            float o[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = acc[i][e] * inv;
-            st_stream(out + 256 * i, pack<bf16>(o));
-        }
-    }
-}
-
 namespace {
 
 constexpr int kPoolThreads = 32 * kPoolWarps;
@@ -397,31 +234,6 @@ cudaError_t run_pool(void* q, void* k, int64_t ld_q, int64_t ld_k, void* pq, voi
     return cudaGetLastError();
 }
 
-template <int SPW>
-cudaError_t run_pool_regs(void* q, void* k, int64_t ld_q, int64_t ld_k, void* pq, void* pk, int64_t ld_pq,
-                          int64_t ld_pk, const void* wq, const void* wk, const int32_t* pos, int32_t grid_H,
-                          int32_t grid_W, int64_t tps, int32_t block, int64_t bps, int64_t n_blocks,
-                          const RopeDev& rope, int64_t n_tokens, float eps, cudaStream_t s)
-{
-    auto kern = k_qk_pool_regs<SPW, SOL_POOL_TPI, SOL_POOL_PARTS>;
-    constexpr int threads = 32 * SOL_POOL_PARTS;
-    if (ctas_per_sm(reinterpret_cast<const void*>(kern), threads, 0) < 1) return cudaErrorInvalidConfiguration;
-    // one CTA per (block, q or k): SMs are refilled as CTAs retire
-    const int64_t grid = 2 * n_blocks < 0x7fffffffLL ? 2 * n_blocks : 0x7fffffffLL;
-    kern<<<(unsigned)grid, threads, 0, s>>>(static_cast<bf16*>(q), static_cast<bf16*>(k), ld_q, ld_k,
-                                       static_cast<bf16*>(pq), static_cast<bf16*>(pk), ld_pq, ld_pk,
-                                       static_cast<const bf16*>(wq), static_cast<const bf16*>(wk), pos, grid_H,
-                                       grid_W, tps, block, bps, n_blocks, rope, n_tokens, eps);
-    return cudaGetLastError();
-}
-
-bool pool_regs_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim)
-{
-    constexpr int heads_step = 2 * SOL_POOL_PARTS;
-    return dt == SOL_DTYPE_BF16 && head_dim == 128 && n_heads % heads_step == 0 && n_heads >= heads_step &&
-           n_heads <= 48;
-}
-
 }  // namespace
 
 size_t qk_pool_smem_bytes(sol_dtype dt, int32_t n_heads, int32_t head_dim)
@@ -441,19 +253,9 @@ cudaError_t launch_qk_rope_pool(sol_dtype dt, void* q, void* k, int64_t ld_q, in
                                 int64_t n_tokens, int32_t n_heads, int32_t head_dim, float eps,
                                 cudaStream_t s)
 {
-    if (pool_regs_fits(dt, n_heads, head_dim)) {
-        switch (n_heads / (2 * SOL_POOL_PARTS)) {  // slots per warp
-#define SOL_POOL_SPW(v)                                                                                            \
-    case v:                                                                                                        \
-        if constexpr (v * 2 * SOL_POOL_PARTS <= 48)                                                                \
-            return run_pool_regs<v>(q, k, ld_q, ld_k, pq, pk, ld_pq, ld_pk, wq, wk, pos, grid_H, grid_W, tps,      \
-                                    block, bps, n_blocks, rope, n_tokens, eps, s);                                 \
-        break;
-            SOL_POOL_SPW(1) SOL_POOL_SPW(2) SOL_POOL_SPW(3) SOL_POOL_SPW(4) SOL_POOL_SPW(5) SOL_POOL_SPW(6)
-            SOL_POOL_SPW(7) SOL_POOL_SPW(8) SOL_POOL_SPW(9) SOL_POOL_SPW(10) SOL_POOL_SPW(11) SOL_POOL_SPW(12)
-#undef SOL_POOL_SPW
-        }
-    }
+    if (qk_pool_stage_fits(dt, n_heads, head_dim, q, k, tps, n_blocks))  // staged rows (k_qk_cta.cu)
+        return launch_qk_pool_stage(q, k, ld_q, ld_k, pq, pk, ld_pq, ld_pk, wq, wk, pos, grid_H, grid_W, tps, block,
+                                    bps, n_blocks, rope, n_tokens, n_heads, eps, s);
     const int lph = head_dim / (dt == SOL_DTYPE_BF16 ? 8 : 4);
 #define ARGS q, k, ld_q, ld_k, pq, pk, ld_pq, ld_pk, wq, wk, pos, grid_H, grid_W, tps, block, bps, n_blocks, rope, n_tokens, n_heads, eps, s
     if (dt == SOL_DTYPE_BF16) {

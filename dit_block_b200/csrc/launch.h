@@ -82,7 +82,15 @@ cudaError_t launch_qk_cta_ex(bool across, bool half, void* q_out, void* k_out, c
                              const void* k, int64_t ld_q, int64_t ld_k, const void* wq, const void* wk,
                              const int32_t* pos, int32_t grid_H, int32_t grid_W, int64_t tps, const RopeDev& rope,
                              int64_t n_tokens, int32_t n_heads, float eps, cudaStream_t s);
-// Error flags of that kernel's bounded wait (bit 1); optionally cleared.  Synchronous.
+// The QKV epilogue with block means, staged (k_qk_cta.cu): bf16, head_dim 128, an even
+// number of heads up to 48, q and k both given.
+bool qk_pool_stage_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim, const void* q, const void* k,
+                        int64_t tps, int64_t n_blocks);
+cudaError_t launch_qk_pool_stage(void* q, void* k, int64_t ld_q, int64_t ld_k, void* pq, void* pk, int64_t ld_pq,
+                                 int64_t ld_pk, const void* wq, const void* wk, const int32_t* pos, int32_t grid_H,
+                                 int32_t grid_W, int64_t tps, int32_t block, int64_t bps, int64_t n_blocks,
+                                 const RopeDev& rope, int64_t n_tokens, int32_t n_heads, float eps, cudaStream_t s);
+// Error flags of these kernels' bounded waits (bit 1); optionally cleared.  Synchronous.
 uint32_t qk_device_error(bool clear);
 
 // QK RMSNorm + 3D RoPE, convention variants (k_qk_ex.cu): `across` = RMS over all heads

@@ -1,6 +1,6 @@
 // qk_math.cuh -- the per-slot arithmetic of QK RMSNorm + interleaved 3D RoPE shared by the
-// staged kernel (k_qk_cta.cu), the row-in-registers kernel (k_qk_regs.cu) and k_qk_pool.cu,
-// whose in-place results must equal the plain epilogue's bit for bit.
+// staged kernels (k_qk_cta.cu: the epilogue and the epilogue with block means) and the
+// row-in-registers kernel (k_qk_regs.cu), whose in-place results must be the same bits.
 //
 // A lane holds 8 consecutive elements (4 interleaved rotary pairs) of a head vector; its
 // RMSNorm weights w[0..7] and its pairs' (cos, sin) are fixed for the row, so the weights

@@ -166,8 +166,10 @@ POOL_CASES = [  # dtype, head_dim, dims, n_heads, grid, samples, audio tokens pe
     (BF, 128, (32, 48, 48), 40, (2, 3, 4), 2, 5, 64),    # packed video+audio, explicit positions
     (torch.float32, 128, (32, 48, 48), 2, (2, 4, 4), 1, 0, 64),
     (torch.float32, 32, (8, 12, 12), 7, (3, 3, 3), 2, 0, 5),
-    (BF, 128, (32, 48, 48), 8, (3, 3, 5), 2, 3, 7),      # register kernel, 1 slot per warp, odd blocks
-    (BF, 128, (32, 48, 48), 48, (2, 2, 3), 1, 0, 5),     # register kernel, 6 slots per warp
+    (BF, 128, (32, 48, 48), 8, (3, 3, 5), 2, 3, 7),      # staged kernel, 1 vector a thread, odd blocks
+    (BF, 128, (32, 48, 48), 48, (2, 2, 3), 1, 0, 5),     # staged kernel at its widest (6 vectors a thread)
+    (BF, 128, (32, 48, 48), 2, (2, 3, 3), 2, 1, 64),     # 2 heads: one warp busy; 19-token blocks
+    (BF, 128, (32, 48, 48), 6, (1, 3, 3), 2, 0, 4),      # blocks of 4, 4 and 1 token (fewer than the ring)
 ]
 
 
