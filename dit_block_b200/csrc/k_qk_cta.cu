@@ -456,6 +456,7 @@ __global__ void __launch_bounds__(kHeadThreads, kPoolCtas)
     if (t1 > (sample + 1) * tps) t1 = (sample + 1) * tps;
     if (t1 > n_tokens) t1 = n_tokens;
     const int cnt = (int)(t1 - t0);
+    if (cnt <= 0) return;  // no block is empty (the host counts them); uniform over the CTA
     bf16* const rows_g = isk ? k : q;
     const int64_t ld = isk ? ld_k : ld_q;
 
