@@ -1,5 +1,5 @@
 """The token-sharded split (dit_block_b200.shard) on CPU: the ranges, the pieces cut at
-sample boundaries, the global positions and stream ids, and -- over two gloo ranks --
+sample boundaries, the global positions and stream ids, and -- over two and four gloo ranks --
 the fp64 oracle run on each rank's pieces reproducing the single-rank oracle over the
 whole sequence bit for bit.  The split needs no collective on the data path; the test
 gathers the ranks' results only to compare them."""
@@ -137,7 +137,10 @@ def _worker(rank, world, port, q):
 
 
 @pytest.mark.timeout(600)
-def test_two_ranks_reproduce_the_single_rank_oracle():
+@pytest.mark.parametrize("world", [2, 4])
+def test_ranks_reproduce_the_single_rank_oracle(world):
+    """Two ranks cut both layouts inside a sample; four ranks also give one rank the end of
+    one sample and the start of the next."""
     import oracle
     oracle.build()
     ctx = mp.get_context("spawn")
@@ -145,7 +148,7 @@ def test_two_ranks_reproduce_the_single_rank_oracle():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         port = s.getsockname()[1]
-    ps = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    ps = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in ps:
         p.start()
     res = [q.get(timeout=300) for _ in ps]
@@ -166,5 +169,7 @@ def test_two_ranks_reproduce_the_single_rank_oracle():
                 for k, v in part.items():
                     assert np.array_equal(v, whole[k][t0:t1]), f"{w.name} rank {rank}: {k}[{t0}:{t1}]"
             assert np.all(covered == 1), f"{w.name}: tokens not covered exactly once"
-        # the cut falls inside a sample for both layouts
-        assert shard.token_ranges(w.n_tokens, 2)[0][1] % w.tokens_per_sample != 0
+        # the first cut falls inside a sample for both layouts
+        assert shard.token_ranges(w.n_tokens, world)[0][1] % w.tokens_per_sample != 0
+    if world == 4:  # a rank whose range spans a sample boundary
+        assert any(len(shard.pieces(PACKED, t0, t1)) > 1 for t0, t1 in shard.token_ranges(PACKED.n_tokens, 4))
