@@ -380,7 +380,7 @@ bool qk_cta_fits(sol_dtype dt, int32_t n_heads, int32_t head_dim, const void* q,
            n_tokens < ((int64_t)1 << 31);
 }
 
-bool qk_cta_ex_fits(sol_dtype dt, bool across, bool half, int32_t n_heads, int32_t head_dim,
+bool qk_cta_ex_fits(sol_dtype dt, bool half, int32_t n_heads, int32_t head_dim,
                     const void* q, const void* k, int64_t n_tokens, int64_t tps, const RopeDev& rope)
 {
     if (!qk_cta_fits(dt, n_heads, head_dim, q, k, n_tokens) || tps >= ((int64_t)1 << 31)) return false;

@@ -243,7 +243,7 @@ cudaError_t launch_qk_ex(sol_dtype dt, bool across, bool half, void* q_out, void
                          int64_t tps, const RopeDev& rope, int64_t n_tokens, int32_t n_heads,
                          int32_t head_dim, float eps, cudaStream_t s)
 {
-    if (qk_cta_ex_fits(dt, across, half, n_heads, head_dim, q, k, n_tokens, tps, rope))  // staged rows (k_qk_cta.cu)
+    if (qk_cta_ex_fits(dt, half, n_heads, head_dim, q, k, n_tokens, tps, rope))  // staged rows (k_qk_cta.cu)
         return launch_qk_cta_ex(across, half, q_out, k_out, os, q, k, ld_q, ld_k, wq, wk, pos, grid_H, grid_W, tps,
                                 rope, n_tokens, n_heads, eps, s);
     const int lph = head_dim / (dt == SOL_DTYPE_BF16 ? 8 : 4);

@@ -76,7 +76,7 @@ cudaError_t launch_qk_cta(void* q_out, void* k_out, int64_t ld_qo, int64_t ld_ko
                           int32_t n_heads, float eps, cudaStream_t s);
 // The same kernel for the convention variants: norm across heads, rotate-half pairs (chunk
 // halves multiples of 4), strided outputs.
-bool qk_cta_ex_fits(sol_dtype dt, bool across, bool half, int32_t n_heads, int32_t head_dim,
+bool qk_cta_ex_fits(sol_dtype dt, bool half, int32_t n_heads, int32_t head_dim,
                     const void* q, const void* k, int64_t n_tokens, int64_t tps, const RopeDev& rope);
 cudaError_t launch_qk_cta_ex(bool across, bool half, void* q_out, void* k_out, const QkOutStrides& os, const void* q,
                              const void* k, int64_t ld_q, int64_t ld_k, const void* wq, const void* wk,
